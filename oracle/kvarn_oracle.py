@@ -1,0 +1,274 @@
+"""Float64 CPU oracle of KVarN-style variance-normalised KV-cache quantisation.
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, obviously correct
+statement of what the CUDA path computes.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+it; the library (``kv_cache_quantization_03_b200``) never does, and this module
+imports nothing from the library.  It shares no code, table or constant
+generator with the kernels.
+
+What it follows
+---------------
+The KVarN pipeline as the pages describe it, one tile (T tokens x d channels
+of one layer / kv-head, keys or values alone) at a time:
+
+1. a Hadamard rotation along head_dim that spreads channel outliers
+   (KVarN project page on open-radar, Key Features, "Variance-Normalized
+   Quantization Pipeline"; KV-Cache tag page on baguaai.com, KVarN item:
+   rotation combined with dual-axis variance normalisation);
+2. an iterative Sinkhorn-like normalisation that equalises the variance of
+   the tile's rows (tokens) and columns (channels), computed per tile with no
+   calibration (same page, "Calibration-Free Operation");
+3. asymmetric round-to-nearest quantisation (same pages; the KV-Cache tag
+   page names RTN);
+4. packing of the codes into the paged cache, one tile per cache block
+   (KVarN project page, "4-bit Keys, 2-bit Values Preset": the tile equals
+   the serving engine's block).
+
+and the consumer: decode attention over the quantised cache with the query
+rotated by the same orthogonal Hadamard, plus the MLA variant in which one
+quantised latent serves as both key and value next to an unquantised rope
+key (KVarN project page, "MLA Model Support").
+
+Readings where the pages are silent (each is a declared choice):
+
+* "variance" is the uncentred second moment (mean of squares); with it the
+  normalisation is Sinkhorn-Knopp scaling of the positive matrix Z*Z, which
+  converges, whereas the centred form does not settle;
+* each iteration normalises the rows first, then the columns; a row or
+  column whose second moment is exactly 0 is left as it is (factor 1);
+* the Hadamard matrix is Sylvester's, of full width d, scaled by 1/sqrt(d);
+* quantisation groups are token rows of the normalised tile: zero point
+  m = row min (a float), step s = (max - min) / (2^b - 1), codes
+  rint((y - m) / s) with ties to even, clamped to [0, 2^b - 1]; s = 0 gives
+  code 0;
+* the row and column factors are folded into what is stored: per token
+  a = r * s and z = r * m, per channel c, all float32 (round to nearest);
+  dequantisation in the rotated domain is (a * q + z) * c;
+* codes are packed little-endian inside each byte, lowest channel in the
+  lowest bits, token rows one after the other; 3-bit codes are two planes
+  per tile: all rows' low 2 bits (2-bit packing), then all rows' high bit
+  (1-bit packing).
+
+All arithmetic is float64 except the float32 rounding of the stored a, z, c.
+Parity of every function here is pinned in tests/test_oracle_pins.py against
+closed forms, library routines, brute force and hand-worked fixtures.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+
+SUPPORTED_BITS = (2, 3, 4, 8)
+
+
+# --------------------------------------------------------------------------
+# 1. Hadamard rotation
+# --------------------------------------------------------------------------
+def hadamard_matrix(n: int) -> np.ndarray:
+    """Sylvester Hadamard matrix of order n (a power of two), int64 entries +-1.
+
+    H_1 = [1];  H_2k = [[H_k, H_k], [H_k, -H_k]].  Unnormalised: H H^T = n I.
+    """
+    if n < 1 or n & (n - 1):
+        raise ValueError("order must be a power of two")
+    h = np.ones((1, 1), dtype=np.int64)
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def rotate(x: np.ndarray) -> np.ndarray:
+    """x H / sqrt(d) along the last axis (float64).
+
+    H / sqrt(d) is symmetric and orthogonal, so the same call undoes itself:
+    rotate(rotate(x)) == x up to rounding.  Dense product, no fast transform.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    return (x @ hadamard_matrix(d).astype(np.float64)) / math.sqrt(d)
+
+
+# --------------------------------------------------------------------------
+# 2. Sinkhorn-like dual-axis variance normalisation
+# --------------------------------------------------------------------------
+def sinkhorn_normalize(z: np.ndarray, n_iter: int, history: Optional[list] = None):
+    """Normalise the second moments of rows and columns of each tile.
+
+    z: [..., T, d] float64 (rotated tile(s)).  Returns (y, r, c) with
+    y: [..., T, d], r: [..., T], c: [..., d] such that z = diag(r) y diag(c).
+
+    Each of the n_iter rounds divides every row by its root-mean-square
+    (over d channels) and multiplies that factor into r, then divides every
+    column by its root-mean-square (over T tokens) and multiplies it into c.
+    A zero root-mean-square leaves its row or column unchanged.  If
+    ``history`` is a list, (y, r, c) after every half-step is appended.
+    """
+    y = np.array(z, dtype=np.float64, copy=True)
+    r = np.ones(y.shape[:-1], dtype=np.float64)
+    c = np.ones(y.shape[:-2] + y.shape[-1:], dtype=np.float64)
+    for _ in range(n_iter):
+        sigma = np.sqrt(np.mean(y * y, axis=-1))            # row RMS, [..., T]
+        f = np.where(sigma > 0, sigma, 1.0)
+        y = y / f[..., :, None]
+        r = r * f
+        if history is not None:
+            history.append((y.copy(), r.copy(), c.copy()))
+        tau = np.sqrt(np.mean(y * y, axis=-2))              # column RMS, [..., d]
+        g = np.where(tau > 0, tau, 1.0)
+        y = y / g[..., None, :]
+        c = c * g
+        if history is not None:
+            history.append((y.copy(), r.copy(), c.copy()))
+    return y, r, c
+
+
+# --------------------------------------------------------------------------
+# 3. Asymmetric round-to-nearest quantisation (per token row)
+# --------------------------------------------------------------------------
+def rtn_rows(y: np.ndarray, bits: int):
+    """Asymmetric RTN of every row of y: [..., T, d] -> (q int64, m, s).
+
+    m = row min, s = (row max - m) / (2^bits - 1),
+    q = clamp(rint((y - m) / s), 0, 2^bits - 1)  (rint rounds half to even);
+    rows with s == 0 get q = 0.
+    """
+    if bits not in SUPPORTED_BITS:
+        raise ValueError("bits must be one of %s" % (SUPPORTED_BITS,))
+    qmax = (1 << bits) - 1
+    m = np.min(y, axis=-1)
+    s = (np.max(y, axis=-1) - m) / qmax
+    safe = np.where(s > 0, s, 1.0)
+    t = (y - m[..., None]) / safe[..., None]
+    q = np.clip(np.rint(t), 0, qmax).astype(np.int64)
+    q = np.where((s > 0)[..., None], q, 0)
+    return q, m, s
+
+
+@dataclasses.dataclass
+class QuantizedTiles:
+    """What one or more quantised tiles store: logical codes and folded scales."""
+    q: np.ndarray   # int64 [..., T, d]   codes in [0, 2^bits - 1]
+    a: np.ndarray   # float32 [..., T]    a = r * s
+    z: np.ndarray   # float32 [..., T]    z = r * m
+    c: np.ndarray   # float32 [..., d]    column factor
+
+
+def quantize_tiles(x: np.ndarray, bits: int, n_iter: int) -> QuantizedTiles:
+    """Rotate, normalise and quantise tiles x: [..., T, d] (any float dtype).
+
+    The tiles are independent; leading axes only batch them.
+    """
+    z = rotate(x)
+    y, r, c = sinkhorn_normalize(z, n_iter)
+    q, m, s = rtn_rows(y, bits)
+    return QuantizedTiles(q=q, a=(r * s).astype(np.float32), z=(r * m).astype(np.float32),
+                          c=c.astype(np.float32))
+
+
+def dequantize_tiles(q, a, z, c, unrotate: bool = True) -> np.ndarray:
+    """(a q + z) c in the rotated domain (float64), then optionally un-rotated."""
+    a = np.asarray(a, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    c = np.asarray(c, dtype=np.float64)
+    zh = (a[..., :, None] * np.asarray(q, dtype=np.float64) + z[..., :, None]) * c[..., None, :]
+    return rotate(zh) if unrotate else zh
+
+
+# --------------------------------------------------------------------------
+# 4. Packing into the cache's byte format
+# --------------------------------------------------------------------------
+def tile_code_bytes(bits: int, tile_tokens: int, head_dim: int) -> int:
+    return tile_tokens * head_dim * bits // 8
+
+
+def _pack_fields(v: np.ndarray, width: int) -> np.ndarray:
+    """Pack [..., n] small ints of `width` bits, 8/width per byte, low bits first."""
+    per = 8 // width
+    v = v.reshape(v.shape[:-1] + (v.shape[-1] // per, per)).astype(np.uint16)
+    out = np.zeros(v.shape[:-1], dtype=np.uint16)
+    for i in range(per):
+        out |= v[..., i] << (width * i)
+    return out.astype(np.uint8)
+
+
+def _unpack_fields(b: np.ndarray, width: int) -> np.ndarray:
+    per = 8 // width
+    b = b.astype(np.uint16)
+    mask = (1 << width) - 1
+    parts = [(b >> (width * i)) & mask for i in range(per)]
+    return np.stack(parts, axis=-1).reshape(b.shape[:-1] + (b.shape[-1] * per,)).astype(np.int64)
+
+
+def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
+    """Logical codes [..., T, d] -> bytes [..., T * d * bits / 8] of one tile each."""
+    q = np.asarray(q)
+    lead, (T, d) = q.shape[:-2], q.shape[-2:]
+    if bits in (2, 4, 8):
+        return _pack_fields(q, bits).reshape(lead + (T * d * bits // 8,))
+    if bits == 3:
+        lo = _pack_fields(q & 3, 2).reshape(lead + (T * d // 4,))
+        hi = _pack_fields(q >> 2, 1).reshape(lead + (T * d // 8,))
+        return np.concatenate([lo, hi], axis=-1)
+    raise ValueError("bits")
+
+
+def unpack_codes(buf: np.ndarray, bits: int, tile_tokens: int, head_dim: int) -> np.ndarray:
+    """Inverse of pack_codes: bytes [..., nbytes] -> int64 codes [..., T, d]."""
+    buf = np.asarray(buf, dtype=np.uint8)
+    lead = buf.shape[:-1]
+    T, d = tile_tokens, head_dim
+    if bits in (2, 4, 8):
+        return _unpack_fields(buf.reshape(lead + (T, d * bits // 8)), bits)
+    if bits == 3:
+        lo = _unpack_fields(buf[..., : T * d // 4].reshape(lead + (T, d // 4)), 2)
+        hi = _unpack_fields(buf[..., T * d // 4:].reshape(lead + (T, d // 8)), 1)
+        return lo | (hi << 2)
+    raise ValueError("bits")
+
+
+# --------------------------------------------------------------------------
+# 5. Decode attention over the quantised cache
+# --------------------------------------------------------------------------
+def _softmax(s: np.ndarray) -> np.ndarray:
+    e = np.exp(s - np.max(s, axis=-1, keepdims=True))
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def decode_attention(q: np.ndarray, k: QuantizedTiles, v: QuantizedTiles,
+                     softmax_scale: float) -> np.ndarray:
+    """One decode step of the G query heads that share one kv-head.
+
+    q: [G, d] (float, un-rotated).  k, v: the kv-head's tiles in token order,
+    q/a/z/c with leading tile axis [n_tiles, T, ...].  Returns o: [G, d]
+    float64, un-rotated.  The query is rotated with the same H as the cache,
+    attention runs in the rotated domain on the dequantised tiles, and the
+    output is rotated back.
+    """
+    d = q.shape[-1]
+    kh = dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=False).reshape(-1, d)
+    vh = dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=False).reshape(-1, d)
+    qr = rotate(q)
+    p = _softmax(softmax_scale * (qr @ kh.T))
+    return rotate(p @ vh)
+
+
+def mla_decode_attention(q: np.ndarray, lat: QuantizedTiles, rope: np.ndarray,
+                         softmax_scale: float) -> np.ndarray:
+    """MLA decode step: one quantised latent serves as key and value.
+
+    q: [H, d + rope_dim] (latent part un-rotated, rope part as is).
+    lat: the latent tiles [n_tiles, T, d]; rope: [n_tiles * T, rope_dim] keys.
+    Score of token t: scale * (rotate(q_lat) . latent_t + q_rope . rope_t);
+    output: rotate back (sum_t p_t latent_t): [H, d] float64.
+    """
+    d = lat.q.shape[-1]
+    ch = dequantize_tiles(lat.q, lat.a, lat.z, lat.c, unrotate=False).reshape(-1, d)
+    q = np.asarray(q, dtype=np.float64)
+    qr = rotate(q[:, :d])
+    s = qr @ ch.T + q[:, d:] @ np.asarray(rope, dtype=np.float64).T
+    p = _softmax(softmax_scale * s)
+    return rotate(p @ ch)

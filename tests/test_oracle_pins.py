@@ -1,0 +1,300 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Closed forms, library routines (scipy's Hadamard, torch's scaled-dot-product
+attention in float64), brute force on tiny inputs, invariants of the method and
+hand-worked fixtures under tests/golden/.  Each test is chosen so that a
+plausible slip in the oracle (a dropped term, a wrong sign or axis, a
+transposed operand, a wrong rounding rule) fails it.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import kvarn_oracle as O
+from kv_cache_quantization_03_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- Hadamard
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 128, 512])
+def test_hadamard_orthogonal_exact(n):
+    h = O.hadamard_matrix(n)
+    assert h.dtype == np.int64
+    assert np.array_equal(h @ h.T, n * np.eye(n, dtype=np.int64))
+    assert np.array_equal(h, h.T)
+
+
+def test_hadamard_small_cases_and_scipy():
+    import scipy.linalg
+    assert np.array_equal(O.hadamard_matrix(2), [[1, 1], [1, -1]])
+    assert np.array_equal(O.hadamard_matrix(4), [[1, 1, 1, 1], [1, -1, 1, -1],
+                                                 [1, 1, -1, -1], [1, -1, -1, 1]])
+    for n in (8, 64, 128, 512):
+        assert np.array_equal(O.hadamard_matrix(n), scipy.linalg.hadamard(n))
+
+
+def test_hadamard_entry_formula():
+    # Sylvester entries: (-1)^popcount(i & j)
+    n = 128
+    h = O.hadamard_matrix(n)
+    i, j = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+    pc = np.vectorize(lambda v: bin(v).count("1"))(i & j)
+    assert np.array_equal(h, np.where(pc % 2 == 0, 1, -1))
+
+
+def test_rotate_roundtrip_and_parseval():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 16, 128)) * 7.0
+    y = O.rotate(x)
+    assert np.max(np.abs(O.rotate(y) - x)) <= 1e-12 * np.max(np.abs(x))
+    assert np.allclose(np.sum(y * y, -1), np.sum(x * x, -1), rtol=1e-12, atol=0)
+    # a single basis vector spreads evenly over all channels (outlier spreading)
+    e = np.zeros(128); e[17] = 1.0
+    assert np.allclose(np.abs(O.rotate(e)), 1 / math.sqrt(128), rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- Sinkhorn
+def test_sinkhorn_closed_form_rank_one_scaling():
+    # Z = diag(u) S diag(v) with S = +-1 reaches Y = S after one round,
+    # with r_i c_j = u_i v_j.
+    rng = np.random.default_rng(2)
+    T, d = 16, 128
+    u = np.exp(rng.uniform(-2, 2, T))
+    v = np.exp(rng.uniform(-2, 2, d))
+    s = np.where(rng.random((T, d)) < 0.5, -1.0, 1.0)
+    z = u[:, None] * s * v[None, :]
+    for n in (1, 4):
+        y, r, c = O.sinkhorn_normalize(z, n)
+        assert np.max(np.abs(y - s)) < 1e-12
+        assert np.max(np.abs(np.outer(r, c) / np.outer(u, v) - 1)) < 1e-12
+
+
+def test_sinkhorn_golden_rank1():
+    fx = _golden("tile_t2_d4_rank1.json")
+    z = np.array(fx["z_rotated"])
+    y, r, c = O.sinkhorn_normalize(z, fx["n_iter"])
+    assert np.allclose(c, fx["c"], rtol=1e-14, atol=0)
+    s = np.array([[1, -1, 1, 1], [-1, 1, 1, -1]], dtype=float)
+    assert np.allclose(y, s, rtol=0, atol=1e-14)
+
+
+def test_sinkhorn_invariant_every_half_step():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-3, 3, 128))
+    hist = []
+    O.sinkhorn_normalize(z, 5, history=hist)
+    assert len(hist) == 10
+    for y, r, c in hist:
+        assert np.max(np.abs(r[:, None] * y * c[None, :] - z)) <= 1e-12 * np.max(np.abs(z))
+
+
+def test_sinkhorn_uncentred_second_moment_not_variance():
+    # rows with a large mean: the reading normalises the mean of squares,
+    # so a centred variance would differ from 1 while the RMS is 1.
+    rng = np.random.default_rng(4)
+    z = rng.standard_normal((16, 128)) + 3.0
+    y, _, _ = O.sinkhorn_normalize(z, 60)
+    rms_rows = np.sqrt(np.mean(y * y, -1))
+    assert np.max(np.abs(rms_rows - 1)) < 1e-9
+    assert np.max(np.abs(np.var(y, -1) - 1)) > 0.5
+
+
+def test_sinkhorn_order_rows_then_columns():
+    # After any number of rounds the column step came last, so the columns are
+    # exactly normalised while the rows are only close.
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-2, 2, (16, 1)))
+    y, _, _ = O.sinkhorn_normalize(z, 2)
+    assert np.max(np.abs(np.sqrt(np.mean(y * y, 0)) - 1)) < 1e-13
+    assert np.max(np.abs(np.sqrt(np.mean(y * y, 1)) - 1)) > 1e-6
+
+
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla"])
+def test_sinkhorn_converges_on_workload_distributions(name):
+    # Row and column second moments equal 1 within 1e-6 after convergence,
+    # on tiles drawn from each workload's distribution.
+    w = W.WORKLOADS[name]
+    small = w.scaled(batch=1, seq_len=64 if not w.mla else 32, num_layers=1)
+    x = W.half_bits_to_f64(W.kv_inputs(small, "k"), w.in_dtype)      # [1, n, H, d]
+    tiles = x[0].reshape(-1, 16, small.num_kv_heads, w.head_dim).transpose(0, 2, 1, 3)
+    y, _, _ = O.sinkhorn_normalize(O.rotate(tiles), 50)
+    assert np.max(np.abs(np.mean(y * y, -1) - 1)) < 1e-6
+    assert np.max(np.abs(np.mean(y * y, -2) - 1)) < 1e-6
+
+
+def test_sinkhorn_zero_rows_and_columns_untouched():
+    z = np.zeros((16, 8))
+    z[3, :] = np.arange(1, 9)
+    y, r, c = O.sinkhorn_normalize(z, 4)
+    assert np.all(np.isfinite(y))
+    assert np.array_equal(np.delete(r, 3), np.ones(15))
+    y0, r0, c0 = O.sinkhorn_normalize(np.zeros((16, 8)), 4)
+    assert np.all(y0 == 0) and np.all(r0 == 1) and np.all(c0 == 1)
+
+
+# ---------------------------------------------------------------- RTN
+def test_rtn_golden_ties_to_even():
+    fx = _golden("rtn_ties.json")
+    q, m, s = O.rtn_rows(np.array(fx["y"]), fx["bits"])
+    assert np.array_equal(q, fx["q"])
+    assert np.array_equal(m, fx["m"]) and np.array_equal(s, fx["s"])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_rtn_is_nearest_level_brute_force(bits):
+    rng = np.random.default_rng(6 + bits)
+    y = rng.standard_normal((64, 16))
+    q, m, s = O.rtn_rows(y, bits)
+    levels = np.arange(1 << bits)
+    recon = m[:, None, None] + s[:, None, None] * levels[None, None, :]
+    err = np.abs(y[:, :, None] - recon)
+    best = np.argmin(err, axis=-1)            # first minimum; no exact ties here
+    assert np.array_equal(q, best)
+    assert np.all(np.abs(y - (m[:, None] + s[:, None] * q)) <= s[:, None] / 2 * (1 + 1e-12))
+    assert np.all(q[np.arange(64), np.argmin(y, 1)] == 0)
+    assert np.all(q[np.arange(64), np.argmax(y, 1)] == (1 << bits) - 1)
+
+
+# ---------------------------------------------------------------- tiles
+def test_quantize_golden_identity_tile():
+    fx = _golden("tile_t2_d2_identity.json")
+    qt = O.quantize_tiles(np.array(fx["x"]), fx["bits"], fx["n_iter"])
+    assert np.array_equal(qt.q, fx["q"])
+    for k in ("a", "z", "c"):
+        assert np.array_equal(getattr(qt, k), np.array(fx[k], dtype=np.float32)), k
+    xr = O.dequantize_tiles(qt.q, qt.a, qt.z, qt.c)
+    assert np.max(np.abs(xr - np.array(fx["x"]))) < 1e-7
+
+
+def test_quantize_golden_rank1_tile():
+    fx = _golden("tile_t2_d4_rank1.json")
+    x = O.rotate(np.array(fx["z_rotated"]))
+    qt = O.quantize_tiles(x, fx["bits"], fx["n_iter"])
+    assert np.array_equal(qt.q, fx["q"])
+    for k in ("a", "z", "c"):
+        assert np.allclose(getattr(qt, k), np.array(fx[k], dtype=np.float32), rtol=2e-7, atol=0), k
+
+
+def test_quantize_homogeneity_and_token_permutation():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-1, 1, 128))
+    base = O.quantize_tiles(x, 4, 4)
+    sc = O.quantize_tiles(x * 8.0, 4, 4)        # power of two: exact scaling
+    assert np.array_equal(sc.q, base.q)
+    assert np.array_equal(sc.a, base.a * 8) and np.array_equal(sc.z, base.z * 8)
+    assert np.array_equal(sc.c, base.c)
+    perm = rng.permutation(16)
+    pm = O.quantize_tiles(x[perm], 4, 4)
+    assert np.array_equal(pm.q, base.q[perm])
+    assert np.allclose(pm.a, base.a[perm], rtol=1e-6) and np.allclose(pm.z, base.z[perm], rtol=1e-6)
+    assert np.allclose(pm.c, base.c, rtol=1e-6)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_dequantize_error_bound(bits):
+    # In the rotated domain each element is off by at most half a step, times
+    # the row and column factors (plus float32 rounding of a, z, c).
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((4, 16, 128)) * np.exp(rng.uniform(-1, 1, (4, 1, 128)))
+    z = O.rotate(x)
+    y, r, c = O.sinkhorn_normalize(z, 4)
+    qt = O.quantize_tiles(x, bits, 4)
+    zh = O.dequantize_tiles(qt.q, qt.a, qt.z, qt.c, unrotate=False)
+    bound = (qt.a.astype(np.float64)[..., None] / 2 + 1e-6 * (np.abs(qt.a)[..., None] * (1 << bits) + np.abs(qt.z)[..., None])) \
+        * qt.c.astype(np.float64)[..., None, :]
+    assert np.all(np.abs(zh - z) <= bound)
+    assert np.allclose(O.dequantize_tiles(qt.q, qt.a, qt.z, qt.c), O.rotate(zh), rtol=0, atol=1e-12)
+
+
+def test_normalisation_does_not_hurt_on_outlier_rows():
+    # Sanity of the method, not of parity: on tiles whose tokens have very
+    # different scales the dual-axis normalisation keeps the error no worse
+    # than rotation + RTN alone.
+    rng = np.random.default_rng(9)
+    x = rng.standard_t(4.0, (64, 16, 128)) * np.exp(rng.uniform(-2, 2, (64, 16, 1)))
+    full = O.quantize_tiles(x, 4, 4)
+    rot = O.quantize_tiles(x, 4, 0)
+    e_full = np.mean((O.dequantize_tiles(full.q, full.a, full.z, full.c) - x) ** 2)
+    e_rot = np.mean((O.dequantize_tiles(rot.q, rot.a, rot.z, rot.c) - x) ** 2)
+    assert e_full <= 1.05 * e_rot
+
+
+# ---------------------------------------------------------------- packing
+def test_packing_golden():
+    fx = _golden("packing.json")
+    for case in fx["cases"]:
+        q = np.array(case["q"])
+        b = O.pack_codes(q, case["bits"])
+        assert list(b) == case["bytes"], case["bits"]
+        assert np.array_equal(O.unpack_codes(b, case["bits"], q.shape[0], q.shape[1]), q)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_unpack_roundtrip(bits):
+    rng = np.random.default_rng(10)
+    q = rng.integers(0, 1 << bits, size=(3, 16, 128))
+    b = O.pack_codes(q, bits)
+    assert b.shape == (3, O.tile_code_bytes(bits, 16, 128)) and b.dtype == np.uint8
+    assert np.array_equal(O.unpack_codes(b, bits, 16, 128), q)
+
+
+# ---------------------------------------------------------------- attention
+def _random_cache(rng, n_tiles, d, bits_k=4, bits_v=4):
+    xk = rng.standard_normal((n_tiles, 16, d)) * 2
+    xv = rng.standard_normal((n_tiles, 16, d))
+    return O.quantize_tiles(xk, bits_k, 4), O.quantize_tiles(xv, bits_v, 4)
+
+
+def test_attention_matches_torch_sdpa_float64():
+    import torch
+    rng = np.random.default_rng(11)
+    k, v = _random_cache(rng, 5, 128, 3, 4)
+    q = rng.standard_normal((4, 128))
+    scale = 1 / math.sqrt(128)
+    o = O.decode_attention(q, k, v, scale)
+    kh = O.dequantize_tiles(k.q, k.a, k.z, k.c).reshape(-1, 128)     # un-rotated
+    vh = O.dequantize_tiles(v.q, v.a, v.z, v.c).reshape(-1, 128)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], torch.from_numpy(kh)[None, None].expand(1, 4, -1, -1),
+        torch.from_numpy(vh)[None, None].expand(1, 4, -1, -1), scale=scale)[0, :, 0, :].numpy()
+    assert np.max(np.abs(o - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_attention_single_token_and_identical_keys():
+    rng = np.random.default_rng(12)
+    k, v = _random_cache(rng, 1, 128)
+    q = rng.standard_normal((2, 128))
+    vh = O.dequantize_tiles(v.q, v.a, v.z, v.c).reshape(-1, 128)
+    one = O.QuantizedTiles(k.q[:, :1], k.a[:, :1], k.z[:, :1], k.c)
+    onev = O.QuantizedTiles(v.q[:, :1], v.a[:, :1], v.z[:, :1], v.c)
+    assert np.allclose(O.decode_attention(q, one, onev, 0.1), vh[:1].repeat(2, 0), rtol=0, atol=1e-12)
+    same = O.QuantizedTiles(np.repeat(k.q[:, :1], 16, 1), np.repeat(k.a[:, :1], 16, 1),
+                            np.repeat(k.z[:, :1], 16, 1), k.c)
+    o = O.decode_attention(q, same, v, 0.3)
+    assert np.allclose(o, vh.mean(0)[None].repeat(2, 0), rtol=0, atol=1e-12)
+
+
+def test_mla_attention_matches_torch_sdpa_float64():
+    import torch
+    rng = np.random.default_rng(13)
+    d, rd, H = 512, 64, 8
+    lat = O.quantize_tiles(rng.standard_normal((3, 16, d)), 4, 4)
+    rope = rng.standard_normal((48, rd))
+    q = rng.standard_normal((H, d + rd))
+    scale = 1 / math.sqrt(d + rd)
+    o = O.mla_decode_attention(q, lat, rope, scale)
+    ch = O.dequantize_tiles(lat.q, lat.a, lat.z, lat.c).reshape(-1, d)     # un-rotated latent
+    key = np.concatenate([ch, rope], 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], torch.from_numpy(key)[None, None].expand(1, H, -1, -1),
+        torch.from_numpy(ch)[None, None].expand(1, H, -1, -1), scale=scale)[0, :, 0, :].numpy()
+    assert np.max(np.abs(o - ref)) <= 1e-12 * np.max(np.abs(ref))
