@@ -1,0 +1,211 @@
+/*
+ * kvq.h -- C ABI of a B200 (sm_100a) library for KVarN-style variance-
+ * normalised KV-cache quantisation and decode attention over the quantised
+ * cache.
+ *
+ * Method (what every call computes), as the KVarN pages state it:
+ *   - KVarN project page (open-radar), Key Features, "Variance-Normalized
+ *     Quantization Pipeline": each tile of the KV cache is rotated with a
+ *     Hadamard transform to spread channel outliers, its variance is
+ *     equalised by an iterative Sinkhorn-like normalisation, and it is then
+ *     quantised with asymmetric round-to-nearest;
+ *   - same page, "Calibration-Free Operation": the statistics are computed
+ *     per tile on the fly;
+ *   - same page, "4-bit Keys, 2-bit Values Preset": keys and values have
+ *     their own bit widths and a tile is one cache block of the serving
+ *     engine ("kvarn_k4v2_g128" = 4-bit K, 2-bit V, 128-token tiles);
+ *   - same page, "MLA Model Support": the compressed latent of multi-head
+ *     latent attention is quantised the same way;
+ *   - KV-Cache tag page (baguaai.com), KVarN item: Hadamard rotation with
+ *     dual-axis variance normalisation, round-to-nearest.
+ *
+ * Declared readings where the pages are silent (tile = T tokens x d
+ * channels of one layer and kv-head; K and V quantised independently):
+ *   Z = X H / sqrt(d)  (Sylvester H, full head_dim);
+ *   n rounds of: divide each row by its root-mean-square, then each column
+ *   by its root-mean-square (a zero RMS leaves its row/column alone); the
+ *   factors accumulate in r (per token) and c (per channel);
+ *   per token row of Y = Z / (r c): m = min, s = (max - min) / (2^b - 1),
+ *   q = rint((Y - m) / s) (ties to even; s = 0 -> q = 0);
+ *   stored: codes q, a = r*s and z = r*m (float32 per token), c (float32
+ *   per channel).  Dequantised rotated value: (a q + z) c.
+ *   Decode attention rotates the query by the same H/sqrt(d), attends in the
+ *   rotated domain with the scales folded into the dot products, and rotates
+ *   the output back.
+ *
+ * Ownership and threading: the caller allocates ALL device memory (the
+ * cache arrays, inputs, outputs, the decode workspace and the device error
+ * word).  The library never allocates, frees or synchronises, except
+ * kvq_read_error, which synchronises the given stream.  Every call that
+ * takes a stream only enqueues work on it (a cudaStream_t passed as void*;
+ * NULL = the legacy default stream) and returns.  Calls are thread-safe.
+ *
+ * Errors: every function returns kvq_status; nothing is thrown across the
+ * ABI.  Host-detectable problems (null pointers, unsupported shapes or bit
+ * widths, a workspace that is too small) are rejected before any launch.
+ * Problems only the device can see (a page id outside [0, num_pages), a
+ * sequence length that is not a multiple of the tile) set bits in the
+ * caller's 32-bit device error word (KVQ_DEVERR_*); the affected tile is
+ * skipped and nothing traps.  Read and clear it with kvq_read_error.
+ *
+ * Cache format (all arrays indexed [layer][page][kv_head][...], one page =
+ * one tile of T tokens):
+ *   codes:      T * d * bits / 8 bytes per (layer, page, head): token rows in
+ *               order, each row's codes packed little-endian inside a byte,
+ *               lowest channel in the lowest bits (2, 4 or 8 bits); 3-bit
+ *               codes are a plane of all rows' low 2 bits (2-bit packing)
+ *               followed by a plane of all rows' high bits (1-bit packing);
+ *   tok_scale:  float32 [T][2] = (a, z) per token;
+ *   chan_scale: float32 [d] = c per channel;
+ *   rope (MLA): bf16 [layer][page][T][rope_dim], unquantised.
+ *
+ * Supported on the GPU: head_dim 128 (GQA) or 512 (MLA latent), tile_tokens
+ * 16, bits_k in {2,3,4,8}, bits_v in {2,4,8}, query group size 1..8 for GQA
+ * and 1..128 heads for MLA; inputs fp16 or bf16.  Other shapes return
+ * KVQ_ERR_UNSUPPORTED.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,         /* null pointer, negative size, inconsistent config */
+  KVQ_ERR_UNSUPPORTED = 2,         /* valid but not built: head_dim, bits, tile, group size */
+  KVQ_ERR_WORKSPACE_TOO_SMALL = 3, /* decode workspace below kvq_decode_workspace_bytes */
+  KVQ_ERR_PARTIAL_TILE = 4,        /* n_tok not a multiple of tile_tokens */
+  KVQ_ERR_BAD_PAGE = 5,            /* reserved for host-side page checks */
+  KVQ_ERR_TIMEOUT = 6,             /* a bounded device wait gave up (see KVQ_DEVERR_TIMEOUT) */
+  KVQ_ERR_CUDA = 7                 /* a CUDA runtime call failed (launch or sync) */
+} kvq_status;
+
+/* Bits of the device error word. */
+#define KVQ_DEVERR_BAD_PAGE 0x1u     /* page id < 0 or >= num_pages: tile skipped */
+#define KVQ_DEVERR_PARTIAL_TILE 0x2u /* seq_len % tile_tokens != 0: tail ignored */
+#define KVQ_DEVERR_TIMEOUT 0x4u      /* an mbarrier wait ran out of iterations */
+#define KVQ_DEVERR_BAD_SEQ 0x8u      /* seq_len < 0 or needs more pages than the block table row */
+
+typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
+
+/* One cache (all layers share it).  Fill it yourself or with
+ * kvq_config_from_string. */
+typedef struct kvq_config {
+  int32_t head_dim;       /* d: 128 (GQA) or 512 (MLA latent); power of two */
+  int32_t num_kv_heads;   /* H_kv (1 for MLA) */
+  int32_t tile_tokens;    /* T == page size in tokens (16) */
+  int32_t bits_k;         /* key (MLA: latent) code width: 2, 3, 4 or 8 */
+  int32_t bits_v;         /* value code width: 2, 4 or 8; ignored when mla */
+  int32_t sinkhorn_iters; /* n >= 0 normalisation rounds (0 = rotation + RTN only) */
+  int32_t hadamard_block; /* must equal head_dim (full-width rotation) */
+  int32_t mla;            /* 1: one latent per token is key and value; no V arrays */
+  int32_t rope_dim;       /* MLA: width of the unquantised bf16 rope key (64) */
+  int32_t num_layers;     /* layers in the pool */
+  int64_t num_pages;      /* pages per layer in the pool */
+  kvq_dtype in_dtype;     /* dtype of the new K/V rows: KVQ_F16 or KVQ_BF16 */
+} kvq_config;
+
+/* Caller-owned device arrays of one cache; byte sizes from kvq_cache_layout
+ * (in this order: k_codes, k_tok_scale, k_chan_scale, v_codes, v_tok_scale,
+ * v_chan_scale, rope).  Unused arrays (V when mla, rope when not) may be
+ * NULL.  Every pointer must be 16-byte aligned. */
+typedef struct kvq_cache_view {
+  void* k_codes;
+  void* k_tok_scale;
+  void* k_chan_scale;
+  void* v_codes;
+  void* v_tok_scale;
+  void* v_chan_scale;
+  void* rope;
+} kvq_cache_view;
+
+/* Parse a KVarN preset name "kvarn_k<K>v<V>_g<T>" (KVarN project page,
+ * "Native vLLM Integration" and "4-bit Keys, 2-bit Values Preset") into
+ * bits_k, bits_v and tile_tokens of *inout; the other fields are left as
+ * they are.  KVQ_ERR_INVALID_ARG if the string does not parse. */
+kvq_status kvq_config_from_string(const char* name, kvq_config* inout);
+
+/* Byte sizes of the seven cache arrays for *cfg (0 for unused arrays).
+ * Host only. */
+kvq_status kvq_cache_layout(const kvq_config* cfg, size_t bytes_out[7]);
+
+/* Quantise n_tok new tokens of every layer into the paged cache (the
+ * whole pipeline: rotation, dual-axis normalisation, asymmetric RTN,
+ * packing).
+ *   k_new, v_new: device, in_dtype [num_layers][n_tok][num_kv_heads][head_dim]
+ *                 (MLA: k_new is the latent [num_layers][n_tok][1][d];
+ *                 v_new is ignored and may be NULL);
+ *   rope_new:     MLA only, device bf16 [num_layers][n_tok][rope_dim],
+ *                 copied into the rope array; NULL otherwise;
+ *   n_tok:        tokens per layer, a multiple of tile_tokens
+ *                 (else KVQ_ERR_PARTIAL_TILE);
+ *   dst_page:     device int32 [n_tok / tile_tokens]: the page that receives
+ *                 tokens [i*T, (i+1)*T) of every layer and kv-head; an id
+ *                 outside [0, num_pages) sets KVQ_DEVERR_BAD_PAGE and that
+ *                 tile is not written;
+ *   dev_error:    device uint32 error word (bits are OR-ed in).
+ * Pages must be distinct within one call. */
+kvq_status kvq_quantize_append(const kvq_config* cfg, const kvq_cache_view* cache,
+                               const void* k_new, const void* v_new, const void* rope_new,
+                               int64_t n_tok, const int32_t* dst_page, uint32_t* dev_error,
+                               void* stream);
+
+/* Dequantise n_pages pages of one layer to float32 (inspection and tests).
+ *   pages:  device int32 [n_pages]; out-of-range ids set KVQ_DEVERR_BAD_PAGE
+ *           and their output is left untouched;
+ *   unrotate: 0 = rotated domain (a q + z) c; 1 = rotated back to the
+ *           input basis;
+ *   k_out, v_out: device float32 [n_pages][num_kv_heads][T][head_dim]
+ *           (v_out ignored when mla). */
+kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache_view* cache, int32_t layer,
+                          const int32_t* pages, int64_t n_pages, int32_t unrotate,
+                          float* k_out, float* v_out, uint32_t* dev_error, void* stream);
+
+/* Bytes of device workspace kvq_decode_attention needs for this shape
+ * (split-KV partial results).  Host only. */
+kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch,
+                                      int32_t num_q_heads, int32_t max_seq_len,
+                                      size_t* bytes);
+
+/* One decode step of attention over the quantised cache of one layer.
+ *   q:           device bf16 [batch][num_q_heads][head_dim (+ rope_dim if mla)],
+ *                un-rotated;
+ *   block_table: device int32 [batch][max_pages_per_seq], pages in token order;
+ *   seq_lens:    device int32 [batch], multiples of tile_tokens (a remainder
+ *                sets KVQ_DEVERR_PARTIAL_TILE and is ignored);
+ *   num_q_heads: a multiple of num_kv_heads; q head h reads kv-head
+ *                h / (num_q_heads / num_kv_heads);
+ *   softmax_scale: multiplies q.k (1/sqrt(128) for GQA, 1/sqrt(576) for MLA);
+ *   out:         device float32 [batch][num_q_heads][head_dim], un-rotated;
+ *                a sequence of length 0 gets zeros;
+ *   workspace:   device scratch of at least kvq_decode_workspace_bytes(...,
+ *                max_seq_len >= every seq_len) bytes, 256-byte aligned; its
+ *                contents need no initialisation and are overwritten. */
+kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache_view* cache, int32_t layer,
+                                const void* q, const int32_t* block_table,
+                                int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                int32_t batch, int32_t num_q_heads, float softmax_scale,
+                                float* out, void* workspace, size_t workspace_bytes,
+                                uint32_t* dev_error, void* stream);
+
+/* Synchronise `stream`, copy the device error word to *host_bits and reset
+ * it to 0.  KVQ_ERR_TIMEOUT if the TIMEOUT bit was set, else KVQ_OK (other
+ * bits are only reported in *host_bits). */
+kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream);
+
+/* Static, human-readable name of a status. */
+const char* kvq_status_string(kvq_status status);
+
+/* Library version as "major.minor.patch". */
+const char* kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

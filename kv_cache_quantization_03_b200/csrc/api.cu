@@ -1,0 +1,277 @@
+// C ABI of the kvq library: argument validation, cache layout sizing,
+// split-KV planning and kernel dispatch.  No allocation, no synchronisation
+// (except kvq_read_error).  Declarations and the method's citations are in
+// include/kvq.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace {
+
+constexpr int kNumSMs = 148;           // B200
+constexpr int kDecodeTargetCtas = 4 * kNumSMs;
+constexpr int kDecodeWarps = 4;        // warps per decode CTA (tiles are dealt round robin)
+constexpr int kMaxGroup = 8;
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+
+kvq_status check_config(const kvq_config* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  if (!is_pow2(c->head_dim) || c->head_dim < 8 || c->head_dim > 1024) return KVQ_ERR_INVALID_ARG;
+  if (c->num_kv_heads <= 0 || c->num_layers <= 0 || c->num_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (!is_pow2(c->tile_tokens) || c->tile_tokens < 8) return KVQ_ERR_INVALID_ARG;
+  if (c->sinkhorn_iters < 0 || c->sinkhorn_iters > 1000) return KVQ_ERR_INVALID_ARG;
+  if (!valid_bits(c->bits_k)) return KVQ_ERR_INVALID_ARG;
+  if (!c->mla && !valid_bits(c->bits_v)) return KVQ_ERR_INVALID_ARG;
+  if (c->in_dtype != KVQ_F16 && c->in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (c->mla) {
+    if (c->num_kv_heads != 1 || c->rope_dim < 0 || (c->rope_dim % 8)) return KVQ_ERR_INVALID_ARG;
+  }
+  if (c->hadamard_block != c->head_dim) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+// Shapes the kernels are built for.
+kvq_status check_gpu_shape(const kvq_config* c) {
+  if (c->mla) return KVQ_ERR_UNSUPPORTED;
+  if (c->head_dim != 128 || c->tile_tokens != 16) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+int64_t slots(const kvq_config* c) { return (int64_t)c->num_layers * c->num_pages * c->num_kv_heads; }
+
+CacheArrays arrays(const kvq_cache_view* v, int which, int bits) {
+  CacheArrays a;
+  a.codes = static_cast<uint8_t*>(which == 0 ? v->k_codes : v->v_codes);
+  a.tok = static_cast<float*>(which == 0 ? v->k_tok_scale : v->v_tok_scale);
+  a.chan = static_cast<float*>(which == 0 ? v->k_chan_scale : v->v_chan_scale);
+  a.bits = bits;
+  return a;
+}
+
+kvq_status check_view(const kvq_config* c, const kvq_cache_view* v) {
+  if (!v) return KVQ_ERR_INVALID_ARG;
+  const void* need[4] = {v->k_codes, v->k_tok_scale, v->k_chan_scale, nullptr};
+  for (int i = 0; i < 3; ++i)
+    if (!need[i] || !aligned16(need[i])) return KVQ_ERR_INVALID_ARG;
+  if (!c->mla) {
+    const void* vv[3] = {v->v_codes, v->v_tok_scale, v->v_chan_scale};
+    for (int i = 0; i < 3; ++i)
+      if (!vv[i] || !aligned16(vv[i])) return KVQ_ERR_INVALID_ARG;
+  } else if (c->rope_dim > 0 && (!v->rope || !aligned16(v->rope))) {
+    return KVQ_ERR_INVALID_ARG;
+  }
+  return KVQ_OK;
+}
+
+struct DecodePlan {
+  int splits;
+  int tiles_per_split;
+};
+
+// Split the tiles of each (sequence, kv-head) so that about kDecodeTargetCtas
+// CTAs run, with at least 4 tiles per warp in a split.
+DecodePlan decode_plan(int64_t pairs, int64_t max_tiles) {
+  DecodePlan d{1, 0};
+  if (pairs <= 0 || max_tiles <= 0) return d;
+  int64_t splits = (kDecodeTargetCtas + pairs - 1) / pairs;
+  const int64_t cap = (max_tiles + 4 * kDecodeWarps - 1) / (4 * kDecodeWarps);
+  if (splits > cap) splits = cap;
+  if (splits < 1) splits = 1;
+  int64_t tps = (max_tiles + splits - 1) / splits;
+  tps = (tps + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps;
+  d.tiles_per_split = (int)tps;
+  d.splits = (int)((max_tiles + tps - 1) / tps);
+  return d;
+}
+
+size_t decode_ws_bytes(int64_t pairs, const DecodePlan& d, int head_dim) {
+  return (size_t)pairs * d.splits * kMaxGroup * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+kvq_status cuda_status(int e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_version(void) { return "0.1.0"; }
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+    case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+    case KVQ_ERR_WORKSPACE_TOO_SMALL: return "KVQ_ERR_WORKSPACE_TOO_SMALL";
+    case KVQ_ERR_PARTIAL_TILE: return "KVQ_ERR_PARTIAL_TILE";
+    case KVQ_ERR_BAD_PAGE: return "KVQ_ERR_BAD_PAGE";
+    case KVQ_ERR_TIMEOUT: return "KVQ_ERR_TIMEOUT";
+    case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+  }
+  return "KVQ_ERR_UNKNOWN";
+}
+
+kvq_status kvq_config_from_string(const char* name, kvq_config* inout) {
+  if (!name || !inout) return KVQ_ERR_INVALID_ARG;
+  int k = 0, v = 0, g = 0;
+  char tail = 0;
+  if (std::sscanf(name, "kvarn_k%dv%d_g%d%c", &k, &v, &g, &tail) != 3) return KVQ_ERR_INVALID_ARG;
+  if (!valid_bits(k) || !valid_bits(v) || !is_pow2(g) || g < 8) return KVQ_ERR_INVALID_ARG;
+  inout->bits_k = k;
+  inout->bits_v = v;
+  inout->tile_tokens = g;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_layout(const kvq_config* c, size_t bytes_out[7]) {
+  if (!bytes_out) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  const size_t n = (size_t)slots(c), T = c->tile_tokens, d = c->head_dim;
+  bytes_out[0] = n * T * d * c->bits_k / 8;
+  bytes_out[1] = n * T * 2 * sizeof(float);
+  bytes_out[2] = n * d * sizeof(float);
+  const bool has_v = !c->mla;
+  bytes_out[3] = has_v ? n * T * d * c->bits_v / 8 : 0;
+  bytes_out[4] = has_v ? n * T * 2 * sizeof(float) : 0;
+  bytes_out[5] = has_v ? n * d * sizeof(float) : 0;
+  bytes_out[6] = c->mla ? (size_t)c->num_layers * c->num_pages * T * c->rope_dim * 2 : 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache, const void* k_new,
+                               const void* v_new, const void* rope_new, int64_t n_tok,
+                               const int32_t* dst_page, uint32_t* dev_error, void* stream) {
+  kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_view(c, cache)) != KVQ_OK) return st;
+  if (n_tok < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_tok % c->tile_tokens) return KVQ_ERR_PARTIAL_TILE;
+  if (n_tok > 0 && (!k_new || !dst_page || (!c->mla && !v_new))) return KVQ_ERR_INVALID_ARG;
+  if (c->mla && c->rope_dim > 0 && n_tok > 0 && !rope_new) return KVQ_ERR_INVALID_ARG;
+  if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new))) return KVQ_ERR_INVALID_ARG;
+  if ((st = check_gpu_shape(c)) != KVQ_OK) return st;
+  if (n_tok == 0) return KVQ_OK;
+  QuantizeParams p{};
+  p.src[0] = k_new;
+  p.src[1] = v_new;
+  p.dst[0] = arrays(cache, 0, c->bits_k);
+  p.dst[1] = arrays(cache, 1, c->bits_v);
+  p.kinds = c->mla ? 1 : 2;
+  p.n_tok = n_tok;
+  p.num_layers = c->num_layers;
+  p.num_heads = c->num_kv_heads;
+  p.num_pages = c->num_pages;
+  p.iters = c->sinkhorn_iters;
+  p.dst_page = dst_page;
+  p.err = dev_error;
+  p.total_tiles = (int64_t)p.kinds * c->num_layers * (n_tok / c->tile_tokens) * c->num_kv_heads;
+  return cuda_status(launch_quantize_d128(p, c->in_dtype == KVQ_F16, stream));
+}
+
+kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
+                          const int32_t* pages, int64_t n_pages, int32_t unrotate, float* k_out,
+                          float* v_out, uint32_t* dev_error, void* stream) {
+  kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_view(c, cache)) != KVQ_OK) return st;
+  if (layer < 0 || layer >= c->num_layers || n_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_pages > 0 && (!pages || !k_out || (!c->mla && !v_out))) return KVQ_ERR_INVALID_ARG;
+  if ((st = check_gpu_shape(c)) != KVQ_OK) return st;
+  if (n_pages == 0) return KVQ_OK;
+  DequantParams p{};
+  p.src[0] = arrays(cache, 0, c->bits_k);
+  p.src[1] = arrays(cache, 1, c->bits_v);
+  p.kinds = c->mla ? 1 : 2;
+  p.layer = layer;
+  p.num_heads = c->num_kv_heads;
+  p.num_pages = c->num_pages;
+  p.pages = pages;
+  p.n_pages = n_pages;
+  p.unrotate = unrotate ? 1 : 0;
+  p.out[0] = k_out;
+  p.out[1] = v_out;
+  p.err = dev_error;
+  return cuda_status(launch_dequantize_d128(p, stream));
+}
+
+kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_t num_q_heads,
+                                      int32_t max_seq_len, size_t* bytes) {
+  kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  if (!bytes || batch < 0 || num_q_heads <= 0 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
+  const int64_t pairs = (int64_t)batch * c->num_kv_heads;
+  const int64_t max_tiles = ((int64_t)max_seq_len + c->tile_tokens - 1) / c->tile_tokens;
+  *bytes = decode_ws_bytes(pairs, decode_plan(pairs, max_tiles), c->head_dim);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
+                                const void* q, const int32_t* block_table, int32_t max_pages_per_seq,
+                                const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                uint32_t* dev_error, void* stream) {
+  kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_view(c, cache)) != KVQ_OK) return st;
+  if (layer < 0 || layer >= c->num_layers || batch < 0 || max_pages_per_seq < 0 || num_q_heads <= 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (num_q_heads % c->num_kv_heads) return KVQ_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (batch > 0 && (!q || !seq_lens || !out || (max_pages_per_seq > 0 && !block_table)))
+    return KVQ_ERR_INVALID_ARG;
+  if (q && !aligned16(q)) return KVQ_ERR_INVALID_ARG;
+  if ((st = check_gpu_shape(c)) != KVQ_OK) return st;
+  const int group = num_q_heads / c->num_kv_heads;
+  if (group > kMaxGroup || c->bits_v == 3) return KVQ_ERR_UNSUPPORTED;
+  if (batch == 0) return KVQ_OK;
+  const int64_t pairs = (int64_t)batch * c->num_kv_heads;
+  const DecodePlan plan = decode_plan(pairs, max_pages_per_seq);
+  const size_t need = decode_ws_bytes(pairs, plan, c->head_dim);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return workspace_bytes < need ? KVQ_ERR_WORKSPACE_TOO_SMALL : KVQ_ERR_INVALID_ARG;
+  if (pairs > 65535) return KVQ_ERR_UNSUPPORTED;
+  DecodeParams p{};
+  p.k = arrays(cache, 0, c->bits_k);
+  p.v = arrays(cache, 1, c->bits_v);
+  p.layer = layer;
+  p.num_kv_heads = c->num_kv_heads;
+  p.num_pages = c->num_pages;
+  p.q = static_cast<const uint16_t*>(q);
+  p.block_table = block_table;
+  p.max_pages = max_pages_per_seq;
+  p.seq_lens = seq_lens;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.group = group;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = p.part_o + (size_t)pairs * plan.splits * kMaxGroup * c->head_dim;
+  p.splits = plan.splits;
+  p.tiles_per_split = plan.tiles_per_split;
+  p.err = dev_error;
+  return cuda_status(launch_decode_d128(p, stream));
+}
+
+kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream) {
+  if (!dev_error || !host_bits) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t bits = 0;
+  if (cudaMemcpyAsync(&bits, dev_error, sizeof(bits), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (cudaMemsetAsync(dev_error, 0, sizeof(uint32_t), s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  *host_bits = bits;
+  return (bits & KVQ_DEVERR_TIMEOUT) ? KVQ_ERR_TIMEOUT : KVQ_OK;
+}
+
+}  // extern "C"

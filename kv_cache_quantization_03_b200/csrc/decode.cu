@@ -1,0 +1,467 @@
+// Decode attention over the quantised cache, head_dim 128, 16-token pages,
+// query groups of 1..8 heads per kv-head (sm_100a).
+//
+// Consumer of the KVarN cache (KVarN project page on open-radar, Key
+// Features, "Variance-Normalized Quantization Pipeline" and "Throughput Above
+// FP16": the cache is read in its quantised form).  The query is rotated with
+// the same Sylvester H/sqrt(128) as the cache, so attention runs in the
+// rotated domain on (a q + z) c with the scales folded in:
+//   score(t, h) = scale * (a_t * sum_j u_hj q_tj + z_t * sum_j u_hj),
+//                 u_h = rotate(q_h) * c_K             (per tile)
+//   out_h      += c_V * (sum_t w_th qv_t + sum_t p_th z_t),  w_th = p_th a_t
+// with an online softmax across tiles, then the output is rotated back.
+//
+// Work split: grid (splits, batch * kv_heads).  Each CTA of 4 warps owns a
+// contiguous range of one sequence's tiles; each warp takes every 4th tile
+// and streams it through its own ring of shared-memory stages filled with
+// 1-D bulk async copies (one mbarrier per stage, bounded waits).  Both
+// contractions of a tile run as m16n8k16 f16 MMAs with fp32 accumulation:
+// codes 0..255 are exact in f16; u and w are rounded to f16.
+//   scores:  D[16 tokens x 8 heads]   = codes_K[16 x 128] * u^T[128 x 8]
+//   values:  D[128 channels x 8 heads] = codes_V^T[128 x 16] * w[16 x 8]
+// The per-channel c_V is applied to each tile's fresh MMA result before it
+// joins the running output.  A second kernel merges the split partials,
+// normalises and rotates back.
+#include <cuda_runtime.h>
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kT = 16;
+constexpr int kDW = 4;      // warps per CTA
+constexpr int kStages = 4;  // ring depth per warp
+constexpr float kNegBig = -1e30f;
+
+struct StageLayout {
+  int kcb, vcb, off_kaz, off_kc, off_v, off_vaz, off_vc, bytes;
+};
+
+__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv) {
+  return StageLayout{kT * kD * bk / 8,
+                     kT * kD * bv / 8,
+                     kT * kD * bk / 8,
+                     kT * kD * bk / 8 + kT * 8,
+                     kT * kD * bk / 8 + kT * 8 + kD * 4,
+                     kT * kD * bk / 8 + kT * 8 + kD * 4 + kT * kD * bv / 8,
+                     kT * kD * bk / 8 + kT * 8 + kD * 4 + kT * kD * bv / 8 + kT * 8,
+                     kT * kD * (bk + bv) / 8 + 2 * (kT * 8 + kD * 4)};
+}
+
+// ---- code pairs -> f16x2 (exact small integers)
+__device__ __forceinline__ uint32_t h2_codes(uint32_t masked) {
+  uint32_t v = masked | 0x64006400u;  // f16 1024 + code in each half
+  __half2 h = *reinterpret_cast<__half2*>(&v);
+  h = __hsub2(h, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Key-side pairing: lane t covers channels 32t..32t+31 of a token row; pair
+// pi (0..15) holds channels (chan(pi), chan(pi) + dist) relative to 32t.
+template <int B>
+__host__ __device__ constexpr int kdist() {
+  return B == 4 ? 4 : (B == 8 ? 2 : 8);
+}
+template <int B>
+__host__ __device__ constexpr int kchan(int pi) {
+  return B == 4 ? 8 * (pi >> 2) + (pi & 3) : (B == 8 ? 4 * (pi >> 1) + (pi & 1) : 16 * (pi >> 3) + (pi & 7));
+}
+
+// Pairs of one token row for the key MMA (16 pairs = 32 codes).
+template <int B>
+__device__ __forceinline__ void key_pairs(const uint8_t* codes, int row, int t, uint32_t (&pr)[16]) {
+  if constexpr (B == 4) {
+    const uint4 w = *reinterpret_cast<const uint4*>(codes + row * 64 + 16 * t);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 2] >> (4 * (pi & 3))) & 0x000F000Fu);
+  } else if constexpr (B == 2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
+    const uint32_t ws[2] = {w.x, w.y};
+#pragma unroll
+    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 3] >> (2 * (pi & 7))) & 0x00030003u);
+  } else if constexpr (B == 8) {
+    const uint4 w0 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t + 16);
+    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 1] >> (8 * (pi & 1))) & 0x00FF00FFu);
+  } else {  // 3 bits: low plane [T][32 B] then high plane [T][16 B]
+    const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
+    const uint32_t hw = *reinterpret_cast<const uint32_t*>(codes + kT * 32 + row * 16 + 4 * t);
+    const uint32_t ws[2] = {w.x, w.y};
+    const uint32_t hs[2] = {__byte_perm(hw, 0u, 0x4140u), __byte_perm(hw, 0u, 0x4342u)};
+    const __half2 four = __halves2half2(__ushort_as_half(0x4400), __ushort_as_half(0x4400));
+#pragma unroll
+    for (int pi = 0; pi < 16; ++pi) {
+      uint32_t lo = h2_codes((ws[pi >> 3] >> (2 * (pi & 7))) & 0x00030003u);
+      uint32_t hi = h2_codes((hs[pi >> 3] >> (pi & 7)) & 0x00010001u);
+      __half2 r = __hfma2(*reinterpret_cast<__half2*>(&hi), four, *reinterpret_cast<__half2*>(&lo));
+      pr[pi] = *reinterpret_cast<uint32_t*>(&r);
+    }
+  }
+}
+
+// Value-side pairs: f16x2 of (token x, token y) at lane g's channel 16g + c.
+template <int B>
+__device__ __forceinline__ void value_pairs(const uint8_t* codes, int rx, int ry, int g, uint32_t (&pr)[16]) {
+  if constexpr (B == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(codes + rx * 64 + 8 * g);
+    const uint2 y = *reinterpret_cast<const uint2*>(codes + ry * 64 + 8 * g);
+    const uint32_t xs[2] = {x.x, x.y}, ys[2] = {y.x, y.y};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t m = __byte_perm(xs[k >> 1], ys[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pr[4 * k + e] = h2_codes((m >> (4 * e)) & 0x000F000Fu);
+    }
+  } else if constexpr (B == 2) {
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(codes + rx * 32 + 4 * g);
+    const uint32_t y = *reinterpret_cast<const uint32_t*>(codes + ry * 32 + 4 * g);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t m = __byte_perm(x, y, k ? 0x7632u : 0x5410u);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pr[8 * k + e] = h2_codes((m >> (2 * e)) & 0x00030003u);
+    }
+  } else {  // 8 bits
+    const uint4 x = *reinterpret_cast<const uint4*>(codes + rx * 128 + 16 * g);
+    const uint4 y = *reinterpret_cast<const uint4*>(codes + ry * 128 + 16 * g);
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t m = __byte_perm(xs[k >> 1], ys[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) pr[2 * k + e] = h2_codes((m >> (8 * e)) & 0x00FF00FFu);
+    }
+  }
+}
+
+__device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+template <int BK, int BV>
+__global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr StageLayout SL = stage_layout(BK, BV);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDW * kStages * SL.bytes);
+  uint8_t* wsm = smem + warp * kStages * SL.bytes;
+  uint64_t* wbar = bars + warp * kStages;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&wbar[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const int pair = blockIdx.y;
+  const int b = pair / p.num_kv_heads, kvh = pair % p.num_kv_heads;
+  const int split = blockIdx.x;
+  int seq = p.seq_lens[b];
+  if (seq < 0) {
+    if (threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+    seq = 0;
+  }
+  int ntiles = seq / kT;
+  if ((seq % kT) && threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_PARTIAL_TILE);
+  if (ntiles > p.max_pages) {
+    if (threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+    ntiles = p.max_pages;
+  }
+  const int t0 = split * p.tiles_per_split;
+  const int t1 = min(t0 + p.tiles_per_split, ntiles);
+  const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
+  const int32_t* btab = p.block_table + (size_t)b * p.max_pages;
+
+  // ---- rotated, pre-scaled query: lane (g, t) keeps head g, channels 32t..32t+31
+  float qr[32];
+  {
+    const bool live = g < p.group;
+    const uint16_t* qp = p.q + ((size_t)b * p.num_q_heads + (size_t)kvh * p.group + (live ? g : 0)) * kD + 32 * t;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = *reinterpret_cast<const uint4*>(qp + 8 * k);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qr[8 * k + 2 * e] = live ? bf16_to_f((uint16_t)(ws[e] & 0xFFFF)) : 0.f;
+        qr[8 * k + 2 * e + 1] = live ? bf16_to_f((uint16_t)(ws[e] >> 16)) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!(i & s)) {
+          const float x = qr[i], y = qr[i + s];
+          qr[i] = x + y;
+          qr[i + s] = x - y;
+        }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      const bool upper = (t & off) != 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, qr[i], off);
+        qr[i] = upper ? (o - qr[i]) : (qr[i] + o);
+      }
+    }
+    const float f = p.scale_log2 * 0.08838834764831845f;  // softmax scale * log2(e) / sqrt(128)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qr[i] *= f;
+  }
+
+  // ---- producer: lane 0 fills stage (i % kStages) with local tile i
+  auto issue = [&](int i) {
+    if (lane != 0) return;
+    uint64_t* bar = &wbar[i % kStages];
+    uint8_t* st = wsm + (i % kStages) * SL.bytes;
+    const int page = btab[t0 + warp + i * kDW];
+    if (page < 0 || page >= p.num_pages) {
+      set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+      mbar_arrive_expect_tx(bar, 0);
+      return;
+    }
+    const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_kv_heads + kvh;
+    mbar_arrive_expect_tx(bar, (uint32_t)SL.bytes);
+    bulk_g2s(st, p.k.codes + slot * SL.kcb, SL.kcb, bar);
+    bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), kT * 8, bar);
+    bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, kD * 4, bar);
+    bulk_g2s(st + SL.off_v, p.v.codes + slot * SL.vcb, SL.vcb, bar);
+    bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), kT * 8, bar);
+    bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, kD * 4, bar);
+  };
+  const int pre = my_n < kStages ? my_n : kStages;
+  for (int i = 0; i < pre; ++i) issue(i);
+  int issued = pre;
+
+  float mrun[2] = {kNegBig, kNegBig};  // running max of heads 2t, 2t+1 (log2 units)
+  float lrun[2] = {0.f, 0.f};          // this lane's share of the running sums
+  f2 O[8][2];                          // [m-block][row g / g+8] x heads (2t, 2t+1)
+#pragma unroll
+  for (int mb = 0; mb < 8; ++mb) O[mb][0] = O[mb][1] = f2{0.f, 0.f};
+  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+
+  bool timed_out = false;
+  for (int i = 0; i < my_n; ++i) {
+    const bool ok = mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
+    if (!__all_sync(0xffffffffu, ok)) {
+      timed_out = true;
+      if (lane == 0) set_error(p.err, KVQ_DEVERR_TIMEOUT);
+      break;
+    }
+    const int page = btab[t0 + warp + i * kDW];
+    if (page >= 0 && page < p.num_pages) {
+      const uint8_t* st = wsm + (i % kStages) * SL.bytes;
+      const float* kaz = reinterpret_cast<const float*>(st + SL.off_kaz);
+      const float* kc = reinterpret_cast<const float*>(st + SL.off_kc);
+      const float* vaz = reinterpret_cast<const float*>(st + SL.off_vaz);
+      const float* vc = reinterpret_cast<const float*>(st + SL.off_vc);
+
+      // u = q~ * c_K on this lane's 32 channels, and its sum
+      float ck[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + 4 * k);
+        ck[4 * k] = c4.x, ck[4 * k + 1] = c4.y, ck[4 * k + 2] = c4.z, ck[4 * k + 3] = c4.w;
+      }
+      float su = 0.f;
+      uint32_t ub[16];
+#pragma unroll
+      for (int pi = 0; pi < 16; ++pi) {
+        const int c0 = kchan<BK>(pi), c1 = c0 + kdist<BK>();
+        const float u0 = qr[c0] * ck[c0], u1 = qr[c1] * ck[c1];
+        su += u0 + u1;
+        ub[pi] = pack_f16x2(u0, u1);
+      }
+      su += __shfl_xor_sync(0xffffffffu, su, 1);
+      su += __shfl_xor_sync(0xffffffffu, su, 2);
+      const float su0 = __shfl_sync(0xffffffffu, su, 8 * t);       // head 2t
+      const float su1 = __shfl_sync(0xffffffffu, su, 8 * t + 4);   // head 2t+1
+
+      // scores: tokens g, g+8 x heads 2t, 2t+1
+      uint32_t kp0[16], kp1[16];
+      key_pairs<BK>(st, g, t, kp0);
+      key_pairs<BK>(st, g + 8, t, kp1);
+      float S[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t a[4] = {kp0[2 * s], kp1[2 * s], kp0[2 * s + 1], kp1[2 * s + 1]};
+        mma16816<true>(S, a, ub[2 * s], ub[2 * s + 1], S);
+      }
+      const float2 az0 = *reinterpret_cast<const float2*>(kaz + 2 * g);
+      const float2 az1 = *reinterpret_cast<const float2*>(kaz + 2 * (g + 8));
+      float sc[4];
+      sc[0] = fmaf(az0.x, S[0], az0.y * su0);
+      sc[1] = fmaf(az0.x, S[1], az0.y * su1);
+      sc[2] = fmaf(az1.x, S[2], az1.y * su0);
+      sc[3] = fmaf(az1.x, S[3], az1.y * su1);
+
+      // online softmax (heads 2t, 2t+1; tokens spread over g)
+      float tm0 = fmaxf(sc[0], sc[2]), tm1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, off));
+        tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
+      }
+      const float mn0 = fmaxf(mrun[0], tm0), mn1 = fmaxf(mrun[1], tm1);
+      const float al0 = exp2f(mrun[0] - mn0), al1 = exp2f(mrun[1] - mn1);
+      mrun[0] = mn0, mrun[1] = mn1;
+      const float p0 = exp2f(sc[0] - mn0), p1 = exp2f(sc[1] - mn1);
+      const float p2 = exp2f(sc[2] - mn0), p3 = exp2f(sc[3] - mn1);
+      lrun[0] = fmaf(lrun[0], al0, p0 + p2);
+      lrun[1] = fmaf(lrun[1], al1, p1 + p3);
+
+      // value weights w = p * a_V / max(a_V) (f16, transposed into B fragments)
+      const float2 vz0 = *reinterpret_cast<const float2*>(vaz + 2 * g);
+      const float2 vz1 = *reinterpret_cast<const float2*>(vaz + 2 * (g + 8));
+      float amax = fmaxf(vz0.x, vz1.x);
+      float bz0 = fmaf(p0, vz0.y, p2 * vz1.y), bz1 = fmaf(p1, vz0.y, p3 * vz1.y);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        bz0 += __shfl_xor_sync(0xffffffffu, bz0, off);
+        bz1 += __shfl_xor_sync(0xffffffffu, bz1, off);
+      }
+      const float ia = amax > 0.f ? 1.f / amax : 0.f;
+      const float r0 = vz0.x * ia, r1 = vz1.x * ia;
+      const uint32_t wb0 = movmatrix_trans(pack_f16x2(p0 * r0, p1 * r0));
+      const uint32_t wb1 = movmatrix_trans(pack_f16x2(p2 * r1, p3 * r1));
+
+      // values: channels 16g + [0,16) x heads 2t, 2t+1
+      uint32_t vp0[16], vp1[16];
+      value_pairs<BV>(st + SL.off_v, 2 * t, 2 * t + 1, g, vp0);
+      value_pairs<BV>(st + SL.off_v, 2 * t + 8, 2 * t + 9, g, vp1);
+      float cv[16];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 c4 = *reinterpret_cast<const float4*>(vc + 16 * g + 4 * k);
+        cv[4 * k] = c4.x, cv[4 * k + 1] = c4.y, cv[4 * k + 2] = c4.z, cv[4 * k + 3] = c4.w;
+      }
+      const f2 alpha = f2{al0, al1}, bz = f2{bz0, bz1}, am = splat2(amax);
+#pragma unroll
+      for (int mb = 0; mb < 8; ++mb) {
+        const uint32_t a[4] = {vp0[2 * mb], vp0[2 * mb + 1], vp1[2 * mb], vp1[2 * mb + 1]};
+        float d[4];
+        mma16816<true>(d, a, wb0, wb1, zero4);
+        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, f2{d[0], d[1]}, bz), mul2(O[mb][0], alpha));
+        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, f2{d[2], d[3]}, bz), mul2(O[mb][1], alpha));
+      }
+    }
+    __syncwarp();
+    if (issued < my_n) {
+      // the stage's shared-memory reads by all lanes precede the async refill
+      if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(issued++);
+    }
+  }
+  if (timed_out) {
+    // Drain: wait (bounded) for every copy this warp still has in flight.
+    for (int i = 0; i < issued; ++i)
+      mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
+  }
+
+  // ---- merge the CTA's warps, write this split's partial
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    lrun[0] += __shfl_xor_sync(0xffffffffu, lrun[0], off);
+    lrun[1] += __shfl_xor_sync(0xffffffffu, lrun[1], off);
+  }
+  __syncthreads();  // every warp is done with its stages
+  float* mo = reinterpret_cast<float*>(smem);                  // [kDW][8 heads][128]
+  float* ml = mo + kDW * 8 * kD;                               // [kDW][8][2]
+#pragma unroll
+  for (int mb = 0; mb < 8; ++mb)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int ch = 16 * g + 2 * mb + r;
+      mo[(warp * 8 + 2 * t) * kD + ch] = O[mb][r].x;
+      mo[(warp * 8 + 2 * t + 1) * kD + ch] = O[mb][r].y;
+    }
+  if (g == 0) {
+    ml[(warp * 8 + 2 * t) * 2] = mrun[0], ml[(warp * 8 + 2 * t) * 2 + 1] = lrun[0];
+    ml[(warp * 8 + 2 * t + 1) * 2] = mrun[1], ml[(warp * 8 + 2 * t + 1) * 2 + 1] = lrun[1];
+  }
+  __syncthreads();
+  const size_t pbase = ((size_t)pair * p.splits + split) * 8;
+  const int ch = threadIdx.x;  // kDW * 32 == 128 == kD
+  for (int h = 0; h < p.group; ++h) {
+    float mx = kNegBig;
+#pragma unroll
+    for (int w = 0; w < kDW; ++w) mx = fmaxf(mx, ml[(w * 8 + h) * 2]);
+    float acc = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDW; ++w) {
+      const float f = exp2f(ml[(w * 8 + h) * 2] - mx);
+      acc = fmaf(f, mo[(w * 8 + h) * kD + ch], acc);
+      l = fmaf(f, ml[(w * 8 + h) * 2 + 1], l);
+    }
+    p.part_o[(pbase + h) * kD + ch] = acc;
+    if (ch == 0) {
+      p.part_ml[(pbase + h) * 2] = mx;
+      p.part_ml[(pbase + h) * 2 + 1] = l;
+    }
+  }
+}
+
+// Merge the splits of one (sequence, kv-head), normalise, rotate back.
+__global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
+  __shared__ float buf[kD];
+  const int pair = blockIdx.x;
+  const int b = pair / p.num_kv_heads, kvh = pair % p.num_kv_heads;
+  const int ch = threadIdx.x;
+  for (int h = 0; h < p.group; ++h) {
+    float mx = kNegBig;
+    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)pair * p.splits + s) * 8 + h) * 2]);
+    float acc = 0.f, l = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const size_t i = ((size_t)pair * p.splits + s) * 8 + h;
+      const float f = exp2f(p.part_ml[i * 2] - mx);
+      acc = fmaf(f, p.part_o[i * kD + ch], acc);
+      l = fmaf(f, p.part_ml[i * 2 + 1], l);
+    }
+    __syncthreads();
+    buf[ch] = l > 0.f ? acc / l : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int s = 1; s < kD; s <<= 1) {
+      const float x = buf[ch & ~s], y = buf[ch | s];
+      __syncthreads();
+      buf[ch] = (ch & s) ? (x - y) : (x + y);
+      __syncthreads();
+    }
+    p.out[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch] = buf[ch] * 0.08838834764831845f;
+  }
+}
+
+template <int BK, int BV>
+int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
+  constexpr StageLayout SL = stage_layout(BK, BV);
+  // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
+  static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
+  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t);
+  auto kern = decode_d128_kernel<BK, BV>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid(p.splits, p.batch * p.num_kv_heads);
+  kern<<<grid, kDW * 32, smem, s>>>(p);
+  combine_d128_kernel<<<p.batch * p.num_kv_heads, kD, 0, s>>>(p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_decode_d128(const DecodeParams& p, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int bk = p.k.bits, bv = p.v.bits;
+#define KVQ_CASE(K, V) \
+  if (bk == K && bv == V) return launch_bk_bv<K, V>(p, s);
+  KVQ_CASE(4, 4) KVQ_CASE(3, 4) KVQ_CASE(2, 4) KVQ_CASE(8, 4)
+  KVQ_CASE(4, 2) KVQ_CASE(3, 2) KVQ_CASE(2, 2) KVQ_CASE(8, 2)
+  KVQ_CASE(4, 8) KVQ_CASE(3, 8) KVQ_CASE(2, 8) KVQ_CASE(8, 8)
+#undef KVQ_CASE
+  return (int)cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

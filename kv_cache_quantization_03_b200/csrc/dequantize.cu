@@ -1,0 +1,72 @@
+// Dequantisation of cache pages to float32 (inspection and tests; not on the
+// decode path).  Rotated domain: (a q + z) c per element; optionally rotated
+// back with H/sqrt(d) (KVarN project page on open-radar, Key Features,
+// "Variance-Normalized Quantization Pipeline": the stored tile is the
+// rotated, normalised one).
+#include <cuda_runtime.h>
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kT = 16;
+
+__device__ __forceinline__ uint32_t read_code(const uint8_t* codes, int bits, int tok, int ch) {
+  if (bits == 3) {
+    const uint32_t lo = (codes[tok * (kD / 4) + ch / 4] >> (2 * (ch % 4))) & 3u;
+    const uint32_t hi = (codes[kT * (kD / 4) + tok * (kD / 8) + ch / 8] >> (ch % 8)) & 1u;
+    return lo | (hi << 2);
+  }
+  const int bit = (tok * kD + ch) * bits;
+  return (codes[bit >> 3] >> (bit & 7)) & ((1u << bits) - 1u);
+}
+
+__global__ void __launch_bounds__(kD) dequantize_d128_kernel(DequantParams p) {
+  __shared__ float tile[kT][kD];
+  const int ch = threadIdx.x;
+  int64_t idx = blockIdx.x;
+  const int head = (int)(idx % p.num_heads);
+  idx /= p.num_heads;
+  const int kind = (int)(idx % p.kinds);
+  const int64_t pi = idx / p.kinds;
+  const int page = p.pages[pi];
+  if (page < 0 || page >= p.num_pages) {
+    if (ch == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+    return;
+  }
+  const CacheArrays src = p.src[kind];
+  const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_heads + head;
+  const uint8_t* codes = src.codes + slot * (kT * kD * src.bits / 8);
+  const float* tok = src.tok + slot * kT * 2;
+  const float c = src.chan[slot * kD + ch];
+  for (int r = 0; r < kT; ++r)
+    tile[r][ch] = fmaf(tok[2 * r], (float)read_code(codes, src.bits, r, ch), tok[2 * r + 1]) * c;
+  __syncthreads();
+  if (p.unrotate) {
+    for (int r = 0; r < kT; ++r) {
+      for (int s = 1; s < kD; s <<= 1) {
+        const float x = tile[r][ch & ~s], y = tile[r][ch | s];
+        __syncthreads();
+        tile[r][ch] = (ch & s) ? (x - y) : (x + y);
+        __syncthreads();
+      }
+      tile[r][ch] *= 0.08838834764831845f;
+    }
+    __syncthreads();
+  }
+  float* out = p.out[kind] + (((size_t)pi * p.num_heads + head) * kT) * kD;
+  for (int r = 0; r < kT; ++r) out[r * kD + ch] = tile[r][ch];
+}
+
+}  // namespace
+
+int launch_dequantize_d128(const DequantParams& p, void* stream) {
+  const int64_t blocks = p.n_pages * p.kinds * p.num_heads;
+  if (blocks == 0) return cudaSuccess;
+  dequantize_d128_kernel<<<(unsigned)blocks, kD, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,77 @@
+// Internal launch parameters shared by the host entry points and kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+// Every spin-wait in a kernel gives up after this many polls and raises
+// KVQ_DEVERR_TIMEOUT (a poll takes well under a microsecond; this bounds a
+// lost transaction to well under a second).
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// One quantised stream (K, V or the MLA latent) of the cache.
+struct CacheArrays {
+  uint8_t* codes;    // [layer][page][head][T*d*bits/8]
+  float* tok;        // [layer][page][head][T][2]
+  float* chan;       // [layer][page][head][d]
+  int bits;
+};
+
+struct QuantizeParams {
+  const void* src[2];   // K, V inputs [layer][n_tok][H][d]
+  CacheArrays dst[2];
+  int kinds;            // 1 (MLA latent only) or 2 (K and V)
+  int64_t n_tok;
+  int num_layers;
+  int num_heads;
+  int64_t num_pages;
+  int iters;
+  const int32_t* dst_page;
+  uint32_t* err;
+  int64_t total_tiles;  // kinds * layers * (n_tok / T) * heads
+};
+
+struct DequantParams {
+  CacheArrays src[2];
+  int kinds;
+  int layer;
+  int num_heads;
+  int64_t num_pages;
+  const int32_t* pages;
+  int64_t n_pages;
+  int unrotate;
+  float* out[2];
+  uint32_t* err;
+};
+
+struct DecodeParams {
+  CacheArrays k, v;
+  int layer;
+  int num_kv_heads;
+  int64_t num_pages;
+  const uint16_t* q;            // bf16 [B][Hq][d]
+  const int32_t* block_table;   // [B][max_pages]
+  int max_pages;
+  const int32_t* seq_lens;      // [B]
+  int batch;
+  int num_q_heads;
+  int group;                    // Hq / Hkv (1..8)
+  float scale_log2;             // softmax_scale * log2(e)
+  float* out;                   // [B][Hq][d]
+  float* part_o;                // [B*Hkv][splits][8][d]  un-normalised partial outputs
+  float* part_ml;               // [B*Hkv][splits][8][2]  (max, sum) in log2 units
+  int splits;
+  int tiles_per_split;
+  uint32_t* err;
+};
+
+// Launchers (defined in the .cu files); return a cudaError_t value.
+int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream);
+int launch_dequantize_d128(const DequantParams& p, void* stream);
+int launch_decode_d128(const DecodeParams& p, void* stream);
+
+}  // namespace kvq

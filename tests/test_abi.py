@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every function include/kvq.h declares, and rejects bad arguments before any
+launch (these calls never reach the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from kv_cache_quantization_03_b200 import build
+    build.build()
+    from kv_cache_quantization_03_b200 import kvq as k
+    return k
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(kvq_\w+)\s*\(", txt, re.M)))
+
+
+def test_every_declared_symbol_is_exported(kvq):
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(kvq.lib, n), n
+    assert set(names) == set(kvq.EXPORTED)
+
+
+def test_status_strings_and_version(kvq):
+    assert kvq.status_string(kvq.KVQ_OK) == "KVQ_OK"
+    assert kvq.status_string(kvq.KVQ_ERR_WORKSPACE_TOO_SMALL) == "KVQ_ERR_WORKSPACE_TOO_SMALL"
+    assert kvq.kvq_version().count(".") == 2
+
+
+def test_config_from_string(kvq):
+    c = kvq.make_config()
+    kvq.kvq_config_from_string("kvarn_k4v2_g128", c)
+    assert (c.bits_k, c.bits_v, c.tile_tokens) == (4, 2, 128)
+    for bad in ("kvarn_k5v2_g128", "kvarn_k4v2_g100", "kvarn_k4v2", "k4v2_g128", "kvarn_k4v2_g128x"):
+        assert kvq.kvq_config_from_string(bad, c, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_cache_layout_sizes(kvq):
+    c = kvq.make_config(num_kv_heads=8, num_layers=2, num_pages=10, bits_k=3, bits_v=4)
+    sizes = kvq.kvq_cache_layout(c)
+    n = 2 * 10 * 8
+    assert sizes == [n * 16 * 128 * 3 // 8, n * 16 * 2 * 4, n * 128 * 4, n * 16 * 128 * 4 // 8,
+                     n * 16 * 2 * 4, n * 128 * 4, 0]
+    m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=4)
+    s = kvq.kvq_cache_layout(m)
+    assert s[3:6] == [0, 0, 0] and s[6] == 4 * 16 * 64 * 2 and s[0] == 4 * 16 * 512 // 2
+
+
+def test_invalid_configs_rejected(kvq):
+    for kw in (dict(head_dim=96), dict(bits_k=5), dict(bits_v=1), dict(num_kv_heads=0),
+               dict(tile_tokens=12), dict(sinkhorn_iters=-1), dict(in_dtype=7)):
+        c = kvq.make_config(num_pages=4, **kw)
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_cache_layout(c)
+    c = kvq.make_config(num_pages=4, hadamard_block=64)
+    out = (ctypes.c_size_t * 7)()
+    assert kvq.lib.kvq_cache_layout(ctypes.byref(c), out) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_host_rejections_before_launch(kvq):
+    c = kvq.make_config(num_kv_heads=2, num_pages=8)
+    fake = 1 << 20                       # aligned non-null "device" pointers; never dereferenced
+    view = kvq.make_view([fake] * 6 + [None])
+    f = kvq.kvq_quantize_append
+    assert f(c, view, fake, fake, None, 17, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_PARTIAL_TILE
+    assert f(c, view, None, fake, None, 16, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert f(c, view, fake + 2, fake, None, 16, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    bad_view = kvq.make_view([fake, None] + [fake] * 4 + [None])
+    assert f(c, bad_view, fake, fake, None, 16, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    d512 = kvq.make_config(head_dim=256, num_kv_heads=2, num_pages=8)
+    assert f(d512, view, fake, fake, None, 16, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
+    assert f(c, view, fake, fake, None, 0, fake, fake, 0, raise_on_error=False) == kvq.KVQ_OK
+    dec = kvq.kvq_decode_attention
+    ws = kvq.kvq_decode_workspace_bytes(c, 4, 8, 1024)
+    assert ws > 0
+    assert dec(c, view, 0, fake, fake, 64, fake, 4, 8, 0.1, fake, fake, ws - 1, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    ws18 = kvq.kvq_decode_workspace_bytes(c, 4, 18, 1024)
+    assert dec(c, view, 0, fake, fake, 64, fake, 4, 18, 0.1, fake, fake, ws18, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED       # group 9 > 8
+    assert dec(c, view, 0, fake, fake, 64, fake, 4, 5, 0.1, fake, fake, ws, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # 5 q heads over 2 kv heads
+    assert dec(c, view, 0, fake, fake, 64, fake, 4, 8, float("nan"), fake, fake, ws, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert dec(c, view, 1, fake, fake, 64, fake, 4, 8, 0.1, fake, fake, ws, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # layer out of range
+    assert dec(c, view, 0, fake, fake, 64, fake, 0, 8, 0.1, fake, fake, ws, fake, 0,
+               raise_on_error=False) == kvq.KVQ_OK                    # empty batch: nothing to do

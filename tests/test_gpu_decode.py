@@ -1,0 +1,103 @@
+"""GPU parity of kvq_decode_attention against the oracle run on the GPU's
+stored codes and scales (tolerance 2e-3 max relative error per head)."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_quantization_03_b200 import kvq, workloads as W
+
+pytestmark = pytest.mark.gpu
+
+from _parity import ATTN_TOL, DecodeRun, QuantRun, attention_error  # noqa: E402
+
+
+def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
+    w = dec.run.w
+    G = dec.hq // w.num_kv_heads
+    worst = 0.0
+    pairs = [(b, h) for b in range(dec.batch) for h in range(w.num_kv_heads)] if pairs is None else pairs
+    for b, h in pairs:
+        ref = dec.oracle(b, h)
+        got = o[b, h * G:(h + 1) * G]
+        if dec.sl[b] // w.tile_tokens == 0:
+            assert np.all(got == 0)
+            continue
+        err = attention_error(got, ref)
+        worst = max(worst, err)
+        assert err <= ATTN_TOL, "seq %d kv-head %d: %g" % (b, h, err)
+    return worst
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("rt1k", {}),
+    ("gqa", dict(batch=3, seq_len=512)),
+    ("long", dict(batch=2, seq_len=2048)),
+])
+def test_decode_parity_small(name, kw):
+    w = W.WORKLOADS[name]
+    w = w.scaled(**kw) if kw else w
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    _check(dec, o)
+
+
+def test_decode_ragged_and_empty_sequences():
+    w = W.WORKLOADS["gqa"].scaled(batch=4, seq_len=1024)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=[1024, 16, 0, 1008])
+    o = dec()
+    assert run.error_bits() == 0
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("group,bits", [(1, (4, 4)), (2, (2, 8)), (8, (8, 2)), (8, (3, 4)), (4, (2, 2))])
+def test_decode_group_sizes_and_bit_widths(group, bits):
+    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=2, seq_len=768), num_q_heads=8 * group,
+                            bits_k=bits[0], bits_v=bits[1])
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    _check(dec, dec())
+
+
+def test_decode_bad_page_sets_error():
+    w = W.WORKLOADS["gqa"].scaled(batch=2, seq_len=256)
+    run = QuantRun(w)
+    bt = W.block_table(w).copy()
+    bt[1, 3] = w.num_pages + 5
+    dec = DecodeRun(run, block_table=bt)
+    o = dec()
+    assert run.error_bits() & 0x1
+    assert np.all(np.isfinite(o))
+    _check(dec, o, pairs=[(0, h) for h in range(w.num_kv_heads)])
+
+
+def test_decode_partial_tile_flag_and_host_errors():
+    w = W.WORKLOADS["gqa"].scaled(batch=2, seq_len=256)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=[256, 250])
+    o = dec()
+    assert run.error_bits() & 0x2
+    # host-side rejections: workspace too small, group > 8, partial append
+    st = kvq.kvq_decode_attention(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, 2, 32,
+                                  0.1, dec.out, dec.ws, 16, run.err, raise_on_error=False)
+    assert st == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    st = kvq.kvq_decode_attention(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, 2, 8 * 16,
+                                  0.1, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED
+    st = kvq.kvq_quantize_append(run.cfg, run.cache.view, run.k, run.v, None, 24, run.dst, run.err,
+                                 raise_on_error=False)
+    assert st == kvq.KVQ_ERR_PARTIAL_TILE
+
+
+def test_decode_deterministic():
+    w = W.WORKLOADS["gqa"].scaled(batch=2, seq_len=1024)
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    a = dec()
+    b = dec()
+    assert np.array_equal(a, b)

@@ -1,0 +1,136 @@
+"""GPU parity of kvq_quantize_append (and kvq_dequantize) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_quantization_03_b200 import workloads as W
+from oracle import kvarn_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+from _parity import (CODE_FLIP_RATE, QuantRun, compare_quantized, oracle_fraction)  # noqa: E402
+
+SMALL = {
+    "rt1k": {},
+    "gqa": dict(batch=2, seq_len=512),
+    "long": dict(batch=1, seq_len=1024),
+    "prefill": dict(seq_len=256, num_layers=3),
+}
+
+
+def _check_all(run: QuantRun, tiles=None, heads=None, layers=None):
+    w = run.w
+    tiles = np.arange(w.n_tok // w.tile_tokens) if tiles is None else np.asarray(tiles)
+    flips = total = 0
+    for which in (("k",) if w.mla else ("k", "v")):
+        bits = w.bits_k if which == "k" else w.bits_v
+        for layer in (range(w.num_layers) if layers is None else layers):
+            for head in (range(w.num_kv_heads) if heads is None else heads):
+                x = run.input_tiles(which, layer, tiles, head)
+                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters)
+                gpu = run.gpu_tiles(which, layer, tiles, head)
+                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters),
+                                           "%s L%d H%d" % (which, layer, head), check_rate=False)
+                total += gpu.q.size
+    assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes" % (flips, total)
+    return flips, total
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_quantize_parity_small(name):
+    w = W.WORKLOADS[name]
+    w = w.scaled(**SMALL[name]) if SMALL[name] else w
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
+
+
+@pytest.mark.parametrize("bits", [(2, 8), (8, 2), (3, 3), (4, 2)])
+def test_quantize_parity_other_bit_widths(bits):
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=1, seq_len=256), bits_k=bits[0], bits_v=bits[1])
+    run = QuantRun(w)
+    _check_all(run)
+
+
+@pytest.mark.parametrize("iters", [0, 1, 9])
+def test_quantize_parity_iteration_counts(iters):
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=1, seq_len=256), sinkhorn_iters=iters)
+    _check_all(QuantRun(w))
+
+
+def _special_tiles():
+    """Degenerate tiles: zeros, a single nonzero, constant rows, a +-1
+    checkerboard, a huge outlier channel, a zero row and a zero column."""
+    T, d = 16, 128
+    rng = np.random.default_rng(21)
+    tiles = []
+    tiles.append(np.zeros((T, d)))
+    t = np.zeros((T, d)); t[5, 17] = 3.0; tiles.append(t)
+    tiles.append(np.repeat(rng.standard_normal((T, 1)), d, axis=1))
+    tiles.append(np.where((np.arange(T)[:, None] + np.arange(d)[None, :]) % 2 == 0, 1.0, -1.0))
+    t = rng.standard_normal((T, d)); t[:, 40] *= 1000.0; tiles.append(t)
+    t = rng.standard_normal((T, d)); t[7, :] = 0.0; tiles.append(t)
+    t = rng.standard_normal((T, d)) * 1e-3; tiles.append(t)
+    t = rng.standard_normal((T, d)) * 1e4; tiles.append(t)
+    x = np.concatenate(tiles, 0).astype(np.float32)        # [n*T, d]
+    return x
+
+
+def test_quantize_parity_degenerate_tiles():
+    import dataclasses
+    x = _special_tiles()
+    n_tok = x.shape[0]
+    w = dataclasses.replace(W.WORKLOADS["gqa"], batch=1, seq_len=n_tok, num_kv_heads=1, num_q_heads=1,
+                            name="special")
+    kb = W._round_to(x, "bf16").reshape(1, n_tok, 1, 128)
+    vb = W._round_to(-x[::-1].copy(), "bf16").reshape(1, n_tok, 1, 128)
+    run = QuantRun(w, inputs=(kb, vb), pages=np.arange(n_tok // 16, dtype=np.int32))
+    assert run.error_bits() == 0
+    _check_all(run)
+    zero = run.gpu_tiles("k", 0, [0], 0)
+    assert np.all(zero.q == 0) and np.all(zero.a == 0) and np.all(zero.z == 0) and np.all(zero.c == 1)
+
+
+def test_quantize_bad_page_sets_error_and_skips_tile():
+    w = W.WORKLOADS["gqa"].scaled(batch=1, seq_len=64)
+    pages = np.array([0, 7, 2, 3], dtype=np.int32)        # pool of 4 pages: 7 is out of range
+    run = QuantRun(w, quantize=False, pages=pages, num_pages=4)
+    canary = run.cache.codes("k")[0, 1].clone()
+    run.cache.codes("k")[0, 1].fill_(0xA5)
+    run.cache.codes("v")[0, 1].fill_(0xA5)
+    run.quantize()
+    assert run.error_bits() & 0x1
+    assert torch.all(run.cache.codes("k")[0, 1] == 0xA5) and torch.all(run.cache.codes("v")[0, 1] == 0xA5)
+    del canary
+    _check_all(run, tiles=[0, 2, 3])
+
+
+def test_quantize_deterministic():
+    w = W.WORKLOADS["gqa"].scaled(batch=1, seq_len=512)
+    run = QuantRun(w)
+    first = {n: t.clone() for n, t in run.cache.arrays.items() if t is not None}
+    run.quantize()
+    for n, t in first.items():
+        assert torch.equal(run.cache.arrays[n], t), n
+
+
+def test_dequantize_matches_oracle_on_stored_codes():
+    from kv_cache_quantization_03_b200 import kvq
+    w = W.WORKLOADS["long"].scaled(batch=1, seq_len=256)
+    run = QuantRun(w)
+    pages = torch.arange(w.num_pages, dtype=torch.int32, device="cuda")
+    for unrot in (0, 1):
+        ko = torch.empty(w.num_pages, w.num_kv_heads, 16, 128, device="cuda")
+        vo = torch.empty_like(ko)
+        kvq.kvq_dequantize(run.cfg, run.cache.view, 0, pages, w.num_pages, unrot, ko, vo, run.err)
+        torch.cuda.synchronize()
+        for which, out in (("k", ko), ("v", vo)):
+            for h in range(w.num_kv_heads):
+                inv = np.argsort(run.pages)                      # page -> tile
+                g = run.gpu_tiles(which, 0, inv, h)              # tiles in page order
+                ref = O.dequantize_tiles(g.q, g.a, g.z, g.c, unrotate=bool(unrot))
+                got = out[:, h].cpu().numpy().astype(np.float64)
+                scale = np.max(np.abs(ref), axis=(-1, -2), keepdims=True)
+                assert np.max(np.abs(got - ref) / scale) < 2e-6
