@@ -16,7 +16,9 @@
 // and streams it through its own ring of shared-memory stages filled with
 // 1-D bulk async copies (one mbarrier per stage, bounded waits).  Both
 // contractions of a tile run as m16n8k16 f16 MMAs with fp32 accumulation:
-// codes 0..255 are exact in f16; u and w are rounded to f16.
+// codes 0..255 are exact in f16; u and w are each carried as an f16 pair
+// hi + lo (two MMAs into one fp32 accumulator), which keeps ~22 significant
+// bits where a single f16 would cost up to 8e-3 of attention accuracy.
 //   scores:  D[16 tokens x 8 heads]   = codes_K[16 x 128] * u^T[128 x 8]
 //   values:  D[128 channels x 8 heads] = codes_V^T[128 x 16] * w[16 x 8]
 // The per-channel c_V is applied to each tile's fresh MMA result before it
@@ -244,11 +246,11 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
   for (int mb = 0; mb < 8; ++mb) O[mb][0] = O[mb][1] = f2{0.f, 0.f};
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
-  bool timed_out = false;
+  int stop = -1;  // local tile whose wait ran out
   for (int i = 0; i < my_n; ++i) {
     const bool ok = mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
     if (!__all_sync(0xffffffffu, ok)) {
-      timed_out = true;
+      stop = i;
       if (lane == 0) set_error(p.err, KVQ_DEVERR_TIMEOUT);
       break;
     }
@@ -268,13 +270,13 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
         ck[4 * k] = c4.x, ck[4 * k + 1] = c4.y, ck[4 * k + 2] = c4.z, ck[4 * k + 3] = c4.w;
       }
       float su = 0.f;
-      uint32_t ub[16];
+      uint32_t ubh[16], ubl[16];  // u = hi + lo, both f16: ~22 significant bits
 #pragma unroll
       for (int pi = 0; pi < 16; ++pi) {
         const int c0 = kchan<BK>(pi), c1 = c0 + kdist<BK>();
         const float u0 = qr[c0] * ck[c0], u1 = qr[c1] * ck[c1];
         su += u0 + u1;
-        ub[pi] = pack_f16x2(u0, u1);
+        split_f16x2(u0, u1, ubh[pi], ubl[pi]);
       }
       su += __shfl_xor_sync(0xffffffffu, su, 1);
       su += __shfl_xor_sync(0xffffffffu, su, 2);
@@ -289,7 +291,8 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t a[4] = {kp0[2 * s], kp1[2 * s], kp0[2 * s + 1], kp1[2 * s + 1]};
-        mma16816<true>(S, a, ub[2 * s], ub[2 * s + 1], S);
+        mma16816<true>(S, a, ubh[2 * s], ubh[2 * s + 1], S);
+        mma16816<true>(S, a, ubl[2 * s], ubl[2 * s + 1], S);
       }
       const float2 az0 = *reinterpret_cast<const float2*>(kaz + 2 * g);
       const float2 az1 = *reinterpret_cast<const float2*>(kaz + 2 * (g + 8));
@@ -327,8 +330,11 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       }
       const float ia = amax > 0.f ? 1.f / amax : 0.f;
       const float r0 = vz0.x * ia, r1 = vz1.x * ia;
-      const uint32_t wb0 = movmatrix_trans(pack_f16x2(p0 * r0, p1 * r0));
-      const uint32_t wb1 = movmatrix_trans(pack_f16x2(p2 * r1, p3 * r1));
+      uint32_t wh0, wl0, wh1, wl1;  // w = hi + lo, both f16
+      split_f16x2(p0 * r0, p1 * r0, wh0, wl0);
+      split_f16x2(p2 * r1, p3 * r1, wh1, wl1);
+      wh0 = movmatrix_trans(wh0), wl0 = movmatrix_trans(wl0);
+      wh1 = movmatrix_trans(wh1), wl1 = movmatrix_trans(wl1);
 
       // values: channels 16g + [0,16) x heads 2t, 2t+1
       uint32_t vp0[16], vp1[16];
@@ -345,7 +351,8 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       for (int mb = 0; mb < 8; ++mb) {
         const uint32_t a[4] = {vp0[2 * mb], vp0[2 * mb + 1], vp1[2 * mb], vp1[2 * mb + 1]};
         float d[4];
-        mma16816<true>(d, a, wb0, wb1, zero4);
+        mma16816<true>(d, a, wh0, wh1, zero4);
+        mma16816<true>(d, a, wl0, wl1, d);
         O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, f2{d[0], d[1]}, bz), mul2(O[mb][0], alpha));
         O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, f2{d[2], d[3]}, bz), mul2(O[mb][1], alpha));
       }
@@ -357,9 +364,9 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       issue(issued++);
     }
   }
-  if (timed_out) {
-    // Drain: wait (bounded) for every copy this warp still has in flight.
-    for (int i = 0; i < issued; ++i)
+  if (stop >= 0) {
+    // Drain: wait (bounded) for the copies this warp still has in flight.
+    for (int i = stop + 1; i < issued; ++i)
       mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
   }
 

@@ -98,6 +98,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// (x, y) = hi + lo with hi = f16(x, y) and lo = f16 of the remainder.
+__device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x, y);
+  const float2 b = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x - b.x, y - b.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
 
 // ---------------------------------------------------------------- memory
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
