@@ -1,0 +1,376 @@
+"""Throughput of the KVarN-style hot path on B200: quantize-append + decode attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa] [--impl kvq|reference]
+
+One step = the whole hot path over one batch of the workload: every new K/V
+row of the batch is rotated, normalised, quantised and packed into the paged
+cache (kvq_quantize_append), then one decode step of attention runs over the
+quantised cache (kvq_decode_attention, split-KV + combine).  The default
+workload is the Llama-3-8B-shaped GQA case: 32 sequences x 8192 tokens, 8 kv /
+32 query heads, head_dim 128, bf16 inputs, 4-bit K and V, 16-token pages.
+
+value  = KV tokens quantized per second (all ranks; one token = all kv-heads'
+         K and V rows of one position), inputs resident in HBM;
+e2e    = the same through the C ABI with the step's inputs copied from pinned
+         host memory and the attention output read back, inside the timing;
+roofline = the quantize kernel (the larger share of the step's bytes) against
+         the measured HBM copy bandwidth; decode_attn gives the decode kernel's
+         algorithmic GB/s and fraction the same way.
+Multi-GPU (torchrun): every rank runs its own shard (own batch, own seed), no
+data-path collective; time = max over ranks.  --impl reference times the
+float64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KV tokens quantized/s; quantized decode-attn HBM GB/s and % of B200 peak"
+UNIT = "tokens/s"
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def algorithmic_bytes(w):
+    """(quantize bytes, decode bytes) one step must move, from the cache format."""
+    T, d, H = w.tile_tokens, w.head_dim, w.num_kv_heads
+    rows = w.num_layers * w.n_tok * H
+    per_row_in = d * 2
+    def cache_row(bits):                       # codes + (a, z) + c share of one row
+        return d * bits / 8 + 8 + d * 4 / T
+    q_bytes = rows * 2 * per_row_in + rows * (cache_row(w.bits_k) + cache_row(w.bits_v))
+    dec_bytes = w.batch * w.seq_len * H * (cache_row(w.bits_k) + cache_row(w.bits_v)) \
+        + w.batch * w.num_q_heads * d * (2 + 4)
+    return q_bytes, dec_bytes
+
+
+def traffic_from_profile(kernel_file: str, profile_name: str):
+    """Bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    src = os.path.join(ROOT, "kv_cache_quantization_03_b200", "csrc", kernel_file)
+    try:
+        txt = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha256_16:\s*([0-9a-f]+)", txt)
+        if m and m.group(2) == sha:
+            return float(m.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- oracle leg
+def oracle_sample_step(w, sample):
+    """Float64 oracle over one (sequence, kv-head) of the workload: quantise its K
+    and V rows, then decode its query group over the sequence.  Returns the token
+    equivalents processed (positions x kv-heads / H_kv)."""
+    import numpy as np
+    from oracle import kvarn_oracle as O
+    from kv_cache_quantization_03_b200 import workloads as W
+    xk, xv, q = sample
+    kt = O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters)
+    vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters)
+    O.decode_attention(q, kt, vt, w.softmax_scale)
+    return xk.shape[0] * xk.shape[1] / w.num_kv_heads
+
+
+def oracle_sample_inputs(w, tokens):
+    import numpy as np
+    from kv_cache_quantization_03_b200 import workloads as W
+    sub = slice(0, max(tokens, W.CHUNK_TOKENS))
+    xk = W.half_bits_to_f64(W.kv_inputs(w, "k", sub)[0, :tokens, 0], w.in_dtype)
+    xv = W.half_bits_to_f64(W.kv_inputs(w, "v", sub)[0, :tokens, 0], w.in_dtype)
+    xk = xk.reshape(-1, w.tile_tokens, w.head_dim)
+    xv = xv.reshape(-1, w.tile_tokens, w.head_dim)
+    q = W.half_bits_to_f64(W.queries(w)[0, :w.group], "bf16")
+    return xk, xv, q
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, budget_s=12.0, tokens=4096):
+    sample = oracle_sample_inputs(w, tokens)
+    t0 = time.perf_counter()
+    done = 0.0
+    n = 0
+    while True:
+        done += oracle_sample_step(w, sample)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": "%d x {quantize K and V of one kv-head over %d tokens of sequence 0 (float64, dense "
+                      "Hadamard) + decode of its %d query heads over them}; %.1f s" % (n, tokens, w.group, dt)}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    tokens = 1024
+    sample = oracle_sample_inputs(w, tokens)
+    for _ in range(args.warmup):
+        oracle_sample_step(w, sample)
+    t0 = time.perf_counter()
+    done = 0.0
+    for _ in range(args.steps):
+        done += oracle_sample_step(w, sample)
+    dt = time.perf_counter() - t0
+    v = done / dt
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(w, args),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": "each step: one kv-head of sequence 0, %d tokens: quantize K and V + "
+                                       "decode of its %d query heads (float64 oracle)" % (tokens, w.group)},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def config_dict(w, args):
+    return {"workload": w.name, "description": w.description, "batch": w.batch, "seq_len": w.seq_len,
+            "num_kv_heads": w.num_kv_heads, "num_q_heads": w.num_q_heads, "head_dim": w.head_dim,
+            "bits_k": w.bits_k, "bits_v": w.bits_v, "tile_tokens": w.tile_tokens,
+            "sinkhorn_iters": w.sinkhorn_iters, "layers": w.num_layers,
+            "parallelism": "dp%d (independent shards)" % args.gpus,
+            "l2": "inputs larger than L2 (K+V bf16 %.2f GB per rank)" % (
+                2 * w.num_layers * w.n_tok * w.num_kv_heads * w.head_dim * 2 / 1e9)}
+
+
+# --------------------------------------------------------------------------- GPU leg
+def run_gpu(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_quantization_03_b200 import kvq, workloads as W
+    from kv_cache_quantization_03_b200.cache import QuantizedCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ws = dataclasses.replace(w, seed=w.seed + 7919 * rank)        # this rank's shard
+
+    cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
+                          bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters,
+                          num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype)
+    cache = QuantizedCache(cfg)
+    kb, vb = W.kv_inputs(ws, "k"), W.kv_inputs(ws, "v")
+    qb, pages = W.queries(ws), W.page_assignment(ws)
+    bt, sl = W.block_table(ws), W.seq_lens(ws)
+    host = {"k": torch.from_numpy(kb.view(np.int16)).pin_memory(),
+            "v": torch.from_numpy(vb.view(np.int16)).pin_memory(),
+            "q": torch.from_numpy(qb.view(np.int16)).pin_memory(),
+            "dst": torch.from_numpy(pages).pin_memory(),
+            "bt": torch.from_numpy(np.ascontiguousarray(bt)).pin_memory(),
+            "sl": torch.from_numpy(sl).pin_memory()}
+    dev = {k: v.cuda() for k, v in host.items()}
+    out = torch.empty(w.batch, w.num_q_heads, w.head_dim, device="cuda")
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws_bytes = kvq.kvq_decode_workspace_bytes(cfg, w.batch, w.num_q_heads, w.seq_len)
+    work = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    s_ptr = stream.cuda_stream
+
+    def quantize():
+        kvq.kvq_quantize_append(cfg, cache.view, dev["k"], dev["v"], None, w.n_tok, dev["dst"], err, s_ptr)
+
+    def decode():
+        kvq.kvq_decode_attention(cfg, cache.view, 0, dev["q"], dev["bt"], w.tiles_per_seq, dev["sl"], w.batch,
+                                 w.num_q_heads, w.softmax_scale, out, work, ws_bytes, err, s_ptr)
+
+    for _ in range(max(args.warmup, 3)):
+        quantize()
+        decode()
+    torch.cuda.synchronize()
+    st, bits = kvq.kvq_read_error(err, s_ptr)
+    if st != kvq.KVQ_OK or bits:
+        raise RuntimeError("device error word %#x after warm-up" % bits)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            quantize()
+            ev[i][1].record(stream)
+            decode()
+            ev[i][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = start.elapsed_time(end) / 1e3
+    t_q = sum(e[0].elapsed_time(e[1]) for e in ev) / K / 1e3
+    t_d = sum(e[1].elapsed_time(e[2]) for e in ev) / K / 1e3
+
+    # end to end: inputs from pinned host memory, output back to the host, each step
+    Ke = max(1, min(K, 10))
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = out.numel() * out.element_size()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        quantize()
+        decode()
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3 / Ke
+    st, bits = kvq.kvq_read_error(err, s_ptr)
+    if st != kvq.KVQ_OK or bits:
+        raise RuntimeError("device error word %#x" % bits)
+
+    t = torch.tensor([elapsed, e2e_s, t_q, t_d], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed, e2e_s, t_q, t_d = t.tolist()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    tokens = w.batch * w.seq_len * world
+    peak, peak_kind = load_peaks()
+    qb_bytes, db_bytes = algorithmic_bytes(w)
+    q_gbs = qb_bytes / t_q / 1e9
+    d_gbs = db_bytes / t_d / 1e9
+    traffic = traffic_from_profile("quantize.cu", "quantize_d128_gqa.md")
+    line = {
+        "metric": METRIC, "value": tokens * K / elapsed, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; see workloads.py)",
+        "config": config_dict(w, args),
+        "roofline": {"kernel": "quantize_d128", "bound": "hbm", "achieved": q_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": q_gbs / peak, "peak_source": peak_kind,
+                     "traffic": traffic, "algorithmic_bytes": qb_bytes},
+        "decode_attn": {"kernel": "decode_d128 + combine", "gbs": d_gbs, "frac_of_measured": d_gbs / peak,
+                        "frac_of_8tbs": d_gbs / 8000.0, "us": 1e6 * t_d, "algorithmic_bytes": db_bytes},
+        "quantize": {"rows_per_s": w.num_layers * w.n_tok * w.num_kv_heads * 2 / t_q, "gbs": q_gbs,
+                     "frac_of_8tbs": q_gbs / 8000.0, "us": 1e6 * t_q},
+        "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling small cases)")
+    ap.add_argument("--seq-len", type=int, default=None, help="override the context length")
+    args = ap.parse_args()
+    from kv_cache_quantization_03_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    if args.batch or args.seq_len:
+        w = w.scaled(batch=args.batch, seq_len=args.seq_len, name="%s-b%d-l%d" % (
+            w.name, args.batch or w.batch, args.seq_len or w.seq_len))
+    if w.mla or w.num_q_heads // w.num_kv_heads > 8:
+        raise SystemExit("bench covers the GQA workloads (rt1k, gqa, long, prefill)")
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()
