@@ -174,6 +174,7 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.dst_page = dst_page;
   p.err = dev_error;
   p.total_tiles = (int64_t)p.kinds * c->num_layers * (n_tok / c->tile_tokens) * c->num_kv_heads;
+  if (p.total_tiles >= (int64_t)1 << 31) return KVQ_ERR_UNSUPPORTED;  // tile ids are 32-bit in the kernel
   return cuda_status(launch_quantize_d128(p, c->in_dtype == KVQ_F16, stream));
 }
 

@@ -53,11 +53,43 @@ __host__ __device__ constexpr StageLayout stage_layout(int bk, int bv) {
 }
 
 // ---- code pairs -> f16x2 (exact small integers)
-__device__ __forceinline__ uint32_t h2_codes(uint32_t masked) {
-  uint32_t v = masked | 0x64006400u;  // f16 1024 + code in each half
+// A field of a 32-bit word masked in place in both halves and OR-ed into the
+// exponent of 1024 reads as the f16 value 1024 + code * 2^shift; one HFMA2
+// (scale 2^-shift, bias -1024 * 2^-shift) leaves the code.
+template <int SHIFT>
+__device__ __forceinline__ uint32_t h2_field(uint32_t word, uint32_t mask) {
+  uint32_t v = (word & (mask << SHIFT)) | 0x64006400u;
   __half2 h = *reinterpret_cast<__half2*>(&v);
-  h = __hsub2(h, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  if constexpr (SHIFT == 0) {
+    h = __hsub2(h, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  } else {
+    constexpr float sc = 1.0f / (1 << SHIFT);
+    const __half2 s2 = __float2half2_rn(sc), b2 = __float2half2_rn(-1024.0f * sc);
+    h = __hfma2(h, s2, b2);
+  }
   return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t h2_codes(uint32_t masked) { return h2_field<0>(masked, 0xFFFFFFFFu); }
+
+// Four code pairs of one word of 4-bit codes: (nibble e, nibble e+4), e = 0..3.
+__device__ __forceinline__ void nib_pairs(uint32_t w, uint32_t* out) {
+  const uint32_t w8 = w >> 8;
+  out[0] = h2_field<0>(w, 0x000F000Fu);
+  out[1] = h2_field<4>(w, 0x000F000Fu);
+  out[2] = h2_field<0>(w8, 0x000F000Fu);
+  out[3] = h2_field<4>(w8, 0x000F000Fu);
+}
+// Eight code pairs of one word of 2-bit codes: (field e, field e+8), e = 0..7.
+__device__ __forceinline__ void crumb_pairs(uint32_t w, uint32_t* out) {
+  const uint32_t w8 = w >> 8;
+  out[0] = h2_field<0>(w, 0x00030003u);
+  out[1] = h2_field<2>(w, 0x00030003u);
+  out[2] = h2_field<4>(w, 0x00030003u);
+  out[3] = h2_field<6>(w, 0x00030003u);
+  out[4] = h2_field<0>(w8, 0x00030003u);
+  out[5] = h2_field<2>(w8, 0x00030003u);
+  out[6] = h2_field<4>(w8, 0x00030003u);
+  out[7] = h2_field<6>(w8, 0x00030003u);
 }
 
 // Key-side pairing: lane t covers channels 32t..32t+31 of a token row; pair
@@ -76,31 +108,35 @@ template <int B>
 __device__ __forceinline__ void key_pairs(const uint8_t* codes, int row, int t, uint32_t (&pr)[16]) {
   if constexpr (B == 4) {
     const uint4 w = *reinterpret_cast<const uint4*>(codes + row * 64 + 16 * t);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 2] >> (4 * (pi & 3))) & 0x000F000Fu);
+    nib_pairs(w.x, pr);
+    nib_pairs(w.y, pr + 4);
+    nib_pairs(w.z, pr + 8);
+    nib_pairs(w.w, pr + 12);
   } else if constexpr (B == 2) {
     const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
-    const uint32_t ws[2] = {w.x, w.y};
-#pragma unroll
-    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 3] >> (2 * (pi & 7))) & 0x00030003u);
+    crumb_pairs(w.x, pr);
+    crumb_pairs(w.y, pr + 8);
   } else if constexpr (B == 8) {
     const uint4 w0 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t);
     const uint4 w1 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t + 16);
     const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int pi = 0; pi < 16; ++pi) pr[pi] = h2_codes((ws[pi >> 1] >> (8 * (pi & 1))) & 0x00FF00FFu);
+    for (int k = 0; k < 8; ++k) {
+      pr[2 * k] = h2_field<0>(ws[k], 0x00FF00FFu);
+      pr[2 * k + 1] = h2_field<0>(ws[k] >> 8, 0x00FF00FFu);
+    }
   } else {  // 3 bits: low plane [T][32 B] then high plane [T][16 B]
     const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
     const uint32_t hw = *reinterpret_cast<const uint32_t*>(codes + kT * 32 + row * 16 + 4 * t);
-    const uint32_t ws[2] = {w.x, w.y};
+    uint32_t lo[16];
+    crumb_pairs(w.x, lo);
+    crumb_pairs(w.y, lo + 8);
     const uint32_t hs[2] = {__byte_perm(hw, 0u, 0x4140u), __byte_perm(hw, 0u, 0x4342u)};
     const __half2 four = __halves2half2(__ushort_as_half(0x4400), __ushort_as_half(0x4400));
 #pragma unroll
     for (int pi = 0; pi < 16; ++pi) {
-      uint32_t lo = h2_codes((ws[pi >> 3] >> (2 * (pi & 7))) & 0x00030003u);
       uint32_t hi = h2_codes((hs[pi >> 3] >> (pi & 7)) & 0x00010001u);
-      __half2 r = __hfma2(*reinterpret_cast<__half2*>(&hi), four, *reinterpret_cast<__half2*>(&lo));
+      __half2 r = __hfma2(*reinterpret_cast<__half2*>(&hi), four, *reinterpret_cast<__half2*>(&lo[pi]));
       pr[pi] = *reinterpret_cast<uint32_t*>(&r);
     }
   }
@@ -115,19 +151,19 @@ __device__ __forceinline__ void value_pairs(const uint8_t* codes, int rx, int ry
     const uint32_t xs[2] = {x.x, x.y}, ys[2] = {y.x, y.y};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+      // bytes 2(k&1), 2(k&1)+1 of both tokens: channels 4k..4k+3, x in the low half
       const uint32_t m = __byte_perm(xs[k >> 1], ys[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pr[4 * k + e] = h2_codes((m >> (4 * e)) & 0x000F000Fu);
+      const uint32_t m8 = m >> 8;
+      pr[4 * k] = h2_field<0>(m, 0x000F000Fu);
+      pr[4 * k + 1] = h2_field<4>(m, 0x000F000Fu);
+      pr[4 * k + 2] = h2_field<0>(m8, 0x000F000Fu);
+      pr[4 * k + 3] = h2_field<4>(m8, 0x000F000Fu);
     }
   } else if constexpr (B == 2) {
     const uint32_t x = *reinterpret_cast<const uint32_t*>(codes + rx * 32 + 4 * g);
     const uint32_t y = *reinterpret_cast<const uint32_t*>(codes + ry * 32 + 4 * g);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint32_t m = __byte_perm(x, y, k ? 0x7632u : 0x5410u);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) pr[8 * k + e] = h2_codes((m >> (2 * e)) & 0x00030003u);
-    }
+    crumb_pairs(__byte_perm(x, y, 0x5410u), pr);
+    crumb_pairs(__byte_perm(x, y, 0x7632u), pr + 8);
   } else {  // 8 bits
     const uint4 x = *reinterpret_cast<const uint4*>(codes + rx * 128 + 16 * g);
     const uint4 y = *reinterpret_cast<const uint4*>(codes + ry * 128 + 16 * g);
@@ -135,10 +171,16 @@ __device__ __forceinline__ void value_pairs(const uint8_t* codes, int rx, int ry
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const uint32_t m = __byte_perm(xs[k >> 1], ys[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) pr[2 * k + e] = h2_codes((m >> (8 * e)) & 0x00FF00FFu);
+      pr[2 * k] = h2_field<0>(m, 0x00FF00FFu);
+      pr[2 * k + 1] = h2_field<0>(m >> 8, 0x00FF00FFu);
     }
   }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -175,7 +217,13 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
   const int t0 = split * p.tiles_per_split;
   const int t1 = min(t0 + p.tiles_per_split, ntiles);
   const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
-  const int32_t* btab = p.block_table + (size_t)b * p.max_pages;
+  // this split's page ids, staged once in shared memory
+  int32_t* spg = reinterpret_cast<int32_t*>(bars + kDW * kStages);
+  {
+    const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
+    for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[i];
+  }
+  __syncthreads();
 
   // ---- rotated, pre-scaled query: lane (g, t) keeps head g, channels 32t..32t+31
   float qr[32];
@@ -220,7 +268,7 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
     if (lane != 0) return;
     uint64_t* bar = &wbar[i % kStages];
     uint8_t* st = wsm + (i % kStages) * SL.bytes;
-    const int page = btab[t0 + warp + i * kDW];
+    const int page = spg[warp + i * kDW];
     if (page < 0 || page >= p.num_pages) {
       set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       mbar_arrive_expect_tx(bar, 0);
@@ -254,7 +302,7 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       if (lane == 0) set_error(p.err, KVQ_DEVERR_TIMEOUT);
       break;
     }
-    const int page = btab[t0 + warp + i * kDW];
+    const int page = spg[warp + i * kDW];
     if (page >= 0 && page < p.num_pages) {
       const uint8_t* st = wsm + (i % kStages) * SL.bytes;
       const float* kaz = reinterpret_cast<const float*>(st + SL.off_kaz);
@@ -310,10 +358,10 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
         tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
       }
       const float mn0 = fmaxf(mrun[0], tm0), mn1 = fmaxf(mrun[1], tm1);
-      const float al0 = exp2f(mrun[0] - mn0), al1 = exp2f(mrun[1] - mn1);
+      const float al0 = ex2(mrun[0] - mn0), al1 = ex2(mrun[1] - mn1);
       mrun[0] = mn0, mrun[1] = mn1;
-      const float p0 = exp2f(sc[0] - mn0), p1 = exp2f(sc[1] - mn1);
-      const float p2 = exp2f(sc[2] - mn0), p3 = exp2f(sc[3] - mn1);
+      const float p0 = ex2(sc[0] - mn0), p1 = ex2(sc[1] - mn1);
+      const float p2 = ex2(sc[2] - mn0), p3 = ex2(sc[3] - mn1);
       lrun[0] = fmaf(lrun[0], al0, p0 + p2);
       lrun[1] = fmaf(lrun[1], al1, p1 + p3);
 
@@ -347,14 +395,18 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
         cv[4 * k] = c4.x, cv[4 * k + 1] = c4.y, cv[4 * k + 2] = c4.z, cv[4 * k + 3] = c4.w;
       }
       const f2 alpha = f2{al0, al1}, bz = f2{bz0, bz1}, am = splat2(amax);
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {  // a running max moved
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) O[mb][0] = mul2(O[mb][0], alpha), O[mb][1] = mul2(O[mb][1], alpha);
+      }
 #pragma unroll
       for (int mb = 0; mb < 8; ++mb) {
         const uint32_t a[4] = {vp0[2 * mb], vp0[2 * mb + 1], vp1[2 * mb], vp1[2 * mb + 1]};
         float d[4];
         mma16816<true>(d, a, wh0, wh1, zero4);
         mma16816<true>(d, a, wl0, wl1, d);
-        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, f2{d[0], d[1]}, bz), mul2(O[mb][0], alpha));
-        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, f2{d[2], d[3]}, bz), mul2(O[mb][1], alpha));
+        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, f2{d[0], d[1]}, bz), O[mb][0]);
+        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, f2{d[2], d[3]}, bz), O[mb][1]);
       }
     }
     __syncwarp();
@@ -401,7 +453,7 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
     float acc = 0.f, l = 0.f;
 #pragma unroll
     for (int w = 0; w < kDW; ++w) {
-      const float f = exp2f(ml[(w * 8 + h) * 2] - mx);
+      const float f = ex2(ml[(w * 8 + h) * 2] - mx);
       acc = fmaf(f, mo[(w * 8 + h) * kD + ch], acc);
       l = fmaf(f, ml[(w * 8 + h) * 2 + 1], l);
     }
@@ -425,7 +477,7 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
     float acc = 0.f, l = 0.f;
     for (int s = 0; s < p.splits; ++s) {
       const size_t i = ((size_t)pair * p.splits + s) * 8 + h;
-      const float f = exp2f(p.part_ml[i * 2] - mx);
+      const float f = ex2(p.part_ml[i * 2] - mx);
       acc = fmaf(f, p.part_o[i * kD + ch], acc);
       l = fmaf(f, p.part_ml[i * 2 + 1], l);
     }
@@ -448,7 +500,8 @@ int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
   constexpr StageLayout SL = stage_layout(BK, BV);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
-  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t);
+  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
+                      ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
   auto kern = decode_d128_kernel<BK, BV>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.splits, p.batch * p.num_kv_heads);

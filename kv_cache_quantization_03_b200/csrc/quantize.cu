@@ -38,7 +38,6 @@ constexpr int kD = 128;
 constexpr int kT = 16;
 constexpr int kWarps = 8;
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: adding it rounds to an integer (ties to even)
-constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 
 // Channel bits carried by the MMA contraction index k = 2t + j0 + 8*j1
@@ -57,74 +56,106 @@ __device__ __forceinline__ uint32_t sign_pair(int m, int k0) {
   return lo | (hi << 16);
 }
 
-__device__ __forceinline__ uint32_t code_of(float t) {
-  return __float_as_uint(t) - kMagicBits;
+// 1/x and 1/sqrt(x) from the hardware approximations plus one Newton step
+// (about 1 ulp), for the few per-row / per-column factors of each tile.
+__device__ __forceinline__ float rcp_nr(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return fmaf(r, fmaf(-x, r, 1.f), r);
+}
+__device__ __forceinline__ float rsqrt_nr(float x) {
+  float y;
+  asm("rsqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y * fmaf(-0.5f * x * y, y, 1.5f);
+}
+
+// Byte 0 of four words, in order: the code held by a magic-number float.
+__device__ __forceinline__ uint32_t gather4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x4000u), 0x7610u);
+}
+// Eight 4-bit codes (byte 0 of each word) -> one word, code i in bits 4i..4i+3.
+__device__ __forceinline__ uint32_t pack_nibbles(const uint32_t* f) {
+  uint32_t u = gather4(f[0], f[1], f[2], f[3]), v = gather4(f[4], f[5], f[6], f[7]);
+  u |= u >> 4;
+  v |= v >> 4;
+  return __byte_perm(u, v, 0x6420u);
+}
+
+struct WarpScratch {
+  float4 col[4][32];  // column partial sums, chunk k of lane (g, t) at [k][4g + (t ^ k)]
+  float4 own[32];     // per-lane owned values (1/c^2 or 1/c), read back by every lane
+};
+
+template <bool F16>
+__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantizeParams& p, uint32_t tile, int g,
+                                          int t, int32_t& page) {
+  const uint32_t H = p.num_heads, ntt = (uint32_t)(p.n_tok / kT);
+  const uint32_t head = tile % H, r1 = tile / H;
+  const uint32_t tt = r1 % ntt, r2 = r1 / ntt;
+  const uint32_t layer = r2 % (uint32_t)p.num_layers, kind = r2 / (uint32_t)p.num_layers;
+  page = __ldg(p.dst_page + tt);
+  const uint16_t* base = static_cast<const uint16_t*>(p.src[kind]) +
+                         (((size_t)layer * p.n_tok + (size_t)tt * kT) * H + head) * kD;
+  const size_t row_stride = (size_t)H * kD;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint16_t* row = base + (size_t)(8 * h + g) * row_stride + 8 * t;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      const uint4 v = ldg_nc_v4(row + 32 * l);
+      L[h][l][0] = v.x, L[h][l][1] = v.y, L[h][l][2] = v.z, L[h][l][3] = v.w;
+    }
+  }
 }
 
 template <bool F16>
-__global__ void __launch_bounds__(kWarps * 32) quantize_d128_kernel(QuantizeParams p) {
+__global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeParams p) {
+  __shared__ WarpScratch scratch[kWarps];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;  // bits 1, 2 of g
+  WarpScratch& sc = scratch[threadIdx.x >> 5];
   uint32_t afrag[4];
   afrag[0] = sign_pair<F16>(g, 2 * t);
   afrag[1] = sign_pair<F16>(g + 8, 2 * t);
   afrag[2] = sign_pair<F16>(g, 2 * t + 8);
   afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8);
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint32_t total = (uint32_t)p.total_tiles;
+  const uint32_t stride = gridDim.x * kWarps;
+  uint32_t tile = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (tile >= total) return;
 
-  const int64_t ntt = p.n_tok / kT;
-  const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-  for (int64_t tile = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); tile < p.total_tiles; tile += nwarps) {
-    int64_t rem = tile;
-    const int head = (int)(rem % p.num_heads);
-    rem /= p.num_heads;
-    const int64_t tt = rem % ntt;
-    rem /= ntt;
-    const int layer = (int)(rem % p.num_layers);
-    const int kind = (int)(rem / p.num_layers);
-    const int page = __ldg(p.dst_page + tt);
-    if (page < 0 || page >= p.num_pages) {
-      if (lane == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
-      continue;
-    }
-    const CacheArrays dst = p.dst[kind];
-
-    // ---- load: lane reads tokens g and g+8, channels 32l + 8t .. +7 (l = 0..3)
-    const uint16_t* base = static_cast<const uint16_t*>(p.src[kind]) +
-                           (((size_t)layer * p.n_tok + (size_t)tt * kT) * p.num_heads + head) * kD;
-    const size_t row_stride = (size_t)p.num_heads * kD;
-    uint32_t L[2][4][4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint16_t* row = base + (size_t)(8 * h + g) * row_stride + 8 * t;
-#pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        const uint4 v = ldg_nc_v4(row + 32 * l);
-        L[h][l][0] = v.x;
-        L[h][l][1] = v.y;
-        L[h][l][2] = v.z;
-        L[h][l][3] = v.w;
-      }
-    }
-
-    // ---- rotation: MMA over channel bits 3..6, then butterflies over bits 0..2
-    // P[h][m3][b] = values of tokens (8h+2t, 8h+2t+1) at channel 16g + 8*m3 + b
+  uint32_t L[2][4][4];
+  int32_t page;
+  load_tile<F16>(L, p, tile, g, t, page);
+  for (; tile < total; tile += stride) {
+    // ---- rotation: MMA over channel bits 3..6 -> P[h][m3][b] = tokens (8h+2t, 8h+2t+1),
+    //      channel 16g + 8*m3 + b; then butterflies over bits 0..2
     f2 P[2][2][8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         const uint32_t sel = (b & 1) ? 0x7632u : 0x5410u;
-        const uint32_t b0 = __byte_perm(L[h][0][b >> 1], L[h][1][b >> 1], sel);
-        const uint32_t b1 = __byte_perm(L[h][2][b >> 1], L[h][3][b >> 1], sel);
         float d[4];
-        mma16816<F16>(d, afrag, b0, b1, zero4);
+        mma16816<F16>(d, afrag, __byte_perm(L[h][0][b >> 1], L[h][1][b >> 1], sel),
+                      __byte_perm(L[h][2][b >> 1], L[h][3][b >> 1], sel), zero4);
         P[h][0][b] = f2{d[0], d[1]};
         P[h][1][b] = f2{d[2], d[3]};
       }
+    const int32_t cur_page = page;
+    const uint32_t cur = tile;
+    if (tile + stride < total) load_tile<F16>(L, p, tile + stride, g, t, page);  // prefetch the next tile
+    if (cur_page < 0 || cur_page >= p.num_pages) {
+      if (lane == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+      continue;
+    }
 #pragma unroll
-      for (int m3 = 0; m3 < 2; ++m3) {
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int s = 1; s < 8; s <<= 1) {
+      for (int m3 = 0; m3 < 2; ++m3)
+#pragma unroll
+        for (int s = 1; s < 8; s <<= 1)
 #pragma unroll
           for (int b = 0; b < 8; ++b) {
             if (b & s) continue;
@@ -132,11 +163,8 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_d128_kernel(QuantizePara
             P[h][m3][b] = add2(x, y);
             P[h][m3][b + s] = sub2(x, y);
           }
-        }
-      }
-    }
 
-    // ---- normalisation on the factors (A = Z^2 kept in registers)
+    // ---- normalisation on the factors; A = Z^2
     f2 A[2][2][8];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -145,158 +173,182 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_d128_kernel(QuantizePara
 #pragma unroll
         for (int b = 0; b < 8; ++b) A[h][m3][b] = mul2(P[h][m3][b], P[h][m3][b]);
 
-    float w[16];   // 1 / c_j^2, j = 8*m3 + b
-    float v[2][2]; // 1 / r_i^2 of tokens 8h + 2t + tp
-    float C[16];   // last column sums
+    float w[16];                          // 1 / c_j^2 of this lane's channels
+    float v[2][2];                        // 1 / r_i^2 of this lane's tokens
+    float v_own = 1.f;                    // token (h = b2, tp = b1) of column t
+    float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);  // channels 16g + 4t .. +3
+    float4 c_tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) w[j] = 1.f, C[j] = 0.f;
-    v[0][0] = v[0][1] = v[1][0] = v[1][1] = 1.f;
+    for (int j = 0; j < 16; ++j) w[j] = 1.f;
     for (int it = 0; it < p.iters; ++it) {
+      // rows: partial sums over 16 channels, reduce-scatter over g, one owner per token
       f2 R[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         R[h] = f2{0.f, 0.f};
 #pragma unroll
-        for (int m3 = 0; m3 < 2; ++m3)
+        for (int j = 0; j < 16; ++j) R[h] = fma2(A[h][j >> 3][j & 7], splat2(w[j]), R[h]);
+      }
+      f2 keep = b2 ? R[1] : R[0];
+      const f2 send = b2 ? R[0] : R[1];
+      keep.x += __shfl_xor_sync(0xffffffffu, send.x, 16);
+      keep.y += __shfl_xor_sync(0xffffffffu, send.y, 16);
+      float rk = b1 ? keep.y : keep.x;
+      rk += __shfl_xor_sync(0xffffffffu, b1 ? keep.x : keep.y, 8);
+      rk += __shfl_xor_sync(0xffffffffu, rk, 4);
+      if (rk > 0.f) v_own = (float)kD * rcp_nr(rk);
 #pragma unroll
-          for (int b = 0; b < 8; ++b) R[h] = fma2(A[h][m3][b], splat2(w[8 * m3 + b]), R[h]);
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tp = 0; tp < 2; ++tp) v[h][tp] = __shfl_sync(0xffffffffu, v_own, (h << 4) | (tp << 3) | t);
+
+      // columns: partial sums over 4 tokens, reduced through shared memory
+      float C[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const f2 acc = fma2(A[1][j >> 3][j & 7], f2{v[1][0], v[1][1]}, mul2(A[0][j >> 3][j & 7], f2{v[0][0], v[0][1]}));
+        C[j] = acc.x + acc.y;
       }
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
+      for (int k = 0; k < 4; ++k)
+        sc.col[k][(lane & ~3) | (t ^ k)] = make_float4(C[4 * k], C[4 * k + 1], C[4 * k + 2], C[4 * k + 3]);
+      __syncwarp();
+      c_tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          R[h].x += __shfl_xor_sync(0xffffffffu, R[h].x, off);
-          R[h].y += __shfl_xor_sync(0xffffffffu, R[h].y, off);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float4 x = sc.col[t][(lane & ~3) | (i ^ t)];
+        c_tot.x += x.x, c_tot.y += x.y, c_tot.z += x.z, c_tot.w += x.w;
       }
+      if (c_tot.x > 0.f) w_own.x = (float)kT * rcp_nr(c_tot.x);
+      if (c_tot.y > 0.f) w_own.y = (float)kT * rcp_nr(c_tot.y);
+      if (c_tot.z > 0.f) w_own.z = (float)kT * rcp_nr(c_tot.z);
+      if (c_tot.w > 0.f) w_own.w = (float)kT * rcp_nr(c_tot.w);
+      sc.own[lane] = w_own;
+      __syncwarp();
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        v[h][0] = R[h].x > 0.f ? (float)kD / R[h].x : v[h][0];
-        v[h][1] = R[h].y > 0.f ? (float)kD / R[h].y : v[h][1];
+      for (int k = 0; k < 4; ++k) {
+        const float4 x = sc.own[(lane & ~3) | k];
+        w[4 * k] = x.x, w[4 * k + 1] = x.y, w[4 * k + 2] = x.z, w[4 * k + 3] = x.w;
       }
-#pragma unroll
-      for (int m3 = 0; m3 < 2; ++m3)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          f2 acc = mul2(A[0][m3][b], f2{v[0][0], v[0][1]});
-          acc = fma2(A[1][m3][b], f2{v[1][0], v[1][1]}, acc);
-          C[8 * m3 + b] = acc.x + acc.y;
-        }
-#pragma unroll
-      for (int off = 1; off < 4; off <<= 1)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) C[j] += __shfl_xor_sync(0xffffffffu, C[j], off);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) w[j] = C[j] > 0.f ? (float)kT / C[j] : w[j];
+      __syncwarp();
     }
 
-    // ---- column factor c and Y' = Z / c
-    float cf[16];
+    // ---- column factor c (owned channels), 1/c to every lane, Y' = Z / c
+    const uint32_t head = cur % (uint32_t)p.num_heads;
+    const uint32_t lk = cur / (uint32_t)p.num_heads / (uint32_t)(p.n_tok / kT);  // layer + layers * kind
+    const uint32_t layer = lk % (uint32_t)p.num_layers;
+    const int kind = (int)(lk / (uint32_t)p.num_layers);
+    const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;
+    const CacheArrays dst = p.dst[kind];
+    {
+      float cv[4], ic[4];
+      const float ct[4] = {c_tot.x, c_tot.y, c_tot.z, c_tot.w};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float c2 = C[j] > 0.f ? C[j] / (float)kT : 1.f;
-      cf[j] = sqrtf(c2);
-      const float ic = 1.f / cf[j];
+      for (int i = 0; i < 4; ++i) {
+        if (p.iters > 0 && ct[i] > 0.f) {
+          const float x = ct[i] * (1.f / kT);
+          ic[i] = rsqrt_nr(x);
+          cv[i] = x * ic[i];
+        } else {
+          ic[i] = 1.f, cv[i] = 1.f;
+        }
+      }
+      *reinterpret_cast<float4*>(dst.chan + slot * kD + 16 * g + 4 * t) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+      sc.own[lane] = make_float4(ic[0], ic[1], ic[2], ic[3]);
+      __syncwarp();
 #pragma unroll
-      for (int h = 0; h < 2; ++h) P[h][j >> 3][j & 7] = mul2(P[h][j >> 3][j & 7], splat2(ic));
+      for (int k = 0; k < 4; ++k) {
+        const float4 x = sc.own[(lane & ~3) | k];
+        const float icj[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * k + e;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) P[h][j >> 3][j & 7] = mul2(P[h][j >> 3][j & 7], splat2(icj[e]));
+        }
+      }
+      __syncwarp();
     }
 
-    // ---- per-token min / max of Y'
+    // ---- per-token min / max of Y': in-lane, then reduce-scatter over g
     float mn[2][2], mx[2][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float a0 = P[h][0][0].x, b0 = P[h][0][0].x, a1 = P[h][0][0].y, b1 = P[h][0][0].y;
+      float a0 = P[h][0][0].x, c0 = a0, a1 = P[h][0][0].y, c1 = a1;
 #pragma unroll
       for (int j = 1; j < 16; j += 2) {
         const f2 u = P[h][j >> 3][j & 7];
         const f2 u2 = (j + 1 < 16) ? P[h][(j + 1) >> 3][(j + 1) & 7] : u;
-        a0 = min3(a0, u.x, u2.x);
-        b0 = max3(b0, u.x, u2.x);
-        a1 = min3(a1, u.y, u2.y);
-        b1 = max3(b1, u.y, u2.y);
+        a0 = min3(a0, u.x, u2.x), c0 = max3(c0, u.x, u2.x);
+        a1 = min3(a1, u.y, u2.y), c1 = max3(c1, u.y, u2.y);
       }
-      mn[h][0] = a0, mx[h][0] = b0, mn[h][1] = a1, mx[h][1] = b1;
+      mn[h][0] = a0, mx[h][0] = c0, mn[h][1] = a1, mx[h][1] = c1;
     }
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1)
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tp = 0; tp < 2; ++tp) {
-          mn[h][tp] = fminf(mn[h][tp], __shfl_xor_sync(0xffffffffu, mn[h][tp], off));
-          mx[h][tp] = fmaxf(mx[h][tp], __shfl_xor_sync(0xffffffffu, mx[h][tp], off));
-        }
-
+    float kmn0 = b2 ? mn[1][0] : mn[0][0], kmn1 = b2 ? mn[1][1] : mn[0][1];
+    float kmx0 = b2 ? mx[1][0] : mx[0][0], kmx1 = b2 ? mx[1][1] : mx[0][1];
+    kmn0 = fminf(kmn0, __shfl_xor_sync(0xffffffffu, b2 ? mn[0][0] : mn[1][0], 16));
+    kmn1 = fminf(kmn1, __shfl_xor_sync(0xffffffffu, b2 ? mn[0][1] : mn[1][1], 16));
+    kmx0 = fmaxf(kmx0, __shfl_xor_sync(0xffffffffu, b2 ? mx[0][0] : mx[1][0], 16));
+    kmx1 = fmaxf(kmx1, __shfl_xor_sync(0xffffffffu, b2 ? mx[0][1] : mx[1][1], 16));
+    float omn = b1 ? kmn1 : kmn0, omx = b1 ? kmx1 : kmx0;
+    omn = fminf(omn, __shfl_xor_sync(0xffffffffu, b1 ? kmn0 : kmn1, 8));
+    omx = fmaxf(omx, __shfl_xor_sync(0xffffffffu, b1 ? kmx0 : kmx1, 8));
+    omn = fminf(omn, __shfl_xor_sync(0xffffffffu, omn, 4));
+    omx = fmaxf(omx, __shfl_xor_sync(0xffffffffu, omx, 4));
     const int bits = dst.bits;
     const float qmax = (float)((1 << bits) - 1);
-    const size_t slot = ((size_t)layer * p.num_pages + page) * p.num_heads + head;
-    const int tile_bytes = kT * kD * bits / 8;
-    uint8_t* codes = dst.codes + slot * tile_bytes;
-    float inv_s[2][2], st[2][2];
+    const float s_own = (omx - omn) / qmax;
+    const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
+    if ((lane & 4) == 0) {  // owner of token 8*b2 + 2t + b1 writes (a, z)
+      float* tokp = dst.tok + slot * (kT * 2);
+      *reinterpret_cast<float2*>(tokp + 2 * (8 * b2 + 2 * t + b1)) = make_float2(s_own * kInvSqrtD, omn * kInvSqrtD);
+    }
+    float mtok[2][2], istok[2][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int tp = 0; tp < 2; ++tp) {
-        const float s = (mx[h][tp] - mn[h][tp]) / qmax;
-        st[h][tp] = s;
-        inv_s[h][tp] = s > 0.f ? 1.f / s : 0.f;
+        const int src = (h << 4) | (tp << 3) | t;
+        mtok[h][tp] = __shfl_sync(0xffffffffu, omn, src);
+        istok[h][tp] = __shfl_sync(0xffffffffu, is_own, src);
       }
 
-    // ---- codes and packing, one token row at a time
+    // ---- codes (magic-number rounding: byte 0 of the float holds the code) and packing
+    const int tile_bytes = kT * kD * bits / 8;
+    uint8_t* codes = dst.codes + slot * tile_bytes;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const f2 m2 = f2{mn[h][0], mn[h][1]}, is2 = f2{inv_s[h][0], inv_s[h][1]};
-      uint32_t q[16][2];
+      const f2 m2 = f2{mtok[h][0], mtok[h][1]}, is2 = f2{istok[h][0], istok[h][1]};
+      uint32_t q[2][16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const f2 tq = add2(mul2(sub2(P[h][j >> 3][j & 7], m2), is2), splat2(kMagic));
-        q[j][0] = code_of(tq.x);
-        q[j][1] = code_of(tq.y);
+        q[0][j] = __float_as_uint(tq.x);
+        q[1][j] = __float_as_uint(tq.y);
       }
 #pragma unroll
       for (int tp = 0; tp < 2; ++tp) {
         const int tok = 8 * h + 2 * t + tp;
+        const uint32_t* f = q[tp];
         if (bits == 4) {
-          uint32_t lo = 0, hi = 0;
-#pragma unroll
-          for (int b = 0; b < 8; ++b) lo |= q[b][tp] << (4 * b), hi |= q[8 + b][tp] << (4 * b);
-          *reinterpret_cast<uint2*>(codes + tok * 64 + 8 * g) = make_uint2(lo, hi);
+          *reinterpret_cast<uint2*>(codes + tok * 64 + 8 * g) = make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
+        } else if (bits == 8) {
+          *reinterpret_cast<uint4*>(codes + tok * 128 + 16 * g) =
+              make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
+                         gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
         } else if (bits == 2) {
           uint32_t wd = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) wd |= q[j][tp] << (2 * j);
+          for (int j = 0; j < 16; ++j) wd |= (f[j] & 3u) << (2 * j);
           *reinterpret_cast<uint32_t*>(codes + tok * 32 + 4 * g) = wd;
-        } else if (bits == 8) {
-          uint32_t wd[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int j = 0; j < 16; ++j) wd[j >> 2] |= q[j][tp] << (8 * (j & 3));
-          *reinterpret_cast<uint4*>(codes + tok * 128 + 16 * g) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         } else {  // 3 bits: low-2-bit plane [T][32 B], then high-bit plane [T][16 B]
           uint32_t lo = 0, hi = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) lo |= (q[j][tp] & 3u) << (2 * j), hi |= (q[j][tp] >> 2) << j;
+          for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
           *reinterpret_cast<uint32_t*>(codes + tok * 32 + 4 * g) = lo;
           *reinterpret_cast<uint16_t*>(codes + kT * 32 + tok * 16 + 2 * g) = (uint16_t)hi;
         }
       }
-    }
-
-    // ---- folded scales
-    if (g == 0) {
-      float* tokp = dst.tok + slot * (kT * 2);
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tp = 0; tp < 2; ++tp) {
-          const int tok = 8 * h + 2 * t + tp;
-          *reinterpret_cast<float2*>(tokp + 2 * tok) =
-              make_float2(st[h][tp] * kInvSqrtD, mn[h][tp] * kInvSqrtD);
-        }
-    }
-    if (t == 0) {
-      float4* cp = reinterpret_cast<float4*>(dst.chan + slot * kD + 16 * g);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) cp[k] = make_float4(cf[4 * k], cf[4 * k + 1], cf[4 * k + 2], cf[4 * k + 3]);
     }
   }
 }
@@ -309,7 +361,7 @@ int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t need = (p.total_tiles + kWarps - 1) / kWarps;
-  const int64_t cap = (int64_t)sms * 8;
+  const int64_t cap = (int64_t)sms;
   const int grid = (int)(need < cap ? need : cap);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (f16)
