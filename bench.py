@@ -340,7 +340,7 @@ def run_gpu(args, w):
         "quantize": {"rows_per_s": w.num_layers * w.n_tok * w.num_kv_heads * 2 / t_q, "gbs": q_gbs,
                      "frac_of_8tbs": q_gbs / 8000.0, "us": 1e6 * t_q},
         "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,  # quantize K, quantize V, decode, combine
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
   float lrun[2] = {0.f, 0.f};          // this lane's share of the running sums
   f2 O[8][2];                          // [m-block][row g / g+8] x heads (2t, 2t+1)
 #pragma unroll
-  for (int mb = 0; mb < 8; ++mb) O[mb][0] = O[mb][1] = f2{0.f, 0.f};
+  for (int mb = 0; mb < 8; ++mb) O[mb][0] = O[mb][1] = make_float2(0.f, 0.f);
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
   int stop = -1;  // local tile whose wait ran out
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
         const float4 c4 = *reinterpret_cast<const float4*>(vc + 16 * g + 4 * k);
         cv[4 * k] = c4.x, cv[4 * k + 1] = c4.y, cv[4 * k + 2] = c4.z, cv[4 * k + 3] = c4.w;
       }
-      const f2 alpha = f2{al0, al1}, bz = f2{bz0, bz1}, am = splat2(amax);
+      const f2 alpha = make_float2(al0, al1), bz = make_float2(bz0, bz1), am = splat2(amax);
       if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {  // a running max moved
 #pragma unroll
         for (int mb = 0; mb < 8; ++mb) O[mb][0] = mul2(O[mb][0], alpha), O[mb][1] = mul2(O[mb][1], alpha);
@@ -405,8 +405,8 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
         float d[4];
         mma16816<true>(d, a, wh0, wh1, zero4);
         mma16816<true>(d, a, wl0, wl1, d);
-        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, f2{d[0], d[1]}, bz), O[mb][0]);
-        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, f2{d[2], d[3]}, bz), O[mb][1]);
+        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, make_float2(d[0], d[1]), bz), O[mb][0]);
+        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, make_float2(d[2], d[3]), bz), O[mb][1]);
       }
     }
     __syncwarp();

@@ -11,43 +11,15 @@
 namespace kvq {
 
 // ---------------------------------------------------------------- fp32 pairs
-// sm_100 executes two fp32 operations per instruction on 64-bit register
-// pairs; these wrappers keep the pairing explicit.
-struct f2 {
-  float x, y;
-};
-
-__device__ __forceinline__ unsigned long long pk(f2 a) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a.x), "f"(a.y));
-  return r;
-}
-__device__ __forceinline__ f2 upk(unsigned long long r) {
-  f2 a;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
-  return a;
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
-}
-__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
-  unsigned long long r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
-}
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-  unsigned long long r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
-  return upk(r);
-}
-__device__ __forceinline__ f2 splat2(float v) { return f2{v, v}; }
+// sm_100 executes two fp32 operations per instruction on a 64-bit register
+// pair (the float2 builtins below); keeping values in float2 lets the
+// compiler allocate the pairs directly.
+using f2 = float2;
+__device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f2 splat2(float v) { return make_float2(v, v); }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;

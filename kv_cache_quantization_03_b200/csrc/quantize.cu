@@ -7,22 +7,25 @@
 // per-token asymmetric round-to-nearest, packing into the tile's cache page.
 //
 // One warp owns one tile.  Lane (g = lane/4, t = lane%4) ends up holding the
-// rotated values of tokens {2t, 2t+1, 2t+8, 2t+9} and channels 16g..16g+15.
+// rotated values of tokens {2t, 2t+1, 2t+8, 2t+9} and channels 16g..16g+15
+// (register pairs hold the two tokens 8h + 2t, 8h + 2t + 1 of one channel).
 //
 // Rotation: the Sylvester matrix factors over the 7 bits of the channel
 // index, H_128 = (x) over bits of H_2.  Bits 3..6 are contracted with one
-// 16x16 +-1 matrix on the tensor cores (mma.sync m16n8k16, exact products,
-// fp32 accumulation; 16 MMAs per tile); bits 0..2 are three in-register
-// butterfly stages on fp32 pairs.  The 1/sqrt(128) factor is not applied to
-// the tile: the column factors c are invariant to a uniform scale of the
-// tile, and a, z are scaled by it at the end.
+// 16x16 +-1 matrix on the tensor cores (mma.sync m16n8k16 with 8 tokens as
+// N: exact products, fp32 accumulation, 16 MMAs per tile); bits 0..2 are
+// three in-register butterfly stages on fp32 pairs.
+// The 1/sqrt(128) factor is not applied to the tile: the column factors c
+// are invariant to a uniform scale, and a, z are scaled by it at the end.
 //
 // Normalisation: the rounds of "divide rows by their RMS, then columns by
 // theirs" are carried out on the factors only.  With A = Z*Z,
 //   r_i^2 = (1/d) sum_j A_ij / c_j^2      (row step; kept if the sum is 0)
 //   c_j^2 = (1/T) sum_i A_ij / r_i^2      (column step; kept if the sum is 0)
 // which is the same recursion as rescaling the tile each half-step, since
-// Y = diag(r)^-1 Z diag(c)^-1 throughout.
+// Y = diag(r)^-1 Z diag(c)^-1 throughout.  Row sums are reduced with
+// shuffles (one lane per token computes its reciprocal); column sums go
+// through the warp's shared memory (each lane owns four channels).
 //
 // Quantisation: a row-wise affine map is invariant to a positive row factor,
 // so codes come from Y' = Z / c directly, and a = r*s = s', z = r*m = m'
@@ -36,8 +39,9 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kT = 16;
-constexpr int kWarps = 8;
-constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: adding it rounds to an integer (ties to even)
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer (ties to even)
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 
 // Channel bits carried by the MMA contraction index k = 2t + j0 + 8*j1
@@ -82,24 +86,39 @@ __device__ __forceinline__ uint32_t pack_nibbles(const uint32_t* f) {
 }
 
 struct WarpScratch {
-  float4 col[4][32];  // column partial sums, chunk k of lane (g, t) at [k][4g + (t ^ k)]
-  float4 own[32];     // per-lane owned values (1/c^2 or 1/c), read back by every lane
+  float4 col[4][32];  // column partials: chunk k of lane (g, t) at [k][4g + (t ^ k)]
+  float4 own[32];     // owned channels 16g + 4t .. +3
+  float4 dup[2][32];  // owned 1/c twice each
 };
 
-template <bool F16>
-__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantizeParams& p, uint32_t tile, int g,
-                                          int t, int32_t& page) {
-  const uint32_t H = p.num_heads, ntt = (uint32_t)(p.n_tok / kT);
-  const uint32_t head = tile % H, r1 = tile / H;
-  const uint32_t tt = r1 % ntt, r2 = r1 / ntt;
-  const uint32_t layer = r2 % (uint32_t)p.num_layers, kind = r2 / (uint32_t)p.num_layers;
+// Quotient by a fixed divisor with a multiply-high (n < 2^31).
+struct FastDiv {
+  uint32_t d, m, s;
+};
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) { return (__umulhi(n, f.m) + n) >> f.s; }
+
+struct QuantLaunch {
+  const uint16_t* src;   // [layer][n_tok][H][d]
+  CacheArrays dst;
+  int64_t n_tok;
+  int num_layers, num_heads;
+  int64_t num_pages;
+  int iters;
+  const int32_t* dst_page;
+  uint32_t* err;
+  uint32_t total;        // layers * (n_tok / T) * heads
+  FastDiv div_h, div_ntt;
+};
+
+__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLaunch& p, uint32_t tile, int g, int t,
+                                          int32_t& page) {
+  const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
+  const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
   page = __ldg(p.dst_page + tt);
-  const uint16_t* base = static_cast<const uint16_t*>(p.src[kind]) +
-                         (((size_t)layer * p.n_tok + (size_t)tt * kT) * H + head) * kD;
-  const size_t row_stride = (size_t)H * kD;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint16_t* row = base + (size_t)(8 * h + g) * row_stride + 8 * t;
+    const uint16_t* row =
+        p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * kD + 8 * t;
 #pragma unroll
     for (int l = 0; l < 4; ++l) {
       const uint4 v = ldg_nc_v4(row + 32 * l);
@@ -108,11 +127,11 @@ __device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const Quantize
   }
 }
 
-template <bool F16>
-__global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeParams p) {
+template <bool F16, int BITS>
+__global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch p) {
   __shared__ WarpScratch scratch[kWarps];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;  // bits 1, 2 of g
+  const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
   WarpScratch& sc = scratch[threadIdx.x >> 5];
   uint32_t afrag[4];
   afrag[0] = sign_pair<F16>(g, 2 * t);
@@ -120,18 +139,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
   afrag[2] = sign_pair<F16>(g, 2 * t + 8);
   afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8);
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint32_t total = (uint32_t)p.total_tiles;
   const uint32_t stride = gridDim.x * kWarps;
   uint32_t tile = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (tile >= total) return;
-
+  if (tile >= p.total) return;
   uint32_t L[2][4][4];
   int32_t page;
-  load_tile<F16>(L, p, tile, g, t, page);
-  for (; tile < total; tile += stride) {
-    // ---- rotation: MMA over channel bits 3..6 -> P[h][m3][b] = tokens (8h+2t, 8h+2t+1),
-    //      channel 16g + 8*m3 + b; then butterflies over bits 0..2
-    f2 P[2][2][8];
+  load_tile(L, p, tile, g, t, page);
+  for (; tile < p.total; tile += stride) {
+    f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -140,12 +155,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
         float d[4];
         mma16816<F16>(d, afrag, __byte_perm(L[h][0][b >> 1], L[h][1][b >> 1], sel),
                       __byte_perm(L[h][2][b >> 1], L[h][3][b >> 1], sel), zero4);
-        P[h][0][b] = f2{d[0], d[1]};
-        P[h][1][b] = f2{d[2], d[3]};
+        P[h][0][b] = make_float2(d[0], d[1]);
+        P[h][1][b] = make_float2(d[2], d[3]);
       }
     const int32_t cur_page = page;
     const uint32_t cur = tile;
-    if (tile + stride < total) load_tile<F16>(L, p, tile + stride, g, t, page);  // prefetch the next tile
+    if (tile + stride < p.total) load_tile(L, p, tile + stride, g, t, page);
     if (cur_page < 0 || cur_page >= p.num_pages) {
       if (lane == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       continue;
@@ -163,66 +178,71 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
             P[h][m3][b] = add2(x, y);
             P[h][m3][b + s] = sub2(x, y);
           }
-
-    // ---- normalisation on the factors; A = Z^2
+    // squares paired along channels: A[h][tp][q] = channels 2q, 2q+1 of token 8h + 2t + tp
     f2 A[2][2][8];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int m3 = 0; m3 < 2; ++m3)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) A[h][m3][b] = mul2(P[h][m3][b], P[h][m3][b]);
-
-    float w[16];                          // 1 / c_j^2 of this lane's channels
-    float v[2][2];                        // 1 / r_i^2 of this lane's tokens
-    float v_own = 1.f;                    // token (h = b2, tp = b1) of column t
-    float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);  // channels 16g + 4t .. +3
-    float4 c_tot = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < 8; ++q) {
+        const f2 x = P[h][q >> 2][2 * (q & 3)], y = P[h][q >> 2][2 * (q & 3) + 1];
+        A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
+        A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
+      }
+    float w[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 1.f;
+    float v_own = 1.f;
+    float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
+    f2 c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
     for (int it = 0; it < p.iters; ++it) {
-      // rows: partial sums over 16 channels, reduce-scatter over g, one owner per token
-      f2 R[2];
+      float R[2][2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        R[h] = f2{0.f, 0.f};
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) R[h] = fma2(A[h][j >> 3][j & 7], splat2(w[j]), R[h]);
-      }
-      f2 keep = b2 ? R[1] : R[0];
-      const f2 send = b2 ? R[0] : R[1];
-      keep.x += __shfl_xor_sync(0xffffffffu, send.x, 16);
-      keep.y += __shfl_xor_sync(0xffffffffu, send.y, 16);
-      float rk = b1 ? keep.y : keep.x;
-      rk += __shfl_xor_sync(0xffffffffu, b1 ? keep.x : keep.y, 8);
+        for (int tp = 0; tp < 2; ++tp) {
+          f2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < 8; q += 2) {
+            acc0 = fma2(A[h][tp][q], make_float2(w[2 * q], w[2 * q + 1]), acc0);
+            acc1 = fma2(A[h][tp][q + 1], make_float2(w[2 * q + 2], w[2 * q + 3]), acc1);
+          }
+          const f2 s2 = add2(acc0, acc1);
+          R[h][tp] = s2.x + s2.y;
+        }
+      float k0 = b2 ? R[1][0] : R[0][0], k1 = b2 ? R[1][1] : R[0][1];
+      k0 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][0] : R[1][0], 16);
+      k1 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][1] : R[1][1], 16);
+      float rk = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 8);
       rk += __shfl_xor_sync(0xffffffffu, rk, 4);
-      if (rk > 0.f) v_own = (float)kD * rcp_nr(rk);
+      const float vn = (float)kD * rcp_nr(rk);
+      v_own = rk > 0.f ? vn : v_own;
+      float v[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int tp = 0; tp < 2; ++tp) v[h][tp] = __shfl_sync(0xffffffffu, v_own, (h << 4) | (tp << 3) | t);
-
-      // columns: partial sums over 4 tokens, reduced through shared memory
-      float C[16];
+      f2 C[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const f2 acc = fma2(A[1][j >> 3][j & 7], f2{v[1][0], v[1][1]}, mul2(A[0][j >> 3][j & 7], f2{v[0][0], v[0][1]}));
-        C[j] = acc.x + acc.y;
-      }
+      for (int q = 0; q < 8; ++q)
+        C[q] = fma2(A[1][1][q], splat2(v[1][1]),
+                    fma2(A[1][0][q], splat2(v[1][0]), fma2(A[0][1][q], splat2(v[0][1]), mul2(A[0][0][q], splat2(v[0][0])))));
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        sc.col[k][(lane & ~3) | (t ^ k)] = make_float4(C[4 * k], C[4 * k + 1], C[4 * k + 2], C[4 * k + 3]);
+        sc.col[k][(lane & ~3) | (t ^ k)] = make_float4(C[2 * k].x, C[2 * k].y, C[2 * k + 1].x, C[2 * k + 1].y);
       __syncwarp();
-      c_tot = make_float4(0.f, 0.f, 0.f, 0.f);
+      c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 x = sc.col[t][(lane & ~3) | (i ^ t)];
-        c_tot.x += x.x, c_tot.y += x.y, c_tot.z += x.z, c_tot.w += x.w;
+        c01 = add2(c01, make_float2(x.x, x.y));
+        c23 = add2(c23, make_float2(x.z, x.w));
       }
-      if (c_tot.x > 0.f) w_own.x = (float)kT * rcp_nr(c_tot.x);
-      if (c_tot.y > 0.f) w_own.y = (float)kT * rcp_nr(c_tot.y);
-      if (c_tot.z > 0.f) w_own.z = (float)kT * rcp_nr(c_tot.z);
-      if (c_tot.w > 0.f) w_own.w = (float)kT * rcp_nr(c_tot.w);
+      const float n0 = (float)kT * rcp_nr(c01.x), n1 = (float)kT * rcp_nr(c01.y);
+      const float n2 = (float)kT * rcp_nr(c23.x), n3 = (float)kT * rcp_nr(c23.y);
+      w_own.x = c01.x > 0.f ? n0 : w_own.x;
+      w_own.y = c01.y > 0.f ? n1 : w_own.y;
+      w_own.z = c23.x > 0.f ? n2 : w_own.z;
+      w_own.w = c23.y > 0.f ? n3 : w_own.w;
       sc.own[lane] = w_own;
       __syncwarp();
 #pragma unroll
@@ -232,45 +252,37 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
       }
       __syncwarp();
     }
-
-    // ---- column factor c (owned channels), 1/c to every lane, Y' = Z / c
-    const uint32_t head = cur % (uint32_t)p.num_heads;
-    const uint32_t lk = cur / (uint32_t)p.num_heads / (uint32_t)(p.n_tok / kT);  // layer + layers * kind
-    const uint32_t layer = lk % (uint32_t)p.num_layers;
-    const int kind = (int)(lk / (uint32_t)p.num_layers);
+    const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
+    const uint32_t layer = fdiv(r1, p.div_ntt);
     const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;
-    const CacheArrays dst = p.dst[kind];
     {
+      const bool norm = p.iters > 0;
+      const float ct[4] = {c01.x, c01.y, c23.x, c23.y};
       float cv[4], ic[4];
-      const float ct[4] = {c_tot.x, c_tot.y, c_tot.z, c_tot.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (p.iters > 0 && ct[i] > 0.f) {
-          const float x = ct[i] * (1.f / kT);
-          ic[i] = rsqrt_nr(x);
-          cv[i] = x * ic[i];
-        } else {
-          ic[i] = 1.f, cv[i] = 1.f;
-        }
+        const float x = ct[i] * (1.f / kT);
+        const float y = rsqrt_nr(x);
+        const bool ok = norm && ct[i] > 0.f;
+        ic[i] = ok ? y : 1.f;
+        cv[i] = ok ? x * y : 1.f;
       }
-      *reinterpret_cast<float4*>(dst.chan + slot * kD + 16 * g + 4 * t) = make_float4(cv[0], cv[1], cv[2], cv[3]);
-      sc.own[lane] = make_float4(ic[0], ic[1], ic[2], ic[3]);
+      *reinterpret_cast<float4*>(p.dst.chan + slot * kD + 16 * g + 4 * t) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+      sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
+      sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
       __syncwarp();
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 x = sc.own[(lane & ~3) | k];
-        const float icj[4] = {x.x, x.y, x.z, x.w};
+      for (int k = 0; k < 8; ++k) {
+        const float4 x = sc.dup[k & 1][(lane & ~3) | (k >> 1)];
+        const int j = 2 * k;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 4 * k + e;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) P[h][j >> 3][j & 7] = mul2(P[h][j >> 3][j & 7], splat2(icj[e]));
+        for (int h = 0; h < 2; ++h) {
+          P[h][j >> 3][j & 7] = mul2(P[h][j >> 3][j & 7], make_float2(x.x, x.y));
+          P[h][(j + 1) >> 3][(j + 1) & 7] = mul2(P[h][(j + 1) >> 3][(j + 1) & 7], make_float2(x.z, x.w));
         }
       }
       __syncwarp();
     }
-
-    // ---- per-token min / max of Y': in-lane, then reduce-scatter over g
     float mn[2][2], mx[2][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -284,41 +296,27 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
       }
       mn[h][0] = a0, mx[h][0] = c0, mn[h][1] = a1, mx[h][1] = c1;
     }
-    float kmn0 = b2 ? mn[1][0] : mn[0][0], kmn1 = b2 ? mn[1][1] : mn[0][1];
-    float kmx0 = b2 ? mx[1][0] : mx[0][0], kmx1 = b2 ? mx[1][1] : mx[0][1];
-    kmn0 = fminf(kmn0, __shfl_xor_sync(0xffffffffu, b2 ? mn[0][0] : mn[1][0], 16));
-    kmn1 = fminf(kmn1, __shfl_xor_sync(0xffffffffu, b2 ? mn[0][1] : mn[1][1], 16));
-    kmx0 = fmaxf(kmx0, __shfl_xor_sync(0xffffffffu, b2 ? mx[0][0] : mx[1][0], 16));
-    kmx1 = fmaxf(kmx1, __shfl_xor_sync(0xffffffffu, b2 ? mx[0][1] : mx[1][1], 16));
-    float omn = b1 ? kmn1 : kmn0, omx = b1 ? kmx1 : kmx0;
-    omn = fminf(omn, __shfl_xor_sync(0xffffffffu, b1 ? kmn0 : kmn1, 8));
-    omx = fmaxf(omx, __shfl_xor_sync(0xffffffffu, b1 ? kmx0 : kmx1, 8));
+    float kmn0 = fminf(b2 ? mn[1][0] : mn[0][0], __shfl_xor_sync(0xffffffffu, b2 ? mn[0][0] : mn[1][0], 16));
+    float kmn1 = fminf(b2 ? mn[1][1] : mn[0][1], __shfl_xor_sync(0xffffffffu, b2 ? mn[0][1] : mn[1][1], 16));
+    float kmx0 = fmaxf(b2 ? mx[1][0] : mx[0][0], __shfl_xor_sync(0xffffffffu, b2 ? mx[0][0] : mx[1][0], 16));
+    float kmx1 = fmaxf(b2 ? mx[1][1] : mx[0][1], __shfl_xor_sync(0xffffffffu, b2 ? mx[0][1] : mx[1][1], 16));
+    float omn = fminf(b1 ? kmn1 : kmn0, __shfl_xor_sync(0xffffffffu, b1 ? kmn0 : kmn1, 8));
+    float omx = fmaxf(b1 ? kmx1 : kmx0, __shfl_xor_sync(0xffffffffu, b1 ? kmx0 : kmx1, 8));
     omn = fminf(omn, __shfl_xor_sync(0xffffffffu, omn, 4));
     omx = fmaxf(omx, __shfl_xor_sync(0xffffffffu, omx, 4));
-    const int bits = dst.bits;
-    const float qmax = (float)((1 << bits) - 1);
-    const float s_own = (omx - omn) / qmax;
+    constexpr float kQmax = (float)((1 << BITS) - 1);
+    const float s_own = (omx - omn) / kQmax;
     const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
-    if ((lane & 4) == 0) {  // owner of token 8*b2 + 2t + b1 writes (a, z)
-      float* tokp = dst.tok + slot * (kT * 2);
-      *reinterpret_cast<float2*>(tokp + 2 * (8 * b2 + 2 * t + b1)) = make_float2(s_own * kInvSqrtD, omn * kInvSqrtD);
-    }
-    float mtok[2][2], istok[2][2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int tp = 0; tp < 2; ++tp) {
-        const int src = (h << 4) | (tp << 3) | t;
-        mtok[h][tp] = __shfl_sync(0xffffffffu, omn, src);
-        istok[h][tp] = __shfl_sync(0xffffffffu, is_own, src);
-      }
-
-    // ---- codes (magic-number rounding: byte 0 of the float holds the code) and packing
-    const int tile_bytes = kT * kD * bits / 8;
-    uint8_t* codes = dst.codes + slot * tile_bytes;
+    if ((lane & 4) == 0)
+      *reinterpret_cast<float2*>(p.dst.tok + slot * (kT * 2) + 2 * (8 * b2 + 2 * t + b1)) =
+          make_float2(s_own * kInvSqrtD, omn * kInvSqrtD);
+    uint8_t* codes = p.dst.codes + slot * (kT * kD * BITS / 8);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const f2 m2 = f2{mtok[h][0], mtok[h][1]}, is2 = f2{istok[h][0], istok[h][1]};
+      const f2 m2 = make_float2(__shfl_sync(0xffffffffu, omn, (h << 4) | t),
+                                __shfl_sync(0xffffffffu, omn, (h << 4) | 8 | t));
+      const f2 is2 = make_float2(__shfl_sync(0xffffffffu, is_own, (h << 4) | t),
+                                 __shfl_sync(0xffffffffu, is_own, (h << 4) | 8 | t));
       uint32_t q[2][16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -330,18 +328,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
       for (int tp = 0; tp < 2; ++tp) {
         const int tok = 8 * h + 2 * t + tp;
         const uint32_t* f = q[tp];
-        if (bits == 4) {
+        if constexpr (BITS == 4) {
           *reinterpret_cast<uint2*>(codes + tok * 64 + 8 * g) = make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
-        } else if (bits == 8) {
+        } else if constexpr (BITS == 8) {
           *reinterpret_cast<uint4*>(codes + tok * 128 + 16 * g) =
               make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
                          gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
-        } else if (bits == 2) {
+        } else if constexpr (BITS == 2) {
           uint32_t wd = 0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) wd |= (f[j] & 3u) << (2 * j);
           *reinterpret_cast<uint32_t*>(codes + tok * 32 + 4 * g) = wd;
-        } else {  // 3 bits: low-2-bit plane [T][32 B], then high-bit plane [T][16 B]
+        } else {
           uint32_t lo = 0, hi = 0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
@@ -353,6 +351,27 @@ __global__ void __launch_bounds__(kWarps * 32, 1) quantize_d128_kernel(QuantizeP
   }
 }
 
+FastDiv make_div(uint32_t d) {
+  FastDiv f{d, 0, 0};
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  f.s = s;
+  f.m = (uint32_t)((((1ull << s) - d) << 32) / d + 1);
+  return f;
+}
+
+template <bool F16>
+int launch_bits(const QuantLaunch& q, int bits, int grid, cudaStream_t s) {
+  switch (bits) {
+    case 2: quantize_d128_kernel<F16, 2><<<grid, kThreads, 0, s>>>(q); break;
+    case 3: quantize_d128_kernel<F16, 3><<<grid, kThreads, 0, s>>>(q); break;
+    case 4: quantize_d128_kernel<F16, 4><<<grid, kThreads, 0, s>>>(q); break;
+    case 8: quantize_d128_kernel<F16, 8><<<grid, kThreads, 0, s>>>(q); break;
+    default: return (int)cudaErrorInvalidValue;
+  }
+  return (int)cudaGetLastError();
+}
+
 }  // namespace
 
 int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream) {
@@ -360,15 +379,30 @@ int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t need = (p.total_tiles + kWarps - 1) / kWarps;
-  const int64_t cap = (int64_t)sms;
-  const int grid = (int)(need < cap ? need : cap);
+  const uint32_t per_kind = (uint32_t)(p.total_tiles / p.kinds);
+  const uint32_t ntt = (uint32_t)(p.n_tok / kT);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (f16)
-    quantize_d128_kernel<true><<<grid, kWarps * 32, 0, s>>>(p);
-  else
-    quantize_d128_kernel<false><<<grid, kWarps * 32, 0, s>>>(p);
-  return (int)cudaGetLastError();
+  for (int kind = 0; kind < p.kinds; ++kind) {
+    QuantLaunch q;
+    q.src = static_cast<const uint16_t*>(p.src[kind]);
+    q.dst = p.dst[kind];
+    q.n_tok = p.n_tok;
+    q.num_layers = p.num_layers;
+    q.num_heads = p.num_heads;
+    q.num_pages = p.num_pages;
+    q.iters = p.iters;
+    q.dst_page = p.dst_page;
+    q.err = p.err;
+    q.total = per_kind;
+    q.div_h = make_div((uint32_t)p.num_heads);
+    q.div_ntt = make_div(ntt);
+    const int64_t need = (per_kind + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sms * 2;
+    const int grid = (int)(need < cap ? need : cap);
+    const int e = f16 ? launch_bits<true>(q, q.dst.bits, grid, s) : launch_bits<false>(q, q.dst.bits, grid, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace kvq
