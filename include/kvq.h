@@ -193,6 +193,28 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache_view* cac
                                 float* out, void* workspace, size_t workspace_bytes,
                                 uint32_t* dev_error, void* stream);
 
+/* kvq_decode_attention for callers that cannot allocate device memory when
+ * they decode (a plug-in whose host process owns all device allocations and
+ * has no scratch hook, or a deployment that forbids allocation after
+ * start-up).  The KVarN pages have no counterpart; this is a deployment
+ * variant of the call above with the same arguments except the workspace.
+ *
+ * The split-KV partial results live in one fixed 8 MiB array of this
+ * library (every GPU that loads the library holds it until the process
+ * exits); nothing is allocated.  Shapes that need more than 8 MiB (see
+ * kvq_decode_workspace_bytes with max_seq_len = max_pages_per_seq *
+ * tile_tokens) return KVQ_ERR_WORKSPACE_TOO_SMALL before any launch.
+ * The first call on a device looks up the array's address on that device,
+ * so make that first call before any stream capture.  All calls share the
+ * array and it keeps the last call's contents (nothing in it needs to start
+ * at zero): calls that overlap on the GPU, on any streams of the process,
+ * race and give wrong results; serialise them. */
+kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache_view* cache,
+                                        int32_t layer, const void* q, const int32_t* block_table,
+                                        int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                        int32_t batch, int32_t num_q_heads, float softmax_scale,
+                                        float* out, uint32_t* dev_error, void* stream);
+
 /* Synchronise `stream`, copy the device error word to *host_bits and reset
  * it to 0.  KVQ_ERR_TIMEOUT if the TIMEOUT bit was set, else KVQ_OK (other
  * bits are only reported in *host_bits). */

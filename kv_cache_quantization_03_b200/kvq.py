@@ -39,8 +39,8 @@ KVQ_F16, KVQ_BF16, KVQ_F32 = 0, 1, 2
 
 EXPORTED = (
     "kvq_config_from_string", "kvq_cache_layout", "kvq_quantize_append", "kvq_dequantize",
-    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_read_error", "kvq_status_string",
-    "kvq_version",
+    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_read_error",
+    "kvq_status_string", "kvq_version",
 )
 
 
@@ -72,6 +72,8 @@ _sig = {
     "kvq_decode_attention": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P,
                                             ctypes.c_size_t, _P, _P]),
+    "kvq_decode_attention_noalloc": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
+                                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "kvq_read_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_version": (ctypes.c_char_p, []),
@@ -176,6 +178,18 @@ def kvq_decode_attention(cfg, view, layer, q, block_table, max_pages_per_seq, se
                                   max_pages_per_seq, _ptr(seq_lens), batch, num_q_heads, float(softmax_scale),
                                   _ptr(out), _ptr(workspace), workspace_bytes, _ptr(dev_error), _stream(stream))
     return _check("kvq_decode_attention", st, raise_on_error)
+
+
+def kvq_decode_attention_noalloc(cfg, view, layer, q, block_table, max_pages_per_seq, seq_lens, batch,
+                                 num_q_heads, softmax_scale, out, dev_error, stream=None, raise_on_error=True) -> int:
+    """kvq_decode_attention with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory when they decode; see
+    include/kvq.h for the size limit and the sharing rules."""
+    st = lib.kvq_decode_attention_noalloc(ctypes.byref(cfg), ctypes.byref(view), layer, _ptr(q), _ptr(block_table),
+                                          max_pages_per_seq, _ptr(seq_lens), batch, num_q_heads,
+                                          float(softmax_scale), _ptr(out), _ptr(dev_error), _stream(stream))
+    return _check("kvq_decode_attention_noalloc", st, raise_on_error)
 
 
 def kvq_read_error(dev_error, stream=None):
