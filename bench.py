@@ -178,8 +178,7 @@ def cpu_baseline(w, budget_s=12.0, tokens=4096):
 
 
 def run_reference(args, w):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if rank_env()[1] != 0:       # under torchrun only rank 0 times the CPU oracle
         return
     tokens = 1024
     sample = oracle_sample_inputs(w, tokens)
@@ -212,6 +211,31 @@ def config_dict(w, args):
                 2 * w.num_layers * w.n_tok * w.num_kv_heads * w.head_dim * 2 / 1e9)}
 
 
+# --------------------------------------------------------------------------- ranks
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def shard(w, rank: int):
+    """This rank's shard of a weak-scaling run: the same shape with its own
+    batch of sequences (a seed of its own); ranks share nothing."""
+    return dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (the slowest rank
+    sets the time); a no-op for one rank."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 # --------------------------------------------------------------------------- GPU leg
 def run_gpu(args, w):
     import numpy as np
@@ -221,15 +245,13 @@ def run_gpu(args, w):
     from kv_cache_quantization_03_b200 import kvq, workloads as W
     from kv_cache_quantization_03_b200.cache import QuantizedCache
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    ws = dataclasses.replace(w, seed=w.seed + 7919 * rank)        # this rank's shard
+    ws = shard(w, rank)
 
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                           bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters,
@@ -312,10 +334,7 @@ def run_gpu(args, w):
     if st != kvq.KVQ_OK or bits:
         raise RuntimeError("device error word %#x" % bits)
 
-    t = torch.tensor([elapsed, e2e_s, t_q, t_d], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed, e2e_s, t_q, t_d = t.tolist()
+    elapsed, e2e_s, t_q, t_d = max_over_ranks([elapsed, e2e_s, t_q, t_d], world, device="cuda")
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:

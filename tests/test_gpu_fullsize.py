@@ -1,0 +1,50 @@
+"""Parity at the workloads' full sizes, in the launch configuration bench.py
+times: the whole workload is quantised (one kvq_quantize_append call) and
+decoded (one kvq_decode_attention call) on the GPU; the float64 oracle then
+checks a seeded sample of tiles and of (sequence, kv-head) outputs."""
+import numpy as np
+import pytest
+
+from kv_cache_quantization_03_b200 import workloads as W
+from oracle import kvarn_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_error,  # noqa: E402
+                     compare_quantized, oracle_fraction)
+
+
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill"])
+def test_fullsize_sampled_parity(name):
+    w = W.WORKLOADS[name]
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    rng = np.random.default_rng(1234)
+    n_tiles = w.n_tok // w.tile_tokens
+    tiles = np.sort(rng.choice(n_tiles, size=min(n_tiles, 160), replace=False))
+    layers = sorted(set(rng.integers(0, w.num_layers, size=3).tolist()))
+    heads = sorted(set(rng.integers(0, w.num_kv_heads, size=2).tolist()))
+    flips = total = 0
+    for which in ("k", "v"):
+        bits = w.bits_k if which == "k" else w.bits_v
+        for layer in layers:
+            for head in heads:
+                x = run.input_tiles(which, layer, tiles, head)
+                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters)
+                gpu = run.gpu_tiles(which, layer, tiles, head)
+                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters),
+                                           "%s %s L%d H%d" % (name, which, layer, head), check_rate=False)
+                total += gpu.q.size
+    assert flips <= CODE_FLIP_RATE * total, "%d flips in %d sampled codes" % (flips, total)
+
+    if name == "prefill":          # the prefill workload measures quantise-append only
+        return
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    G = w.group
+    pairs = {(int(rng.integers(0, w.batch)), int(rng.integers(0, w.num_kv_heads))) for _ in range(3)}
+    for b, h in sorted(pairs):
+        err = attention_error(o[b, h * G:(h + 1) * G], dec.oracle(b, h))
+        assert err <= ATTN_TOL, "%s seq %d kv-head %d: %g" % (name, b, h, err)
