@@ -39,11 +39,18 @@ kvq_status check_config(const kvq_config* c) {
   return KVQ_OK;
 }
 
-// Shapes the kernels are built for.
+// Shapes the quantize and dequantize kernels are built for: 16-token tiles,
+// head_dim 128 for K/V caches, 512 for an MLA latent.
 kvq_status check_gpu_shape(const kvq_config* c) {
-  if (c->mla) return KVQ_ERR_UNSUPPORTED;
-  if (c->head_dim != 128 || c->tile_tokens != 16) return KVQ_ERR_UNSUPPORTED;
+  if (c->tile_tokens != 16) return KVQ_ERR_UNSUPPORTED;
+  if (c->head_dim != (c->mla ? 512 : 128)) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
+}
+
+// Shapes the decode kernels are built for (MLA: 512-channel latent, 64 rope).
+kvq_status check_decode_shape(const kvq_config* c) {
+  if (c->mla && c->rope_dim != 64) return KVQ_ERR_UNSUPPORTED;
+  return check_gpu_shape(c);
 }
 
 int64_t slots(const kvq_config* c) { return (int64_t)c->num_layers * c->num_pages * c->num_kv_heads; }
@@ -95,6 +102,27 @@ DecodePlan decode_plan(int64_t pairs, int64_t max_tiles) {
 
 size_t decode_ws_bytes(int64_t pairs, const DecodePlan& d, int head_dim) {
   return (size_t)pairs * d.splits * kMaxGroup * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+// MLA: one CTA pair per (sequence, split), one CTA per SM; about six waves,
+// at least two 32-token steps per split, an even number of tiles per split.
+constexpr int kMlaHeads = 128;
+DecodePlan decode_plan_mla(int64_t batch, int64_t max_tiles) {
+  DecodePlan d{1, 2};
+  if (batch <= 0 || max_tiles <= 0) return d;
+  int64_t splits = (3 * kNumSMs + batch - 1) / batch;
+  const int64_t cap = (max_tiles + 3) / 4;
+  if (splits > cap) splits = cap;
+  if (splits < 1) splits = 1;
+  int64_t tps = (max_tiles + splits - 1) / splits;
+  tps = (tps + 1) / 2 * 2;
+  d.tiles_per_split = (int)tps;
+  d.splits = (int)((max_tiles + tps - 1) / tps);
+  return d;
+}
+
+size_t decode_ws_bytes_mla(int64_t batch, const DecodePlan& d) {
+  return (size_t)batch * d.splits * kMlaHeads * (512 + 2) * sizeof(float);
 }
 
 kvq_status cuda_status(int e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
@@ -175,7 +203,11 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.err = dev_error;
   p.total_tiles = (int64_t)p.kinds * c->num_layers * (n_tok / c->tile_tokens) * c->num_kv_heads;
   if (p.total_tiles >= (int64_t)1 << 31) return KVQ_ERR_UNSUPPORTED;  // tile ids are 32-bit in the kernel
-  return cuda_status(launch_quantize_d128(p, c->in_dtype == KVQ_F16, stream));
+  p.rope_src = (c->mla && c->rope_dim > 0) ? rope_new : nullptr;
+  p.rope_dst = cache->rope;
+  p.rope_dim = c->rope_dim;
+  if (p.rope_src && !aligned16(p.rope_src)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, stream));
 }
 
 kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
@@ -201,7 +233,7 @@ kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int3
   p.out[0] = k_out;
   p.out[1] = v_out;
   p.err = dev_error;
-  return cuda_status(launch_dequantize_d128(p, stream));
+  return cuda_status(launch_dequantize(p, c->head_dim, stream));
 }
 
 kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_t num_q_heads,
@@ -211,7 +243,8 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_
   if (!bytes || batch < 0 || num_q_heads <= 0 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
   const int64_t pairs = (int64_t)batch * c->num_kv_heads;
   const int64_t max_tiles = ((int64_t)max_seq_len + c->tile_tokens - 1) / c->tile_tokens;
-  *bytes = decode_ws_bytes(pairs, decode_plan(pairs, max_tiles), c->head_dim);
+  *bytes = c->mla ? decode_ws_bytes_mla(batch, decode_plan_mla(batch, max_tiles))
+                  : decode_ws_bytes(pairs, decode_plan(pairs, max_tiles), c->head_dim);
   return KVQ_OK;
 }
 
@@ -230,7 +263,38 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
   if (batch > 0 && (!q || !seq_lens || !out || (max_pages_per_seq > 0 && !block_table)))
     return KVQ_ERR_INVALID_ARG;
   if (q && !aligned16(q)) return KVQ_ERR_INVALID_ARG;
-  if ((st = check_gpu_shape(c)) != KVQ_OK) return st;
+  if ((st = check_decode_shape(c)) != KVQ_OK) return st;
+  if (c->mla) {
+    if (num_q_heads > kMlaHeads) return KVQ_ERR_UNSUPPORTED;
+    if (batch == 0) return KVQ_OK;
+    if (batch > 65535) return KVQ_ERR_UNSUPPORTED;
+    const DecodePlan plan = decode_plan_mla(batch, max_pages_per_seq);
+    const size_t need = decode_ws_bytes_mla(batch, plan);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return workspace_bytes < need ? KVQ_ERR_WORKSPACE_TOO_SMALL : KVQ_ERR_INVALID_ARG;
+    MlaDecodeParams m{};
+    m.codes = static_cast<const uint8_t*>(cache->k_codes);
+    m.tok = static_cast<const float*>(cache->k_tok_scale);
+    m.chan = static_cast<const float*>(cache->k_chan_scale);
+    m.rope = static_cast<const uint16_t*>(cache->rope);
+    m.bits = c->bits_k;
+    m.layer = layer;
+    m.num_pages = c->num_pages;
+    m.q = static_cast<const uint16_t*>(q);
+    m.block_table = block_table;
+    m.max_pages = max_pages_per_seq;
+    m.seq_lens = seq_lens;
+    m.batch = batch;
+    m.num_q_heads = num_q_heads;
+    m.scale_log2 = softmax_scale * 1.4426950408889634f;
+    m.out = out;
+    m.part_o = static_cast<float*>(workspace);
+    m.part_ml = m.part_o + (size_t)batch * plan.splits * kMlaHeads * 512;
+    m.splits = plan.splits;
+    m.tiles_per_split = plan.tiles_per_split;
+    m.err = dev_error;
+    return cuda_status(launch_decode_mla(m, stream));
+  }
   const int group = num_q_heads / c->num_kv_heads;
   if (group > kMaxGroup || c->bits_v == 3) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;

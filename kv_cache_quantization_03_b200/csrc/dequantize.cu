@@ -10,9 +10,9 @@
 namespace kvq {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kT = 16;
 
+template <int kD>
 __device__ __forceinline__ uint32_t read_code(const uint8_t* codes, int bits, int tok, int ch) {
   if (bits == 3) {
     const uint32_t lo = (codes[tok * (kD / 4) + ch / 4] >> (2 * (ch % 4))) & 3u;
@@ -23,7 +23,8 @@ __device__ __forceinline__ uint32_t read_code(const uint8_t* codes, int bits, in
   return (codes[bit >> 3] >> (bit & 7)) & ((1u << bits) - 1u);
 }
 
-__global__ void __launch_bounds__(kD) dequantize_d128_kernel(DequantParams p) {
+template <int kD>
+__global__ void __launch_bounds__(kD) dequantize_kernel(DequantParams p) {
   __shared__ float tile[kT][kD];
   const int ch = threadIdx.x;
   int64_t idx = blockIdx.x;
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(kD) dequantize_d128_kernel(DequantParams p) {
   const float* tok = src.tok + slot * kT * 2;
   const float c = src.chan[slot * kD + ch];
   for (int r = 0; r < kT; ++r)
-    tile[r][ch] = fmaf(tok[2 * r], (float)read_code(codes, src.bits, r, ch), tok[2 * r + 1]) * c;
+    tile[r][ch] = fmaf(tok[2 * r], (float)read_code<kD>(codes, src.bits, r, ch), tok[2 * r + 1]) * c;
   __syncthreads();
   if (p.unrotate) {
     for (int r = 0; r < kT; ++r) {
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(kD) dequantize_d128_kernel(DequantParams p) {
         tile[r][ch] = (ch & s) ? (x - y) : (x + y);
         __syncthreads();
       }
-      tile[r][ch] *= 0.08838834764831845f;
+      tile[r][ch] *= rsqrtf((float)kD);
     }
     __syncthreads();
   }
@@ -62,10 +63,16 @@ __global__ void __launch_bounds__(kD) dequantize_d128_kernel(DequantParams p) {
 
 }  // namespace
 
-int launch_dequantize_d128(const DequantParams& p, void* stream) {
+int launch_dequantize(const DequantParams& p, int head_dim, void* stream) {
   const int64_t blocks = p.n_pages * p.kinds * p.num_heads;
   if (blocks == 0) return cudaSuccess;
-  dequantize_d128_kernel<<<(unsigned)blocks, kD, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128)
+    dequantize_kernel<128><<<(unsigned)blocks, 128, 0, s>>>(p);
+  else if (head_dim == 512)
+    dequantize_kernel<512><<<(unsigned)blocks, 512, 0, s>>>(p);
+  else
+    return (int)cudaErrorInvalidValue;
   return (int)cudaGetLastError();
 }
 

@@ -33,6 +33,9 @@ struct QuantizeParams {
   const int32_t* dst_page;
   uint32_t* err;
   int64_t total_tiles;  // kinds * layers * (n_tok / T) * heads
+  const void* rope_src; // MLA rope keys [layer][n_tok][rope_dim] bf16, or null
+  void* rope_dst;       // cache rope array [layer][page][T][rope_dim]
+  int rope_dim;
 };
 
 struct DequantParams {
@@ -69,9 +72,33 @@ struct DecodeParams {
   uint32_t* err;
 };
 
+struct MlaDecodeParams {
+  const uint8_t* codes;         // latent codes [layer][page][T*512*bits/8]
+  const float* tok;             // [layer][page][T][2]
+  const float* chan;            // [layer][page][512]
+  const uint16_t* rope;         // bf16 [layer][page][T][64]
+  int bits;
+  int layer;
+  int64_t num_pages;
+  const uint16_t* q;            // bf16 [B][Hq][576]
+  const int32_t* block_table;   // [B][max_pages]
+  int max_pages;
+  const int32_t* seq_lens;      // [B]
+  int batch;
+  int num_q_heads;              // <= 128
+  float scale_log2;
+  float* out;                   // [B][Hq][512]
+  float* part_o;                // [B][splits][128][512]
+  float* part_ml;               // [B][splits][128][2]
+  int splits;
+  int tiles_per_split;          // even
+  uint32_t* err;
+};
+
 // Launchers (defined in the .cu files); return a cudaError_t value.
-int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream);
-int launch_dequantize_d128(const DequantParams& p, void* stream);
+int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* stream);
+int launch_dequantize(const DequantParams& p, int head_dim, void* stream);
 int launch_decode_d128(const DecodeParams& p, void* stream);
+int launch_decode_mla(const MlaDecodeParams& p, void* stream);
 
 }  // namespace kvq

@@ -1,4 +1,5 @@
-// Quantize-append for head_dim 128, 16-token tiles (sm_100a).
+// Quantize-append for head_dim 128 (GQA) and 512 (MLA latent), 16-token tiles
+// (sm_100a).
 //
 // Computes, per tile of 16 tokens x 128 channels of one (layer, kv-head,
 // K-or-V), the KVarN pipeline (KVarN project page on open-radar, Key
@@ -6,9 +7,14 @@
 // along head_dim, Sinkhorn-like row/column second-moment normalisation,
 // per-token asymmetric round-to-nearest, packing into the tile's cache page.
 //
-// One warp owns one tile.  Lane (g = lane/4, t = lane%4) ends up holding the
-// rotated values of tokens {2t, 2t+1, 2t+8, 2t+9} and channels 16g..16g+15
-// (register pairs hold the two tokens 8h + 2t, 8h + 2t + 1 of one channel).
+// One warp owns one 128-channel block of a tile (head_dim 128: the whole
+// tile; 512: four warps share a tile).  Lane (g = lane/4, t = lane%4) ends up
+// holding the rotated values of tokens {2t, 2t+1, 2t+8, 2t+9} and channels
+// 16g..16g+15 of its block (register pairs hold the two tokens 8h + 2t,
+// 8h + 2t + 1 of one channel).  For 512 channels, H_512 = H_4 (x) H_128: each
+// warp applies H_128 to its block, then the four blocks are combined with the
+// signs of H_4 through shared memory; row sums and row min/max are combined
+// across the four warps the same way, column sums stay within a warp.
 //
 // Rotation: the Sylvester matrix factors over the 7 bits of the channel
 // index, H_128 = (x) over bits of H_2.  Bits 3..6 are contracted with one
@@ -37,12 +43,11 @@
 namespace kvq {
 namespace {
 
-constexpr int kD = 128;
+constexpr int kBlk = 128;                  // channels per warp (one 128-channel block of a tile)
 constexpr int kT = 16;
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer (ties to even)
-constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 
 // Channel bits carried by the MMA contraction index k = 2t + j0 + 8*j1
 // (t = lane%4 of the B fragment): bits 3,4 <- t, bit 5 <- j0, bit 6 <- j1.
@@ -98,7 +103,7 @@ struct FastDiv {
 __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) { return (__umulhi(n, f.m) + n) >> f.s; }
 
 struct QuantLaunch {
-  const uint16_t* src;   // [layer][n_tok][H][d]
+  const uint16_t* src;   // [layer][n_tok][H][D]
   CacheArrays dst;
   int64_t n_tok;
   int num_layers, num_heads;
@@ -108,17 +113,28 @@ struct QuantLaunch {
   uint32_t* err;
   uint32_t total;        // layers * (n_tok / T) * heads
   FastDiv div_h, div_ntt;
+  const uint16_t* rope_src;  // MLA: [layer][n_tok][rope_dim] bf16, copied into rope_dst; else null
+  uint16_t* rope_dst;        // [layer][page][T][rope_dim]
+  int rope_dim;
 };
 
-__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLaunch& p, uint32_t tile, int g, int t,
-                                          int32_t& page) {
+// Shared memory of one tile whose 512 channels are split over four warps.
+struct TileShare {
+  float2 x[4][32][32];   // per block, per register pair, per lane: values for the H_4 combination
+  float row[2][4][kT];   // row partial sums, double-buffered by round parity
+  float2 mm[4][kT];      // per block and token: (min, max)
+};
+
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLaunch& p, uint32_t tile, int blk, int g,
+                                          int t, int32_t& page) {
   const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
   const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
   page = __ldg(p.dst_page + tt);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint16_t* row =
-        p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * kD + 8 * t;
+    const uint16_t* row = p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * D +
+                          kBlk * blk + 8 * t;
 #pragma unroll
     for (int l = 0; l < 4; ++l) {
       const uint4 v = ldg_nc_v4(row + 32 * l);
@@ -127,26 +143,37 @@ __device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLau
   }
 }
 
-template <bool F16, int BITS>
-__global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch p) {
+template <int W>
+__device__ __forceinline__ void tile_sync() {
+  if constexpr (W > 1) __syncthreads();  // one tile per CTA when its blocks span warps
+}
+
+template <bool F16, int BITS, int D>
+__global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(QuantLaunch p) {
+  constexpr int W = D / kBlk;     // warps per tile
+  constexpr int TPC = kWarps / W; // tiles per CTA
   __shared__ WarpScratch scratch[kWarps];
+  __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int warp = threadIdx.x >> 5, blk = warp % W, slot_id = warp / W;
   const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
-  WarpScratch& sc = scratch[threadIdx.x >> 5];
+  WarpScratch& sc = scratch[warp];
+  TileShare& sh = share[0];
   uint32_t afrag[4];
   afrag[0] = sign_pair<F16>(g, 2 * t);
   afrag[1] = sign_pair<F16>(g + 8, 2 * t);
   afrag[2] = sign_pair<F16>(g, 2 * t + 8);
   afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8);
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint32_t stride = gridDim.x * kWarps;
-  uint32_t tile = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (tile >= p.total) return;
+  const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.044194173824159216f;
+  const uint32_t stride = gridDim.x * TPC;
+  uint32_t tile = blockIdx.x * TPC + slot_id;
+  if (tile >= p.total) return;  // every warp of a tile leaves together
   uint32_t L[2][4][4];
   int32_t page;
-  load_tile(L, p, tile, g, t, page);
+  load_tile<D>(L, p, tile, blk, g, t, page);
   for (; tile < p.total; tile += stride) {
-    f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b
+    f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b of the block
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -160,10 +187,20 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
       }
     const int32_t cur_page = page;
     const uint32_t cur = tile;
-    if (tile + stride < p.total) load_tile(L, p, tile + stride, g, t, page);
-    if (cur_page < 0 || cur_page >= p.num_pages) {
-      if (lane == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+    const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
+    const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
+    if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
+    if (cur_page < 0 || cur_page >= p.num_pages) {  // same decision in every warp of the tile
+      if (lane == 0 && blk == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       continue;
+    }
+    const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;
+    if (p.rope_src && blk == 0) {  // MLA: the tile's rope rows go to the page unquantised
+      const int rd = p.rope_dim;
+      const uint16_t* rs = p.rope_src + ((size_t)layer * p.n_tok + (size_t)tt * kT) * rd;
+      uint16_t* rdst = p.rope_dst + ((size_t)layer * p.num_pages + cur_page) * kT * rd;
+      for (int i = lane * 8; i < kT * rd; i += 32 * 8)
+        *reinterpret_cast<uint4*>(rdst + i) = *reinterpret_cast<const uint4*>(rs + i);
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -178,6 +215,21 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
             P[h][m3][b] = add2(x, y);
             P[h][m3][b + s] = sub2(x, y);
           }
+    if constexpr (W > 1) {  // channel bits 7, 8: H_4 across the four blocks of the tile
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sh.x[blk][i][lane] = P[i >> 4][(i >> 3) & 1][i & 7];
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        f2 acc = sh.x[0][i][lane];
+#pragma unroll
+        for (int k = 1; k < W; ++k) {
+          const f2 y = sh.x[k][i][lane];
+          acc = (__popc(blk & k) & 1) ? sub2(acc, y) : add2(acc, y);
+        }
+        P[i >> 4][(i >> 3) & 1][i & 7] = acc;
+      }
+    }
     // squares paired along channels: A[h][tp][q] = channels 2q, 2q+1 of token 8h + 2t + tp
     f2 A[2][2][8];
 #pragma unroll
@@ -213,8 +265,16 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
       k0 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][0] : R[1][0], 16);
       k1 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][1] : R[1][1], 16);
       float rk = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 8);
-      rk += __shfl_xor_sync(0xffffffffu, rk, 4);
-      const float vn = (float)kD * rcp_nr(rk);
+      rk += __shfl_xor_sync(0xffffffffu, rk, 4);  // token 8*b2 + 2t + b1, this block's channels
+      if constexpr (W > 1) {
+        const int tok = 8 * b2 + 2 * t + b1;
+        if ((lane & 4) == 0) sh.row[it & 1][blk][tok] = rk;
+        __syncthreads();
+        rk = sh.row[it & 1][0][tok];
+#pragma unroll
+        for (int k = 1; k < W; ++k) rk += sh.row[it & 1][k][tok];
+      }
+      const float vn = (float)D * rcp_nr(rk);
       v_own = rk > 0.f ? vn : v_own;
       float v[2][2];
 #pragma unroll
@@ -252,9 +312,6 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
       }
       __syncwarp();
     }
-    const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
-    const uint32_t layer = fdiv(r1, p.div_ntt);
-    const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;
     {
       const bool norm = p.iters > 0;
       const float ct[4] = {c01.x, c01.y, c23.x, c23.y};
@@ -267,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
         ic[i] = ok ? y : 1.f;
         cv[i] = ok ? x * y : 1.f;
       }
-      *reinterpret_cast<float4*>(p.dst.chan + slot * kD + 16 * g + 4 * t) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+      *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
+          make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
       __syncwarp();
@@ -304,13 +362,23 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
     float omx = fmaxf(b1 ? kmx1 : kmx0, __shfl_xor_sync(0xffffffffu, b1 ? kmx0 : kmx1, 8));
     omn = fminf(omn, __shfl_xor_sync(0xffffffffu, omn, 4));
     omx = fmaxf(omx, __shfl_xor_sync(0xffffffffu, omx, 4));
+    if constexpr (W > 1) {
+      const int tok = 8 * b2 + 2 * t + b1;
+      if ((lane & 4) == 0) sh.mm[blk][tok] = make_float2(omn, omx);
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < W; ++k) {
+        const float2 x = sh.mm[k][tok];
+        omn = fminf(omn, x.x), omx = fmaxf(omx, x.y);
+      }
+    }
     constexpr float kQmax = (float)((1 << BITS) - 1);
     const float s_own = (omx - omn) / kQmax;
     const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
-    if ((lane & 4) == 0)
+    if ((lane & 4) == 0 && blk == 0)
       *reinterpret_cast<float2*>(p.dst.tok + slot * (kT * 2) + 2 * (8 * b2 + 2 * t + b1)) =
-          make_float2(s_own * kInvSqrtD, omn * kInvSqrtD);
-    uint8_t* codes = p.dst.codes + slot * (kT * kD * BITS / 8);
+          make_float2(s_own * inv_sqrt_d, omn * inv_sqrt_d);
+    uint8_t* codes = p.dst.codes + slot * (kT * D * BITS / 8);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const f2 m2 = make_float2(__shfl_sync(0xffffffffu, omn, (h << 4) | t),
@@ -328,26 +396,29 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_d128_kernel(QuantLaunch 
       for (int tp = 0; tp < 2; ++tp) {
         const int tok = 8 * h + 2 * t + tp;
         const uint32_t* f = q[tp];
+        constexpr int row_bytes = D * BITS / 8, seg = kBlk * BITS / 8;
         if constexpr (BITS == 4) {
-          *reinterpret_cast<uint2*>(codes + tok * 64 + 8 * g) = make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
+          *reinterpret_cast<uint2*>(codes + tok * row_bytes + seg * blk + 8 * g) =
+              make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
         } else if constexpr (BITS == 8) {
-          *reinterpret_cast<uint4*>(codes + tok * 128 + 16 * g) =
+          *reinterpret_cast<uint4*>(codes + tok * row_bytes + seg * blk + 16 * g) =
               make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
                          gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
         } else if constexpr (BITS == 2) {
           uint32_t wd = 0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) wd |= (f[j] & 3u) << (2 * j);
-          *reinterpret_cast<uint32_t*>(codes + tok * 32 + 4 * g) = wd;
-        } else {
+          *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = wd;
+        } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
           uint32_t lo = 0, hi = 0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
-          *reinterpret_cast<uint32_t*>(codes + tok * 32 + 4 * g) = lo;
-          *reinterpret_cast<uint16_t*>(codes + kT * 32 + tok * 16 + 2 * g) = (uint16_t)hi;
+          *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
+          *reinterpret_cast<uint16_t*>(codes + kT * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) = (uint16_t)hi;
         }
       }
     }
+    tile_sync<W>();  // shared tile buffers are reused by the next tile
   }
 }
 
@@ -360,13 +431,13 @@ FastDiv make_div(uint32_t d) {
   return f;
 }
 
-template <bool F16>
+template <bool F16, int D>
 int launch_bits(const QuantLaunch& q, int bits, int grid, cudaStream_t s) {
   switch (bits) {
-    case 2: quantize_d128_kernel<F16, 2><<<grid, kThreads, 0, s>>>(q); break;
-    case 3: quantize_d128_kernel<F16, 3><<<grid, kThreads, 0, s>>>(q); break;
-    case 4: quantize_d128_kernel<F16, 4><<<grid, kThreads, 0, s>>>(q); break;
-    case 8: quantize_d128_kernel<F16, 8><<<grid, kThreads, 0, s>>>(q); break;
+    case 2: quantize_kernel<F16, 2, D><<<grid, kThreads, 0, s>>>(q); break;
+    case 3: quantize_kernel<F16, 3, D><<<grid, kThreads, 0, s>>>(q); break;
+    case 4: quantize_kernel<F16, 4, D><<<grid, kThreads, 0, s>>>(q); break;
+    case 8: quantize_kernel<F16, 8, D><<<grid, kThreads, 0, s>>>(q); break;
     default: return (int)cudaErrorInvalidValue;
   }
   return (int)cudaGetLastError();
@@ -374,7 +445,7 @@ int launch_bits(const QuantLaunch& q, int bits, int grid, cudaStream_t s) {
 
 }  // namespace
 
-int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream) {
+int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* stream) {
   if (p.total_tiles == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -396,10 +467,20 @@ int launch_quantize_d128(const QuantizeParams& p, bool f16, void* stream) {
     q.total = per_kind;
     q.div_h = make_div((uint32_t)p.num_heads);
     q.div_ntt = make_div(ntt);
-    const int64_t need = (per_kind + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)sms * 2;
+    q.rope_src = kind == 0 ? static_cast<const uint16_t*>(p.rope_src) : nullptr;
+    q.rope_dst = static_cast<uint16_t*>(p.rope_dst);
+    q.rope_dim = p.rope_dim;
+    const int tpc = head_dim == 128 ? kWarps : kWarps / (head_dim / kBlk);
+    const int64_t need = (per_kind + tpc - 1) / tpc;
+    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 2 : 4);
     const int grid = (int)(need < cap ? need : cap);
-    const int e = f16 ? launch_bits<true>(q, q.dst.bits, grid, s) : launch_bits<false>(q, q.dst.bits, grid, s);
+    int e;
+    if (head_dim == 128)
+      e = f16 ? launch_bits<true, 128>(q, q.dst.bits, grid, s) : launch_bits<false, 128>(q, q.dst.bits, grid, s);
+    else if (head_dim == 512)
+      e = f16 ? launch_bits<true, 512>(q, q.dst.bits, grid, s) : launch_bits<false, 512>(q, q.dst.bits, grid, s);
+    else
+      e = (int)cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

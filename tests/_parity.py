@@ -48,13 +48,16 @@ class QuantRun:
         self.pages = W.page_assignment(w) if pages is None else np.asarray(pages, dtype=np.int32)
         self.k = torch.from_numpy(self.k_bits.view(np.int16)).cuda()
         self.v = None if w.mla else torch.from_numpy(self.v_bits.view(np.int16)).cuda()
+        self.rope_bits = W.rope_inputs(w) if (w.mla and w.rope_dim) else None
+        self.rope = None if self.rope_bits is None else torch.from_numpy(self.rope_bits.view(np.int16)).cuda()
         self.dst = torch.from_numpy(self.pages).cuda()
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
         if quantize:
             self.quantize()
 
     def quantize(self):
-        kvq.kvq_quantize_append(self.cfg, self.cache.view, self.k, self.v, None, self.w.n_tok, self.dst, self.err)
+        kvq.kvq_quantize_append(self.cfg, self.cache.view, self.k, self.v, self.rope, self.w.n_tok, self.dst,
+                                self.err)
         torch.cuda.synchronize()
 
     def error_bits(self):
@@ -166,6 +169,16 @@ class DecodeRun:
         w = self.run.w
         G = self.hq // w.num_kv_heads
         n = int(self.sl[b]) // w.tile_tokens
+        if w.mla:
+            q = W.half_bits_to_f64(self.q_bits[b], "bf16")
+            if n == 0:
+                return np.zeros((G, w.head_dim))
+            pages = self.bt[b, :n]
+            lat = gpu_pages(self.run, "k", 0, pages, 0)
+            rope_all = self.run.cache["rope"].view(w.num_layers, -1, w.tile_tokens, w.rope_dim)
+            pg = torch.as_tensor(np.asarray(pages, dtype=np.int64)).cuda()
+            rope = rope_all[0, pg].float().cpu().numpy().astype(np.float64).reshape(-1, w.rope_dim)
+            return O.mla_decode_attention(q, lat, rope, w.softmax_scale)
         q = W.half_bits_to_f64(self.q_bits[b, kvh * G:(kvh + 1) * G], "bf16")
         if n == 0:
             return np.zeros((G, w.head_dim))

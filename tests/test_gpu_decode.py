@@ -46,6 +46,26 @@ def test_decode_parity_small(name, kw):
     _check(dec, o)
 
 
+@pytest.mark.parametrize("kw", [dict(batch=2, seq_len=512), dict(batch=3, seq_len=304)])
+def test_mla_decode_parity(kw):
+    w = W.WORKLOADS["mla"].scaled(**kw)
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    _check(dec, o)
+
+
+def test_mla_decode_fewer_heads_ragged():
+    w = dataclasses.replace(W.WORKLOADS["mla"].scaled(batch=3, seq_len=256), num_q_heads=16)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=[256, 48, 0])
+    o = dec()
+    assert run.error_bits() == 0
+    _check(dec, o)
+
+
 def test_decode_ragged_and_empty_sequences():
     w = W.WORKLOADS["gqa"].scaled(batch=4, seq_len=1024)
     run = QuantRun(w)

@@ -14,7 +14,7 @@ from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_er
                      compare_quantized, oracle_fraction)
 
 
-@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill"])
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla"])
 def test_fullsize_sampled_parity(name):
     w = W.WORKLOADS[name]
     run = QuantRun(w)
@@ -25,7 +25,7 @@ def test_fullsize_sampled_parity(name):
     layers = sorted(set(rng.integers(0, w.num_layers, size=3).tolist()))
     heads = sorted(set(rng.integers(0, w.num_kv_heads, size=2).tolist()))
     flips = total = 0
-    for which in ("k", "v"):
+    for which in (("k",) if w.mla else ("k", "v")):
         bits = w.bits_k if which == "k" else w.bits_v
         for layer in layers:
             for head in heads:

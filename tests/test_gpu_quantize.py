@@ -15,6 +15,7 @@ SMALL = {
     "gqa": dict(batch=2, seq_len=512),
     "long": dict(batch=1, seq_len=1024),
     "prefill": dict(seq_len=256, num_layers=3),
+    "mla": dict(batch=2, seq_len=256),
 }
 
 
@@ -107,6 +108,16 @@ def test_quantize_bad_page_sets_error_and_skips_tile():
     _check_all(run, tiles=[0, 2, 3])
 
 
+def test_mla_rope_rows_copied_to_their_pages():
+    w = W.WORKLOADS["mla"].scaled(batch=2, seq_len=128)
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    rope = run.cache["rope"].view(w.num_layers, w.num_pages, 16, w.rope_dim).cpu().view(torch.int16).numpy()
+    src = run.rope_bits.view(np.int16).reshape(w.num_layers, -1, 16, w.rope_dim)
+    for tile, page in enumerate(run.pages):
+        assert np.array_equal(rope[0, page], src[0, tile])
+
+
 def test_quantize_deterministic():
     w = W.WORKLOADS["gqa"].scaled(batch=1, seq_len=512)
     run = QuantRun(w)
@@ -116,17 +127,19 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-def test_dequantize_matches_oracle_on_stored_codes():
+@pytest.mark.parametrize("name", ["long", "mla"])
+def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
-    w = W.WORKLOADS["long"].scaled(batch=1, seq_len=256)
+    w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
     run = QuantRun(w)
     pages = torch.arange(w.num_pages, dtype=torch.int32, device="cuda")
     for unrot in (0, 1):
-        ko = torch.empty(w.num_pages, w.num_kv_heads, 16, 128, device="cuda")
+        ko = torch.empty(w.num_pages, w.num_kv_heads, 16, w.head_dim, device="cuda")
         vo = torch.empty_like(ko)
-        kvq.kvq_dequantize(run.cfg, run.cache.view, 0, pages, w.num_pages, unrot, ko, vo, run.err)
+        kvq.kvq_dequantize(run.cfg, run.cache.view, 0, pages, w.num_pages, unrot, ko, None if w.mla else vo,
+                           run.err)
         torch.cuda.synchronize()
-        for which, out in (("k", ko), ("v", vo)):
+        for which, out in ((("k", ko),) if w.mla else (("k", ko), ("v", vo))):
             for h in range(w.num_kv_heads):
                 inv = np.argsort(run.pages)                      # page -> tile
                 g = run.gpu_tiles(which, 0, inv, h)              # tiles in page order
