@@ -51,9 +51,26 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def load_tensor_peak():
+    """Dense f16/bf16 tensor peak for a kernel timed inside a long step (sustained)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops_sustained"]), "measured sustained"
+    except Exception:
+        return 1400.0, "fallback sustained"
+
+
 def algorithmic_bytes(w):
     """(quantize bytes, decode bytes) one step must move, from the cache format."""
     T, d, H = w.tile_tokens, w.head_dim, w.num_kv_heads
+    if w.mla:
+        lat_row = d * w.bits_k / 8 + 8 + d * 4 / T          # codes + (a, z) + channel-scale share
+        rope_row = w.rope_dim * 2
+        tokens = w.num_layers * w.n_tok
+        q_bytes = tokens * (d * 2 + rope_row) + tokens * (lat_row + rope_row)
+        dec_bytes = w.batch * w.seq_len * (lat_row + rope_row) + w.batch * w.num_q_heads * ((d + w.rope_dim) * 2 + d * 4)
+        return q_bytes, dec_bytes
     rows = w.num_layers * w.n_tok * H
     per_row_in = d * 2
     def cache_row(bits):                       # codes + (a, z) + c share of one row
@@ -135,6 +152,9 @@ def oracle_sample_step(w, sample):
     from kv_cache_quantization_03_b200 import workloads as W
     xk, xv, q = sample
     kt = O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters)
+    if w.mla:   # xv holds the rope keys
+        O.mla_decode_attention(q, kt, xv, w.softmax_scale)
+        return xk.shape[0] * xk.shape[1]
     vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters)
     O.decode_attention(q, kt, vt, w.softmax_scale)
     return xk.shape[0] * xk.shape[1] / w.num_kv_heads
@@ -145,8 +165,13 @@ def oracle_sample_inputs(w, tokens):
     from kv_cache_quantization_03_b200 import workloads as W
     sub = slice(0, max(tokens, W.CHUNK_TOKENS))
     xk = W.half_bits_to_f64(W.kv_inputs(w, "k", sub)[0, :tokens, 0], w.in_dtype)
-    xv = W.half_bits_to_f64(W.kv_inputs(w, "v", sub)[0, :tokens, 0], w.in_dtype)
     xk = xk.reshape(-1, w.tile_tokens, w.head_dim)
+    if w.mla:
+        small = w.scaled(batch=1, seq_len=tokens)
+        rope = W.half_bits_to_f64(W.rope_inputs(small)[0], "bf16")
+        q = W.half_bits_to_f64(W.queries(w)[0], "bf16")
+        return xk, rope, q
+    xv = W.half_bits_to_f64(W.kv_inputs(w, "v", sub)[0, :tokens, 0], w.in_dtype)
     xv = xv.reshape(-1, w.tile_tokens, w.head_dim)
     q = W.half_bits_to_f64(W.queries(w)[0, :w.group], "bf16")
     return xk, xv, q
@@ -254,18 +279,20 @@ def run_gpu(args, w):
     ws = shard(w, rank)
 
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
-                          bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters,
-                          num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype)
+                          bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
+                          rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype)
     cache = QuantizedCache(cfg)
-    kb, vb = W.kv_inputs(ws, "k"), W.kv_inputs(ws, "v")
     qb, pages = W.queries(ws), W.page_assignment(ws)
     bt, sl = W.block_table(ws), W.seq_lens(ws)
-    host = {"k": torch.from_numpy(kb.view(np.int16)).pin_memory(),
-            "v": torch.from_numpy(vb.view(np.int16)).pin_memory(),
-            "q": torch.from_numpy(qb.view(np.int16)).pin_memory(),
-            "dst": torch.from_numpy(pages).pin_memory(),
-            "bt": torch.from_numpy(np.ascontiguousarray(bt)).pin_memory(),
-            "sl": torch.from_numpy(sl).pin_memory()}
+    host = {"k": torch.from_numpy(W.kv_inputs(ws, "k").view(np.int16)).pin_memory()}
+    if w.mla:
+        host["rope"] = torch.from_numpy(W.rope_inputs(ws).view(np.int16)).pin_memory()
+    else:
+        host["v"] = torch.from_numpy(W.kv_inputs(ws, "v").view(np.int16)).pin_memory()
+    host.update({"q": torch.from_numpy(qb.view(np.int16)).pin_memory(),
+                 "dst": torch.from_numpy(pages).pin_memory(),
+                 "bt": torch.from_numpy(np.ascontiguousarray(bt)).pin_memory(),
+                 "sl": torch.from_numpy(sl).pin_memory()})
     dev = {k: v.cuda() for k, v in host.items()}
     out = torch.empty(w.batch, w.num_q_heads, w.head_dim, device="cuda")
     out_host = torch.empty_like(out, device="cpu").pin_memory()
@@ -276,7 +303,8 @@ def run_gpu(args, w):
     s_ptr = stream.cuda_stream
 
     def quantize():
-        kvq.kvq_quantize_append(cfg, cache.view, dev["k"], dev["v"], None, w.n_tok, dev["dst"], err, s_ptr)
+        kvq.kvq_quantize_append(cfg, cache.view, dev["k"], dev.get("v"), dev.get("rope"), w.n_tok, dev["dst"], err,
+                                s_ptr)
 
     def decode():
         kvq.kvq_decode_attention(cfg, cache.view, 0, dev["q"], dev["bt"], w.tiles_per_seq, dev["sl"], w.batch,
@@ -345,7 +373,7 @@ def run_gpu(args, w):
     qb_bytes, db_bytes = algorithmic_bytes(w)
     q_gbs = qb_bytes / t_q / 1e9
     d_gbs = db_bytes / t_d / 1e9
-    traffic = traffic_from_profile("quantize.cu", "quantize_d128_gqa.md")
+    traffic = traffic_from_profile("quantize.cu", "quantize_d128_gqa.md") if not w.mla else None
     line = {
         "metric": METRIC, "value": tokens * K / elapsed, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / K, "higher_is_better": True, "scaling": "weak",
@@ -359,9 +387,20 @@ def run_gpu(args, w):
         "quantize": {"rows_per_s": w.num_layers * w.n_tok * w.num_kv_heads * 2 / t_q, "gbs": q_gbs,
                      "frac_of_8tbs": q_gbs / 8000.0, "us": 1e6 * t_q},
         "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * K,  # quantize K, quantize V, decode, combine
+        "gpu_launches": (3 if w.mla else 4) * K,  # quantize (K[, V]), decode, combine
         "clocks": clk.summary(),
     }
+    if w.mla:   # decode attention is a dense contraction over 128 heads: tensor-bound
+        flops = 2.0 * w.batch * w.seq_len * w.num_q_heads * (w.head_dim + w.rope_dim + w.head_dim)
+        tf = flops / t_d / 1e12
+        tpeak = load_tensor_peak()
+        line["decode_attn"].update({"tflops": tf, "frac_of_tensor_peak": tf / tpeak[0], "tensor_peak": tpeak[0],
+                                    "tensor_peak_source": tpeak[1], "flops": flops})
+        if t_d >= t_q:
+            line["roofline"] = {"kernel": "decode_mla (tcgen05)", "bound": "tensor", "achieved": tf,
+                                "peak": tpeak[0], "unit": "TFLOP/s", "frac": tf / tpeak[0],
+                                "peak_source": tpeak[1] + " bf16 dense (f16 same rate)", "traffic": None,
+                                "algorithmic_flops": flops}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))
@@ -383,8 +422,8 @@ def main():
     if args.batch or args.seq_len:
         w = w.scaled(batch=args.batch, seq_len=args.seq_len, name="%s-b%d-l%d" % (
             w.name, args.batch or w.batch, args.seq_len or w.seq_len))
-    if w.mla or w.num_q_heads // w.num_kv_heads > 8:
-        raise SystemExit("bench covers the GQA workloads (rt1k, gqa, long, prefill)")
+    if not w.mla and w.num_q_heads // w.num_kv_heads > 8:
+        raise SystemExit("GQA decode covers query groups of up to 8 heads")
     if args.impl == "reference":
         run_reference(args, w)
     else:

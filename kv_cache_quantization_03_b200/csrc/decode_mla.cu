@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   const uint32_t peer = rank ^ 1u;
   for (int c = 0; c < nchunks; ++c) {
     // a. raw chunk arrived
-    ok &= mbar_wait_bounded(&bar_stage[c & 1], (uint32_t)(c >> 1) & 1u, kWaitLimit);
+    ok &= mbar_wait_bounded(&bar_stage[c & 1], (uint32_t)(c >> 1) & 1u, ok ? kWaitLimit : 0u);
     // b. dequantise into Kb[c & 1]: thread -> token tid / 8, 32 channels of this half
     {
       const uint8_t* st = smem + kOffSt + (c & 1) * kStageBytes;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
     // d. scores: own partial to the peer, full scores, online softmax, P
     float sc[32];
     if (warp < 4) {
-      ok &= mbar_wait_bounded(bar_s, (uint32_t)c & 1u, kWaitLimit);
+      ok &= mbar_wait_bounded(bar_s, (uint32_t)c & 1u, ok ? kWaitLimit : 0u);
       tc_fence_after();
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kHalf, sc);
       const uint32_t dst = peer_addr(s_base + kOffSx + (c & 1) * kSxBytes + tid * 128, peer);
@@ -315,28 +315,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
     cluster_sync();
     if (warp < 4) {
       const float* sx = reinterpret_cast<const float*>(smem + kOffSx + (c & 1) * kSxBytes) + tid * 32;
+      bool tv[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int lt = 2 * c + j;
+        tv[j] = lt < ntl && spg[lt] >= 0 && spg[lt] < p.num_pages;
+      }
       float mx = kNegBig;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int lt = 2 * c + (i >> 4);
-        const bool valid = lt < ntl && spg[lt] >= 0 && spg[lt] < p.num_pages;
-        sc[i] = valid ? sc[i] + sx[i] : kNegBig;
+        sc[i] = tv[i >> 4] ? sc[i] + sx[i] : kNegBig;
         mx = fmaxf(mx, sc[i]);
       }
-      if (c > 0) ok &= mbar_wait_bounded(bar_pv, (uint32_t)(c - 1) & 1u, kWaitLimit);  // P and O are free
+      if (c > 0) ok &= mbar_wait_bounded(bar_pv, (uint32_t)(c - 1) & 1u, ok ? kWaitLimit : 0u);  // P and O are free
       tc_fence_after();
-      if (mx > m_run + 8.f) {       // rescale (lazily): the accumulated output and sum follow the new max
-        const float alpha = ex2f(m_run - mx);
-        if (c > 0 && l_run > 0.f) {
-          for (int c0 = 0; c0 < kHalf; c0 += 32) {
-            float o[32];
-            const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + c0;
-            tmem_ld32(ta, o);
+      // lazy rescale: a head whose max grew by more than 2^8 moves its running max;
+      // the TMEM accesses are warp-wide, so the whole warp joins (factor 1 where unchanged)
+      const bool grow = mx > m_run + 8.f;
+      const float alpha = grow ? ex2f(m_run - mx) : 1.f;
+      if (__any_sync(0xffffffffu, grow && c > 0)) {
+        for (int c0 = 0; c0 < kHalf; c0 += 32) {
+          float o[32];
+          const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + c0;
+          tmem_ld32(ta, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(ta, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(ta, o);
         }
+      }
+      if (grow) {
         l_run *= alpha;
         m_run = mx;
       }
@@ -344,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       float ls = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float p0 = ex2f(sc[2 * i] - m_run), p1 = ex2f(sc[2 * i + 1] - m_run);
+        const float p0 = tv[i >> 3] ? ex2f(sc[2 * i] - m_run) : 0.f;
+        const float p1 = tv[i >> 3] ? ex2f(sc[2 * i + 1] - m_run) : 0.f;
         ls += p0 + p1;
         pk[i] = pack_f16x2(p0, p1);
       }
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   if (warp < 4) {
     float* po = p.part_o + (((size_t)b * p.splits + split) * kH + tid) * kLat + rank * kHalf;
     if (nchunks > 0) {
-      ok &= mbar_wait_bounded(bar_pv, (uint32_t)(nchunks - 1) & 1u, kWaitLimit);
+      ok &= mbar_wait_bounded(bar_pv, (uint32_t)(nchunks - 1) & 1u, ok ? kWaitLimit : 0u);
       tc_fence_after();
       for (int c0 = 0; c0 < kHalf; c0 += 32) {
         float o[32];

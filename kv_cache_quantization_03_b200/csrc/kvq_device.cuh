@@ -102,11 +102,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// Bounded wait on an mbarrier phase.  Returns false (and gives up) after
-// `limit` polls, so a lost transaction can never hang the GPU.
+// Bounded wait on an mbarrier phase.  Gives up (returns false) after about
+// `limit` nanoseconds of global time, so a lost transaction can never hang
+// the GPU; limit 0 returns at once unless the phase is already complete.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t i = 0; i < limit; ++i) {
+  uint64_t t0 = 0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (;;) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
@@ -114,8 +117,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    uint64_t t1;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+    if (t1 - t0 >= limit) return false;
   }
-  return false;
 }
 // 1-D bulk copy global -> shared, completion counted on `bar` in bytes.
 // dst, src 16-byte aligned; bytes a multiple of 16.

@@ -8,10 +8,9 @@
 
 namespace kvq {
 
-// Every spin-wait in a kernel gives up after this many polls and raises
-// KVQ_DEVERR_TIMEOUT (a poll takes well under a microsecond; this bounds a
-// lost transaction to well under a second).
-constexpr uint32_t kWaitLimit = 1u << 22;
+// Every spin-wait in a kernel gives up after this many nanoseconds (1 s of
+// GPU global time) and raises KVQ_DEVERR_TIMEOUT.
+constexpr uint32_t kWaitLimit = 1000000000u;
 
 // One quantised stream (K, V or the MLA latent) of the cache.
 struct CacheArrays {
