@@ -103,34 +103,48 @@ __host__ __device__ constexpr int kchan(int pi) {
   return B == 4 ? 8 * (pi >> 2) + (pi & 3) : (B == 8 ? 4 * (pi >> 1) + (pi & 1) : 16 * (pi >> 3) + (pi & 7));
 }
 
-// Pairs of one token row for the key MMA (16 pairs = 32 codes).
+// Each lane t works on the 32 channels 32t..32t+31 in a "slot" order rotated
+// by rot(t) channels: slot i is channel 32t + (i + rot(t)) % 32.  With the
+// rotation the lanes t = 0..3 read the per-channel key scales from different
+// shared-memory banks; codes, scales and the query use the same slot order.
+template <int B>
+__device__ __forceinline__ int rot_channels(int t) {
+  return (B == 4 || B == 8) ? 8 * t : 16 * (t & 1);
+}
+
+// Pairs of one token row for the key MMA (16 pairs = 32 codes), slot order.
 template <int B>
 __device__ __forceinline__ void key_pairs(const uint8_t* codes, int row, int t, uint32_t (&pr)[16]) {
-  if constexpr (B == 4) {
-    const uint4 w = *reinterpret_cast<const uint4*>(codes + row * 64 + 16 * t);
-    nib_pairs(w.x, pr);
-    nib_pairs(w.y, pr + 4);
-    nib_pairs(w.z, pr + 8);
-    nib_pairs(w.w, pr + 12);
-  } else if constexpr (B == 2) {
-    const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
-    crumb_pairs(w.x, pr);
-    crumb_pairs(w.y, pr + 8);
-  } else if constexpr (B == 8) {
-    const uint4 w0 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t);
-    const uint4 w1 = *reinterpret_cast<const uint4*>(codes + row * 128 + 32 * t + 16);
-    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  if constexpr (B == 4) {  // slot word m = channel word (m + t) % 4
+    const uint8_t* r = codes + row * 64 + 16 * t;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) nib_pairs(*reinterpret_cast<const uint32_t*>(r + 4 * ((m + t) & 3)), pr + 4 * m);
+  } else if constexpr (B == 2) {  // slot word m = channel word (m + t) % 2
+    const uint8_t* r = codes + row * 32 + 8 * t;
+    crumb_pairs(*reinterpret_cast<const uint32_t*>(r + 4 * (t & 1)), pr);
+    crumb_pairs(*reinterpret_cast<const uint32_t*>(r + 4 * ((t + 1) & 1)), pr + 8);
+  } else if constexpr (B == 8) {  // slot word m = channel word (m + 2t) % 8
+    const uint8_t* r = codes + row * 128 + 32 * t;
+    uint32_t ws[8];
+#pragma unroll
+    for (int m = 0; m < 8; m += 2) {
+      const uint2 x = *reinterpret_cast<const uint2*>(r + 4 * ((m + 2 * t) & 7));
+      ws[m] = x.x, ws[m + 1] = x.y;
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       pr[2 * k] = h2_field<0>(ws[k], 0x00FF00FFu);
       pr[2 * k + 1] = h2_field<0>(ws[k] >> 8, 0x00FF00FFu);
     }
-  } else {  // 3 bits: low plane [T][32 B] then high plane [T][16 B]
-    const uint2 w = *reinterpret_cast<const uint2*>(codes + row * 32 + 8 * t);
-    const uint32_t hw = *reinterpret_cast<const uint32_t*>(codes + kT * 32 + row * 16 + 4 * t);
+  } else {  // 3 bits: low plane [T][32 B] then high plane [T][16 B]; rotation by 16 (t & 1)
+    const uint8_t* r = codes + row * 32 + 8 * t;
+    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r + 4 * (t & 1));
+    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r + 4 * ((t + 1) & 1));
+    uint32_t hw = *reinterpret_cast<const uint32_t*>(codes + kT * 32 + row * 16 + 4 * t);
+    hw = (t & 1) ? __funnelshift_r(hw, hw, 16) : hw;
     uint32_t lo[16];
-    crumb_pairs(w.x, lo);
-    crumb_pairs(w.y, lo + 8);
+    crumb_pairs(w0, lo);
+    crumb_pairs(w1, lo + 8);
     const uint32_t hs[2] = {__byte_perm(hw, 0u, 0x4140u), __byte_perm(hw, 0u, 0x4342u)};
     const __half2 four = __halves2half2(__ushort_as_half(0x4400), __ushort_as_half(0x4400));
 #pragma unroll
@@ -259,8 +273,16 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       }
     }
     const float f = p.scale_log2 * 0.08838834764831845f;  // softmax scale * log2(e) / sqrt(128)
+    // into slot order (once per CTA, through this warp's not-yet-used stage memory)
+    float* scr = reinterpret_cast<float*>(wsm) + lane * 33;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) qr[i] *= f;
+    for (int i = 0; i < 32; ++i) scr[i] = qr[i] * f;
+    __syncwarp();
+    const int rot = rot_channels<BK>(t);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qr[i] = scr[(i + rot) & 31];
+    __syncwarp();
+    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
 
   // ---- producer: lane 0 fills stage (i % kStages) with local tile i
@@ -311,21 +333,23 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       const float* vc = reinterpret_cast<const float*>(st + SL.off_vc);
 
       // u = q~ * c_K on this lane's 32 channels, and its sum
-      float ck[32];
+      float ck[32];  // slot order
+      const int rq = rot_channels<BK>(t) >> 2;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + 4 * k);
+        const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + 4 * ((k + rq) & 7));
         ck[4 * k] = c4.x, ck[4 * k + 1] = c4.y, ck[4 * k + 2] = c4.z, ck[4 * k + 3] = c4.w;
       }
-      float su = 0.f;
+      f2 su2 = make_float2(0.f, 0.f);
       uint32_t ubh[16], ubl[16];  // u = hi + lo, both f16: ~22 significant bits
 #pragma unroll
       for (int pi = 0; pi < 16; ++pi) {
         const int c0 = kchan<BK>(pi), c1 = c0 + kdist<BK>();
-        const float u0 = qr[c0] * ck[c0], u1 = qr[c1] * ck[c1];
-        su += u0 + u1;
-        split_f16x2(u0, u1, ubh[pi], ubl[pi]);
+        const f2 u = make_float2(qr[c0] * ck[c0], qr[c1] * ck[c1]);
+        su2 = add2(su2, u);
+        split_f16x2(u.x, u.y, ubh[pi], ubl[pi]);
       }
+      float su = su2.x + su2.y;
       su += __shfl_xor_sync(0xffffffffu, su, 1);
       su += __shfl_xor_sync(0xffffffffu, su, 2);
       const float su0 = __shfl_sync(0xffffffffu, su, 8 * t);       // head 2t

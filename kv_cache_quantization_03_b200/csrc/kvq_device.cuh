@@ -73,8 +73,8 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // (x, y) = hi + lo with hi = f16(x, y) and lo = f16 of the remainder.
 __device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(x, y);
-  const float2 b = __half22float2(h);
-  const __half2 l = __floats2half2_rn(x - b.x, y - b.y);
+  const float2 r = sub2(make_float2(x, y), __half22float2(h));
+  const __half2 l = __floats2half2_rn(r.x, r.y);
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }

@@ -149,11 +149,13 @@ __device__ __forceinline__ void tile_sync() {
 }
 
 template <bool F16, int BITS, int D>
-__global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(QuantLaunch p) {
+__global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(QuantLaunch p) {
   constexpr int W = D / kBlk;     // warps per tile
   constexpr int TPC = kWarps / W; // tiles per CTA
+  constexpr bool kPark = (W == 1);  // park the rotated tile in shared memory during the rounds
   __shared__ WarpScratch scratch[kWarps];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
+  __shared__ float4 parked[kPark ? kWarps : 1][16][32];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int warp = threadIdx.x >> 5, blk = warp % W, slot_id = warp / W;
   const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
@@ -240,6 +242,14 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(
         A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
         A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
       }
+    // park the rotated values in shared memory until the factors are known
+    if constexpr (kPark) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const f2 x = P[i >> 3][(i >> 2) & 1][2 * (i & 3)], y = P[i >> 3][(i >> 2) & 1][2 * (i & 3) + 1];
+        parked[warp][i][lane] = make_float4(x.x, x.y, y.x, y.y);
+      }
+    }
     float w[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 1.f;
@@ -274,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(
 #pragma unroll
         for (int k = 1; k < W; ++k) rk += sh.row[it & 1][k][tok];
       }
-      const float vn = (float)D * rcp_nr(rk);
-      v_own = rk > 0.f ? vn : v_own;
+      // a zero row (rk = 0) only ever multiplies zeros, so its factor may be anything finite
+      v_own = (float)D * rcp_nr(fmaxf(rk, 1e-30f));
       float v[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -297,12 +307,11 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(
         c01 = add2(c01, make_float2(x.x, x.y));
         c23 = add2(c23, make_float2(x.z, x.w));
       }
-      const float n0 = (float)kT * rcp_nr(c01.x), n1 = (float)kT * rcp_nr(c01.y);
-      const float n2 = (float)kT * rcp_nr(c23.x), n3 = (float)kT * rcp_nr(c23.y);
-      w_own.x = c01.x > 0.f ? n0 : w_own.x;
-      w_own.y = c01.y > 0.f ? n1 : w_own.y;
-      w_own.z = c23.x > 0.f ? n2 : w_own.z;
-      w_own.w = c23.y > 0.f ? n3 : w_own.w;
+      // likewise a zero column; its stored factor is set to 1 after the rounds
+      w_own.x = (float)kT * rcp_nr(fmaxf(c01.x, 1e-30f));
+      w_own.y = (float)kT * rcp_nr(fmaxf(c01.y, 1e-30f));
+      w_own.z = (float)kT * rcp_nr(fmaxf(c23.x, 1e-30f));
+      w_own.w = (float)kT * rcp_nr(fmaxf(c23.y, 1e-30f));
       sc.own[lane] = w_own;
       __syncwarp();
 #pragma unroll
@@ -328,6 +337,14 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 2 : 1)) quantize_kernel(
           make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
+      if constexpr (kPark) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 x = parked[warp][i][lane];
+          P[i >> 3][(i >> 2) & 1][2 * (i & 3)] = make_float2(x.x, x.y);
+          P[i >> 3][(i >> 2) & 1][2 * (i & 3) + 1] = make_float2(x.z, x.w);
+        }
+      }
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -472,7 +489,7 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* strea
     q.rope_dim = p.rope_dim;
     const int tpc = head_dim == 128 ? kWarps : kWarps / (head_dim / kBlk);
     const int64_t need = (per_kind + tpc - 1) / tpc;
-    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 2 : 4);
+    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 3 : 4);
     const int grid = (int)(need < cap ? need : cap);
     int e;
     if (head_dim == 128)
