@@ -4,6 +4,7 @@
 // include/kvq.h.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -104,25 +105,29 @@ size_t decode_ws_bytes(int64_t pairs, const DecodePlan& d, int head_dim) {
   return (size_t)pairs * d.splits * kMaxGroup * ((size_t)head_dim + 2) * sizeof(float);
 }
 
-// MLA: one CTA pair per (sequence, split), one CTA per SM; about six waves,
-// at least two 32-token steps per split, an even number of tiles per split.
+// MLA: one CTA pair per (sequence, split), one CTA per SM, so kNumSMs / 2
+// pairs run at once.  The split count minimises (waves) x (32-token chunks
+// per split + a fixed cost of about four chunks for the query fetch, the
+// output write and the combine); a split has an even number of tiles.
 constexpr int kMlaHeads = 128;
 DecodePlan decode_plan_mla(int64_t batch, int64_t max_tiles) {
   DecodePlan d{1, 2};
   if (batch <= 0 || max_tiles <= 0) return d;
-  int64_t splits = (3 * kNumSMs + batch - 1) / batch;
-  const int64_t cap = (max_tiles + 3) / 4;
-  if (splits > cap) splits = cap;
-  if (splits < 1) splits = 1;
-  int64_t tps = (max_tiles + splits - 1) / splits;
-  tps = (tps + 1) / 2 * 2;
+  const int64_t slots = kNumSMs / 2, chunks = (max_tiles + 1) / 2;
+  int64_t best = 1, best_cost = INT64_MAX;
+  for (int64_t s = 1; s <= chunks && s <= 64; ++s) {
+    const int64_t per = (chunks + s - 1) / s, waves = (batch * s + slots - 1) / slots;
+    const int64_t cost = waves * (per + 4);
+    if (cost < best_cost) best_cost = cost, best = s;
+  }
+  const int64_t tps = 2 * ((chunks + best - 1) / best);
   d.tiles_per_split = (int)tps;
   d.splits = (int)((max_tiles + tps - 1) / tps);
   return d;
 }
 
 size_t decode_ws_bytes_mla(int64_t batch, const DecodePlan& d) {
-  return (size_t)batch * d.splits * kMlaHeads * (512 + 2) * sizeof(float);
+  return (size_t)batch * d.splits * kMlaHeads * (512 + 2) * sizeof(float) + mla_qprep_bytes(batch);
 }
 
 kvq_status cuda_status(int e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
@@ -292,6 +297,7 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
     m.part_ml = m.part_o + (size_t)batch * plan.splits * kMlaHeads * 512;
     m.splits = plan.splits;
     m.tiles_per_split = plan.tiles_per_split;
+    m.qprep = reinterpret_cast<uint8_t*>(m.part_ml + (size_t)batch * plan.splits * kMlaHeads * 2);
     m.err = dev_error;
     return cuda_status(launch_decode_mla(m, stream));
   }

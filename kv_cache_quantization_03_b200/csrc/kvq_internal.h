@@ -91,6 +91,7 @@ struct MlaDecodeParams {
   float* part_ml;               // [B][splits][128][2]
   int splits;
   int tiles_per_split;          // even
+  uint8_t* qprep;               // [B][2][128 x 288 f16]: rotated queries in the score-operand layout
   uint32_t* err;
 };
 
@@ -99,5 +100,6 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* strea
 int launch_dequantize(const DequantParams& p, int head_dim, void* stream);
 int launch_decode_d128(const DecodeParams& p, void* stream);
 int launch_decode_mla(const MlaDecodeParams& p, void* stream);
+size_t mla_qprep_bytes(int64_t batch);  // workspace for the prepared MLA queries
 
 }  // namespace kvq
