@@ -16,7 +16,7 @@ using namespace kvq;
 namespace {
 
 constexpr int kNumSMs = 148;           // B200
-constexpr int kDecodeTargetCtas = 4 * kNumSMs;
+constexpr int kDecodeCtasPerSm = 4;      // resident decode CTAs per SM (registers and shared memory)
 constexpr int kDecodeWarps = 4;        // warps per decode CTA (tiles are dealt round robin)
 constexpr int kMaxGroup = 8;
 
@@ -85,16 +85,23 @@ struct DecodePlan {
   int tiles_per_split;
 };
 
-// Split the tiles of each (sequence, kv-head) so that about kDecodeTargetCtas
-// CTAs run, with at least 4 tiles per warp in a split.
+// Split the tiles of each (sequence, kv-head) over CTAs.  kDecodeCtasPerSm
+// CTAs fit on an SM at once, so the split count minimises (waves) x (tiles
+// per warp + a fixed cost of about six tiles for the prologue, the merge of
+// the CTA's warps and the combine), with at least 4 tiles per warp.
 DecodePlan decode_plan(int64_t pairs, int64_t max_tiles) {
   DecodePlan d{1, 0};
   if (pairs <= 0 || max_tiles <= 0) return d;
-  int64_t splits = (kDecodeTargetCtas + pairs - 1) / pairs;
+  const int64_t slots = (int64_t)kDecodeCtasPerSm * kNumSMs;
   const int64_t cap = (max_tiles + 4 * kDecodeWarps - 1) / (4 * kDecodeWarps);
-  if (splits > cap) splits = cap;
-  if (splits < 1) splits = 1;
-  int64_t tps = (max_tiles + splits - 1) / splits;
+  int64_t best = 1, best_cost = INT64_MAX;
+  for (int64_t s = 1; s <= cap && s <= 256; ++s) {
+    const int64_t per_warp = (max_tiles + s * kDecodeWarps - 1) / (s * kDecodeWarps);
+    const int64_t waves = (pairs * s + slots - 1) / slots;
+    const int64_t cost = waves * (per_warp + 6);
+    if (cost < best_cost) best_cost = cost, best = s;
+  }
+  int64_t tps = (max_tiles + best - 1) / best;
   tps = (tps + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps;
   d.tiles_per_split = (int)tps;
   d.splits = (int)((max_tiles + tps - 1) / tps);

@@ -34,7 +34,8 @@ namespace {
 constexpr int kD = 128;
 constexpr int kT = 16;
 constexpr int kDW = 4;      // warps per CTA
-constexpr int kStages = 4;  // ring depth per warp
+constexpr int kStages = 3;  // ring depth per warp
+constexpr int kQStride = 132;  // floats per head row of the shared rotated query (padded: no bank conflicts)
 constexpr float kNegBig = -1e30f;
 
 struct StageLayout {
@@ -200,7 +201,7 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 template <int BK, int BV>
-__global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr StageLayout SL = stage_layout(BK, BV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -232,16 +233,18 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
   const int t1 = min(t0 + p.tiles_per_split, ntiles);
   const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
   // this split's page ids, staged once in shared memory
-  int32_t* spg = reinterpret_cast<int32_t*>(bars + kDW * kStages);
+  float* qs = reinterpret_cast<float*>(bars + kDW * kStages);     // [8][kQStride] rotated query
+  int32_t* spg = reinterpret_cast<int32_t*>(qs + 8 * kQStride);
   {
     const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
     for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[i];
   }
   __syncthreads();
 
-  // ---- rotated, pre-scaled query: lane (g, t) keeps head g, channels 32t..32t+31
-  float qr[32];
-  {
+  // ---- rotated, pre-scaled query of the CTA's 8 heads into shared memory (warp 0:
+  // lane (g, t) computes head g, channels 32t..32t+31)
+  if (warp == 0) {
+    float qr[32];
     const bool live = g < p.group;
     const uint16_t* qp = p.q + ((size_t)b * p.num_q_heads + (size_t)kvh * p.group + (live ? g : 0)) * kD + 32 * t;
 #pragma unroll
@@ -273,17 +276,12 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       }
     }
     const float f = p.scale_log2 * 0.08838834764831845f;  // softmax scale * log2(e) / sqrt(128)
-    // into slot order (once per CTA, through this warp's not-yet-used stage memory)
-    float* scr = reinterpret_cast<float*>(wsm) + lane * 33;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) scr[i] = qr[i] * f;
-    __syncwarp();
-    const int rot = rot_channels<BK>(t);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) qr[i] = scr[(i + rot) & 31];
-    __syncwarp();
-    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4*>(qs + g * kQStride + 32 * t + i) =
+          make_float4(qr[i] * f, qr[i + 1] * f, qr[i + 2] * f, qr[i + 3] * f);
   }
+  __syncthreads();
 
   // ---- producer: lane 0 fills stage (i % kStages) with local tile i
   auto issue = [&](int i) {
@@ -332,22 +330,28 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       const float* vaz = reinterpret_cast<const float*>(st + SL.off_vaz);
       const float* vc = reinterpret_cast<const float*>(st + SL.off_vc);
 
-      // u = q~ * c_K on this lane's 32 channels, and its sum
-      float ck[32];  // slot order
-      const int rq = rot_channels<BK>(t) >> 2;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + 4 * ((k + rq) & 7));
-        ck[4 * k] = c4.x, ck[4 * k + 1] = c4.y, ck[4 * k + 2] = c4.z, ck[4 * k + 3] = c4.w;
-      }
+      // u = q~ * c_K on this lane's 32 channels (slot order), and its sum
+      float u[32];
       f2 su2 = make_float2(0.f, 0.f);
+      {
+        const int rq = rot_channels<BK>(t) >> 2;
+        const float* qg = qs + g * kQStride + 32 * t;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int kk = 4 * ((k + rq) & 7);
+          const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + kk);
+          const float4 q4 = *reinterpret_cast<const float4*>(qg + kk);
+          const f2 a = mul2(make_float2(q4.x, q4.y), make_float2(c4.x, c4.y));
+          const f2 d = mul2(make_float2(q4.z, q4.w), make_float2(c4.z, c4.w));
+          su2 = add2(su2, add2(a, d));
+          u[4 * k] = a.x, u[4 * k + 1] = a.y, u[4 * k + 2] = d.x, u[4 * k + 3] = d.y;
+        }
+      }
       uint32_t ubh[16], ubl[16];  // u = hi + lo, both f16: ~22 significant bits
 #pragma unroll
       for (int pi = 0; pi < 16; ++pi) {
         const int c0 = kchan<BK>(pi), c1 = c0 + kdist<BK>();
-        const f2 u = make_float2(qr[c0] * ck[c0], qr[c1] * ck[c1]);
-        su2 = add2(su2, u);
-        split_f16x2(u.x, u.y, ubh[pi], ubl[pi]);
+        split_f16x2(u[c0], u[c1], ubh[pi], ubl[pi]);
       }
       float su = su2.x + su2.y;
       su += __shfl_xor_sync(0xffffffffu, su, 1);
@@ -359,13 +363,14 @@ __global__ void __launch_bounds__(kDW * 32) decode_d128_kernel(DecodeParams p) {
       uint32_t kp0[16], kp1[16];
       key_pairs<BK>(st, g, t, kp0);
       key_pairs<BK>(st, g + 8, t, kp1);
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
+      float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f};  // two independent MMA chains
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t a[4] = {kp0[2 * s], kp1[2 * s], kp0[2 * s + 1], kp1[2 * s + 1]};
-        mma16816<true>(S, a, ubh[2 * s], ubh[2 * s + 1], S);
-        mma16816<true>(S, a, ubl[2 * s], ubl[2 * s + 1], S);
+        mma16816<true>(Sh, a, ubh[2 * s], ubh[2 * s + 1], Sh);
+        mma16816<true>(Sl, a, ubl[2 * s], ubl[2 * s + 1], Sl);
       }
+      const float S[4] = {Sh[0] + Sl[0], Sh[1] + Sl[1], Sh[2] + Sl[2], Sh[3] + Sl[3]};
       const float2 az0 = *reinterpret_cast<const float2*>(kaz + 2 * g);
       const float2 az1 = *reinterpret_cast<const float2*>(kaz + 2 * (g + 8));
       float sc[4];
@@ -524,7 +529,7 @@ int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
   constexpr StageLayout SL = stage_layout(BK, BV);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
-  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
+  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) + 8 * kQStride * 4 +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
   auto kern = decode_d128_kernel<BK, BV>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

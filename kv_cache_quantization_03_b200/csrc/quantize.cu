@@ -82,12 +82,19 @@ __device__ __forceinline__ float rsqrt_nr(float x) {
 __device__ __forceinline__ uint32_t gather4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x4000u), 0x7610u);
 }
-// Eight 4-bit codes (byte 0 of each word) -> one word, code i in bits 4i..4i+3.
+// The words hold magic-number floats: bits 0..21 are the code, bits above
+// them a constant whose low byte is 0.  So f0 + (f1 << 4) carries the two
+// codes in its low byte: eight 4-bit codes -> one word, code i in bits
+// 4i..4i+3.
 __device__ __forceinline__ uint32_t pack_nibbles(const uint32_t* f) {
-  uint32_t u = gather4(f[0], f[1], f[2], f[3]), v = gather4(f[4], f[5], f[6], f[7]);
-  u |= u >> 4;
-  v |= v >> 4;
-  return __byte_perm(u, v, 0x6420u);
+  return gather4(f[0] + (f[1] << 4), f[2] + (f[3] << 4), f[4] + (f[5] << 4), f[6] + (f[7] << 4));
+}
+// Sixteen 2-bit codes -> one word, code i in bits 2i..2i+1.
+__device__ __forceinline__ uint32_t pack_crumbs(const uint32_t* f) {
+  uint32_t b[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) b[k] = f[4 * k] + (f[4 * k + 1] << 2) + (f[4 * k + 2] << 4) + (f[4 * k + 3] << 6);
+  return gather4(b[0], b[1], b[2], b[3]);
 }
 
 struct WarpScratch {
@@ -405,7 +412,9 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
       uint32_t q[2][16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const f2 tq = add2(mul2(sub2(P[h][j >> 3][j & 7], m2), is2), splat2(kMagic));
+        // (y - m) / s rounded to the nearest integer (ties to even) by the
+        // single rounding of the fused multiply-add into the magic number
+        const f2 tq = fma2(sub2(P[h][j >> 3][j & 7], m2), is2, splat2(kMagic));
         q[0][j] = __float_as_uint(tq.x);
         q[1][j] = __float_as_uint(tq.y);
       }
@@ -422,10 +431,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
               make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
                          gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
         } else if constexpr (BITS == 2) {
-          uint32_t wd = 0;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) wd |= (f[j] & 3u) << (2 * j);
-          *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = wd;
+          *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = pack_crumbs(f);
         } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
           uint32_t lo = 0, hi = 0;
 #pragma unroll
