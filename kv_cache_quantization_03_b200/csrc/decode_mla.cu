@@ -9,33 +9,33 @@
 //
 // All heads of a sequence (M = 128) share every tile, so both contractions
 // run on the tensor cores with the tile dequantised once to f16 in shared
-// memory: scores = Q K^T, out += P V.  128 x 512 fp32 output accumulators
-// would fill all of an SM's tensor memory, so a cluster of two CTAs shares
-// each (sequence, split): CTA r owns latent channels [256r, 256r + 256) of
-// the output and rope channels [32r, 32r + 32) of the score, computes the
-// partial score over its 288 channels, and the two partial score blocks are
-// exchanged through distributed shared memory.
+// memory: S = Q K^T (K = 576), out += P V.  128 x 512 fp32 output
+// accumulators would fill all of an SM's tensor memory, so two CTAs share
+// each (sequence, split): CTA r accumulates output channels [256r, 256r+256).
+// Both compute the full scores and the same softmax, so no data moves
+// between them.  The query's first 288 channels sit in tensor memory as the
+// MMA's A operand, the other 288 in shared memory.
 //
 // Each CTA is a pipeline of three roles connected by mbarriers:
-//   warp 8 (one thread)  bulk copies of the raw tiles into a ring of stages,
-//                        and the tcgen05 MMAs: S(c) = Q K(c)^T into one of
-//                        two TMEM score buffers, then O += P(c-1) V(c-1);
-//   warps 4-7            dequantise a 32-token chunk, (a q + z) c in fp32,
-//                        to f16 in the no-swizzle core-matrix operand layout
-//                        (three buffers, so they run up to two chunks ahead);
-//   warps 0-3            one thread per head (a TMEM lane): load the partial
-//                        score, send it to the peer CTA, add the peer's
-//                        partial, online softmax with lazy rescaling of the
-//                        TMEM output (only when the running max grows by
-//                        more than 2^8), P in f16 to shared memory.
-// The softmax of chunk c-1 overlaps the dequantisation of chunk c+1 and the
-// score MMA of chunk c.  Every wait is bounded in time (1 s of global time);
-// a wait that runs out raises KVQ_DEVERR_TIMEOUT and the remaining waits of
-// that thread are skipped, so the kernel always terminates.
+//   warp 20 (one thread)  bulk copies of the raw tiles into a ring of stages,
+//                         and the tcgen05 MMAs: S(c) into one of two TMEM
+//                         score buffers, then O += P(c-1) V(c-1);
+//   warps 4-19            dequantise a 32-token chunk, (a q + z) c in fp32,
+//                         to f16 in the no-swizzle core-matrix operand layout
+//                         (three buffers, two at 8 bits, so the dequantisation
+//                         of chunk c+1 overlaps the MMAs of chunk c);
+//   warps 0-3             one thread per head (a TMEM lane): online softmax
+//                         with lazy rescaling of the TMEM output (only when
+//                         the running max grows by more than 2^8), P in f16
+//                         to tensor memory, where it is the A operand of P V.
+// Every wait is bounded in time (1 s of global time); a wait that runs out
+// raises KVQ_DEVERR_TIMEOUT and the remaining waits of that thread are
+// skipped, so the kernel always terminates.
 //
-// The rotated, pre-scaled f16 query of every (sequence, latent half) is
-// built once by mla_prep_q_kernel in exactly the shared-memory operand
-// layout, and each CTA fetches its 72 KB with one bulk copy.
+// mla_prep_q_kernel builds the rotated, pre-scaled f16 query of every
+// sequence once: channels [0, 288) row-major (loaded into tensor memory by
+// the softmax threads), channels [288, 576) in the shared-memory operand
+// layout (one bulk copy).
 #include <cuda_runtime.h>
 
 #include "kvq_device.cuh"
@@ -44,45 +44,52 @@ namespace kvq {
 namespace {
 
 constexpr int kT = 16;
-constexpr int kLat = 512, kHalf = 256, kRope = 64, kRopeHalf = 32;
-constexpr int kK = kHalf + kRopeHalf;  // 288: K extent of this CTA's score operands
-constexpr int kH = 128;                // M: heads (rows beyond num_q_heads are zero)
-constexpr int kChunk = 32;             // tokens per step (two tiles)
-constexpr int kDqWarps = 4;
-constexpr int kThreads = 9 * 32;       // softmax 0-3, dequantisation 4-7, copies + MMA 8
-constexpr int kNB = 3;                 // dequantised chunk buffers
+constexpr int kLat = 512, kRope = 64, kKf = kLat + kRope;  // 576: K extent of the scores
+constexpr int kKT = 288;             // query channels [0, 288) in tensor memory
+constexpr int kKS = kKf - kKT;       // query channels [288, 576) in shared memory
+constexpr int kHalf = 256;           // output channels per CTA
+constexpr int kH = 128;              // M: heads (rows beyond num_q_heads are zero)
+constexpr int kChunk = 32;           // tokens per step (two tiles)
+constexpr int kDqWarps = 16;
+constexpr int kThreads = (4 + kDqWarps + 1) * 32;  // softmax 0-3, dequantisation 4-19, copies + MMA 20
 constexpr float kNegBig = -1e30f;
+// TMEM columns: O [0,256), S [256,320), Q [320,464), P [464,496)
+constexpr uint32_t kTmemS = 256, kTmemQ = 320, kTmemP = 464;
 
 // byte offsets in shared memory
-constexpr int kSbo = kK / 8 * 128;           // 4608: next 8 rows of a K-major operand
-constexpr int kQsBytes = kH * kK * 2;        // 73728
-constexpr int kKbBytes = kChunk * kK * 2;    // 18432 per buffer
-constexpr int kPsBytes = kH * kChunk * 2;    // 8192 per buffer
-constexpr int kSxBytes = kH * kChunk * 4;    // 16384 per buffer
+constexpr int kSboQ = kKS / 8 * 128;         // 4608: next 8 rows of the shared query part
+constexpr int kSboK = kKf / 8 * 128;         // 9216: next 8 rows of a dequantised chunk
+constexpr int kQsBytes = kH * kKS * 2;       // 73728
+constexpr int kQtBytes = kH * kKT * 2;       // 73728
+constexpr int kKbBytes = kChunk * kKf * 2;   // 36864 per buffer
 constexpr int kOffQs = 0;
 constexpr int kOffKb = kOffQs + kQsBytes;
-constexpr int kOffPs = kOffKb + kNB * kKbBytes;
-constexpr int kOffSx = kOffPs + 2 * kPsBytes;
-constexpr int kOffSt = kOffSx + 2 * kSxBytes;
-// a stage holds two tiles: codes | (a, z) | channel scales of this CTA's half | rope
+__host__ __device__ constexpr int num_kb(int bits) { return bits == 8 ? 2 : 3; }  // dequantised chunk buffers
+__host__ __device__ constexpr int st_offset(int bits) { return kOffKb + num_kb(bits) * kKbBytes; }
+// a stage holds two tiles: codes | (a, z) | channel scales | rope
 __host__ __device__ constexpr int tile_code_bytes(int bits) { return kT * kLat * bits / 8; }
 __host__ __device__ constexpr int stage_bytes(int bits) {
-  return 2 * (tile_code_bytes(bits) + kT * 8 + kHalf * 4 + kT * kRope * 2);
+  return 2 * (tile_code_bytes(bits) + kT * 8 + kLat * 4 + kT * kRope * 2);
 }
-__host__ __device__ constexpr int num_stages(int bits) { return bits == 8 ? 2 : 3; }
-__host__ __device__ constexpr int bar_offset(int bits) { return kOffSt + num_stages(bits) * stage_bytes(bits); }
-// full[3] dq[kNB] sfull[2] pfull[2] pv[4] sxf[2] sxe[2] qf[1], then the TMEM address
-constexpr int kNumBars = 3 + kNB + 2 + 2 + 4 + 2 + 2 + 1;
-__host__ __device__ constexpr int smem_bytes(int bits) { return bar_offset(bits) + kNumBars * 8 + 16; }
-static_assert(smem_bytes(8) <= 232448 && smem_bytes(4) <= 232448, "shared memory");
+constexpr int kNS = 2;  // raw-tile stages
+__host__ __device__ constexpr int bar_offset(int bits) { return st_offset(bits) + kNS * stage_bytes(bits); }
+// full[2] dq[3] sfull[2] pfull[2] pv[4] qf qt, the TMEM address, then the tile-validity bits
+constexpr int kNumBars = kNS + 3 + 2 + 2 + 4 + 2;
+__host__ __device__ constexpr int vmask_offset(int bits) { return bar_offset(bits) + kNumBars * 8 + 8; }
+__host__ __device__ constexpr int smem_bytes(int bits, int tiles_per_split) {
+  return vmask_offset(bits) + ((tiles_per_split + 31) / 32) * 4;
+}
+static_assert(smem_bytes(4, 8192) <= 232448 && smem_bytes(8, 8192) <= 232448, "shared memory");
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
 }
-// K-major core-matrix layout offset of element (row, k), kSbo bytes per 8 rows
-__host__ __device__ __forceinline__ uint32_t km_off(int row, int k) {
-  return (row >> 3) * kSbo + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+// No-swizzle core-matrix layout offset of element (row, k): 8 x 8 blocks of
+// 16-bit elements (128 B, one row of 16 B per row), k-blocks 128 B apart,
+// row-blocks `sbo` bytes apart.
+__host__ __device__ __forceinline__ uint32_t cm_off(int row, int k, int sbo) {
+  return (row >> 3) * sbo + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
 }
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
   asm volatile("{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;}" ::"r"(
@@ -122,49 +129,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t peer) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(peer));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-// Arrive (count 1) on an mbarrier of the peer CTA; orders this thread's
-// earlier shared-memory accesses of the cluster before it.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 __device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Bounded wait with cluster-scope acquire: for phases completed by the peer.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  const uint32_t a = smem_u32(bar);
-  uint64_t t0 = 0;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-    uint64_t t1;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
-    if (t1 - t0 >= limit) return false;
-  }
 }
 
 __device__ __forceinline__ float bf16f(uint32_t b) { return __uint_as_float(b << 16); }
@@ -198,29 +164,44 @@ __device__ __forceinline__ void codes8(const uint8_t* codes, int tr, int ch0, fl
   for (int e = 0; e < 8; ++e) q[e] = __uint_as_float(0x4B000000u | c[e]) - 8388608.0f;  // exact small integers
 }
 
+
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                                uint32_t acc) {
+  asm volatile("{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;}" ::"r"(
+                   tmem_d),
+               "r"(tmem_a), "l"(db), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams p) {
-  constexpr int NS = num_stages(BITS), SB = stage_bytes(BITS), CB = tile_code_bytes(BITS);
-  constexpr int kStAz = 2 * CB, kStC = kStAz + 2 * kT * 8, kStRope = kStC + 2 * kHalf * 4;
+  constexpr int NS = kNS, NB = num_kb(BITS), SB = stage_bytes(BITS), CB = tile_code_bytes(BITS);
+  constexpr int kOffSt = st_offset(BITS);
+  constexpr int kStAz = 2 * CB, kStC = kStAz + 2 * kT * 8, kStRope = kStC + 2 * kLat * 4;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;  // latent half owned by this CTA
-  const int split = blockIdx.x >> 1, b = blockIdx.y;
+  const int r = blockIdx.x & 1, split = blockIdx.x >> 1, b = blockIdx.y;  // r: output half
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + bar_offset(BITS));
-  uint64_t* dq = full + 3;
-  uint64_t* sfull = dq + kNB;
+  uint64_t* dq = full + kNS;
+  uint64_t* sfull = dq + 3;
   uint64_t* pfull = sfull + 2;
   uint64_t* pv = pfull + 2;
-  uint64_t* sxf = pv + 4;
-  uint64_t* sxe = sxf + 2;
-  uint64_t* qf = sxe + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qf + 1);
+  uint64_t* qf = pv + 4;
+  uint64_t* qt = qf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qt + 1);
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + vmask_offset(BITS));
   const uint32_t s_base = smem_u32(smem);
 
   const int seq_raw = p.seq_lens[b];
   int ntiles = seq_raw < 0 ? 0 : seq_raw / kT;
   if (ntiles > p.max_pages) ntiles = p.max_pages;
-  if (split == 0 && rank == 0 && tid == 0) {
+  if (split == 0 && r == 0 && tid == 0) {
     if (seq_raw < 0 || seq_raw / kT > p.max_pages) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
     if (seq_raw % kT) set_error(p.err, KVQ_DEVERR_PARTIAL_TILE);
   }
@@ -229,27 +210,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   const int ntl = t1 > t0 ? t1 - t0 : 0;
   const int nchunks = (ntl + 1) / 2;
   const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
-  auto tile_ok = [&](int lt) {
-    if (lt >= ntl) return false;
-    const int pg = __ldg(btab + lt);
-    return pg >= 0 && pg < p.num_pages;
-  };
+  const uint8_t* qprep = p.qprep + (size_t)b * (kQsBytes + kQtBytes);
+
+  // which tiles of the split have a valid page (bit lt of vmask)
+  for (int i = tid; i < (ntl + 31) / 32; i += kThreads) vmask[i] = 0u;
+  __syncthreads();
+  for (int lt = tid; lt < ntl; lt += kThreads) {
+    const int pg = btab[lt];
+    if (pg >= 0 && pg < p.num_pages) atomicOr(&vmask[lt >> 5], 1u << (lt & 31));
+    else if (r == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+  }
+  auto tile_ok = [&](int lt) { return lt < ntl && ((vmask[lt >> 5] >> (lt & 31)) & 1u); };
 
   if (tid == 0) {
 #pragma unroll
     for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
 #pragma unroll
-    for (int i = 0; i < kNB; ++i) mbar_init(&dq[i], kDqWarps * 32);
+    for (int i = 0; i < NB; ++i) mbar_init(&dq[i], kDqWarps * 32);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], kH);
-      mbar_init(&sxf[i], kH);
-      mbar_init(&sxe[i], kH);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) mbar_init(&pv[i], 1);
     mbar_init(qf, 1);
+    mbar_init(qt, kH);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -259,34 +245,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();  // both CTAs' barriers exist before any remote arrive
-  const uint32_t tmem = *tmem_slot;  // columns [0, 256): output half; [256, 320): two score buffers
+  const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 8) {
+  if (warp == 4 + kDqWarps) {
     // ---------------------------------------------------------------- copies + MMA (one thread)
     if (lane == 0) {
       mbar_arrive_expect_tx(qf, kQsBytes);
-      bulk_g2s(smem + kOffQs, p.qprep + ((size_t)b * 2 + rank) * kQsBytes, kQsBytes, qf);
+      bulk_g2s(smem + kOffQs, qprep, kQsBytes, qf);
       auto issue = [&](int c) {  // raw chunk c into stage c % NS
         uint64_t* bar = &full[c % NS];
         uint8_t* st = smem + kOffSt + (c % NS) * SB;
         uint32_t bytes = 0;
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          if (tile_ok(2 * c + j)) bytes += CB + kT * 8 + kHalf * 4 + kT * kRope * 2;
+          if (tile_ok(2 * c + j)) bytes += CB + kT * 8 + kLat * 4 + kT * kRope * 2;
         mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int lt = 2 * c + j;
-          if (!tile_ok(lt)) {
-            if (lt < ntl) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
-            continue;
-          }
-          const size_t slot = (size_t)p.layer * p.num_pages + __ldg(btab + lt);
+          if (!tile_ok(2 * c + j)) continue;
+          const size_t slot = (size_t)p.layer * p.num_pages + btab[2 * c + j];
           bulk_g2s(st + j * CB, p.codes + slot * CB, CB, bar);
           bulk_g2s(st + kStAz + j * kT * 8, p.tok + slot * kT * 2, kT * 8, bar);
-          bulk_g2s(st + kStC + j * kHalf * 4, p.chan + slot * kLat + rank * kHalf, kHalf * 4, bar);
+          bulk_g2s(st + kStC + j * kLat * 4, p.chan + slot * kLat, kLat * 4, bar);
           bulk_g2s(st + kStRope + j * kT * kRope * 2, p.rope + slot * kT * kRope, kT * kRope * 2, bar);
         }
       };
@@ -294,33 +275,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       for (int c = 0; c < pre; ++c) issue(c);
       const uint32_t idesc_s = (1u << 4) | ((uint32_t)(kChunk >> 3) << 17) | ((uint32_t)(kH >> 4) << 24);
       const uint32_t idesc_pv = (1u << 4) | (1u << 16) | ((uint32_t)(kHalf >> 3) << 17) | ((uint32_t)(kH >> 4) << 24);
-      const uint32_t qs = s_base + kOffQs;
+      const uint64_t dq0 = umma_desc(s_base + kOffQs, 128, kSboQ), dk0 = umma_desc(s_base + kOffKb, 128, kSboK);
+      const uint64_t dv0 = umma_desc(s_base + kOffKb + r * (kHalf / 8) * 128, kSboK, 128);
       ok &= mbar_wait_bounded(qf, 0u, kWaitLimit);
+      ok &= mbar_wait_bounded(qt, 0u, ok ? kWaitLimit : 0u);
       for (int c = 0; c <= nchunks; ++c) {
         if (c < nchunks) {
           // chunk c is dequantised; its raw stage is free again
-          ok &= mbar_wait_bounded(&dq[c % kNB], (uint32_t)(c / kNB) & 1u, ok ? kWaitLimit : 0u);
+          ok &= mbar_wait_bounded(&dq[c % NB], (uint32_t)(c / NB) & 1u, ok ? kWaitLimit : 0u);
           if (c + NS < nchunks) {
             proxy_fence();
             issue(c + NS);
           }
           tc_fence_after();
-          const uint32_t kb = s_base + kOffKb + (c % kNB) * kKbBytes;
-#pragma unroll 1
-          for (int s = 0; s < kK / 16; ++s)
-            umma_f16(tmem + kHalf + 32 * (c & 1), umma_desc(qs + s * 256, 128, kSbo), umma_desc(kb + s * 256, 128, kSbo),
-                     idesc_s, s > 0);
+          // descriptors advance by 256 B (16 in the address field) per 16-channel step
+          const uint64_t dk = dk0 + (uint64_t)((c % NB) * (kKbBytes >> 4));
+          const uint32_t d = tmem + kTmemS + 32 * (c & 1);
+#pragma unroll
+          for (int s = 0; s < kKT / 16; ++s)  // query channels [0, 288) from tensor memory
+            umma_f16_tmem_a(d, tmem + kTmemQ + 8 * s, dk + 16 * s, idesc_s, s > 0);
+#pragma unroll
+          for (int s = 0; s < kKS / 16; ++s)  // [288, 576) from shared memory
+            umma_f16(d, dq0 + 16 * s, dk + (kKT / 8) * 8 + 16 * s, idesc_s, 1u);
           umma_commit(&sfull[c & 1]);
         }
         if (c >= 1) {
           const int x = c - 1;
           ok &= mbar_wait_bounded(&pfull[x & 1], (uint32_t)(x >> 1) & 1u, ok ? kWaitLimit : 0u);
           tc_fence_after();
-          const uint32_t ps = s_base + kOffPs + (x & 1) * kPsBytes, kb = s_base + kOffKb + (x % kNB) * kKbBytes;
+          const uint64_t dv = dv0 + (uint64_t)((x % NB) * (kKbBytes >> 4));
 #pragma unroll
-          for (int s = 0; s < kChunk / 16; ++s)
-            umma_f16(tmem, umma_desc(ps + s * 256, 128, 512), umma_desc(kb + s * 2 * kSbo, kSbo, 128), idesc_pv,
-                     (x > 0 || s > 0) ? 1u : 0u);
+          for (int s = 0; s < kChunk / 16; ++s)  // A = P(x) in tensor memory
+            umma_f16_tmem_a(tmem, tmem + kTmemP + 16 * (x & 1) + 8 * s, dv + s * 2 * (kSboK >> 4), idesc_pv,
+                            (x > 0 || s > 0) ? 1u : 0u);
           umma_commit(&pv[x & 3]);
         }
       }
@@ -330,144 +317,129 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- dequantisation
-    // Lane l converts latent channels 8l..8l+7 of this half for the chunk rows
-    // 8 dw + ((l + it) & 7), it = 0..7 (both the code loads and the operand
-    // stores are free of bank conflicts), then 8 rope channels of one row.
-    const int dw = warp - 4, j = dw >> 1;
+    // Warp dw covers tile j = dw / 8, latent channels 256 gh + 8 lane .. + 7
+    // (gh = (dw / 4) % 2) of the tile rows 8 rh + ((lane + it + 4 hf) % 8),
+    // it = 0..3 (rh = (dw / 2) % 2, hf = dw % 2): code loads and operand
+    // stores are free of bank conflicts.  Warps 0..7 then convert 8 rope
+    // channels of one row each, spread the same way.
+    const int dw = warp - 4, j = dw >> 3, gh = (dw >> 2) & 1, rh = (dw >> 1) & 1, hf = dw & 1;
+    const int ch0 = kHalf * gh + 8 * lane;
+    const int ri = lane & 7, rP = (lane >> 3) + 4 * ((dw >> 2) & 1);
+    const int rrow = 8 * (dw & 3) + ((ri + rP) & 7), rgrp = ri;  // rope (dw < 8): chunk row, 8-channel group
     for (int c = 0; c < nchunks; ++c) {
       ok &= mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, ok ? kWaitLimit : 0u);
-      if (c >= kNB)  // PV(c - kNB) has read this operand buffer
-        ok &= mbar_wait_bounded(&pv[(c - kNB) & 3], (uint32_t)((c - kNB) >> 2) & 1u, ok ? kWaitLimit : 0u);
+      if (c >= NB)  // PV(c - NB) has read this operand buffer
+        ok &= mbar_wait_bounded(&pv[(c - NB) & 3], (uint32_t)((c - NB) >> 2) & 1u, ok ? kWaitLimit : 0u);
       const uint8_t* st = smem + kOffSt + (c % NS) * SB;
-      uint8_t* kb = smem + kOffKb + (c % kNB) * kKbBytes;
+      uint8_t* kb = smem + kOffKb + (c % NB) * kKbBytes;
       const bool valid = tile_ok(2 * c + j);
       f2 cc[4];
       {
-        const float4* cp = reinterpret_cast<const float4*>(st + kStC + j * kHalf * 4) + 2 * lane;
+        const float4* cp = reinterpret_cast<const float4*>(st + kStC + j * kLat * 4 + ch0 * 4);
         const float4 c0 = cp[0], c1 = cp[1];
         cc[0] = make_float2(c0.x, c0.y), cc[1] = make_float2(c0.z, c0.w);
         cc[2] = make_float2(c1.x, c1.y), cc[3] = make_float2(c1.z, c1.w);
       }
-#pragma unroll 2
-      for (int it = 0; it < 8; ++it) {
-        const int tr = 8 * (dw & 1) + ((lane + it) & 7);
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int tr = 8 * rh + ((lane + it + 4 * hf) & 7);
         const float2 az = *reinterpret_cast<const float2*>(st + kStAz + j * kT * 8 + tr * 8);
         float q[8];
-        codes8<BITS>(st + j * CB, tr, kHalf * (int)rank + 8 * lane, q);
+        codes8<BITS>(st + j * CB, tr, ch0, q);
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const f2 v = mul2(fma2(splat2(az.x), make_float2(q[2 * e], q[2 * e + 1]), splat2(az.y)), cc[e]);
           pk[e] = valid ? pack_f16x2(v.x, v.y) : 0u;
         }
-        *reinterpret_cast<uint4*>(kb + km_off(16 * j + tr, 8 * lane)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(kb + cm_off(16 * j + tr, ch0, kSboK)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      {
-        const int row = 8 * dw + (lane & 7), grp = lane >> 3;
-        const bool v2 = tile_ok(2 * c + (row >> 4));
-        const uint4 r = *reinterpret_cast<const uint4*>(st + kStRope + (row >> 4) * kT * kRope * 2 +
-                                                        (row & 15) * kRope * 2 + (kRopeHalf * rank + 8 * grp) * 2);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+      if (dw < 8) {
+        const int jj = rrow >> 4;
+        const bool v2 = tile_ok(2 * c + jj);
+        const uint4 w4 = *reinterpret_cast<const uint4*>(st + kStRope + jj * kT * kRope * 2 + (rrow & 15) * kRope * 2 +
+                                                         rgrp * 16);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) pk[e] = v2 ? pack_f16x2(bf16f(w[e] & 0xFFFFu), bf16f(w[e] >> 16)) : 0u;
-        *reinterpret_cast<uint4*>(kb + km_off(row, kHalf + 8 * grp)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(kb + cm_off(rrow, kLat + 8 * rgrp, kSboK)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       proxy_fence();
-      mbar_arrive_local(&dq[c % kNB]);
+      mbar_arrive_local(&dq[c % NB]);
     }
   } else {
     // ---------------------------------------------------------------- softmax, one thread per head
     const int h = tid;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t sx_peer = peer_addr(s_base + kOffSx, peer);
-    const uint32_t sxf_peer = peer_addr(smem_u32(sxf), peer), sxe_peer = peer_addr(smem_u32(sxe), peer);
-    float m_run = kNegBig, l_run = 0.f;
-    float prev[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) prev[i] = 0.f;
-    for (int c = 0; c <= nchunks; ++c) {
-      float cur[32];
-      if (c < nchunks) {
-        // own partial score of chunk c -> row h of the peer's exchange buffer c & 1
-        ok &= mbar_wait_bounded(&sfull[c & 1], (uint32_t)(c >> 1) & 1u, ok ? kWaitLimit : 0u);
-        tc_fence_after();
-        tmem_ld32(tmem + lane_base + kHalf + 32 * (c & 1), cur);
-        if (c >= 2)  // the peer has read chunk c - 2 out of that buffer
-          ok &= mbar_wait_cluster(&sxe[c & 1], (uint32_t)((c - 2) >> 1) & 1u, ok ? kWaitLimit : 0u);
-        const uint32_t dst = sx_peer + (c & 1) * kSxBytes + h * 128;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)  // 16-byte chunk i of the row at i ^ (h & 7): no bank conflicts
-          st_cluster_v4(dst + 16 * (i ^ (h & 7)), cur[4 * i], cur[4 * i + 1], cur[4 * i + 2], cur[4 * i + 3]);
-        mbar_arrive_remote(sxf_peer + 8 * (c & 1));
-      }
-      if (c >= 1) {
-        const int x = c - 1;
-        ok &= mbar_wait_cluster(&sxf[x & 1], (uint32_t)(x >> 1) & 1u, ok ? kWaitLimit : 0u);
-        const float4* sx = reinterpret_cast<const float4*>(smem + kOffSx + (x & 1) * kSxBytes + h * 128);
-        float sc[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 v = sx[i ^ (h & 7)];
-          sc[4 * i] = prev[4 * i] + v.x, sc[4 * i + 1] = prev[4 * i + 1] + v.y;
-          sc[4 * i + 2] = prev[4 * i + 2] + v.z, sc[4 * i + 3] = prev[4 * i + 3] + v.w;
-        }
-        mbar_arrive_remote(sxe_peer + 8 * (x & 1));
-        const bool tv[2] = {tile_ok(2 * x), tile_ok(2 * x + 1)};
-        float mx = kNegBig;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sc[i] = tv[i >> 4] ? sc[i] : kNegBig;
-          mx = fmaxf(mx, sc[i]);
-        }
-        // lazy rescale; the TMEM accesses are warp-wide, so the whole warp
-        // joins (factor 1 where a head's max did not grow)
-        const bool grow = mx > m_run + 8.f;
-        const float alpha = grow ? ex2f(m_run - mx) : 1.f;
-        if (__any_sync(0xffffffffu, grow && x > 0)) {
-          ok &= mbar_wait_bounded(&pv[(x - 1) & 3], (uint32_t)((x - 1) >> 2) & 1u, ok ? kWaitLimit : 0u);
-          tc_fence_after();
+    {  // query channels [0, 288) of head h into tensor memory: f16 pairs, lane h
+      const uint4* src = reinterpret_cast<const uint4*>(qprep + kQsBytes + (size_t)h * kKT * 2);
 #pragma unroll 1
-          for (int c0 = 0; c0 < kHalf; c0 += 32) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + c0, o);
+      for (int k = 0; k < kKT / 32; ++k) {
+        uint32_t v[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tmem + lane_base + c0, o);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const uint4 x = src[4 * k + i];
+          v[4 * i] = x.x, v[4 * i + 1] = x.y, v[4 * i + 2] = x.z, v[4 * i + 3] = x.w;
         }
-        if (grow) {
-          l_run *= alpha;
-          m_run = mx;
-        }
-        if (x >= 2)  // PV(x - 2) has read P buffer x & 1
-          ok &= mbar_wait_bounded(&pv[(x - 2) & 3], (uint32_t)((x - 2) >> 2) & 1u, ok ? kWaitLimit : 0u);
-        uint32_t pk[16];
-        float ls = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = tv[i >> 3] ? ex2f(sc[2 * i] - m_run) : 0.f;
-          const float p1 = tv[i >> 3] ? ex2f(sc[2 * i + 1] - m_run) : 0.f;
-          ls += p0 + p1;
-          pk[i] = pack_f16x2(p0, p1);
-        }
-        l_run += ls;
-        uint8_t* ps = smem + kOffPs + (x & 1) * kPsBytes;
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8)
-          *reinterpret_cast<uint4*>(ps + (h >> 3) * 512 + g8 * 128 + (h & 7) * 16) =
-              make_uint4(pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
-        proxy_fence();
-        tc_fence_before();
-        mbar_arrive_local(&pfull[x & 1]);
+        tmem_st16(tmem + lane_base + kTmemQ + 16 * k, v);
       }
-      if (c < nchunks) {
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive_local(qt);
+    }
+    float m_run = kNegBig, l_run = 0.f;
+    for (int x = 0; x < nchunks; ++x) {
+      ok &= mbar_wait_bounded(&sfull[x & 1], (uint32_t)(x >> 1) & 1u, ok ? kWaitLimit : 0u);
+      tc_fence_after();
+      float sc[32];
+      tmem_ld32(tmem + lane_base + kTmemS + 32 * (x & 1), sc);
+      const bool tv[2] = {tile_ok(2 * x), tile_ok(2 * x + 1)};
+      float mx = kNegBig;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) prev[i] = cur[i];
+      for (int i = 0; i < 32; ++i) {
+        sc[i] = tv[i >> 4] ? sc[i] : kNegBig;
+        mx = fmaxf(mx, sc[i]);
       }
+      // lazy rescale; the TMEM accesses are warp-wide, so the whole warp
+      // joins (factor 1 where a head's max did not grow)
+      const bool grow = mx > m_run + 8.f;
+      const float alpha = grow ? ex2f(m_run - mx) : 1.f;
+      if (__any_sync(0xffffffffu, grow && x > 0)) {
+        ok &= mbar_wait_bounded(&pv[(x - 1) & 3], (uint32_t)((x - 1) >> 2) & 1u, ok ? kWaitLimit : 0u);
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHalf; c0 += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + c0, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tmem + lane_base + c0, o);
+        }
+      }
+      if (grow) {
+        l_run *= alpha;
+        m_run = mx;
+      }
+      if (x >= 2)  // PV(x - 2) has read P buffer x & 1
+        ok &= mbar_wait_bounded(&pv[(x - 2) & 3], (uint32_t)((x - 2) >> 2) & 1u, ok ? kWaitLimit : 0u);
+      uint32_t pk[16];
+      float ls = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float p0 = tv[i >> 3] ? ex2f(sc[2 * i] - m_run) : 0.f;
+        const float p1 = tv[i >> 3] ? ex2f(sc[2 * i + 1] - m_run) : 0.f;
+        ls += p0 + p1;
+        pk[i] = pack_f16x2(p0, p1);
+      }
+      l_run += ls;
+      tmem_st16(tmem + lane_base + kTmemP + 16 * (x & 1), pk);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive_local(&pfull[x & 1]);
     }
     // ---- epilogue: this split's partial output half, (max, sum) per head
-    float* po = p.part_o + (((size_t)b * p.splits + split) * kH + h) * kLat + rank * kHalf;
+    float* po = p.part_o + (((size_t)b * p.splits + split) * kH + h) * kLat + r * kHalf;
     if (nchunks > 0) {
       const int x = nchunks - 1;
       ok &= mbar_wait_bounded(&pv[x & 3], (uint32_t)(x >> 2) & 1u, ok ? kWaitLimit : 0u);
@@ -483,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
     } else {
       for (int c0 = 0; c0 < kHalf; c0 += 4) *reinterpret_cast<float4*>(po + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (rank == 0) {
+    if (r == 0) {
       float* pm = p.part_ml + (((size_t)b * p.splits + split) * kH + h) * 2;
       pm[0] = m_run;
       pm[1] = l_run;
@@ -492,40 +464,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   if (!ok) set_error(p.err, KVQ_DEVERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // no DSMEM traffic may target a CTA that has exited
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
 
-// Rotated, pre-scaled f16 queries of one (sequence, latent half r), in the
-// K-major core-matrix layout of the score operand: channels [0, 256) hold
-// (H_512 q_lat)[256r + i] * scale * log2(e) / sqrt(512), which is
-// H_256 (q[0:256] + (-1)^r q[256:512]) since H_512 = H_2 (x) H_256; channels
-// [256, 288) hold rope channels [32r, 32r + 32) * scale * log2(e).
-// One warp per head: lane l keeps elements 8l..8l+7; index bits 0..2 are
-// butterflies in registers, bits 3..7 shuffles.
+// Rotated, pre-scaled f16 queries of one sequence: element k of head h is
+// (H_512 q_lat)[k] * scale * log2(e) / sqrt(512) for k < 512 and
+// q_rope[k - 512] * scale * log2(e) after; k in [0, 288) row-major, k in
+// [288, 576) in the shared-memory operand layout.  One warp per head: lane l
+// keeps latent elements 16l..16l+15; index bits 0..3 are butterflies in
+// registers, bits 4..8 shuffles.
 __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
-  const int b = blockIdx.x, r = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* out = p.qprep + ((size_t)b * 2 + r) * kQsBytes;
-  const float sgn = r ? -1.f : 1.f;
+  const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* out_s = p.qprep + (size_t)b * (kQsBytes + kQtBytes);
+  uint8_t* out_t = out_s + kQsBytes;
   const float f = p.scale_log2 * 0.044194173824159216f;  // 1 / sqrt(512)
   for (int h = warp; h < kH; h += 8) {
-    float v[8];
+    float v[16];
     const bool live = h < p.num_q_heads;
-    const uint16_t* qh = p.q + ((size_t)b * p.num_q_heads + (live ? h : 0)) * (kLat + kRope);
-    {
-      const uint4 lo = *reinterpret_cast<const uint4*>(qh + 8 * lane);
-      const uint4 hi = *reinterpret_cast<const uint4*>(qh + kHalf + 8 * lane);
-      const uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w}, c[4] = {hi.x, hi.y, hi.z, hi.w};
+    const uint16_t* qh = p.q + ((size_t)b * p.num_q_heads + (live ? h : 0)) * kKf;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint4 x = *reinterpret_cast<const uint4*>(qh + 16 * lane + 8 * k);
+      const uint32_t a[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        v[2 * e] = live ? bf16f(a[e] & 0xFFFFu) + sgn * bf16f(c[e] & 0xFFFFu) : 0.f;
-        v[2 * e + 1] = live ? bf16f(a[e] >> 16) + sgn * bf16f(c[e] >> 16) : 0.f;
+        v[8 * k + 2 * e] = live ? bf16f(a[e] & 0xFFFFu) : 0.f;
+        v[8 * k + 2 * e + 1] = live ? bf16f(a[e] >> 16) : 0.f;
       }
     }
 #pragma unroll
-    for (int s = 1; s < 8; s <<= 1)
+    for (int s = 1; s < 16; s <<= 1)
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 16; ++i)
         if (!(i & s)) {
           const float x = v[i], y = v[i + s];
           v[i] = x + y;
@@ -535,22 +505,32 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
     for (int off = 1; off < 32; off <<= 1) {
       const bool upper = (lane & off) != 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float o = __shfl_xor_sync(0xffffffffu, v[i], off);
         v[i] = upper ? (o - v[i]) : (v[i] + o);
       }
     }
-    *reinterpret_cast<uint4*>(out + km_off(h, 8 * lane)) =
-        make_uint4(pack_f16x2(v[0] * f, v[1] * f), pack_f16x2(v[2] * f, v[3] * f), pack_f16x2(v[4] * f, v[5] * f),
-                   pack_f16x2(v[6] * f, v[7] * f));
-    if (lane < 4) {
-      const uint4 w = *reinterpret_cast<const uint4*>(qh + kLat + kRopeHalf * r + 8 * lane);
-      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+    uint4 w[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      w[k] = make_uint4(pack_f16x2(v[8 * k] * f, v[8 * k + 1] * f), pack_f16x2(v[8 * k + 2] * f, v[8 * k + 3] * f),
+                        pack_f16x2(v[8 * k + 4] * f, v[8 * k + 5] * f), pack_f16x2(v[8 * k + 6] * f, v[8 * k + 7] * f));
+    const int k0 = 16 * lane;
+    if (k0 < kKT) {
+      *reinterpret_cast<uint4*>(out_t + (size_t)(h * kKT + k0) * 2) = w[0];
+      *reinterpret_cast<uint4*>(out_t + (size_t)(h * kKT + k0 + 8) * 2) = w[1];
+    } else {
+      *reinterpret_cast<uint4*>(out_s + cm_off(h, k0 - kKT, kSboQ)) = w[0];
+      *reinterpret_cast<uint4*>(out_s + cm_off(h, k0 + 8 - kKT, kSboQ)) = w[1];
+    }
+    if (lane < kRope / 8) {
+      const uint4 x = *reinterpret_cast<const uint4*>(qh + kLat + 8 * lane);
+      const uint32_t a[4] = {x.x, x.y, x.z, x.w};
       uint32_t pk[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         pk[e] = live ? pack_f16x2(bf16f(a[e] & 0xFFFFu) * p.scale_log2, bf16f(a[e] >> 16) * p.scale_log2) : 0u;
-      *reinterpret_cast<uint4*>(out + km_off(h, kHalf + 8 * lane)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(out_s + cm_off(h, kLat - kKT + 8 * lane, kSboQ)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
 }
@@ -581,7 +561,7 @@ __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
 
 template <int BITS>
 int launch_mla_bits(const MlaDecodeParams& p, cudaStream_t s) {
-  const int smem = smem_bytes(BITS);
+  const int smem = smem_bytes(BITS, p.tiles_per_split);
   cudaError_t e = cudaFuncSetAttribute(decode_mla_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   cudaLaunchConfig_t cfg = {};
@@ -589,23 +569,16 @@ int launch_mla_bits(const MlaDecodeParams& p, cudaStream_t s) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   return (int)cudaLaunchKernelEx(&cfg, decode_mla_kernel<BITS>, p);
 }
 
 }  // namespace
 
-size_t mla_qprep_bytes(int64_t batch) { return (size_t)batch * 2 * kQsBytes; }
+size_t mla_qprep_bytes(int64_t batch) { return (size_t)batch * (kQsBytes + kQtBytes); }
 
 int launch_decode_mla(const MlaDecodeParams& p, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  mla_prep_q_kernel<<<dim3(p.batch, 2, 1), 256, 0, s>>>(p);
+  mla_prep_q_kernel<<<p.batch, 256, 0, s>>>(p);
   int e = (int)cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (p.bits) {
