@@ -17,9 +17,9 @@
 // MMA's A operand, the other 288 in shared memory.
 //
 // Each CTA is a pipeline of three roles connected by mbarriers:
-//   warp 20 (one thread)  bulk copies of the raw tiles into a ring of stages,
-//                         and the tcgen05 MMAs: S(c) into one of two TMEM
-//                         score buffers, then O += P(c-1) V(c-1);
+//   warp 21 (one thread)  bulk copies of the raw tiles into a ring of stages;
+//   warp 20 (one thread)  the tcgen05 MMAs: S(c) into one of two TMEM score
+//                         buffers, then O += P(c-1) V(c-1);
 //   warps 4-19            dequantise a 32-token chunk, (a q + z) c in fp32,
 //                         to f16 in the no-swizzle core-matrix operand layout
 //                         (three buffers, two at 8 bits, so the dequantisation
@@ -51,7 +51,8 @@ constexpr int kHalf = 256;           // output channels per CTA
 constexpr int kH = 128;              // M: heads (rows beyond num_q_heads are zero)
 constexpr int kChunk = 32;           // tokens per step (two tiles)
 constexpr int kDqWarps = 16;
-constexpr int kThreads = (4 + kDqWarps + 1) * 32;  // softmax 0-3, dequantisation 4-19, copies + MMA 20
+constexpr int kThreads = (4 + kDqWarps + 2) * 32;  // softmax 0-3, dequantisation 4-19, MMA 20, copies 21
+constexpr int kMmaWarp = 4 + kDqWarps, kCopyWarp = kMmaWarp + 1;
 constexpr float kNegBig = -1e30f;
 // TMEM columns: O [0,256), S [256,320), Q [320,464), P [464,496)
 constexpr uint32_t kTmemS = 256, kTmemQ = 320, kTmemP = 464;
@@ -248,12 +249,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 4 + kDqWarps) {
-    // ---------------------------------------------------------------- copies + MMA (one thread)
+  if (warp == kCopyWarp) {
+    // ---------------------------------------------------------------- bulk copies (one thread)
     if (lane == 0) {
       mbar_arrive_expect_tx(qf, kQsBytes);
       bulk_g2s(smem + kOffQs, qprep, kQsBytes, qf);
-      auto issue = [&](int c) {  // raw chunk c into stage c % NS
+      // page ids of chunk c (two tiles); the loop loads them one chunk ahead
+      auto pages_of = [&](int c, int (&pg)[2]) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) pg[j] = 2 * c + j < ntl ? btab[2 * c + j] : -1;
+      };
+      auto issue = [&](int c, const int (&pg)[2]) {  // raw chunk c into stage c % NS
         uint64_t* bar = &full[c % NS];
         uint8_t* st = smem + kOffSt + (c % NS) * SB;
         uint32_t bytes = 0;
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (!tile_ok(2 * c + j)) continue;
-          const size_t slot = (size_t)p.layer * p.num_pages + btab[2 * c + j];
+          const size_t slot = (size_t)p.layer * p.num_pages + pg[j];
           bulk_g2s(st + j * CB, p.codes + slot * CB, CB, bar);
           bulk_g2s(st + kStAz + j * kT * 8, p.tok + slot * kT * 2, kT * 8, bar);
           bulk_g2s(st + kStC + j * kLat * 4, p.chan + slot * kLat, kLat * 4, bar);
@@ -272,7 +278,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
         }
       };
       const int pre = nchunks < NS ? nchunks : NS;
-      for (int c = 0; c < pre; ++c) issue(c);
+      for (int c = 0; c < pre; ++c) {
+        int pg[2];
+        pages_of(c, pg);
+        issue(c, pg);
+      }
+      int pg_next[2];
+      pages_of(NS, pg_next);
+      for (int c = 0; c + NS < nchunks; ++c) {
+        // chunk c is dequantised: its stage is free again
+        ok &= mbar_wait_bounded(&dq[c % NB], (uint32_t)(c / NB) & 1u, ok ? kWaitLimit : 0u);
+        proxy_fence();
+        issue(c + NS, pg_next);
+        pages_of(c + NS + 1, pg_next);  // in flight until the next chunk
+      }
+      ok &= mbar_wait_bounded(qf, 0u, ok ? kWaitLimit : 0u);
+      // no bulk copy may still be writing when the CTA exits
+      for (int c = nchunks > NS ? nchunks - NS : 0; c < nchunks; ++c)
+        ok &= mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, ok ? kWaitLimit : 0u);
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA (one thread)
+    if (lane == 0) {
       const uint32_t idesc_s = (1u << 4) | ((uint32_t)(kChunk >> 3) << 17) | ((uint32_t)(kH >> 4) << 24);
       const uint32_t idesc_pv = (1u << 4) | (1u << 16) | ((uint32_t)(kHalf >> 3) << 17) | ((uint32_t)(kH >> 4) << 24);
       const uint64_t dq0 = umma_desc(s_base + kOffQs, 128, kSboQ), dk0 = umma_desc(s_base + kOffKb, 128, kSboK);
@@ -281,12 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       ok &= mbar_wait_bounded(qt, 0u, ok ? kWaitLimit : 0u);
       for (int c = 0; c <= nchunks; ++c) {
         if (c < nchunks) {
-          // chunk c is dequantised; its raw stage is free again
           ok &= mbar_wait_bounded(&dq[c % NB], (uint32_t)(c / NB) & 1u, ok ? kWaitLimit : 0u);
-          if (c + NS < nchunks) {
-            proxy_fence();
-            issue(c + NS);
-          }
           tc_fence_after();
           // descriptors advance by 256 B (16 in the address field) per 16-channel step
           const uint64_t dk = dk0 + (uint64_t)((c % NB) * (kKbBytes >> 4));
@@ -311,9 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
           umma_commit(&pv[x & 3]);
         }
       }
-      // no bulk copy may still be writing when the CTA exits
-      for (int c = nchunks > NS ? nchunks - NS : 0; c < nchunks; ++c)
-        ok &= mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, ok ? kWaitLimit : 0u);
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- dequantisation
