@@ -150,19 +150,79 @@ __device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLau
   }
 }
 
+// Channel bits 0..6 of the 128-channel block: bits 3..6 on the tensor cores
+// (16 MMAs), bits 0..2 as three butterfly stages on fp32 pairs.
+template <bool F16>
+__device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const uint32_t (&afrag)[4], f2 (&P)[2][2][8]) {
+  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const uint32_t sel = (b & 1) ? 0x7632u : 0x5410u;
+      float d[4];
+      mma16816<F16>(d, afrag, __byte_perm(L[h][0][b >> 1], L[h][1][b >> 1], sel),
+                    __byte_perm(L[h][2][b >> 1], L[h][3][b >> 1], sel), zero4);
+      P[h][0][b] = make_float2(d[0], d[1]);
+      P[h][1][b] = make_float2(d[2], d[3]);
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int m3 = 0; m3 < 2; ++m3)
+#pragma unroll
+      for (int s = 1; s < 8; s <<= 1)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (b & s) continue;
+          const f2 x = P[h][m3][b], y = P[h][m3][b + s];
+          P[h][m3][b] = add2(x, y);
+          P[h][m3][b + s] = sub2(x, y);
+        }
+}
+
+// Raw tile of 16 tokens x 128 channels staged per lane in shared memory by
+// cp.async: slot [h * 4 + l][lane] holds what load_tile keeps in L[h][l].
+__device__ __forceinline__ void stage_tile(uint4 (*dst)[32], const QuantLaunch& p, uint32_t tile, int g, int t,
+                                           int lane, int32_t& page) {
+  const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
+  const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
+  page = __ldg(p.dst_page + tt);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint16_t* row = p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * kBlk + 8 * t;
+#pragma unroll
+    for (int l = 0; l < 4; ++l)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&dst[h * 4 + l][lane])), "l"(row + 32 * l)
+                   : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void read_staged(const uint4 (*src)[32], int lane, uint32_t (&L)[2][4][4]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 v = src[i][lane];
+    L[i >> 2][i & 3][0] = v.x, L[i >> 2][i & 3][1] = v.y, L[i >> 2][i & 3][2] = v.z, L[i >> 2][i & 3][3] = v.w;
+  }
+}
+
 template <int W>
 __device__ __forceinline__ void tile_sync() {
   if constexpr (W > 1) __syncthreads();  // one tile per CTA when its blocks span warps
 }
 
 template <bool F16, int BITS, int D>
-__global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(QuantLaunch p) {
+__global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(QuantLaunch p) {
   constexpr int W = D / kBlk;     // warps per tile
   constexpr int TPC = kWarps / W; // tiles per CTA
-  constexpr bool kPark = (W == 1);  // park the rotated tile in shared memory during the rounds
+  // head_dim 128: the raw tiles are staged in shared memory by cp.async (the
+  // next one while the current one is processed) and the rotated tile is
+  // recomputed from the raw one after the rounds instead of being held in
+  // registers, which keeps the kernel at 128 registers (four CTAs per SM).
+  constexpr bool kStage = (W == 1);
   __shared__ WarpScratch scratch[kWarps];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
-  __shared__ float4 parked[kPark ? kWarps : 1][16][32];
+  __shared__ uint4 staged[kStage ? kWarps : 1][2][8][32];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int warp = threadIdx.x >> 5, blk = warp % W, slot_id = warp / W;
   const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
@@ -173,32 +233,30 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
   afrag[1] = sign_pair<F16>(g + 8, 2 * t);
   afrag[2] = sign_pair<F16>(g, 2 * t + 8);
   afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8);
-  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
   const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.044194173824159216f;
   const uint32_t stride = gridDim.x * TPC;
   uint32_t tile = blockIdx.x * TPC + slot_id;
   if (tile >= p.total) return;  // every warp of a tile leaves together
   uint32_t L[2][4][4];
   int32_t page;
-  load_tile<D>(L, p, tile, blk, g, t, page);
-  for (; tile < p.total; tile += stride) {
+  if constexpr (kStage)
+    stage_tile(staged[warp][0], p, tile, g, t, lane, page);
+  else
+    load_tile<D>(L, p, tile, blk, g, t, page);
+  for (int buf = 0; tile < p.total; tile += stride, buf ^= 1) {
     f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b of the block
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const uint32_t sel = (b & 1) ? 0x7632u : 0x5410u;
-        float d[4];
-        mma16816<F16>(d, afrag, __byte_perm(L[h][0][b >> 1], L[h][1][b >> 1], sel),
-                      __byte_perm(L[h][2][b >> 1], L[h][3][b >> 1], sel), zero4);
-        P[h][0][b] = make_float2(d[0], d[1]);
-        P[h][1][b] = make_float2(d[2], d[3]);
-      }
     const int32_t cur_page = page;
+    if constexpr (kStage) {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");  // this lane's copies of the current tile
+      read_staged(staged[warp][buf], lane, L);
+      if (tile + stride < p.total) stage_tile(staged[warp][buf ^ 1], p, tile + stride, g, t, lane, page);
+    }
+    hadamard128<F16>(L, afrag, P);
     const uint32_t cur = tile;
     const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
     const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
-    if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
+    if constexpr (!kStage)
+      if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
     if (cur_page < 0 || cur_page >= p.num_pages) {  // same decision in every warp of the tile
       if (lane == 0 && blk == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       continue;
@@ -211,19 +269,6 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
       for (int i = lane * 8; i < kT * rd; i += 32 * 8)
         *reinterpret_cast<uint4*>(rdst + i) = *reinterpret_cast<const uint4*>(rs + i);
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int m3 = 0; m3 < 2; ++m3)
-#pragma unroll
-        for (int s = 1; s < 8; s <<= 1)
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            if (b & s) continue;
-            const f2 x = P[h][m3][b], y = P[h][m3][b + s];
-            P[h][m3][b] = add2(x, y);
-            P[h][m3][b + s] = sub2(x, y);
-          }
     if constexpr (W > 1) {  // channel bits 7, 8: H_4 across the four blocks of the tile
 #pragma unroll
       for (int i = 0; i < 32; ++i) sh.x[blk][i][lane] = P[i >> 4][(i >> 3) & 1][i & 7];
@@ -249,14 +294,6 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
         A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
         A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
       }
-    // park the rotated values in shared memory until the factors are known
-    if constexpr (kPark) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const f2 x = P[i >> 3][(i >> 2) & 1][2 * (i & 3)], y = P[i >> 3][(i >> 2) & 1][2 * (i & 3) + 1];
-        parked[warp][i][lane] = make_float4(x.x, x.y, y.x, y.y);
-      }
-    }
     float w[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 1.f;
@@ -344,13 +381,9 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 3 : 1)) quantize_kernel(
           make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
-      if constexpr (kPark) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 x = parked[warp][i][lane];
-          P[i >> 3][(i >> 2) & 1][2 * (i & 3)] = make_float2(x.x, x.y);
-          P[i >> 3][(i >> 2) & 1][2 * (i & 3) + 1] = make_float2(x.z, x.w);
-        }
+      if constexpr (kStage) {  // the rotated tile again, from the staged raw tile
+        read_staged(staged[warp][buf], lane, L);
+        hadamard128<F16>(L, afrag, P);
       }
       __syncwarp();
 #pragma unroll
@@ -495,7 +528,7 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* strea
     q.rope_dim = p.rope_dim;
     const int tpc = head_dim == 128 ? kWarps : kWarps / (head_dim / kBlk);
     const int64_t need = (per_kind + tpc - 1) / tpc;
-    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 3 : 4);
+    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 4 : 2);  // resident CTAs per SM
     const int grid = (int)(need < cap ? need : cap);
     int e;
     if (head_dim == 128)
