@@ -47,6 +47,8 @@ constexpr int kBlk = 128;                  // channels per warp (one 128-channel
 constexpr int kT = 16;
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
+template <int D>
+constexpr int log2_dt() { return D == 128 ? 3 : 5; }  // log2(d / T)
 constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer (ties to even)
 
 // Channel bits carried by the MMA contraction index k = 2t + j0 + 8*j1
@@ -71,6 +73,12 @@ __device__ __forceinline__ float rcp_nr(float x) {
   float r;
   asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
   return fmaf(r, fmaf(-x, r, 1.f), r);
+}
+// 1/x from the hardware approximation alone (for the per-round factors).
+__device__ __forceinline__ float rcp_fast(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 __device__ __forceinline__ float rsqrt_nr(float x) {
   float y;
@@ -216,13 +224,15 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
   constexpr int W = D / kBlk;     // warps per tile
   constexpr int TPC = kWarps / W; // tiles per CTA
   // head_dim 128: the raw tiles are staged in shared memory by cp.async (the
-  // next one while the current one is processed) and the rotated tile is
-  // recomputed from the raw one after the rounds instead of being held in
-  // registers, which keeps the kernel at 128 registers (four CTAs per SM).
+  // next one while the current one is processed) and the rotated tile waits
+  // out the rounds in tensor memory (64 columns of the warp's lane quarter),
+  // which keeps the kernel at 128 registers (four CTAs per SM).
   constexpr bool kStage = (W == 1);
+  constexpr int kLogDT = log2_dt<D>();
   __shared__ WarpScratch scratch[kWarps];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
   __shared__ uint4 staged[kStage ? kWarps : 1][2][8][32];
+  __shared__ uint32_t tmem_slot;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int warp = threadIdx.x >> 5, blk = warp % W, slot_id = warp / W;
   const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
@@ -236,13 +246,26 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
   const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.044194173824159216f;
   const uint32_t stride = gridDim.x * TPC;
   uint32_t tile = blockIdx.x * TPC + slot_id;
-  if (tile >= p.total) return;  // every warp of a tile leaves together
+  if constexpr (!kStage)
+    if (tile >= p.total) return;  // every warp of a tile leaves together
+  uint32_t tpark = 0;             // this warp's 64 TMEM columns
+  if constexpr (kStage) {
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;" ::"r"(smem_u32(&tmem_slot)));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    tpark = tmem_slot + ((uint32_t)(warp * 32) << 16);
+  }
   uint32_t L[2][4][4];
-  int32_t page;
-  if constexpr (kStage)
-    stage_tile(staged[warp][0], p, tile, g, t, lane, page);
-  else
+  int32_t page = 0;
+  if constexpr (kStage) {
+    if (tile < p.total) stage_tile(staged[warp][0], p, tile, g, t, lane, page);
+  } else {
     load_tile<D>(L, p, tile, blk, g, t, page);
+  }
   for (int buf = 0; tile < p.total; tile += stride, buf ^= 1) {
     f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b of the block
     const int32_t cur_page = page;
@@ -294,6 +317,18 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
         A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
         A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
       }
+    if constexpr (kStage) {  // park the rotated tile in tensor memory until the factors are known
+      float v[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const f2 x = P[half][i >> 3][i & 7];
+          v[2 * i] = x.x, v[2 * i + 1] = x.y;
+        }
+        tmem_st32(tpark + 32 * half, v);
+      }
+    }
     float w[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 1.f;
@@ -329,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
         for (int k = 1; k < W; ++k) rk += sh.row[it & 1][k][tok];
       }
       // a zero row (rk = 0) only ever multiplies zeros, so its factor may be anything finite
-      v_own = (float)D * rcp_nr(fmaxf(rk, 1e-30f));
+      v_own = rcp_fast(fmaxf(rk, 1e-30f));
       float v[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -352,10 +387,10 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
         c23 = add2(c23, make_float2(x.z, x.w));
       }
       // likewise a zero column; its stored factor is set to 1 after the rounds
-      w_own.x = (float)kT * rcp_nr(fmaxf(c01.x, 1e-30f));
-      w_own.y = (float)kT * rcp_nr(fmaxf(c01.y, 1e-30f));
-      w_own.z = (float)kT * rcp_nr(fmaxf(c23.x, 1e-30f));
-      w_own.w = (float)kT * rcp_nr(fmaxf(c23.y, 1e-30f));
+      w_own.x = rcp_fast(fmaxf(c01.x, 1e-30f));
+      w_own.y = rcp_fast(fmaxf(c01.y, 1e-30f));
+      w_own.z = rcp_fast(fmaxf(c23.x, 1e-30f));
+      w_own.w = rcp_fast(fmaxf(c23.y, 1e-30f));
       sc.own[lane] = w_own;
       __syncwarp();
 #pragma unroll
@@ -367,11 +402,15 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
     }
     {
       const bool norm = p.iters > 0;
+      // The rounds use v = 1 / R and w = 1 / C instead of d / R and T / C:
+      // every factor then differs from the textbook one by a power of two,
+      // and after n rounds c^2 = C / T = C' (d / T)^n, an exact scaling.
+      const float c2_scale = ldexpf(1.f, kLogDT * p.iters);
       const float ct[4] = {c01.x, c01.y, c23.x, c23.y};
       float cv[4], ic[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float x = ct[i] * (1.f / kT);
+        const float x = ct[i] * c2_scale;
         const float y = rsqrt_nr(x);
         const bool ok = norm && ct[i] > 0.f;
         ic[i] = ok ? y : 1.f;
@@ -381,9 +420,14 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
           make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
-      if constexpr (kStage) {  // the rotated tile again, from the staged raw tile
-        read_staged(staged[warp][buf], lane, L);
-        hadamard128<F16>(L, afrag, P);
+      if constexpr (kStage) {  // the rotated tile back from tensor memory
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float v[32];
+          tmem_ld32(tpark + 32 * half, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) P[half][i >> 3][i & 7] = make_float2(v[2 * i], v[2 * i + 1]);
+        }
       }
       __syncwarp();
 #pragma unroll
@@ -475,6 +519,11 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
       }
     }
     tile_sync<W>();  // shared tile buffers are reused by the next tile
+  }
+  if constexpr (kStage) {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;" ::"r"(tmem_slot));
   }
 }
 
