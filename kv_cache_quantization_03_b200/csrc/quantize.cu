@@ -220,14 +220,15 @@ __device__ __forceinline__ void tile_sync() {
 }
 
 template <bool F16, int BITS, int D>
-__global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(QuantLaunch p) {
+__global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(QuantLaunch p) {
   constexpr int W = D / kBlk;     // warps per tile
   constexpr int TPC = kWarps / W; // tiles per CTA
-  // head_dim 128: the raw tiles are staged in shared memory by cp.async (the
-  // next one while the current one is processed) and the rotated tile waits
-  // out the rounds in tensor memory (64 columns of the warp's lane quarter),
-  // which keeps the kernel at 128 registers (four CTAs per SM).
+  // The rotated tile waits out the rounds in tensor memory (64 columns of the
+  // warp's lane quarter).  At head_dim 128 the raw tiles are also staged in
+  // shared memory by cp.async (the next one while the current one is
+  // processed), which keeps that kernel at 128 registers (four CTAs per SM).
   constexpr bool kStage = (W == 1);
+  constexpr bool kPark = true;
   constexpr int kLogDT = log2_dt<D>();
   __shared__ WarpScratch scratch[kWarps];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
@@ -246,10 +247,8 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
   const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.044194173824159216f;
   const uint32_t stride = gridDim.x * TPC;
   uint32_t tile = blockIdx.x * TPC + slot_id;
-  if constexpr (!kStage)
-    if (tile >= p.total) return;  // every warp of a tile leaves together
   uint32_t tpark = 0;             // this warp's 64 TMEM columns
-  if constexpr (kStage) {
+  if constexpr (kPark) {
     if (warp == 0) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;" ::"r"(smem_u32(&tmem_slot)));
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -264,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
   if constexpr (kStage) {
     if (tile < p.total) stage_tile(staged[warp][0], p, tile, g, t, lane, page);
   } else {
-    load_tile<D>(L, p, tile, blk, g, t, page);
+    if (tile < p.total) load_tile<D>(L, p, tile, blk, g, t, page);
   }
   for (int buf = 0; tile < p.total; tile += stride, buf ^= 1) {
     f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b of the block
@@ -317,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
         A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
         A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
       }
-    if constexpr (kStage) {  // park the rotated tile in tensor memory until the factors are known
+    if constexpr (kPark) {  // park the rotated tile in tensor memory until the factors are known
       float v[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -420,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
           make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
-      if constexpr (kStage) {  // the rotated tile back from tensor memory
+      if constexpr (kPark) {  // the rotated tile back from tensor memory
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float v[32];
@@ -520,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 1)) quantize_kernel(
     }
     tile_sync<W>();  // shared tile buffers are reused by the next tile
   }
-  if constexpr (kStage) {
+  if constexpr (kPark) {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;" ::"r"(tmem_slot));
@@ -577,7 +576,7 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* strea
     q.rope_dim = p.rope_dim;
     const int tpc = head_dim == 128 ? kWarps : kWarps / (head_dim / kBlk);
     const int64_t need = (per_kind + tpc - 1) / tpc;
-    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 4 : 2);  // resident CTAs per SM
+    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 4 : 3);  // resident CTAs per SM
     const int grid = (int)(need < cap ? need : cap);
     int e;
     if (head_dim == 128)
