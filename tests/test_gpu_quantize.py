@@ -108,6 +108,28 @@ def test_quantize_bad_page_sets_error_and_skips_tile():
     _check_all(run, tiles=[0, 2, 3])
 
 
+@pytest.mark.parametrize("name", ["rt1k", "mla"])
+def test_quantize_single_tile(name):
+    # One tile per call: at head_dim 128 three of the CTA's four warps have no
+    # tile and go straight to the CTA's final barrier; at 512 one CTA works.
+    w = W.WORKLOADS[name].scaled(batch=1, seq_len=16)
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
+
+
+def test_mla_quantize_bad_page_sets_error_and_skips_tile():
+    # head_dim 512: the four warps of a tile leave it together on a bad page
+    w = W.WORKLOADS["mla"].scaled(batch=1, seq_len=64)
+    pages = np.array([0, 9, 2, 3], dtype=np.int32)        # pool of 4 pages: 9 is out of range
+    run = QuantRun(w, quantize=False, pages=pages, num_pages=4)
+    run.cache.codes("k")[0, 1].fill_(0xA5)
+    run.quantize()
+    assert run.error_bits() & 0x1
+    assert torch.all(run.cache.codes("k")[0, 1] == 0xA5)
+    _check_all(run, tiles=[0, 2, 3])
+
+
 def test_mla_rope_rows_copied_to_their_pages():
     w = W.WORKLOADS["mla"].scaled(batch=2, seq_len=128)
     run = QuantRun(w)
