@@ -255,8 +255,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_
   if (!bytes || batch < 0 || num_q_heads <= 0 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
   const int64_t pairs = (int64_t)batch * c->num_kv_heads;
   const int64_t max_tiles = ((int64_t)max_seq_len + c->tile_tokens - 1) / c->tile_tokens;
+  const int nh = decode_kv_heads_per_cta(num_q_heads / c->num_kv_heads, c->num_kv_heads);
   *bytes = c->mla ? decode_ws_bytes_mla(batch, decode_plan_mla(batch, max_tiles))
-                  : decode_ws_bytes(pairs, decode_plan(pairs, max_tiles), c->head_dim);
+                  : decode_ws_bytes(pairs, decode_plan(pairs / nh, max_tiles), c->head_dim);
   return KVQ_OK;
 }
 
@@ -312,7 +313,8 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
   if (group > kMaxGroup || c->bits_v == 3) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;
   const int64_t pairs = (int64_t)batch * c->num_kv_heads;
-  const DecodePlan plan = decode_plan(pairs, max_pages_per_seq);
+  // one CTA covers decode_kv_heads_per_cta adjacent kv-heads of a sequence
+  const DecodePlan plan = decode_plan(pairs / decode_kv_heads_per_cta(group, c->num_kv_heads), max_pages_per_seq);
   const size_t need = decode_ws_bytes(pairs, plan, c->head_dim);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return workspace_bytes < need ? KVQ_ERR_WORKSPACE_TOO_SMALL : KVQ_ERR_INVALID_ARG;

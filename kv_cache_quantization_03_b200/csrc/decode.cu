@@ -42,16 +42,20 @@ struct StageLayout {
   int kcb, vcb, off_kaz, off_kc, off_v, off_vaz, off_vc, bytes;
 };
 
-__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv) {
-  return StageLayout{kT * kD * bk / 8,
-                     kT * kD * bv / 8,
-                     kT * kD * bk / 8,
-                     kT * kD * bk / 8 + kT * 8,
-                     kT * kD * bk / 8 + kT * 8 + kD * 4,
-                     kT * kD * bk / 8 + kT * 8 + kD * 4 + kT * kD * bv / 8,
-                     kT * kD * bk / 8 + kT * 8 + kD * 4 + kT * kD * bv / 8 + kT * 8,
-                     kT * kD * (bk + bv) / 8 + 2 * (kT * 8 + kD * 4)};
+// One stage: the tile of nh adjacent kv-heads (their pages are contiguous in
+// every cache array): K codes | K (a, z) | K c | V codes | V (a, z) | V c.
+__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv, int nh) {
+  return StageLayout{nh * kT * kD * bk / 8,
+                     nh * kT * kD * bv / 8,
+                     nh * (kT * kD * bk / 8),
+                     nh * (kT * kD * bk / 8 + kT * 8),
+                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4),
+                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4) + nh * kT * kD * bv / 8,
+                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4) + nh * (kT * kD * bv / 8 + kT * 8),
+                     nh * (kT * kD * (bk + bv) / 8 + 2 * (kT * 8 + kD * 4))};
 }
+// Ring depth per warp: 3 stages of one kv-head, 2 of a pair (four CTAs per SM).
+__host__ __device__ constexpr int num_stages(int nh) { return nh == 2 ? 2 : kStages; }
 
 // ---- code pairs -> f16x2 (exact small integers)
 // A field of a 32-bit word masked in place in both halves and OR-ed into the
@@ -200,10 +204,19 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-template <int BK, int BV>
+// NH = 1: one kv-head per CTA, its (up to 8) query heads on the MMA's 8
+// columns.  NH = 2 (groups of at most 4 query heads): two adjacent kv-heads
+// per CTA; head slot n (column n of the MMAs) is query head n % 4 of kv-head
+// n / 4.  Lane (g, t) computes u for slot g and owns the score/output columns
+// 2t, 2t+1, i.e. kv-head hs = t / 2.  The score MMAs run once per kv-head
+// (each lane keeps the result of its own kv-head); for P V each kv-head's
+// weights are masked to its own columns, so both MMAs add into one result.
+template <int BK, int BV, int NH>
 __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr StageLayout SL = stage_layout(BK, BV);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH);
+  constexpr int kStages = num_stages(NH);
+  constexpr int KCB = SL.kcb / NH, VCB = SL.vcb / NH;  // code bytes of one kv-head's tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDW * kStages * SL.bytes);
   uint8_t* wsm = smem + warp * kStages * SL.bytes;
@@ -215,8 +228,8 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   }
   __syncwarp();
 
-  const int pair = blockIdx.y;
-  const int b = pair / p.num_kv_heads, kvh = pair % p.num_kv_heads;
+  const int kvh_per_seq = p.num_kv_heads / NH;
+  const int b = blockIdx.y / kvh_per_seq, kvh = (blockIdx.y % kvh_per_seq) * NH;  // first kv-head of the CTA
   const int split = blockIdx.x;
   int seq = p.seq_lens[b];
   if (seq < 0) {
@@ -245,8 +258,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   // lane (g, t) computes head g, channels 32t..32t+31)
   if (warp == 0) {
     float qr[32];
-    const bool live = g < p.group;
-    const uint16_t* qp = p.q + ((size_t)b * p.num_q_heads + (size_t)kvh * p.group + (live ? g : 0)) * kD + 32 * t;
+    const int hh = NH == 2 ? (g & 3) : g, hk = NH == 2 ? kvh + (g >> 2) : kvh;  // slot g: head hh of kv-head hk
+    const bool live = hh < p.group;
+    const uint16_t* qp = p.q + ((size_t)b * p.num_q_heads + (size_t)hk * p.group + (live ? hh : 0)) * kD + 32 * t;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint4 w = *reinterpret_cast<const uint4*>(qp + 8 * k);
@@ -296,12 +310,12 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     }
     const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_kv_heads + kvh;
     mbar_arrive_expect_tx(bar, (uint32_t)SL.bytes);
-    bulk_g2s(st, p.k.codes + slot * SL.kcb, SL.kcb, bar);
-    bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), kT * 8, bar);
-    bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, kD * 4, bar);
-    bulk_g2s(st + SL.off_v, p.v.codes + slot * SL.vcb, SL.vcb, bar);
-    bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), kT * 8, bar);
-    bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, kD * 4, bar);
+    bulk_g2s(st, p.k.codes + slot * KCB, SL.kcb, bar);
+    bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), NH * kT * 8, bar);
+    bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, NH * kD * 4, bar);
+    bulk_g2s(st + SL.off_v, p.v.codes + slot * VCB, SL.vcb, bar);
+    bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), NH * kT * 8, bar);
+    bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, NH * kD * 4, bar);
   };
   const int pre = my_n < kStages ? my_n : kStages;
   for (int i = 0; i < pre; ++i) issue(i);
@@ -325,10 +339,11 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     const int page = spg[warp + i * kDW];
     if (page >= 0 && page < p.num_pages) {
       const uint8_t* st = wsm + (i % kStages) * SL.bytes;
-      const float* kaz = reinterpret_cast<const float*>(st + SL.off_kaz);
-      const float* kc = reinterpret_cast<const float*>(st + SL.off_kc);
-      const float* vaz = reinterpret_cast<const float*>(st + SL.off_vaz);
-      const float* vc = reinterpret_cast<const float*>(st + SL.off_vc);
+      const int hu = NH == 2 ? (g >> 2) : 0, hs = NH == 2 ? (t >> 1) : 0;  // kv-head of this lane's u / columns
+      const float* kaz = reinterpret_cast<const float*>(st + SL.off_kaz) + hs * 2 * kT;
+      const float* kc = reinterpret_cast<const float*>(st + SL.off_kc) + hu * kD;
+      const float* vaz = reinterpret_cast<const float*>(st + SL.off_vaz) + hs * 2 * kT;
+      const float* vc = reinterpret_cast<const float*>(st + SL.off_vc) + hs * kD;
 
       // u = q~ * c_K on this lane's 32 channels (slot order), and its sum
       float u[32];
@@ -359,18 +374,25 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       const float su0 = __shfl_sync(0xffffffffu, su, 8 * t);       // head 2t
       const float su1 = __shfl_sync(0xffffffffu, su, 8 * t + 4);   // head 2t+1
 
-      // scores: tokens g, g+8 x heads 2t, 2t+1
-      uint32_t kp0[16], kp1[16];
-      key_pairs<BK>(st, g, t, kp0);
-      key_pairs<BK>(st, g + 8, t, kp1);
-      float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f};  // two independent MMA chains
+      // scores: tokens g, g+8 x heads 2t, 2t+1 (each kv-head's codes against all
+      // columns; a lane keeps its own kv-head's result)
+      float S[4];
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint32_t a[4] = {kp0[2 * s], kp1[2 * s], kp0[2 * s + 1], kp1[2 * s + 1]};
-        mma16816<true>(Sh, a, ubh[2 * s], ubh[2 * s + 1], Sh);
-        mma16816<true>(Sl, a, ubl[2 * s], ubl[2 * s + 1], Sl);
+      for (int h = 0; h < NH; ++h) {
+        uint32_t kp0[16], kp1[16];
+        key_pairs<BK>(st + h * KCB, g, t, kp0);
+        key_pairs<BK>(st + h * KCB, g + 8, t, kp1);
+        float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f};  // two independent MMA chains
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint32_t a[4] = {kp0[2 * s], kp1[2 * s], kp0[2 * s + 1], kp1[2 * s + 1]};
+          mma16816<true>(Sh, a, ubh[2 * s], ubh[2 * s + 1], Sh);
+          mma16816<true>(Sl, a, ubl[2 * s], ubl[2 * s + 1], Sl);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (h == 0 || hs == h) S[e] = Sh[e] + Sl[e];
       }
-      const float S[4] = {Sh[0] + Sl[0], Sh[1] + Sl[1], Sh[2] + Sl[2], Sh[3] + Sl[3]};
       const float2 az0 = *reinterpret_cast<const float2*>(kaz + 2 * g);
       const float2 az1 = *reinterpret_cast<const float2*>(kaz + 2 * (g + 8));
       float sc[4];
@@ -414,9 +436,6 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       wh1 = movmatrix_trans(wh1), wl1 = movmatrix_trans(wl1);
 
       // values: channels 16g + [0,16) x heads 2t, 2t+1
-      uint32_t vp0[16], vp1[16];
-      value_pairs<BV>(st + SL.off_v, 2 * t, 2 * t + 1, g, vp0);
-      value_pairs<BV>(st + SL.off_v, 2 * t + 8, 2 * t + 9, g, vp1);
       float cv[16];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -429,13 +448,23 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
         for (int mb = 0; mb < 8; ++mb) O[mb][0] = mul2(O[mb][0], alpha), O[mb][1] = mul2(O[mb][1], alpha);
       }
 #pragma unroll
-      for (int mb = 0; mb < 8; ++mb) {
-        const uint32_t a[4] = {vp0[2 * mb], vp0[2 * mb + 1], vp1[2 * mb], vp1[2 * mb + 1]};
-        float d[4];
-        mma16816<true>(d, a, wh0, wh1, zero4);
-        mma16816<true>(d, a, wl0, wl1, d);
-        O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, make_float2(d[0], d[1]), bz), O[mb][0]);
-        O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, make_float2(d[2], d[3]), bz), O[mb][1]);
+      for (int h = 0; h < NH; ++h) {
+        // B fragments of kv-head h: lane (g, t) holds column g, zero outside h's columns
+        const bool mine = NH == 1 || (g >> 2) == h;
+        const uint32_t bh0 = mine ? wh0 : 0u, bh1 = mine ? wh1 : 0u, bl0 = mine ? wl0 : 0u, bl1 = mine ? wl1 : 0u;
+        const f2 bzh = (NH == 1 || hs == h) ? bz : make_float2(0.f, 0.f);
+        uint32_t vp0[16], vp1[16];
+        value_pairs<BV>(st + SL.off_v + h * VCB, 2 * t, 2 * t + 1, g, vp0);
+        value_pairs<BV>(st + SL.off_v + h * VCB, 2 * t + 8, 2 * t + 9, g, vp1);
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) {
+          const uint32_t a[4] = {vp0[2 * mb], vp0[2 * mb + 1], vp1[2 * mb], vp1[2 * mb + 1]};
+          float d[4];
+          mma16816<true>(d, a, bh0, bh1, zero4);
+          mma16816<true>(d, a, bl0, bl1, d);
+          O[mb][0] = fma2(splat2(cv[2 * mb]), fma2(am, make_float2(d[0], d[1]), bzh), O[mb][0]);
+          O[mb][1] = fma2(splat2(cv[2 * mb + 1]), fma2(am, make_float2(d[2], d[3]), bzh), O[mb][1]);
+        }
       }
     }
     __syncwarp();
@@ -473,9 +502,11 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     ml[(warp * 8 + 2 * t + 1) * 2] = mrun[1], ml[(warp * 8 + 2 * t + 1) * 2 + 1] = lrun[1];
   }
   __syncthreads();
-  const size_t pbase = ((size_t)pair * p.splits + split) * 8;
   const int ch = threadIdx.x;  // kDW * 32 == 128 == kD
-  for (int h = 0; h < p.group; ++h) {
+  for (int h = 0; h < 8; ++h) {  // head slot h: query head h % 4 of kv-head kvh + h / 4 when NH = 2
+    const int hh = NH == 2 ? (h & 3) : h, hk = NH == 2 ? kvh + (h >> 2) : kvh;
+    if (hh >= p.group) continue;
+    const size_t pbase = (((size_t)b * p.num_kv_heads + hk) * p.splits + split) * 8 + hh;
     float mx = kNegBig;
 #pragma unroll
     for (int w = 0; w < kDW; ++w) mx = fmaxf(mx, ml[(w * 8 + h) * 2]);
@@ -486,10 +517,10 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       acc = fmaf(f, mo[(w * 8 + h) * kD + ch], acc);
       l = fmaf(f, ml[(w * 8 + h) * 2 + 1], l);
     }
-    p.part_o[(pbase + h) * kD + ch] = acc;
+    p.part_o[pbase * kD + ch] = acc;
     if (ch == 0) {
-      p.part_ml[(pbase + h) * 2] = mx;
-      p.part_ml[(pbase + h) * 2 + 1] = l;
+      p.part_ml[pbase * 2] = mx;
+      p.part_ml[pbase * 2 + 1] = l;
     }
   }
 }
@@ -524,16 +555,17 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
   }
 }
 
-template <int BK, int BV>
+template <int BK, int BV, int NH>
 int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
-  constexpr StageLayout SL = stage_layout(BK, BV);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH);
+  constexpr int kStages = num_stages(NH);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
   const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) + 8 * kQStride * 4 +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
-  auto kern = decode_d128_kernel<BK, BV>;
+  auto kern = decode_d128_kernel<BK, BV, NH>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  dim3 grid(p.splits, p.batch * p.num_kv_heads);
+  dim3 grid(p.splits, p.batch * p.num_kv_heads / NH);
   kern<<<grid, kDW * 32, smem, s>>>(p);
   combine_d128_kernel<<<p.batch * p.num_kv_heads, kD, 0, s>>>(p);
   return (int)cudaGetLastError();
@@ -541,11 +573,14 @@ int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
 
 }  // namespace
 
+int decode_kv_heads_per_cta(int group, int num_kv_heads) { return (group <= 4 && num_kv_heads % 2 == 0) ? 2 : 1; }
+
 int launch_decode_d128(const DecodeParams& p, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bk = p.k.bits, bv = p.v.bits;
+  const bool pairs = decode_kv_heads_per_cta(p.group, p.num_kv_heads) == 2;
 #define KVQ_CASE(K, V) \
-  if (bk == K && bv == V) return launch_bk_bv<K, V>(p, s);
+  if (bk == K && bv == V) return pairs ? launch_bk_bv<K, V, 2>(p, s) : launch_bk_bv<K, V, 1>(p, s);
   KVQ_CASE(4, 4) KVQ_CASE(3, 4) KVQ_CASE(2, 4) KVQ_CASE(8, 4)
   KVQ_CASE(4, 2) KVQ_CASE(3, 2) KVQ_CASE(2, 2) KVQ_CASE(8, 2)
   KVQ_CASE(4, 8) KVQ_CASE(3, 8) KVQ_CASE(2, 8) KVQ_CASE(8, 8)

@@ -99,6 +99,8 @@ struct MlaDecodeParams {
 int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* stream);
 int launch_dequantize(const DequantParams& p, int head_dim, void* stream);
 int launch_decode_d128(const DecodeParams& p, void* stream);
+// kv-heads one GQA decode CTA covers (2 for groups of at most 4 query heads)
+int decode_kv_heads_per_cta(int group, int num_kv_heads);
 int launch_decode_mla(const MlaDecodeParams& p, void* stream);
 size_t mla_qprep_bytes(int64_t batch);  // workspace for the prepared MLA queries
 
