@@ -35,7 +35,6 @@ constexpr int kD = 128;
 constexpr int kT = 16;
 constexpr int kDW = 4;      // warps per CTA
 constexpr int kStages = 3;  // ring depth per warp
-constexpr int kQStride = 132;  // floats per head row of the shared rotated query (padded: no bank conflicts)
 constexpr float kNegBig = -1e30f;
 
 struct StageLayout {
@@ -246,17 +245,25 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   const int t1 = min(t0 + p.tiles_per_split, ntiles);
   const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
   // this split's page ids, staged once in shared memory
-  float* qs = reinterpret_cast<float*>(bars + kDW * kStages);     // [8][kQStride] rotated query
-  int32_t* spg = reinterpret_cast<int32_t*>(qs + 8 * kQStride);
+  int32_t* spg = reinterpret_cast<int32_t*>(bars + kDW * kStages);
   {
     const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
     for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[i];
   }
+  __shared__ uint32_t tmem_slot;
+  if (warp == 0) {  // 32 TMEM columns: each warp keeps its lanes' rotated query in its lane quarter
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 32;" ::"r"(smem_u32(&tmem_slot)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tq = tmem_slot + ((uint32_t)(warp * 32) << 16);
 
-  // ---- rotated, pre-scaled query of the CTA's 8 heads into shared memory (warp 0:
-  // lane (g, t) computes head g, channels 32t..32t+31)
-  if (warp == 0) {
+  // ---- rotated, pre-scaled query of the CTA's 8 heads: lane (g, t) computes head
+  // slot g, channels 32t..32t+31, puts them in its slot order (through this
+  // warp's not-yet-used stage memory) and keeps them in tensor memory
+  {
     float qr[32];
     const int hh = NH == 2 ? (g & 3) : g, hk = NH == 2 ? kvh + (g >> 2) : kvh;  // slot g: head hh of kv-head hk
     const bool live = hh < p.group;
@@ -290,12 +297,17 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       }
     }
     const float f = p.scale_log2 * 0.08838834764831845f;  // softmax scale * log2(e) / sqrt(128)
+    float* scr = reinterpret_cast<float*>(wsm) + lane * 33;
 #pragma unroll
-    for (int i = 0; i < 32; i += 4)
-      *reinterpret_cast<float4*>(qs + g * kQStride + 32 * t + i) =
-          make_float4(qr[i] * f, qr[i + 1] * f, qr[i + 2] * f, qr[i + 3] * f);
+    for (int i = 0; i < 32; ++i) scr[i] = qr[i] * f;
+    __syncwarp();
+    const int rot = rot_channels<BK>(t);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qr[i] = scr[(i + rot) & 31];
+    __syncwarp();
+    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the stage refills
+    tmem_st32(tq, qr);
   }
-  __syncthreads();
 
   // ---- producer: lane 0 fills stage (i % kStages) with local tile i
   auto issue = [&](int i) {
@@ -350,14 +362,14 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       f2 su2 = make_float2(0.f, 0.f);
       {
         const int rq = rot_channels<BK>(t) >> 2;
-        const float* qg = qs + g * kQStride + 32 * t;
+        float qv[32];  // slot order
+        tmem_ld32(tq, qv);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int kk = 4 * ((k + rq) & 7);
           const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + kk);
-          const float4 q4 = *reinterpret_cast<const float4*>(qg + kk);
-          const f2 a = mul2(make_float2(q4.x, q4.y), make_float2(c4.x, c4.y));
-          const f2 d = mul2(make_float2(q4.z, q4.w), make_float2(c4.z, c4.w));
+          const f2 a = mul2(make_float2(qv[4 * k], qv[4 * k + 1]), make_float2(c4.x, c4.y));
+          const f2 d = mul2(make_float2(qv[4 * k + 2], qv[4 * k + 3]), make_float2(c4.z, c4.w));
           su2 = add2(su2, add2(a, d));
           u[4 * k] = a.x, u[4 * k + 1] = a.y, u[4 * k + 2] = d.x, u[4 * k + 3] = d.y;
         }
@@ -486,7 +498,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     lrun[0] += __shfl_xor_sync(0xffffffffu, lrun[0], off);
     lrun[1] += __shfl_xor_sync(0xffffffffu, lrun[1], off);
   }
-  __syncthreads();  // every warp is done with its stages
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();  // every warp is done with its stages and its tensor memory
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 32;" ::"r"(tmem_slot));
   float* mo = reinterpret_cast<float*>(smem);                  // [kDW][8 heads][128]
   float* ml = mo + kDW * 8 * kD;                               // [kDW][8][2]
 #pragma unroll
@@ -561,7 +575,7 @@ int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
   constexpr int kStages = num_stages(NH);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
-  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) + 8 * kQStride * 4 +
+  const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
   auto kern = decode_d128_kernel<BK, BV, NH>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
