@@ -1,7 +1,7 @@
 """Helpers of the parity tests: run the CUDA path through the C ABI, run the
 float64 oracle on the same seeded inputs, compare with the stated tolerances.
 
-Tolerances (the benchmark spec's, readings as stated in the oracle's header):
+Tolerances (readings as stated in the oracle's header):
 * codes: identical, except +-1 flips where the oracle's (y - m) / s lies within
   1e-4 of a half-integer (a rounding tie the float32 kernel may resolve the
   other way); such flips on at most 1e-5 of the elements;
