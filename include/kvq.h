@@ -59,10 +59,11 @@
  *   chan_scale: float32 [d] = c per channel;
  *   rope (MLA): bf16 [layer][page][T][rope_dim], unquantised.
  *
- * Supported on the GPU: head_dim 128 (GQA) or 512 (MLA latent), tile_tokens
- * 16, bits_k in {2,3,4,8}, bits_v in {2,4,8}, query group size 1..8 for GQA
- * and 1..128 heads for MLA; inputs fp16 or bf16.  Other shapes return
- * KVQ_ERR_UNSUPPORTED.
+ * Supported on the GPU: head_dim 128 (GQA) with tile_tokens 16, 32, 64 or
+ * 128 (the shipped "4-bit Keys, 2-bit Values Preset" uses 128), or 512 (MLA
+ * latent) with tile_tokens 16; bits_k in {2,3,4,8}, bits_v in {2,4,8}, query
+ * group size 1..8 for GQA and 1..128 heads for MLA; inputs fp16 or bf16.
+ * Other shapes return KVQ_ERR_UNSUPPORTED.
  */
 #ifndef KVQ_H_
 #define KVQ_H_
@@ -98,7 +99,7 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
 typedef struct kvq_config {
   int32_t head_dim;       /* d: 128 (GQA) or 512 (MLA latent); power of two */
   int32_t num_kv_heads;   /* H_kv (1 for MLA) */
-  int32_t tile_tokens;    /* T == page size in tokens (16) */
+  int32_t tile_tokens;    /* T == page size in tokens (16; 32, 64, 128 at head_dim 128) */
   int32_t bits_k;         /* key (MLA: latent) code width: 2, 3, 4 or 8 */
   int32_t bits_v;         /* value code width: 2, 4 or 8; ignored when mla */
   int32_t sinkhorn_iters; /* n >= 0 normalisation rounds (0 = rotation + RTN only) */

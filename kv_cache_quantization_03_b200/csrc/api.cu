@@ -40,12 +40,19 @@ kvq_status check_config(const kvq_config* c) {
   return KVQ_OK;
 }
 
-// Shapes the quantize and dequantize kernels are built for: 16-token tiles,
-// head_dim 128 for K/V caches, 512 for an MLA latent.
+// Shapes the kernels are built for: head_dim 128 K/V caches with tiles of
+// 16, 32, 64 or 128 tokens; a 512-wide MLA latent with 16-token tiles.
 kvq_status check_gpu_shape(const kvq_config* c) {
-  if (c->tile_tokens != 16) return KVQ_ERR_UNSUPPORTED;
   if (c->head_dim != (c->mla ? 512 : 128)) return KVQ_ERR_UNSUPPORTED;
+  if (c->mla ? c->tile_tokens != 16 : (c->tile_tokens < 16 || c->tile_tokens > 128)) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
+}
+
+// 16-token decode tiles per page, as a power of two.
+int sub_log2(const kvq_config* c) {
+  int s = 0;
+  while ((16 << s) < c->tile_tokens) ++s;
+  return s;
 }
 
 // Shapes the decode kernels are built for (MLA: 512-channel latent, 64 rope).
@@ -219,7 +226,7 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.rope_dst = cache->rope;
   p.rope_dim = c->rope_dim;
   if (p.rope_src && !aligned16(p.rope_src)) return KVQ_ERR_INVALID_ARG;
-  return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, stream));
+  return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, c->tile_tokens, stream));
 }
 
 kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
@@ -242,6 +249,7 @@ kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int3
   p.pages = pages;
   p.n_pages = n_pages;
   p.unrotate = unrotate ? 1 : 0;
+  p.tile_tokens = c->tile_tokens;
   p.out[0] = k_out;
   p.out[1] = v_out;
   p.err = dev_error;
@@ -257,7 +265,7 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_
   const int64_t max_tiles = ((int64_t)max_seq_len + c->tile_tokens - 1) / c->tile_tokens;
   const int nh = decode_kv_heads_per_cta(num_q_heads / c->num_kv_heads, c->num_kv_heads);
   *bytes = c->mla ? decode_ws_bytes_mla(batch, decode_plan_mla(batch, max_tiles))
-                  : decode_ws_bytes(pairs, decode_plan(pairs / nh, max_tiles), c->head_dim);
+                  : decode_ws_bytes(pairs, decode_plan(pairs / nh, max_tiles << sub_log2(c)), c->head_dim);
   return KVQ_OK;
 }
 
@@ -314,7 +322,8 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
   if (batch == 0) return KVQ_OK;
   const int64_t pairs = (int64_t)batch * c->num_kv_heads;
   // one CTA covers decode_kv_heads_per_cta adjacent kv-heads of a sequence
-  const DecodePlan plan = decode_plan(pairs / decode_kv_heads_per_cta(group, c->num_kv_heads), max_pages_per_seq);
+  const DecodePlan plan = decode_plan(pairs / decode_kv_heads_per_cta(group, c->num_kv_heads),
+                                      (int64_t)max_pages_per_seq << sub_log2(c));
   const size_t need = decode_ws_bytes(pairs, plan, c->head_dim);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return workspace_bytes < need ? KVQ_ERR_WORKSPACE_TOO_SMALL : KVQ_ERR_INVALID_ARG;
@@ -338,6 +347,7 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
   p.part_ml = p.part_o + (size_t)pairs * plan.splits * kMaxGroup * c->head_dim;
   p.splits = plan.splits;
   p.tiles_per_split = plan.tiles_per_split;
+  p.sub_log2 = sub_log2(c);
   p.err = dev_error;
   return cuda_status(launch_decode_d128(p, stream));
 }

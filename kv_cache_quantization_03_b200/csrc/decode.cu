@@ -1,5 +1,5 @@
-// Decode attention over the quantised cache, head_dim 128, 16-token pages,
-// query groups of 1..8 heads per kv-head (sm_100a).
+// Decode attention over the quantised cache, head_dim 128, pages of 16..128
+// tokens, query groups of 1..8 heads per kv-head (sm_100a).
 //
 // Consumer of the KVarN cache (KVarN project page on open-radar, Key
 // Features, "Variance-Normalized Quantization Pipeline" and "Throughput Above
@@ -11,10 +11,13 @@
 //   out_h      += c_V * (sum_t w_th qv_t + sum_t p_th z_t),  w_th = p_th a_t
 // with an online softmax across tiles, then the output is rotated back.
 //
-// Work split: grid (splits, batch * kv_heads).  Each CTA of 4 warps owns a
-// contiguous range of one sequence's tiles; each warp takes every 4th tile
-// and streams it through its own ring of shared-memory stages filled with
-// 1-D bulk async copies (one mbarrier per stage, bounded waits).  Both
+// Work split: grid (splits, batch * kv_heads).  The unit of work is a tile of
+// 16 tokens: a whole page, or one of the 16-token slices of a longer page
+// (each slice reads its rows of codes and token scales and the page's channel
+// scales).  Each CTA of 4 warps owns a contiguous range of one sequence's
+// tiles; each warp takes every 4th tile and streams it through its own ring
+// of shared-memory stages filled with 1-D bulk async copies (one mbarrier per
+// stage, bounded waits).  Both
 // contractions of a tile run as m16n8k16 f16 MMAs with fp32 accumulation:
 // codes 0..255 are exact in f16; u and w are each carried as an f16 pair
 // hi + lo (two MMAs into one fp32 accumulator), which keeps ~22 significant
@@ -235,20 +238,22 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     if (threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
     seq = 0;
   }
-  int ntiles = seq / kT;
-  if ((seq % kT) && threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_PARTIAL_TILE);
-  if (ntiles > p.max_pages) {
+  const int page_tokens = kT << p.sub_log2;
+  int npages = seq / page_tokens;
+  if ((seq % page_tokens) && threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_PARTIAL_TILE);
+  if (npages > p.max_pages) {
     if (threadIdx.x == 0 && split == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
-    ntiles = p.max_pages;
+    npages = p.max_pages;
   }
+  const int ntiles = npages << p.sub_log2;  // 16-token tiles
   const int t0 = split * p.tiles_per_split;
   const int t1 = min(t0 + p.tiles_per_split, ntiles);
   const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
-  // this split's page ids, staged once in shared memory
+  // the page id of each of this split's tiles, staged once in shared memory
   int32_t* spg = reinterpret_cast<int32_t*>(bars + kDW * kStages);
   {
-    const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
-    for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[i];
+    const int32_t* btab = p.block_table + (size_t)b * p.max_pages;
+    for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[(t0 + i) >> p.sub_log2];
   }
   __shared__ uint32_t tmem_slot;
   if (warp == 0) {  // 32 TMEM columns: each warp keeps its lanes' rotated query in its lane quarter
@@ -314,7 +319,8 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     if (lane != 0) return;
     uint64_t* bar = &wbar[i % kStages];
     uint8_t* st = wsm + (i % kStages) * SL.bytes;
-    const int page = spg[warp + i * kDW];
+    const int li = warp + i * kDW;
+    const int page = spg[li];
     if (page < 0 || page >= p.num_pages) {
       set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       mbar_arrive_expect_tx(bar, 0);
@@ -322,12 +328,34 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     }
     const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_kv_heads + kvh;
     mbar_arrive_expect_tx(bar, (uint32_t)SL.bytes);
-    bulk_g2s(st, p.k.codes + slot * KCB, SL.kcb, bar);
-    bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), NH * kT * 8, bar);
-    bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, NH * kD * 4, bar);
-    bulk_g2s(st + SL.off_v, p.v.codes + slot * VCB, SL.vcb, bar);
-    bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), NH * kT * 8, bar);
-    bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, NH * kD * 4, bar);
+    if (p.sub_log2 == 0) {  // 16-token pages: the nh kv-heads' pages are contiguous in every array
+      bulk_g2s(st, p.k.codes + slot * KCB, SL.kcb, bar);
+      bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), NH * kT * 8, bar);
+      bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, NH * kD * 4, bar);
+      bulk_g2s(st + SL.off_v, p.v.codes + slot * VCB, SL.vcb, bar);
+      bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), NH * kT * 8, bar);
+      bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, NH * kD * 4, bar);
+      return;
+    }
+    // longer pages: slice `sub` of each kv-head's page, in the same stage layout
+    const int spt = 1 << p.sub_log2, sub = (t0 + li) & (spt - 1);
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const size_t sh = slot + h;
+      const uint8_t* kc = p.k.codes + sh * (size_t)(spt * KCB);
+      if constexpr (BK == 3) {  // the slice's rows of the low-bit plane, then of the high-bit plane
+        bulk_g2s(st + h * KCB, kc + sub * (kT * kD / 4), kT * kD / 4, bar);
+        bulk_g2s(st + h * KCB + kT * kD / 4, kc + spt * (kT * kD / 4) + sub * (kT * kD / 8), kT * kD / 8, bar);
+      } else {
+        bulk_g2s(st + h * KCB, kc + sub * KCB, KCB, bar);
+      }
+      bulk_g2s(st + SL.off_kaz + h * (kT * 8), p.k.tok + (sh * spt + sub) * (kT * 2), kT * 8, bar);
+      bulk_g2s(st + SL.off_kc + h * (kD * 4), p.k.chan + sh * kD, kD * 4, bar);
+      static_assert(BV != 3, "3-bit values have two planes");
+      bulk_g2s(st + SL.off_v + h * VCB, p.v.codes + (sh * spt + sub) * VCB, VCB, bar);
+      bulk_g2s(st + SL.off_vaz + h * (kT * 8), p.v.tok + (sh * spt + sub) * (kT * 2), kT * 8, bar);
+      bulk_g2s(st + SL.off_vc + h * (kD * 4), p.v.chan + sh * kD, kD * 4, bar);
+    }
   };
   const int pre = my_n < kStages ? my_n : kStages;
   for (int i = 0; i < pre; ++i) issue(i);

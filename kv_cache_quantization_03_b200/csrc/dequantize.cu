@@ -10,13 +10,13 @@
 namespace kvq {
 namespace {
 
-constexpr int kT = 16;
+constexpr int kT = 16;  // rows per pass
 
 template <int kD>
-__device__ __forceinline__ uint32_t read_code(const uint8_t* codes, int bits, int tok, int ch) {
+__device__ __forceinline__ uint32_t read_code(const uint8_t* codes, int bits, int T, int tok, int ch) {
   if (bits == 3) {
     const uint32_t lo = (codes[tok * (kD / 4) + ch / 4] >> (2 * (ch % 4))) & 3u;
-    const uint32_t hi = (codes[kT * (kD / 4) + tok * (kD / 8) + ch / 8] >> (ch % 8)) & 1u;
+    const uint32_t hi = (codes[T * (kD / 4) + tok * (kD / 8) + ch / 8] >> (ch % 8)) & 1u;
     return lo | (hi << 2);
   }
   const int bit = (tok * kD + ch) * bits;
@@ -38,27 +38,32 @@ __global__ void __launch_bounds__(kD) dequantize_kernel(DequantParams p) {
     return;
   }
   const CacheArrays src = p.src[kind];
+  const int T = p.tile_tokens;
   const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_heads + head;
-  const uint8_t* codes = src.codes + slot * (kT * kD * src.bits / 8);
-  const float* tok = src.tok + slot * kT * 2;
+  const uint8_t* codes = src.codes + slot * ((size_t)T * kD * src.bits / 8);
+  const float* tok = src.tok + slot * T * 2;
   const float c = src.chan[slot * kD + ch];
-  for (int r = 0; r < kT; ++r)
-    tile[r][ch] = fmaf(tok[2 * r], (float)read_code<kD>(codes, src.bits, r, ch), tok[2 * r + 1]) * c;
-  __syncthreads();
-  if (p.unrotate) {
-    for (int r = 0; r < kT; ++r) {
-      for (int s = 1; s < kD; s <<= 1) {
-        const float x = tile[r][ch & ~s], y = tile[r][ch | s];
-        __syncthreads();
-        tile[r][ch] = (ch & s) ? (x - y) : (x + y);
-        __syncthreads();
-      }
-      tile[r][ch] *= rsqrtf((float)kD);
-    }
+  float* out = p.out[kind] + (((size_t)pi * p.num_heads + head) * T) * kD;
+  for (int r0 = 0; r0 < T; r0 += kT) {  // kT rows at a time
+    for (int r = 0; r < kT; ++r)
+      tile[r][ch] =
+          fmaf(tok[2 * (r0 + r)], (float)read_code<kD>(codes, src.bits, T, r0 + r, ch), tok[2 * (r0 + r) + 1]) * c;
     __syncthreads();
+    if (p.unrotate) {
+      for (int r = 0; r < kT; ++r) {
+        for (int s = 1; s < kD; s <<= 1) {
+          const float x = tile[r][ch & ~s], y = tile[r][ch | s];
+          __syncthreads();
+          tile[r][ch] = (ch & s) ? (x - y) : (x + y);
+          __syncthreads();
+        }
+        tile[r][ch] *= rsqrtf((float)kD);
+      }
+      __syncthreads();
+    }
+    for (int r = 0; r < kT; ++r) out[(r0 + r) * kD + ch] = tile[r][ch];
+    __syncthreads();  // the tile is rewritten by the next rows
   }
-  float* out = p.out[kind] + (((size_t)pi * p.num_heads + head) * kT) * kD;
-  for (int r = 0; r < kT; ++r) out[r * kD + ch] = tile[r][ch];
 }
 
 }  // namespace

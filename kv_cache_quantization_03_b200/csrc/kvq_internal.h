@@ -46,6 +46,7 @@ struct DequantParams {
   const int32_t* pages;
   int64_t n_pages;
   int unrotate;
+  int tile_tokens;      // T: rows per page (a multiple of 16)
   float* out[2];
   uint32_t* err;
 };
@@ -67,7 +68,8 @@ struct DecodeParams {
   float* part_o;                // [B*Hkv][splits][8][d]  un-normalised partial outputs
   float* part_ml;               // [B*Hkv][splits][8][2]  (max, sum) in log2 units
   int splits;
-  int tiles_per_split;
+  int tiles_per_split;          // in 16-token sub-tiles
+  int sub_log2;                 // log2(16-token sub-tiles per page): 0 for 16-token pages, 3 for 128
   uint32_t* err;
 };
 
@@ -96,7 +98,7 @@ struct MlaDecodeParams {
 };
 
 // Launchers (defined in the .cu files); return a cudaError_t value.
-int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* stream);
+int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, int tile_tokens, void* stream);
 int launch_dequantize(const DequantParams& p, int head_dim, void* stream);
 int launch_decode_d128(const DecodeParams& p, void* stream);
 // kv-heads one GQA decode CTA covers (2 for groups of at most 4 query heads)

@@ -1,14 +1,16 @@
-// Quantize-append for head_dim 128 (GQA) and 512 (MLA latent), 16-token tiles
-// (sm_100a).
+// Quantize-append for head_dim 128 (GQA; tiles of 16, 32, 64 or 128 tokens)
+// and 512 (MLA latent; 16-token tiles) (sm_100a).
 //
-// Computes, per tile of 16 tokens x 128 channels of one (layer, kv-head,
+// Computes, per tile of T tokens x d channels of one (layer, kv-head,
 // K-or-V), the KVarN pipeline (KVarN project page on open-radar, Key
 // Features, "Variance-Normalized Quantization Pipeline"): Hadamard rotation
 // along head_dim, Sinkhorn-like row/column second-moment normalisation,
 // per-token asymmetric round-to-nearest, packing into the tile's cache page.
 //
-// One warp owns one 128-channel block of a tile (head_dim 128: the whole
-// tile; 512: four warps share a tile).  Lane (g = lane/4, t = lane%4) ends up
+// One warp owns 16 tokens x one 128-channel block of a tile (head_dim 128,
+// T = 16: the whole tile; 512: four warps share a tile across channels;
+// T = 16 TW: TW warps share it across tokens, and their column sums are added
+// through shared memory once per round).  Lane (g = lane/4, t = lane%4) ends up
 // holding the rotated values of tokens {2t, 2t+1, 2t+8, 2t+9} and channels
 // 16g..16g+15 of its block (register pairs hold the two tokens 8h + 2t,
 // 8h + 2t + 1 of one channel).  For 512 channels, H_512 = H_4 (x) H_128: each
@@ -44,11 +46,14 @@ namespace kvq {
 namespace {
 
 constexpr int kBlk = 128;                  // channels per warp (one 128-channel block of a tile)
-constexpr int kT = 16;
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-template <int D>
-constexpr int log2_dt() { return D == 128 ? 3 : 5; }  // log2(d / T)
+constexpr int kT = 16;                     // tokens per warp
+constexpr int kWarps = 4;                  // warps per CTA, unless a tile needs more
+// Warps per CTA: four, or one tile's TW token slices when that is more.
+template <int TW>
+constexpr int cta_warps() { return TW > kWarps ? TW : kWarps; }
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+template <int D, int TW>
+constexpr int log2_dt() { return ilog2(D) - ilog2(kT * TW); }  // log2(d / T), may be <= 0
 constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer (ties to even)
 
 // Channel bits carried by the MMA contraction index k = 2t + j0 + 8*j1
@@ -147,7 +152,7 @@ __device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLau
   const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
   page = __ldg(p.dst_page + tt);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < 2; ++h) {  // (16-token tiles only)
     const uint16_t* row = p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * D +
                           kBlk * blk + 8 * t;
 #pragma unroll
@@ -189,16 +194,20 @@ __device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const 
         }
 }
 
-// Raw tile of 16 tokens x 128 channels staged per lane in shared memory by
-// cp.async: slot [h * 4 + l][lane] holds what load_tile keeps in L[h][l].
-__device__ __forceinline__ void stage_tile(uint4 (*dst)[32], const QuantLaunch& p, uint32_t tile, int g, int t,
+// Raw 16 tokens x 128 channels (token slice wt of a tile of TW slices)
+// staged per lane in shared memory by cp.async: slot [h * 4 + l][lane] holds
+// what load_tile keeps in L[h][l].
+template <int TW>
+__device__ __forceinline__ void stage_tile(uint4 (*dst)[32], const QuantLaunch& p, uint32_t tile, int wt, int g, int t,
                                            int lane, int32_t& page) {
   const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
   const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
   page = __ldg(p.dst_page + tt);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint16_t* row = p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * kBlk + 8 * t;
+    const uint16_t* row =
+        p.src + (((size_t)layer * p.n_tok + (size_t)tt * (kT * TW) + kT * wt + 8 * h + g) * p.num_heads + head) * kBlk +
+        8 * t;
 #pragma unroll
     for (int l = 0; l < 4; ++l)
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&dst[h * 4 + l][lane])), "l"(row + 32 * l)
@@ -218,24 +227,40 @@ template <int W>
 __device__ __forceinline__ void tile_sync() {
   if constexpr (W > 1) __syncthreads();  // one tile per CTA when its blocks span warps
 }
+// The TW warps of one tile (tile slot `slot` of the CTA) meet at a named barrier.
+template <int TW>
+__device__ __forceinline__ void slice_sync(int slot) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(TW * 32) : "memory");
+}
 
-template <bool F16, int BITS, int D>
-__global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(QuantLaunch p) {
-  constexpr int W = D / kBlk;     // warps per tile
-  constexpr int TPC = kWarps / W; // tiles per CTA
+// Raw-tile staging buffers of a CTA (dynamic shared memory): two tiles per warp.
+template <int TW>
+constexpr size_t stage_bytes() { return (size_t)cta_warps<TW>() * 2 * 8 * 32 * sizeof(uint4); }
+
+template <bool F16, int BITS, int D, int TW>
+__global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_warps<TW>() : 3))
+    quantize_kernel(QuantLaunch p) {
+  static_assert(TW == 1 || D == kBlk, "tiles longer than 16 tokens need head_dim 128");
+  constexpr int kCW = cta_warps<TW>();
+  constexpr int W = D / kBlk;     // warps per tile along channels
+  constexpr int kTile = kT * TW;  // tokens per tile
+  constexpr int TPC = kCW / (W * TW);  // tiles per CTA
   // The rotated tile waits out the rounds in tensor memory (64 columns of the
   // warp's lane quarter).  At head_dim 128 the raw tiles are also staged in
   // shared memory by cp.async (the next one while the current one is
   // processed), which keeps that kernel at 128 registers (four CTAs per SM).
   constexpr bool kStage = (W == 1);
   constexpr bool kPark = true;
-  constexpr int kLogDT = log2_dt<D>();
-  __shared__ WarpScratch scratch[kWarps];
+  constexpr int kLogDT = log2_dt<D, TW>();
+  constexpr int kTmemCols = 64 * (kCW / 4);  // 64 columns per warp, four lane quarters
+  __shared__ WarpScratch scratch[kCW];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
-  __shared__ uint4 staged[kStage ? kWarps : 1][2][8][32];
+  __shared__ float4 colw[TW > 1 ? TPC : 1][2][TW][32];  // column partials of the token slices, by round parity
+  extern __shared__ uint4 dyn_smem[];
+  uint4(*staged)[2][8][32] = reinterpret_cast<uint4(*)[2][8][32]>(dyn_smem);  // [kCW] when kStage
   __shared__ uint32_t tmem_slot;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int warp = threadIdx.x >> 5, blk = warp % W, slot_id = warp / W;
+  const int warp = threadIdx.x >> 5, blk = warp % W, wt = (warp / W) % TW, slot_id = warp / (W * TW);
   const int b1 = (lane >> 3) & 1, b2 = (lane >> 4) & 1;
   WarpScratch& sc = scratch[warp];
   TileShare& sh = share[0];
@@ -250,18 +275,21 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
   uint32_t tpark = 0;             // this warp's 64 TMEM columns
   if constexpr (kPark) {
     if (warp == 0) {
-      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;" ::"r"(smem_u32(&tmem_slot)));
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                   "n"(kTmemCols));
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    tpark = tmem_slot + ((uint32_t)(warp * 32) << 16);
+    // a warp reaches the TMEM lanes 32 (warp % 4) .. +31 only
+    tpark = tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) + 64 * (warp >> 2);
   }
   uint32_t L[2][4][4];
   int32_t page = 0;
+  uint32_t rounds = 0;  // rounds done by this warp (parity of the column-partial buffer)
   if constexpr (kStage) {
-    if (tile < p.total) stage_tile(staged[warp][0], p, tile, g, t, lane, page);
+    if (tile < p.total) stage_tile<TW>(staged[warp][0], p, tile, wt, g, t, lane, page);
   } else {
     if (tile < p.total) load_tile<D>(L, p, tile, blk, g, t, page);
   }
@@ -271,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
     if constexpr (kStage) {
       asm volatile("cp.async.wait_group 0;" ::: "memory");  // this lane's copies of the current tile
       read_staged(staged[warp][buf], lane, L);
-      if (tile + stride < p.total) stage_tile(staged[warp][buf ^ 1], p, tile + stride, g, t, lane, page);
+      if (tile + stride < p.total) stage_tile<TW>(staged[warp][buf ^ 1], p, tile + stride, wt, g, t, lane, page);
     }
     hadamard128<F16>(L, afrag, P);
     const uint32_t cur = tile;
@@ -280,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
     if constexpr (!kStage)
       if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
     if (cur_page < 0 || cur_page >= p.num_pages) {  // same decision in every warp of the tile
-      if (lane == 0 && blk == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+      if (lane == 0 && blk == 0 && wt == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       continue;
     }
     const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;
@@ -385,6 +413,20 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
         c01 = add2(c01, make_float2(x.x, x.y));
         c23 = add2(c23, make_float2(x.z, x.w));
       }
+      if constexpr (TW > 1) {  // add the token slices' sums, in slice order (same result in every warp)
+        float4(*cw)[32] = colw[slot_id][rounds & 1];
+        cw[wt][lane] = make_float4(c01.x, c01.y, c23.x, c23.y);
+        slice_sync<TW>(slot_id);
+        float4 x = cw[0][lane];
+        c01 = make_float2(x.x, x.y), c23 = make_float2(x.z, x.w);
+#pragma unroll
+        for (int k = 1; k < TW; ++k) {
+          x = cw[k][lane];
+          c01 = add2(c01, make_float2(x.x, x.y));
+          c23 = add2(c23, make_float2(x.z, x.w));
+        }
+        ++rounds;
+      }
       // likewise a zero column; its stored factor is set to 1 after the rounds
       w_own.x = rcp_fast(fmaxf(c01.x, 1e-30f));
       w_own.y = rcp_fast(fmaxf(c01.y, 1e-30f));
@@ -415,8 +457,9 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
         ic[i] = ok ? y : 1.f;
         cv[i] = ok ? x * y : 1.f;
       }
-      *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
-          make_float4(cv[0], cv[1], cv[2], cv[3]);
+      if (wt == 0)
+        *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
+            make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
       if constexpr (kPark) {  // the rotated tile back from tensor memory
@@ -476,9 +519,9 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
     const float s_own = (omx - omn) / kQmax;
     const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
     if ((lane & 4) == 0 && blk == 0)
-      *reinterpret_cast<float2*>(p.dst.tok + slot * (kT * 2) + 2 * (8 * b2 + 2 * t + b1)) =
+      *reinterpret_cast<float2*>(p.dst.tok + slot * (kTile * 2) + 2 * (kT * wt + 8 * b2 + 2 * t + b1)) =
           make_float2(s_own * inv_sqrt_d, omn * inv_sqrt_d);
-    uint8_t* codes = p.dst.codes + slot * (kT * D * BITS / 8);
+    uint8_t* codes = p.dst.codes + slot * (kTile * D * BITS / 8);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const f2 m2 = make_float2(__shfl_sync(0xffffffffu, omn, (h << 4) | t),
@@ -496,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
       }
 #pragma unroll
       for (int tp = 0; tp < 2; ++tp) {
-        const int tok = 8 * h + 2 * t + tp;
+        const int tok = kT * wt + 8 * h + 2 * t + tp;  // row of the tile
         const uint32_t* f = q[tp];
         constexpr int row_bytes = D * BITS / 8, seg = kBlk * BITS / 8;
         if constexpr (BITS == 4) {
@@ -513,7 +556,8 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
 #pragma unroll
           for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
           *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
-          *reinterpret_cast<uint16_t*>(codes + kT * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) = (uint16_t)hi;
+          *reinterpret_cast<uint16_t*>(codes + kTile * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) =
+              (uint16_t)hi;
         }
       }
     }
@@ -522,7 +566,8 @@ __global__ void __launch_bounds__(kThreads, (D == 128 ? 4 : 3)) quantize_kernel(
   if constexpr (kPark) {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;" ::"r"(tmem_slot));
+    if (warp == 0)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "n"(kTmemCols));
   }
 }
 
@@ -535,27 +580,54 @@ FastDiv make_div(uint32_t d) {
   return f;
 }
 
-template <bool F16, int D>
-int launch_bits(const QuantLaunch& q, int bits, int grid, cudaStream_t s) {
+template <bool F16, int BITS, int D, int TW>
+void launch_one(const QuantLaunch& q, int sms, cudaStream_t s) {
+  constexpr int kCW = cta_warps<TW>(), tpc = kCW / ((D / kBlk) * TW);
+  constexpr size_t dyn = D == kBlk ? stage_bytes<TW>() : 0;  // raw-tile staging at head_dim 128
+  const int64_t need = (q.total + tpc - 1) / tpc;
+  const int64_t cap = (int64_t)sms * (D == kBlk ? 16 / kCW : 3);  // resident CTAs per SM
+  const int grid = (int)(need < cap ? need : cap);
+  auto kern = quantize_kernel<F16, BITS, D, TW>;
+  // static + dynamic shared memory may pass 48 KB, which needs the opt-in
+  if (dyn > 0) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  kern<<<grid, kCW * 32, dyn, s>>>(q);
+}
+
+template <bool F16, int D, int TW>
+int launch_bits(const QuantLaunch& q, int bits, int sms, cudaStream_t s) {
   switch (bits) {
-    case 2: quantize_kernel<F16, 2, D><<<grid, kThreads, 0, s>>>(q); break;
-    case 3: quantize_kernel<F16, 3, D><<<grid, kThreads, 0, s>>>(q); break;
-    case 4: quantize_kernel<F16, 4, D><<<grid, kThreads, 0, s>>>(q); break;
-    case 8: quantize_kernel<F16, 8, D><<<grid, kThreads, 0, s>>>(q); break;
+    case 2: launch_one<F16, 2, D, TW>(q, sms, s); break;
+    case 3: launch_one<F16, 3, D, TW>(q, sms, s); break;
+    case 4: launch_one<F16, 4, D, TW>(q, sms, s); break;
+    case 8: launch_one<F16, 8, D, TW>(q, sms, s); break;
     default: return (int)cudaErrorInvalidValue;
   }
   return (int)cudaGetLastError();
 }
 
+template <bool F16>
+int launch_shape(const QuantLaunch& q, int head_dim, int tile_tokens, int sms, cudaStream_t s) {
+  const int bits = q.dst.bits;
+  if (head_dim == 512 && tile_tokens == 16) return launch_bits<F16, 512, 1>(q, bits, sms, s);
+  if (head_dim != 128) return (int)cudaErrorInvalidValue;
+  switch (tile_tokens) {
+    case 16: return launch_bits<F16, 128, 1>(q, bits, sms, s);
+    case 32: return launch_bits<F16, 128, 2>(q, bits, sms, s);
+    case 64: return launch_bits<F16, 128, 4>(q, bits, sms, s);
+    case 128: return launch_bits<F16, 128, 8>(q, bits, sms, s);
+    default: return (int)cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
-int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* stream) {
+int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, int tile_tokens, void* stream) {
   if (p.total_tiles == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const uint32_t per_kind = (uint32_t)(p.total_tiles / p.kinds);
-  const uint32_t ntt = (uint32_t)(p.n_tok / kT);
+  const uint32_t ntt = (uint32_t)(p.n_tok / tile_tokens);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int kind = 0; kind < p.kinds; ++kind) {
     QuantLaunch q;
@@ -574,17 +646,8 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, void* strea
     q.rope_src = kind == 0 ? static_cast<const uint16_t*>(p.rope_src) : nullptr;
     q.rope_dst = static_cast<uint16_t*>(p.rope_dst);
     q.rope_dim = p.rope_dim;
-    const int tpc = head_dim == 128 ? kWarps : kWarps / (head_dim / kBlk);
-    const int64_t need = (per_kind + tpc - 1) / tpc;
-    const int64_t cap = (int64_t)sms * (head_dim == 128 ? 4 : 3);  // resident CTAs per SM
-    const int grid = (int)(need < cap ? need : cap);
-    int e;
-    if (head_dim == 128)
-      e = f16 ? launch_bits<true, 128>(q, q.dst.bits, grid, s) : launch_bits<false, 128>(q, q.dst.bits, grid, s);
-    else if (head_dim == 512)
-      e = f16 ? launch_bits<true, 512>(q, q.dst.bits, grid, s) : launch_bits<false, 512>(q, q.dst.bits, grid, s);
-    else
-      e = (int)cudaErrorInvalidValue;
+    const int e = f16 ? launch_shape<true>(q, head_dim, tile_tokens, sms, s)
+                      : launch_shape<false>(q, head_dim, tile_tokens, sms, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -23,6 +23,8 @@ prefill 16384 tok x 32 layers x 8 kv-heads, d = 128, bf16 N(0,1) times a
 mla    64 seq x 32768 tok, latent 512 (4-bit) + rope 64 (bf16), 128
        absorbed query heads, bf16 N(0,1) latents with round(0.01*512) = 5
        outlier dims x25
+g128   the shipped preset kvarn_k4v2_g128 on the gqa shapes and
+       distribution: 4-bit K, 2-bit V, 128-token tiles (= pages)
 =====  ==================================================================
 
 All draws use numpy's PCG64 with the seed of the workload; the values are
@@ -97,6 +99,8 @@ WORKLOADS: Dict[str, Workload] = {
                         description="prefill append, 16384 tokens x 32 layers x 8 kv-heads"),
     "mla": Workload("mla", 64, 32768, 1, 128, 512, 4, 4, 4, 5, mla=True, rope_dim=64,
                     description="MLA latent cache, 64 x 32768 ctx, latent 512 + rope 64"),
+    "g128": Workload("g128", 32, 8192, 8, 32, 128, 4, 2, 4, 6, tile_tokens=128,
+                     description="preset kvarn_k4v2_g128 (4-bit K, 2-bit V, 128-token pages), gqa shapes"),
 }
 
 
@@ -132,7 +136,7 @@ def outlier_channels(w: Workload, layer: int, head: int, which: str) -> np.ndarr
         return np.array([3, 17, 64, 101])
     if w.mla:
         n = round(0.01 * w.head_dim)
-    elif w.name.startswith("gqa"):
+    elif _base_name(w) in ("gqa", "g128"):
         n = round(0.02 * w.head_dim)
     else:
         return np.zeros(0, dtype=np.int64)
@@ -170,8 +174,8 @@ def kv_inputs(w: Workload, which: str, tokens: Optional[slice] = None) -> np.nda
         r = _rng(w.seed, 10 * kind)
         scale = np.exp(r.uniform(math.log(0.1), math.log(10.0), size=(L, 1, H, d))).astype(np.float32)
     outl = None
-    if base in ("rt1k", "gqa", "mla"):
-        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0}[base]
+    if base in ("rt1k", "gqa", "mla", "g128"):
+        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0, "g128": 15.0}[base]
         outl = np.ones((L, 1, H, d), dtype=np.float32)
         for layer in range(L):
             for h in range(H):

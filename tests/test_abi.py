@@ -96,3 +96,27 @@ def test_host_rejections_before_launch(kvq):
                raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # layer out of range
     assert dec(c, view, 0, fake, fake, 64, fake, 0, 8, 0.1, fake, fake, ws, fake, 0,
                raise_on_error=False) == kvq.KVQ_OK                    # empty batch: nothing to do
+
+
+def test_tile_lengths_accepted_and_rejected(kvq):
+    # head_dim 128 caches take 16..128-token tiles; the MLA latent 16 only
+    fake = 1 << 20
+    view = kvq.make_view([fake] * 6 + [None])
+    f = kvq.kvq_quantize_append
+    for T, want in ((8, kvq.KVQ_ERR_UNSUPPORTED), (16, kvq.KVQ_OK), (32, kvq.KVQ_OK), (128, kvq.KVQ_OK),
+                    (256, kvq.KVQ_ERR_UNSUPPORTED)):
+        c = kvq.make_config(num_kv_heads=2, num_pages=8, tile_tokens=T)
+        assert f(c, view, fake, fake, None, 0, fake, fake, 0, raise_on_error=False) == want, T
+        assert f(c, view, fake, fake, None, T // 2, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_PARTIAL_TILE
+    m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=1, rope_dim=64, num_pages=8, tile_tokens=128)
+    mview = kvq.make_view([fake] * 3 + [None] * 3 + [fake])
+    assert f(m, mview, fake, None, fake, 0, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_decode_workspace_counts_16_token_tiles(kvq):
+    # decode works on 16-token tiles whatever the page length, so the split
+    # plan (and the workspace) depends on the context length only
+    for seq in (128, 1024, 8192, 131072):
+        sizes = {T: kvq.kvq_decode_workspace_bytes(kvq.make_config(num_kv_heads=8, num_pages=8, tile_tokens=T),
+                                                   32, 32, seq) for T in (16, 32, 64, 128)}
+        assert len(set(sizes.values())) == 1, (seq, sizes)

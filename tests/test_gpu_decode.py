@@ -34,6 +34,7 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("rt1k", {}),
     ("gqa", dict(batch=3, seq_len=512)),
     ("long", dict(batch=2, seq_len=2048)),
+    ("g128", dict(batch=3, seq_len=1024)),
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]
@@ -82,6 +83,41 @@ def test_decode_group_sizes_and_bit_widths(group, bits):
     run = QuantRun(w)
     dec = DecodeRun(run)
     _check(dec, dec())
+
+
+def test_decode_long_pages_ragged_and_empty():
+    # 128-token pages read as eight 16-token tiles; a split may start mid-page
+    w = W.WORKLOADS["g128"].scaled(batch=4, seq_len=2048)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=[2048, 128, 0, 1920])
+    o = dec()
+    assert run.error_bits() == 0
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("tile,group,bits", [(32, 8, (3, 4)), (64, 4, (3, 2)), (128, 1, (8, 8)), (64, 2, (2, 4))])
+def test_decode_tile_lengths(tile, group, bits):
+    # 3-bit keys come from the two planes of the page; one or two kv-heads per CTA
+    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=2, seq_len=1024), tile_tokens=tile,
+                            num_q_heads=8 * group, bits_k=bits[0], bits_v=bits[1])
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    _check(dec, o)
+
+
+def test_decode_long_pages_bad_page_and_partial():
+    w = W.WORKLOADS["g128"].scaled(batch=2, seq_len=512)
+    run = QuantRun(w)
+    bt = W.block_table(w).copy()
+    bt[1, 2] = w.num_pages + 3
+    dec = DecodeRun(run, block_table=bt, seq_lens=[500, 512])
+    o = dec()
+    bits = run.error_bits()
+    assert bits & 0x1 and bits & 0x2          # bad page in sequence 1, partial page in sequence 0
+    assert np.all(np.isfinite(o))
+    _check(dec, o, pairs=[(0, h) for h in range(w.num_kv_heads)])   # sequence 0: its three whole pages
 
 
 def test_decode_bad_page_sets_error():

@@ -14,7 +14,7 @@ from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_er
                      compare_quantized, oracle_fraction)
 
 
-@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla"])
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128"])
 def test_fullsize_sampled_parity(name):
     w = W.WORKLOADS[name]
     run = QuantRun(w)

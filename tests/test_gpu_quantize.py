@@ -16,6 +16,7 @@ SMALL = {
     "long": dict(batch=1, seq_len=1024),
     "prefill": dict(seq_len=256, num_layers=3),
     "mla": dict(batch=2, seq_len=256),
+    "g128": dict(batch=2, seq_len=512),
 }
 
 
@@ -55,10 +56,22 @@ def test_quantize_parity_other_bit_widths(bits):
 
 
 @pytest.mark.parametrize("iters", [0, 1, 9])
-def test_quantize_parity_iteration_counts(iters):
+@pytest.mark.parametrize("name", ["gqa", "g128"])
+def test_quantize_parity_iteration_counts(name, iters):
     import dataclasses
-    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=1, seq_len=256), sinkhorn_iters=iters)
+    w = dataclasses.replace(W.WORKLOADS[name].scaled(batch=1, seq_len=256), sinkhorn_iters=iters)
     _check_all(QuantRun(w))
+
+
+@pytest.mark.parametrize("tile,bits", [(32, (3, 4)), (64, (4, 8)), (128, (3, 2)), (128, (8, 4))])
+def test_quantize_parity_tile_lengths(tile, bits):
+    # 2, 4 or 8 warps share a tile's column sums; 3-bit planes span the whole page
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=1, seq_len=512), tile_tokens=tile, bits_k=bits[0],
+                            bits_v=bits[1])
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
 
 
 def _special_tiles():
@@ -79,19 +92,23 @@ def _special_tiles():
     return x
 
 
-def test_quantize_parity_degenerate_tiles():
+@pytest.mark.parametrize("tile", [16, 128])
+def test_quantize_parity_degenerate_tiles(tile):
+    # at 128 tokens the eight blocks form one tile: zero rows, a constant block,
+    # a huge outlier column and a 1e7 spread of magnitudes in one normalisation
     import dataclasses
     x = _special_tiles()
     n_tok = x.shape[0]
     w = dataclasses.replace(W.WORKLOADS["gqa"], batch=1, seq_len=n_tok, num_kv_heads=1, num_q_heads=1,
-                            name="special")
+                            name="special", tile_tokens=tile)
     kb = W._round_to(x, "bf16").reshape(1, n_tok, 1, 128)
     vb = W._round_to(-x[::-1].copy(), "bf16").reshape(1, n_tok, 1, 128)
-    run = QuantRun(w, inputs=(kb, vb), pages=np.arange(n_tok // 16, dtype=np.int32))
+    run = QuantRun(w, inputs=(kb, vb), pages=np.arange(n_tok // tile, dtype=np.int32))
     assert run.error_bits() == 0
     _check_all(run)
-    zero = run.gpu_tiles("k", 0, [0], 0)
-    assert np.all(zero.q == 0) and np.all(zero.a == 0) and np.all(zero.z == 0) and np.all(zero.c == 1)
+    if tile == 16:
+        zero = run.gpu_tiles("k", 0, [0], 0)
+        assert np.all(zero.q == 0) and np.all(zero.a == 0) and np.all(zero.z == 0) and np.all(zero.c == 1)
 
 
 def test_quantize_bad_page_sets_error_and_skips_tile():
@@ -108,14 +125,29 @@ def test_quantize_bad_page_sets_error_and_skips_tile():
     _check_all(run, tiles=[0, 2, 3])
 
 
-@pytest.mark.parametrize("name", ["rt1k", "mla"])
+@pytest.mark.parametrize("name", ["rt1k", "mla", "g128"])
 def test_quantize_single_tile(name):
     # One tile per call: at head_dim 128 three of the CTA's four warps have no
-    # tile and go straight to the CTA's final barrier; at 512 one CTA works.
-    w = W.WORKLOADS[name].scaled(batch=1, seq_len=16)
+    # tile and go straight to the CTA's final barrier; at 512 one CTA works;
+    # a 128-token tile is one CTA of eight warps.
+    w = W.WORKLOADS[name]
+    w = w.scaled(batch=1, seq_len=w.tile_tokens)
     run = QuantRun(w)
     assert run.error_bits() == 0
     _check_all(run)
+
+
+def test_long_tile_bad_page_sets_error_and_skips_tile():
+    # 128-token tiles: the eight warps of a tile leave it together on a bad page
+    w = W.WORKLOADS["g128"].scaled(batch=1, seq_len=512)
+    pages = np.array([0, 1, 6, 3], dtype=np.int32)        # pool of 4 pages: 6 is out of range
+    run = QuantRun(w, quantize=False, pages=pages, num_pages=4)
+    run.cache.codes("k")[0, 2].fill_(0xA5)
+    run.cache.codes("v")[0, 2].fill_(0xA5)
+    run.quantize()
+    assert run.error_bits() & 0x1
+    assert torch.all(run.cache.codes("k")[0, 2] == 0xA5) and torch.all(run.cache.codes("v")[0, 2] == 0xA5)
+    _check_all(run, tiles=[0, 1, 3])
 
 
 def test_mla_quantize_bad_page_sets_error_and_skips_tile():
@@ -149,14 +181,14 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-@pytest.mark.parametrize("name", ["long", "mla"])
+@pytest.mark.parametrize("name", ["long", "mla", "g128"])
 def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
     w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
     run = QuantRun(w)
     pages = torch.arange(w.num_pages, dtype=torch.int32, device="cuda")
     for unrot in (0, 1):
-        ko = torch.empty(w.num_pages, w.num_kv_heads, 16, w.head_dim, device="cuda")
+        ko = torch.empty(w.num_pages, w.num_kv_heads, w.tile_tokens, w.head_dim, device="cuda")
         vo = torch.empty_like(ko)
         kvq.kvq_dequantize(run.cfg, run.cache.view, 0, pages, w.num_pages, unrot, ko, None if w.mla else vo,
                            run.err)

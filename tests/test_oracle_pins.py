@@ -63,11 +63,12 @@ def test_rotate_roundtrip_and_parseval():
 
 
 # ---------------------------------------------------------------- Sinkhorn
-def test_sinkhorn_closed_form_rank_one_scaling():
+@pytest.mark.parametrize("T", [16, 128])
+def test_sinkhorn_closed_form_rank_one_scaling(T):
     # Z = diag(u) S diag(v) with S = +-1 reaches Y = S after one round,
     # with r_i c_j = u_i v_j.
     rng = np.random.default_rng(2)
-    T, d = 16, 128
+    d = 128
     u = np.exp(rng.uniform(-2, 2, T))
     v = np.exp(rng.uniform(-2, 2, d))
     s = np.where(rng.random((T, d)) < 0.5, -1.0, 1.0)
@@ -118,14 +119,14 @@ def test_sinkhorn_order_rows_then_columns():
     assert np.max(np.abs(np.sqrt(np.mean(y * y, 1)) - 1)) > 1e-6
 
 
-@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla"])
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128"])
 def test_sinkhorn_converges_on_workload_distributions(name):
     # Row and column second moments equal 1 within 1e-6 after convergence,
-    # on tiles drawn from each workload's distribution.
+    # on tiles drawn from each workload's distribution (with its tile length).
     w = W.WORKLOADS[name]
-    small = w.scaled(batch=1, seq_len=64 if not w.mla else 32, num_layers=1)
+    small = w.scaled(batch=1, seq_len=max(w.tile_tokens, 64 if not w.mla else 32), num_layers=1)
     x = W.half_bits_to_f64(W.kv_inputs(small, "k"), w.in_dtype)      # [1, n, H, d]
-    tiles = x[0].reshape(-1, 16, small.num_kv_heads, w.head_dim).transpose(0, 2, 1, 3)
+    tiles = x[0].reshape(-1, w.tile_tokens, small.num_kv_heads, w.head_dim).transpose(0, 2, 1, 3)
     y, _, _ = O.sinkhorn_normalize(O.rotate(tiles), 50)
     assert np.max(np.abs(np.mean(y * y, -1) - 1)) < 1e-6
     assert np.max(np.abs(np.mean(y * y, -2) - 1)) < 1e-6
@@ -238,13 +239,26 @@ def test_packing_golden():
         assert np.array_equal(O.unpack_codes(b, case["bits"], q.shape[0], q.shape[1]), q)
 
 
+@pytest.mark.parametrize("T", [16, 128])
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
-def test_pack_unpack_roundtrip(bits):
+def test_pack_unpack_roundtrip(bits, T):
     rng = np.random.default_rng(10)
-    q = rng.integers(0, 1 << bits, size=(3, 16, 128))
+    q = rng.integers(0, 1 << bits, size=(3, T, 128))
     b = O.pack_codes(q, bits)
-    assert b.shape == (3, O.tile_code_bytes(bits, 16, 128)) and b.dtype == np.uint8
-    assert np.array_equal(O.unpack_codes(b, bits, 16, 128), q)
+    assert b.shape == (3, O.tile_code_bytes(bits, T, 128)) and b.dtype == np.uint8
+    assert np.array_equal(O.unpack_codes(b, bits, T, 128), q)
+
+
+def test_packing_three_bit_planes_span_the_page():
+    # 128-token page, code 5 = 0b101 at token 127, channel 9: its low bits
+    # sit in the low-bit plane's last row, its high bit in the high-bit plane
+    # that starts after all 128 rows of the low plane (128 * 32 bytes).
+    q = np.zeros((128, 128), dtype=np.int64)
+    q[127, 9] = 5
+    b = O.pack_codes(q, 3)
+    nz = np.flatnonzero(b)
+    assert list(nz) == [127 * 32 + 2, 128 * 32 + 127 * 16 + 1]
+    assert b[127 * 32 + 2] == 0b01 << 2 and b[128 * 32 + 127 * 16 + 1] == 1 << 1
 
 
 # ---------------------------------------------------------------- attention
