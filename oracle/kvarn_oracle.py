@@ -256,6 +256,36 @@ def decode_attention(q: np.ndarray, k: QuantizedTiles, v: QuantizedTiles,
     return rotate(p @ vh)
 
 
+def decode_attention_with_tail(q: np.ndarray, k: Optional[QuantizedTiles], v: Optional[QuantizedTiles],
+                               k_tail: np.ndarray, v_tail: np.ndarray, softmax_scale: float) -> np.ndarray:
+    """Decode step over a sequence whose newest tokens do not fill a tile yet.
+
+    The cache holds the sequence's whole tiles; the last L < T tokens (the
+    tail) are kept at input precision until their tile fills (the pages say
+    nothing on this; the reading: a serving engine appends token by token,
+    so the tokens past the last whole tile stay unquantised, and attention
+    runs over all of the sequence's keys).
+
+    q: [G, d] un-rotated; k, v: the kv-head's quantised tiles in token order
+    (or None for none); k_tail, v_tail: [L, d] tail rows.  Written in the
+    input basis: the tiles are dequantised and rotated back, the tail rows
+    join them as they are, then plain softmax attention.  Returns [G, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[-1]
+    keys = [np.asarray(k_tail, dtype=np.float64).reshape(-1, d)]
+    vals = [np.asarray(v_tail, dtype=np.float64).reshape(-1, d)]
+    if k is not None and k.q.shape[0] > 0:
+        keys.insert(0, dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=True).reshape(-1, d))
+        vals.insert(0, dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=True).reshape(-1, d))
+    kk = np.concatenate(keys, 0)
+    vv = np.concatenate(vals, 0)
+    if kk.shape[0] == 0:
+        return np.zeros((q.shape[0], d))
+    p = _softmax(softmax_scale * (q @ kk.T))
+    return p @ vv
+
+
 def mla_decode_attention(q: np.ndarray, lat: QuantizedTiles, rope: np.ndarray,
                          softmax_scale: float) -> np.ndarray:
     """MLA decode step: one quantised latent serves as key and value.

@@ -297,6 +297,44 @@ def test_attention_single_token_and_identical_keys():
     assert np.allclose(o, vh.mean(0)[None].repeat(2, 0), rtol=0, atol=1e-12)
 
 
+def test_tail_attention_reduces_to_cache_attention_without_tail():
+    # two formulations: rotated-domain attention on the cache vs the input-basis
+    # attention with an empty tail
+    rng = np.random.default_rng(31)
+    k, v = _random_cache(rng, 5, 128, 3, 2)
+    q = rng.standard_normal((4, 128))
+    a = O.decode_attention(q, k, v, 1 / math.sqrt(128))
+    b = O.decode_attention_with_tail(q, k, v, np.zeros((0, 128)), np.zeros((0, 128)), 1 / math.sqrt(128))
+    assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_tail_attention_matches_torch_sdpa_on_tail_only():
+    import torch
+    rng = np.random.default_rng(32)
+    kt, vt = rng.standard_normal((11, 128)), rng.standard_normal((11, 128))
+    q = rng.standard_normal((8, 128))
+    o = O.decode_attention_with_tail(q, None, None, kt, vt, 0.09)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None], torch.from_numpy(kt)[None, None].expand(1, 8, 11, 128),
+        torch.from_numpy(vt)[None, None].expand(1, 8, 11, 128), scale=0.09)[0, :, 0].numpy()
+    assert np.max(np.abs(o - ref)) < 1e-12
+    assert np.all(O.decode_attention_with_tail(q, None, None, np.zeros((0, 128)), np.zeros((0, 128)), 0.09) == 0)
+
+
+def test_tail_attention_tokens_may_move_between_cache_and_tail():
+    # the last tile's dequantised rows given as tail rows change nothing: the
+    # result depends on the set of keys only
+    rng = np.random.default_rng(33)
+    k, v = _random_cache(rng, 4, 128)
+    q = rng.standard_normal((2, 128))
+    full = O.decode_attention_with_tail(q, k, v, np.zeros((0, 128)), np.zeros((0, 128)), 0.1)
+    head = O.QuantizedTiles(k.q[:3], k.a[:3], k.z[:3], k.c[:3]), O.QuantizedTiles(v.q[:3], v.a[:3], v.z[:3], v.c[:3])
+    kt = O.dequantize_tiles(k.q[3:], k.a[3:], k.z[3:], k.c[3:], unrotate=True)[0]
+    vt = O.dequantize_tiles(v.q[3:], v.a[3:], v.z[3:], v.c[3:], unrotate=True)[0]
+    moved = O.decode_attention_with_tail(q, head[0], head[1], kt, vt, 0.1)
+    assert np.max(np.abs(full - moved)) < 1e-12
+
+
 def test_mla_attention_matches_torch_sdpa_float64():
     import torch
     rng = np.random.default_rng(13)
