@@ -146,9 +146,11 @@ kvq_status kvq_cache_layout(const kvq_config* cfg, size_t bytes_out[7]);
  *   n_tok:        tokens per layer, a multiple of tile_tokens
  *                 (else KVQ_ERR_PARTIAL_TILE);
  *   dst_page:     device int32 [n_tok / tile_tokens]: the page that receives
- *                 tokens [i*T, (i+1)*T) of every layer and kv-head; an id
- *                 outside [0, num_pages) sets KVQ_DEVERR_BAD_PAGE and that
- *                 tile is not written;
+ *                 tokens [i*T, (i+1)*T) of every layer and kv-head; -1
+ *                 skips that tile (no error: quantise-on-fill passes a
+ *                 whole tail buffer and skips the tails that are not full);
+ *                 any other id outside [0, num_pages) sets
+ *                 KVQ_DEVERR_BAD_PAGE and that tile is not written;
  *   dev_error:    device uint32 error word (bits are OR-ed in).
  * Pages must be distinct within one call. */
 kvq_status kvq_quantize_append(const kvq_config* cfg, const kvq_cache_view* cache,
@@ -193,6 +195,30 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache_view* cac
                                 int32_t batch, int32_t num_q_heads, float softmax_scale,
                                 float* out, void* workspace, size_t workspace_bytes,
                                 uint32_t* dev_error, void* stream);
+
+/* kvq_decode_attention for sequences whose newest tokens do not fill a page
+ * yet (GQA caches).  The KVarN pages are silent on partial tiles; here the
+ * last tail_lens[b] < T tokens of sequence b stay unquantised in a tail
+ * buffer and attention runs over its cached tokens and its tail together
+ * (a tail token is scored with q . k and weighted by its value row as is;
+ * the result is the softmax over all of the sequence's keys).
+ *   k_tail, v_tail: device, in_dtype [num_layers][batch][tile_tokens]
+ *                [num_kv_heads][head_dim], 16-byte aligned: rows 0 ..
+ *                tail_lens[b] - 1 of sequence b are its tail in this layer;
+ *                the same layout as kvq_quantize_append's input with
+ *                n_tok = batch * tile_tokens, so full tails are quantised in
+ *                one append call (dst_page[b] = -1 skips the others);
+ *   tail_lens:   device int32 [batch], 0 .. tile_tokens (a value outside
+ *                sets KVQ_DEVERR_BAD_SEQ and the tail is ignored);
+ * the other arguments and the workspace are those of kvq_decode_attention.
+ * MLA caches and tiles longer than 128 tokens return KVQ_ERR_UNSUPPORTED. */
+kvq_status kvq_decode_attention_tail(const kvq_config* cfg, const kvq_cache_view* cache, int32_t layer,
+                                     const void* q, const int32_t* block_table,
+                                     int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                     const void* k_tail, const void* v_tail, const int32_t* tail_lens,
+                                     int32_t batch, int32_t num_q_heads, float softmax_scale,
+                                     float* out, void* workspace, size_t workspace_bytes,
+                                     uint32_t* dev_error, void* stream);
 
 /* kvq_decode_attention for callers that cannot allocate device memory when
  * they decode (a plug-in whose host process owns all device allocations and

@@ -269,11 +269,17 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* c, int32_t batch, int32_
   return KVQ_OK;
 }
 
-kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
-                                const void* q, const int32_t* block_table, int32_t max_pages_per_seq,
-                                const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
-                                float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
-                                uint32_t* dev_error, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Decode attention over the cache, plus the unquantised tails when k_tail is
+// given (GQA caches only).
+kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t layer, const void* q,
+                  const int32_t* block_table, int32_t max_pages_per_seq, const int32_t* seq_lens,
+                  const void* k_tail, const void* v_tail, const int32_t* tail_lens, int32_t batch,
+                  int32_t num_q_heads, float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                  uint32_t* dev_error, void* stream) {
   kvq_status st = check_config(c);
   if (st != KVQ_OK) return st;
   if ((st = check_view(c, cache)) != KVQ_OK) return st;
@@ -349,7 +355,40 @@ kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache
   p.tiles_per_split = plan.tiles_per_split;
   p.sub_log2 = sub_log2(c);
   p.err = dev_error;
+  p.k_tail = static_cast<const uint16_t*>(k_tail);
+  p.v_tail = static_cast<const uint16_t*>(v_tail);
+  p.tail_lens = tail_lens;
+  p.tail_f16 = c->in_dtype == KVQ_F16;
+  p.tail_tokens = c->tile_tokens;
   return cuda_status(launch_decode_d128(p, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
+                                const void* q, const int32_t* block_table, int32_t max_pages_per_seq,
+                                const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                uint32_t* dev_error, void* stream) {
+  return decode(c, cache, layer, q, block_table, max_pages_per_seq, seq_lens, nullptr, nullptr, nullptr, batch,
+                num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error, stream);
+}
+
+kvq_status kvq_decode_attention_tail(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
+                                     const void* q, const int32_t* block_table, int32_t max_pages_per_seq,
+                                     const int32_t* seq_lens, const void* k_tail, const void* v_tail,
+                                     const int32_t* tail_lens, int32_t batch, int32_t num_q_heads,
+                                     float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                     uint32_t* dev_error, void* stream) {
+  if (c && c->mla) return check_config(c) == KVQ_OK ? KVQ_ERR_UNSUPPORTED : check_config(c);
+  if (batch > 0 && (!k_tail || !v_tail || !tail_lens)) return KVQ_ERR_INVALID_ARG;
+  if ((k_tail && !aligned16(k_tail)) || (v_tail && !aligned16(v_tail))) return KVQ_ERR_INVALID_ARG;
+  if (c && c->tile_tokens > 128) return KVQ_ERR_UNSUPPORTED;
+  return decode(c, cache, layer, q, block_table, max_pages_per_seq, seq_lens, batch > 0 ? k_tail : nullptr,
+                v_tail, tail_lens, batch, num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error,
+                stream);
 }
 
 kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream) {

@@ -567,14 +567,82 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   }
 }
 
-// Merge the splits of one (sequence, kv-head), normalise, rotate back.
+// Merge the splits of one (sequence, kv-head), rotate back, normalise.  With
+// a tail, its tokens join as one more partial: their scores q . k and their
+// value sum are taken in the input basis (the rotation is orthogonal, so
+// q~ . k~ = q . k), and that sum is added after the splits' sum is rotated
+// back.
+constexpr int kMaxTail = 128;
 __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
   __shared__ float buf[kD];
+  __shared__ float tq[8][kD];        // tail: the group's query heads
+  __shared__ float ts[8][kMaxTail];  // tail: scores (log2 units), then softmax numerators
+  __shared__ float tov[8][kD];       // tail: sum_t p_t v_t per head
+  __shared__ float tml[8][2];        // tail: (max, sum) per head
   const int pair = blockIdx.x;
   const int b = pair / p.num_kv_heads, kvh = pair % p.num_kv_heads;
-  const int ch = threadIdx.x;
+  const int ch = threadIdx.x, warp = ch >> 5, lane = ch & 31;
+  int L = 0;
+  if (p.k_tail) {
+    L = p.tail_lens[b];
+    if (L < 0 || L > p.tail_tokens || L > kMaxTail) {
+      if (ch == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+      L = 0;
+    }
+  }
+  if (L > 0) {
+    const size_t row_stride = (size_t)p.num_kv_heads * kD;  // elements between tail tokens
+    const size_t base = (((size_t)p.layer * p.batch + b) * p.tail_tokens * p.num_kv_heads + kvh) * kD;
+    const uint16_t* kt = p.k_tail + base;
+    const uint16_t* vt = p.v_tail + base;
+    auto elem = [&](uint16_t x) { return p.tail_f16 ? __half2float(__ushort_as_half(x)) : bf16_to_f(x); };
+    for (int h = 0; h < p.group; ++h)
+      tq[h][ch] = bf16_to_f(p.q[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch]);
+    __syncthreads();
+    for (int t = warp; t < L; t += kD / 32) {  // warp w: tokens w, w + 4, ...; lane: channels 4 lane .. +3
+      const uint2 raw = *reinterpret_cast<const uint2*>(kt + t * row_stride + 4 * lane);
+      const float k4[4] = {elem((uint16_t)(raw.x & 0xFFFF)), elem((uint16_t)(raw.x >> 16)),
+                           elem((uint16_t)(raw.y & 0xFFFF)), elem((uint16_t)(raw.y >> 16))};
+      for (int h = 0; h < p.group; ++h) {
+        float s = tq[h][4 * lane] * k4[0];
+        s = fmaf(tq[h][4 * lane + 1], k4[1], s);
+        s = fmaf(tq[h][4 * lane + 2], k4[2], s);
+        s = fmaf(tq[h][4 * lane + 3], k4[3], s);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) ts[h][t] = s * p.scale_log2;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < p.group; h += kD / 32) {
+      float m = kNegBig;
+      for (int t = lane; t < L; t += 32) m = fmaxf(m, ts[h][t]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      float l = 0.f;
+      for (int t = lane; t < L; t += 32) {
+        const float e = ex2(ts[h][t] - m);
+        ts[h][t] = e;
+        l += e;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      if (lane == 0) tml[h][0] = m, tml[h][1] = l;
+    }
+    __syncthreads();
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int t = 0; t < L; ++t) {
+      const float v = elem(vt[t * row_stride + ch]);
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < p.group) acc[h] = fmaf(ts[h][t], v, acc[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < p.group) tov[h][ch] = acc[h];
+  }
   for (int h = 0; h < p.group; ++h) {
-    float mx = kNegBig;
+    float mx = L > 0 ? tml[h][0] : kNegBig;
     for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)pair * p.splits + s) * 8 + h) * 2]);
     float acc = 0.f, l = 0.f;
     for (int s = 0; s < p.splits; ++s) {
@@ -584,7 +652,7 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
       l = fmaf(f, p.part_ml[i * 2 + 1], l);
     }
     __syncthreads();
-    buf[ch] = l > 0.f ? acc / l : 0.f;
+    buf[ch] = acc;
     __syncthreads();
 #pragma unroll
     for (int s = 1; s < kD; s <<= 1) {
@@ -593,7 +661,13 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
       buf[ch] = (ch & s) ? (x - y) : (x + y);
       __syncthreads();
     }
-    p.out[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch] = buf[ch] * 0.08838834764831845f;
+    float o = buf[ch] * 0.08838834764831845f;
+    if (L > 0) {
+      const float f = ex2(tml[h][0] - mx);
+      o = fmaf(f, tov[h][ch], o);
+      l = fmaf(f, tml[h][1], l);
+    }
+    p.out[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch] = l > 0.f ? o / l : 0.f;
   }
 }
 

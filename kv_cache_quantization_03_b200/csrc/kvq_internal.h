@@ -71,6 +71,13 @@ struct DecodeParams {
   int tiles_per_split;          // in 16-token sub-tiles
   int sub_log2;                 // log2(16-token sub-tiles per page): 0 for 16-token pages, 3 for 128
   uint32_t* err;
+  // unquantised tail of each sequence (the newest tokens short of a whole
+  // page), merged by the combine kernel; k_tail == nullptr: no tail
+  const uint16_t* k_tail;       // [layers][B][T][Hkv][d], fp16 or bf16
+  const uint16_t* v_tail;
+  const int32_t* tail_lens;     // [B], 0..T
+  int tail_f16;                 // 1: fp16 rows, 0: bf16
+  int tail_tokens;              // T
 };
 
 struct MlaDecodeParams {

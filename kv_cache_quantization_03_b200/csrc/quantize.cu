@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
     if constexpr (!kStage)
       if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
     if (cur_page < 0 || cur_page >= p.num_pages) {  // same decision in every warp of the tile
-      if (lane == 0 && blk == 0 && wt == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
+      // page -1: the caller skips this tile (a sequence whose tail is not full)
+      if (cur_page != -1 && lane == 0 && blk == 0 && wt == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
       continue;
     }
     const size_t slot = ((size_t)layer * p.num_pages + cur_page) * p.num_heads + head;

@@ -39,7 +39,8 @@ KVQ_F16, KVQ_BF16, KVQ_F32 = 0, 1, 2
 
 EXPORTED = (
     "kvq_config_from_string", "kvq_cache_layout", "kvq_quantize_append", "kvq_dequantize",
-    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_read_error",
+    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_tail",
+    "kvq_decode_attention_noalloc", "kvq_read_error",
     "kvq_status_string", "kvq_version",
 )
 
@@ -72,6 +73,9 @@ _sig = {
     "kvq_decode_attention": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P,
                                             ctypes.c_size_t, _P, _P]),
+    "kvq_decode_attention_tail": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
+                                                 _P, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P,
+                                                 _P, ctypes.c_size_t, _P, _P]),
     "kvq_decode_attention_noalloc": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "kvq_read_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -178,6 +182,16 @@ def kvq_decode_attention(cfg, view, layer, q, block_table, max_pages_per_seq, se
                                   max_pages_per_seq, _ptr(seq_lens), batch, num_q_heads, float(softmax_scale),
                                   _ptr(out), _ptr(workspace), workspace_bytes, _ptr(dev_error), _stream(stream))
     return _check("kvq_decode_attention", st, raise_on_error)
+
+
+def kvq_decode_attention_tail(cfg, view, layer, q, block_table, max_pages_per_seq, seq_lens, k_tail, v_tail,
+                              tail_lens, batch, num_q_heads, softmax_scale, out, workspace, workspace_bytes,
+                              dev_error, stream=None, raise_on_error=True) -> int:
+    st = lib.kvq_decode_attention_tail(ctypes.byref(cfg), ctypes.byref(view), layer, _ptr(q), _ptr(block_table),
+                                       max_pages_per_seq, _ptr(seq_lens), _ptr(k_tail), _ptr(v_tail),
+                                       _ptr(tail_lens), batch, num_q_heads, float(softmax_scale), _ptr(out),
+                                       _ptr(workspace), workspace_bytes, _ptr(dev_error), _stream(stream))
+    return _check("kvq_decode_attention_tail", st, raise_on_error)
 
 
 def kvq_decode_attention_noalloc(cfg, view, layer, q, block_table, max_pages_per_seq, seq_lens, batch,

@@ -212,6 +212,21 @@ def queries(w: Workload) -> np.ndarray:
     return _round_to(x, "bf16")
 
 
+def tail_inputs(w: Workload, which: str) -> np.ndarray:
+    """Unquantised tail buffer: uint16 bits [layers][B][T][H_kv][d] in the
+    workload's input dtype, N(0,1) (only rows below each tail length are read)."""
+    r = _rng(w.seed, 6 if which == "k" else 7)
+    x = r.standard_normal(size=(w.num_layers, w.batch, w.tile_tokens, w.num_kv_heads, w.head_dim),
+                          dtype=np.float32)
+    return _round_to(x, w.in_dtype)
+
+
+def tail_lens(w: Workload) -> np.ndarray:
+    """Tail length of every sequence: int32 [B], uniform in [0, T)."""
+    r = _rng(w.seed, 8)
+    return r.integers(0, w.tile_tokens, size=w.batch).astype(np.int32)
+
+
 def page_assignment(w: Workload) -> np.ndarray:
     """Physical page of every tile, in append order (sequence-major): int32 [n_tok / T].
 

@@ -164,6 +164,36 @@ class DecodeRun:
         torch.cuda.synchronize()
         return self.out.cpu().numpy().astype(np.float64)
 
+    def with_tail(self, k_tail_bits, v_tail_bits, tail_lens, layer=0):
+        """kvq_decode_attention_tail with the given tail buffers; returns the output."""
+        w = self.run.w
+        self.k_tail_bits, self.v_tail_bits = k_tail_bits, v_tail_bits
+        self.tl = np.asarray(tail_lens, dtype=np.int32)
+        kt = torch.from_numpy(k_tail_bits.view(np.int16)).cuda()
+        vt = torch.from_numpy(v_tail_bits.view(np.int16)).cuda()
+        tl = torch.from_numpy(self.tl).cuda()
+        kvq.kvq_decode_attention_tail(self.run.cfg, self.run.cache.view, layer, self.q, self.bt_d, self.maxp,
+                                      self.sl_d, kt, vt, tl, self.batch, self.hq, w.softmax_scale, self.out,
+                                      self.ws, self.ws_bytes, self.run.err)
+        torch.cuda.synchronize()
+        return self.out.cpu().numpy().astype(np.float64)
+
+    def oracle_tail(self, b: int, kvh: int, layer=0, tail_len=None) -> np.ndarray:
+        """Oracle output with the tail rows of (layer, sequence b, kv-head kvh): [G, d]."""
+        w = self.run.w
+        G = self.hq // w.num_kv_heads
+        n = int(self.sl[b]) // w.tile_tokens
+        L = int(self.tl[b]) if tail_len is None else tail_len
+        q = W.half_bits_to_f64(self.q_bits[b, kvh * G:(kvh + 1) * G], "bf16")
+        kt = W.half_bits_to_f64(self.k_tail_bits[layer, b, :L, kvh], w.in_dtype)
+        vt = W.half_bits_to_f64(self.v_tail_bits[layer, b, :L, kvh], w.in_dtype)
+        k = v = None
+        if n:
+            pages = self.bt[b, :n]
+            k = gpu_pages(self.run, "k", layer, pages, kvh)
+            v = gpu_pages(self.run, "v", layer, pages, kvh)
+        return O.decode_attention_with_tail(q, k, v, kt, vt, w.softmax_scale)
+
     def oracle(self, b: int, kvh: int) -> np.ndarray:
         """Oracle output of the query heads of (sequence b, kv-head kvh): [G, d]."""
         w = self.run.w
