@@ -81,15 +81,28 @@ def hadamard_matrix(n: int) -> np.ndarray:
     return h
 
 
-def rotate(x: np.ndarray) -> np.ndarray:
-    """x H / sqrt(d) along the last axis (float64).
+def block_hadamard_matrix(d: int, block: int) -> np.ndarray:
+    """Block-diagonal Hadamard of order d: d / block copies of H_block on the
+    diagonal, int64 (the "block-diagonal Hadamard rotation" of the SAW-INT4
+    entry on the Hugging Face paper listing; blocks are runs of consecutive
+    channels).  block == d gives the full Sylvester matrix."""
+    if d % block:
+        raise ValueError("block must divide d")
+    return np.kron(np.eye(d // block, dtype=np.int64), hadamard_matrix(block))
 
-    H / sqrt(d) is symmetric and orthogonal, so the same call undoes itself:
+
+def rotate(x: np.ndarray, block: Optional[int] = None) -> np.ndarray:
+    """x H / sqrt(b) along the last axis (float64), H the Sylvester matrix of
+    the full width d (block None or d) or the block-diagonal one of order d
+    with blocks of b channels.
+
+    H / sqrt(b) is symmetric and orthogonal, so the same call undoes itself:
     rotate(rotate(x)) == x up to rounding.  Dense product, no fast transform.
     """
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
-    return (x @ hadamard_matrix(d).astype(np.float64)) / math.sqrt(d)
+    b = d if block is None else block
+    return (x @ block_hadamard_matrix(d, b).astype(np.float64)) / math.sqrt(b)
 
 
 # --------------------------------------------------------------------------
@@ -157,25 +170,26 @@ class QuantizedTiles:
     c: np.ndarray   # float32 [..., d]    column factor
 
 
-def quantize_tiles(x: np.ndarray, bits: int, n_iter: int) -> QuantizedTiles:
+def quantize_tiles(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] = None) -> QuantizedTiles:
     """Rotate, normalise and quantise tiles x: [..., T, d] (any float dtype).
 
-    The tiles are independent; leading axes only batch them.
+    The tiles are independent; leading axes only batch them.  block: the
+    rotation's block (None = full width).
     """
-    z = rotate(x)
+    z = rotate(x, block)
     y, r, c = sinkhorn_normalize(z, n_iter)
     q, m, s = rtn_rows(y, bits)
     return QuantizedTiles(q=q, a=(r * s).astype(np.float32), z=(r * m).astype(np.float32),
                           c=c.astype(np.float32))
 
 
-def dequantize_tiles(q, a, z, c, unrotate: bool = True) -> np.ndarray:
+def dequantize_tiles(q, a, z, c, unrotate: bool = True, block: Optional[int] = None) -> np.ndarray:
     """(a q + z) c in the rotated domain (float64), then optionally un-rotated."""
     a = np.asarray(a, dtype=np.float64)
     z = np.asarray(z, dtype=np.float64)
     c = np.asarray(c, dtype=np.float64)
     zh = (a[..., :, None] * np.asarray(q, dtype=np.float64) + z[..., :, None]) * c[..., None, :]
-    return rotate(zh) if unrotate else zh
+    return rotate(zh, block) if unrotate else zh
 
 
 # --------------------------------------------------------------------------
@@ -239,7 +253,7 @@ def _softmax(s: np.ndarray) -> np.ndarray:
 
 
 def decode_attention(q: np.ndarray, k: QuantizedTiles, v: QuantizedTiles,
-                     softmax_scale: float) -> np.ndarray:
+                     softmax_scale: float, block: Optional[int] = None) -> np.ndarray:
     """One decode step of the G query heads that share one kv-head.
 
     q: [G, d] (float, un-rotated).  k, v: the kv-head's tiles in token order,
@@ -251,13 +265,14 @@ def decode_attention(q: np.ndarray, k: QuantizedTiles, v: QuantizedTiles,
     d = q.shape[-1]
     kh = dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=False).reshape(-1, d)
     vh = dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=False).reshape(-1, d)
-    qr = rotate(q)
+    qr = rotate(q, block)
     p = _softmax(softmax_scale * (qr @ kh.T))
-    return rotate(p @ vh)
+    return rotate(p @ vh, block)
 
 
 def decode_attention_with_tail(q: np.ndarray, k: Optional[QuantizedTiles], v: Optional[QuantizedTiles],
-                               k_tail: np.ndarray, v_tail: np.ndarray, softmax_scale: float) -> np.ndarray:
+                               k_tail: np.ndarray, v_tail: np.ndarray, softmax_scale: float,
+                               block: Optional[int] = None) -> np.ndarray:
     """Decode step over a sequence whose newest tokens do not fill a tile yet.
 
     The cache holds the sequence's whole tiles; the last L < T tokens (the
@@ -276,8 +291,8 @@ def decode_attention_with_tail(q: np.ndarray, k: Optional[QuantizedTiles], v: Op
     keys = [np.asarray(k_tail, dtype=np.float64).reshape(-1, d)]
     vals = [np.asarray(v_tail, dtype=np.float64).reshape(-1, d)]
     if k is not None and k.q.shape[0] > 0:
-        keys.insert(0, dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=True).reshape(-1, d))
-        vals.insert(0, dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=True).reshape(-1, d))
+        keys.insert(0, dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=True, block=block).reshape(-1, d))
+        vals.insert(0, dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=True, block=block).reshape(-1, d))
     kk = np.concatenate(keys, 0)
     vv = np.concatenate(vals, 0)
     if kk.shape[0] == 0:

@@ -51,6 +51,47 @@ def test_hadamard_entry_formula():
     assert np.array_equal(h, np.where(pc % 2 == 0, 1, -1))
 
 
+@pytest.mark.parametrize("block", [8, 16, 32, 64, 128])
+def test_block_hadamard_orthogonal_and_block_local(block):
+    B = O.block_hadamard_matrix(128, block)
+    assert np.array_equal(B @ B.T, block * np.eye(128, dtype=np.int64))
+    # a spike in channel 37 spreads over its own block of channels only
+    e = np.zeros(128); e[37] = 1.0
+    r = O.rotate(e, block)
+    lo = 37 // block * block
+    assert np.allclose(np.abs(r[lo:lo + block]), 1 / math.sqrt(block), rtol=0, atol=1e-15)
+    assert np.all(r[:lo] == 0) and np.all(r[lo + block:] == 0)
+    x = np.random.default_rng(40).standard_normal((3, 128))
+    assert np.max(np.abs(O.rotate(O.rotate(x, block), block) - x)) < 1e-12
+
+
+@pytest.mark.parametrize("block", [8, 32])
+def test_full_rotation_factors_through_the_block_rotation(block):
+    # Sylvester: H_d = H_(d/b) (x) H_b = (H_(d/b) (x) I_b)(I_(d/b) (x) H_b), so the
+    # full rotation is the block rotation followed by H_(d/b) across the blocks
+    x = np.random.default_rng(41).standard_normal((4, 128))
+    across = np.kron(O.hadamard_matrix(128 // block), np.eye(block)) / math.sqrt(128 // block)
+    assert np.max(np.abs(O.rotate(x, block) @ across - O.rotate(x))) < 1e-12
+    assert np.array_equal(O.block_hadamard_matrix(128, 128), O.hadamard_matrix(128))
+
+
+def test_block_rotation_attention_matches_plain_attention_on_dequantised_rows():
+    # decode with a block rotation equals plain attention on the rows the cache
+    # decodes to (dequantised and rotated back with the same blocks)
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((2, 3, 16, 128))
+    k = O.quantize_tiles(x[0], 4, 0, block=32)
+    v = O.quantize_tiles(x[1], 4, 0, block=32)
+    q = rng.standard_normal((4, 128))
+    o = O.decode_attention(q, k, v, 0.1, block=32)
+    kk = O.dequantize_tiles(k.q, k.a, k.z, k.c, block=32).reshape(-1, 128)
+    vv = O.dequantize_tiles(v.q, v.a, v.z, v.c, block=32).reshape(-1, 128)
+    s = 0.1 * q @ kk.T
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    assert np.max(np.abs(o - p @ vv)) < 1e-12
+
+
 def test_rotate_roundtrip_and_parseval():
     rng = np.random.default_rng(1)
     x = rng.standard_normal((5, 16, 128)) * 7.0
