@@ -151,12 +151,12 @@ def oracle_sample_step(w, sample):
     from oracle import kvarn_oracle as O
     from kv_cache_quantization_03_b200 import workloads as W
     xk, xv, q = sample
-    kt = O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters)
+    kt = O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters, w.block)
     if w.mla:   # xv holds the rope keys
         O.mla_decode_attention(q, kt, xv, w.softmax_scale)
         return xk.shape[0] * xk.shape[1]
-    vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters)
-    O.decode_attention(q, kt, vt, w.softmax_scale)
+    vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters, w.block)
+    O.decode_attention(q, kt, vt, w.softmax_scale, block=w.block)
     return xk.shape[0] * xk.shape[1] / w.num_kv_heads
 
 
@@ -230,7 +230,8 @@ def config_dict(w, args):
     return {"workload": w.name, "description": w.description, "batch": w.batch, "seq_len": w.seq_len,
             "num_kv_heads": w.num_kv_heads, "num_q_heads": w.num_q_heads, "head_dim": w.head_dim,
             "bits_k": w.bits_k, "bits_v": w.bits_v, "tile_tokens": w.tile_tokens,
-            "sinkhorn_iters": w.sinkhorn_iters, "layers": w.num_layers,
+            "sinkhorn_iters": w.sinkhorn_iters, "hadamard_block": w.hadamard_block or w.head_dim,
+            "layers": w.num_layers,
             "parallelism": "dp%d (independent shards)" % args.gpus,
             "l2": "inputs larger than L2 (K+V bf16 %.2f GB per rank)" % (
                 2 * w.num_layers * w.n_tok * w.num_kv_heads * w.head_dim * 2 / 1e9)}
@@ -280,7 +281,8 @@ def run_gpu(args, w):
 
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                           bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
-                          rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype)
+                          rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype,
+                          hadamard_block=w.hadamard_block or None)
     cache = QuantizedCache(cfg)
     qb, pages = W.queries(ws), W.page_assignment(ws)
     bt, sl = W.block_table(ws), W.seq_lens(ws)

@@ -103,7 +103,10 @@ typedef struct kvq_config {
   int32_t bits_k;         /* key (MLA: latent) code width: 2, 3, 4 or 8 */
   int32_t bits_v;         /* value code width: 2, 4 or 8; ignored when mla */
   int32_t sinkhorn_iters; /* n >= 0 normalisation rounds (0 = rotation + RTN only) */
-  int32_t hadamard_block; /* must equal head_dim (full-width rotation) */
+  int32_t hadamard_block; /* channels per block of the rotation: head_dim = the full
+                           * Sylvester rotation; 8..head_dim/2 (K/V caches only) = a
+                           * block-diagonal rotation of consecutive channels (the
+                           * SAW-INT4 entry on the Hugging Face paper listing) */
   int32_t mla;            /* 1: one latent per token is key and value; no V arrays */
   int32_t rope_dim;       /* MLA: width of the unquantised bf16 rope key (64) */
   int32_t num_layers;     /* layers in the pool */

@@ -36,7 +36,9 @@ kvq_status check_config(const kvq_config* c) {
   if (c->mla) {
     if (c->num_kv_heads != 1 || c->rope_dim < 0 || (c->rope_dim % 8)) return KVQ_ERR_INVALID_ARG;
   }
-  if (c->hadamard_block != c->head_dim) return KVQ_ERR_UNSUPPORTED;
+  if (!is_pow2(c->hadamard_block) || c->hadamard_block > c->head_dim) return KVQ_ERR_INVALID_ARG;
+  // block-diagonal rotations (blocks of 8 .. head_dim channels) for K/V caches; the MLA latent full width
+  if (c->hadamard_block < 8 || (c->mla && c->hadamard_block != c->head_dim)) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 
@@ -225,6 +227,7 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.rope_src = (c->mla && c->rope_dim > 0) ? rope_new : nullptr;
   p.rope_dst = cache->rope;
   p.rope_dim = c->rope_dim;
+  p.hblock = c->hadamard_block;
   if (p.rope_src && !aligned16(p.rope_src)) return KVQ_ERR_INVALID_ARG;
   return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, c->tile_tokens, stream));
 }
@@ -250,6 +253,7 @@ kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int3
   p.n_pages = n_pages;
   p.unrotate = unrotate ? 1 : 0;
   p.tile_tokens = c->tile_tokens;
+  p.hblock = c->hadamard_block;
   p.out[0] = k_out;
   p.out[1] = v_out;
   p.err = dev_error;
@@ -360,6 +364,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   p.tail_lens = tail_lens;
   p.tail_f16 = c->in_dtype == KVQ_F16;
   p.tail_tokens = c->tile_tokens;
+  p.hblock = c->hadamard_block;
   return cuda_status(launch_decode_d128(p, stream));
 }
 

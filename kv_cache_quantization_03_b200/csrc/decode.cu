@@ -283,17 +283,22 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
         qr[8 * k + 2 * e + 1] = live ? bf16_to_f((uint16_t)(ws[e] >> 16)) : 0.f;
       }
     }
+    // H over channel bits 0..4 in registers, bits 5 and 6 across the lanes t;
+    // a block-diagonal rotation (blocks of hblock channels) stops at its block
 #pragma unroll
     for (int s = 1; s < 32; s <<= 1)
+      if (s < p.hblock) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (!(i & s)) {
-          const float x = qr[i], y = qr[i + s];
-          qr[i] = x + y;
-          qr[i + s] = x - y;
-        }
+        for (int i = 0; i < 32; ++i)
+          if (!(i & s)) {
+            const float x = qr[i], y = qr[i + s];
+            qr[i] = x + y;
+            qr[i + s] = x - y;
+          }
+      }
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
+      if (32 * off >= p.hblock) break;
       const bool upper = (t & off) != 0;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
         qr[i] = upper ? (o - qr[i]) : (qr[i] + o);
       }
     }
-    const float f = p.scale_log2 * 0.08838834764831845f;  // softmax scale * log2(e) / sqrt(128)
+    const float f = p.scale_log2 * inv_sqrt_pow2(p.hblock);  // softmax scale * log2(e) / sqrt(block)
     float* scr = reinterpret_cast<float*>(wsm) + lane * 33;
 #pragma unroll
     for (int i = 0; i < 32; ++i) scr[i] = qr[i] * f;
@@ -654,14 +659,13 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
     __syncthreads();
     buf[ch] = acc;
     __syncthreads();
-#pragma unroll
-    for (int s = 1; s < kD; s <<= 1) {
+    for (int s = 1; s < p.hblock; s <<= 1) {  // H / sqrt(b) on each block of b = hblock channels
       const float x = buf[ch & ~s], y = buf[ch | s];
       __syncthreads();
       buf[ch] = (ch & s) ? (x - y) : (x + y);
       __syncthreads();
     }
-    float o = buf[ch] * 0.08838834764831845f;
+    float o = buf[ch] * inv_sqrt_pow2(p.hblock);
     if (L > 0) {
       const float f = ex2(tml[h][0] - mx);
       o = fmaf(f, tov[h][ch], o);

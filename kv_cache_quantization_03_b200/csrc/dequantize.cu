@@ -49,15 +49,15 @@ __global__ void __launch_bounds__(kD) dequantize_kernel(DequantParams p) {
       tile[r][ch] =
           fmaf(tok[2 * (r0 + r)], (float)read_code<kD>(codes, src.bits, T, r0 + r, ch), tok[2 * (r0 + r) + 1]) * c;
     __syncthreads();
-    if (p.unrotate) {
+    if (p.unrotate) {  // H / sqrt(b) on each block of b = hblock channels
       for (int r = 0; r < kT; ++r) {
-        for (int s = 1; s < kD; s <<= 1) {
+        for (int s = 1; s < p.hblock; s <<= 1) {
           const float x = tile[r][ch & ~s], y = tile[r][ch | s];
           __syncthreads();
           tile[r][ch] = (ch & s) ? (x - y) : (x + y);
           __syncthreads();
         }
-        tile[r][ch] *= rsqrtf((float)kD);
+        tile[r][ch] *= inv_sqrt_pow2(p.hblock);
       }
       __syncthreads();
     }

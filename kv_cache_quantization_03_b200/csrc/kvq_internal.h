@@ -8,6 +8,16 @@
 
 namespace kvq {
 
+// 1/sqrt(b) for a power of two b, correctly rounded: 2^(-k/2) for b = 2^k,
+// k even, else sqrt(2) (rounded once) times the power of two 2^(-(k+1)/2).
+inline __host__ __device__ float inv_sqrt_pow2(int b) {
+  int k = 0;
+  while ((1 << k) < b) ++k;
+  float r = (k & 1) ? 1.41421356237309505f : 1.0f;
+  for (int i = 0; i < (k + 1) / 2; ++i) r *= 0.5f;
+  return r;
+}
+
 // Every spin-wait in a kernel gives up after this many nanoseconds (1 s of
 // GPU global time) and raises KVQ_DEVERR_TIMEOUT.
 constexpr uint32_t kWaitLimit = 1000000000u;
@@ -35,6 +45,7 @@ struct QuantizeParams {
   const void* rope_src; // MLA rope keys [layer][n_tok][rope_dim] bf16, or null
   void* rope_dst;       // cache rope array [layer][page][T][rope_dim]
   int rope_dim;
+  int hblock;           // Hadamard block: channels per diagonal block (head_dim = full width)
 };
 
 struct DequantParams {
@@ -47,6 +58,7 @@ struct DequantParams {
   int64_t n_pages;
   int unrotate;
   int tile_tokens;      // T: rows per page (a multiple of 16)
+  int hblock;           // Hadamard block
   float* out[2];
   uint32_t* err;
 };
@@ -78,6 +90,7 @@ struct DecodeParams {
   const int32_t* tail_lens;     // [B], 0..T
   int tail_f16;                 // 1: fp16 rows, 0: bf16
   int tail_tokens;              // T
+  int hblock;                   // Hadamard block: 8 .. 128 channels
 };
 
 struct MlaDecodeParams {

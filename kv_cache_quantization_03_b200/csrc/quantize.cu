@@ -64,12 +64,19 @@ __device__ __forceinline__ int k_bits(int k) {
 // Channel bits of the MMA output row m = g + 8*m3: bit 3 <- m3, bits 4..6 <- g.
 __device__ __forceinline__ int m_bits(int m) { return ((m >> 3) << 3) | ((m & 7) << 4); }
 
+// Entry (m, k) of the 16x16 factor over channel bits 3..6: the product over
+// those bits of H_2 entries, or, for bits at or above a block-diagonal
+// rotation's block (mask `out`), of identity entries.
 template <bool F16>
-__device__ __forceinline__ uint32_t sign_pair(int m, int k0) {
+__device__ __forceinline__ uint32_t sign_entry(int m, int k, uint32_t out) {
   const uint32_t one = F16 ? 0x3C00u : 0x3F80u, neg = F16 ? 0xBC00u : 0xBF80u;
-  const uint32_t lo = (__popc(m_bits(m) & k_bits(k0)) & 1) ? neg : one;
-  const uint32_t hi = (__popc(m_bits(m) & k_bits(k0 + 1)) & 1) ? neg : one;
-  return lo | (hi << 16);
+  const uint32_t mb = m_bits(m), kb = k_bits(k);
+  if ((mb ^ kb) & out) return 0u;
+  return (__popc(mb & kb & ~out) & 1) ? neg : one;
+}
+template <bool F16>
+__device__ __forceinline__ uint32_t sign_pair(int m, int k0, uint32_t out) {
+  return sign_entry<F16>(m, k0, out) | (sign_entry<F16>(m, k0 + 1, out) << 16);
 }
 
 // 1/x and 1/sqrt(x) from the hardware approximations plus one Newton step
@@ -136,6 +143,8 @@ struct QuantLaunch {
   const uint16_t* rope_src;  // MLA: [layer][n_tok][rope_dim] bf16, copied into rope_dst; else null
   uint16_t* rope_dst;        // [layer][page][T][rope_dim]
   int rope_dim;
+  int hblock;                // Hadamard block (8 .. 128 channels; 512 for the MLA latent)
+  float inv_sqrt_b;          // 1/sqrt(hblock)
 };
 
 // Shared memory of one tile whose 512 channels are split over four warps.
@@ -265,11 +274,13 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
   WarpScratch& sc = scratch[warp];
   TileShare& sh = share[0];
   uint32_t afrag[4];
-  afrag[0] = sign_pair<F16>(g, 2 * t);
-  afrag[1] = sign_pair<F16>(g + 8, 2 * t);
-  afrag[2] = sign_pair<F16>(g, 2 * t + 8);
-  afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8);
-  const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.044194173824159216f;
+  const uint32_t out_bits = D == kBlk ? 0x78u & ~(uint32_t)(p.hblock - 1) : 0u;  // channel bits 3..6 outside a block
+  afrag[0] = sign_pair<F16>(g, 2 * t, out_bits);
+  afrag[1] = sign_pair<F16>(g + 8, 2 * t, out_bits);
+  afrag[2] = sign_pair<F16>(g, 2 * t + 8, out_bits);
+  afrag[3] = sign_pair<F16>(g + 8, 2 * t + 8, out_bits);
+  // 1/sqrt(block) (1/sqrt(d) for the full rotation)
+  const float inv_sqrt_d = D == kBlk ? p.inv_sqrt_b : 0.044194173824159216f;
   const uint32_t stride = gridDim.x * TPC;
   uint32_t tile = blockIdx.x * TPC + slot_id;
   uint32_t tpark = 0;             // this warp's 64 TMEM columns
@@ -647,6 +658,8 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, int tile_to
     q.rope_src = kind == 0 ? static_cast<const uint16_t*>(p.rope_src) : nullptr;
     q.rope_dst = static_cast<uint16_t*>(p.rope_dst);
     q.rope_dim = p.rope_dim;
+    q.hblock = p.hblock;
+    q.inv_sqrt_b = inv_sqrt_pow2(p.hblock);
     const int e = f16 ? launch_shape<true>(q, head_dim, tile_tokens, sms, s)
                       : launch_shape<false>(q, head_dim, tile_tokens, sms, s);
     if (e != cudaSuccess) return e;

@@ -4,7 +4,9 @@ float64 oracle on the same seeded inputs, compare with the stated tolerances.
 Tolerances (readings as stated in the oracle's header):
 * codes: identical, except +-1 flips where the oracle's (y - m) / s lies within
   1e-4 of a half-integer (a rounding tie the float32 kernel may resolve the
-  other way); such flips on at most 1e-5 of the elements;
+  other way); such flips on at most 1e-5 of the elements, not counting flips
+  at exact ties (the oracle's fraction within 1e-9 of 1/2), where both codes
+  are equally near and either is acceptable;
 * a, z, c: |gpu - oracle| <= 1e-6 |oracle| + 1e-30;
 * attention: per (sequence, head) max_j |o_j - o'_j| / max_j |o'_j| <= 2e-3,
   with the oracle run on the GPU's stored codes and scales.
@@ -22,6 +24,7 @@ from oracle import kvarn_oracle as O
 
 CODE_TIE_BAND = 1e-4
 CODE_FLIP_RATE = 1e-5
+CODE_EXACT_TIE = 1e-9   # an exact tie in real arithmetic, up to the oracle's float64 rounding
 SCALE_RTOL = 1e-6
 ATTN_TOL = 2e-3
 
@@ -30,7 +33,8 @@ def config_for(w: W.Workload, num_pages=None) -> kvq.kvq_config:
     return kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                            bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                            rope_dim=w.rope_dim, num_layers=w.num_layers,
-                           num_pages=w.num_pages if num_pages is None else num_pages, in_dtype=w.in_dtype)
+                           num_pages=w.num_pages if num_pages is None else num_pages, in_dtype=w.in_dtype,
+                           hadamard_block=w.hadamard_block or None)
 
 
 class QuantRun:
@@ -82,9 +86,9 @@ class QuantRun:
         return W.half_bits_to_f64(src[layer, idx, head, :], w.in_dtype)   # [n, T, d]
 
 
-def oracle_fraction(x: np.ndarray, bits: int, n_iter: int) -> np.ndarray:
+def oracle_fraction(x: np.ndarray, bits: int, n_iter: int, block=None) -> np.ndarray:
     """The oracle's (y - m) / s of every element (to locate rounding ties)."""
-    y, _, _ = O.sinkhorn_normalize(O.rotate(x), n_iter)
+    y, _, _ = O.sinkhorn_normalize(O.rotate(x, block), n_iter)
     m = y.min(-1, keepdims=True)
     s = (y.max(-1, keepdims=True) - m) / ((1 << bits) - 1)
     return (y - m) / np.where(s > 0, s, 1.0)
@@ -92,7 +96,8 @@ def oracle_fraction(x: np.ndarray, bits: int, n_iter: int) -> np.ndarray:
 
 def compare_quantized(gpu: O.QuantizedTiles, ora: O.QuantizedTiles, frac: np.ndarray, label="",
                       check_rate=True):
-    """Asserts the code and scale tolerances; returns the number of tie flips.
+    """Asserts the code and scale tolerances; returns the number of tie flips
+    that count toward the rate (those not at an exact tie).
 
     With check_rate=False the caller aggregates the flip count over several
     comparisons and checks the 1e-5 rate itself."""
@@ -103,6 +108,7 @@ def compare_quantized(gpu: O.QuantizedTiles, ora: O.QuantizedTiles, frac: np.nda
         f = frac[diff]
         dist = np.abs(f - np.floor(f) - 0.5)
         assert np.all(dist <= CODE_TIE_BAND), "%s: flip away from a tie (distance %g)" % (label, dist.max())
+        nflip = int((dist > CODE_EXACT_TIE).sum())
     if check_rate:
         assert nflip <= CODE_FLIP_RATE * gpu.q.size, "%s: %d flips in %d codes" % (label, nflip, gpu.q.size)
     for name in ("a", "z", "c"):
@@ -192,7 +198,7 @@ class DecodeRun:
             pages = self.bt[b, :n]
             k = gpu_pages(self.run, "k", layer, pages, kvh)
             v = gpu_pages(self.run, "v", layer, pages, kvh)
-        return O.decode_attention_with_tail(q, k, v, kt, vt, w.softmax_scale)
+        return O.decode_attention_with_tail(q, k, v, kt, vt, w.softmax_scale, block=w.block)
 
     def oracle(self, b: int, kvh: int) -> np.ndarray:
         """Oracle output of the query heads of (sequence b, kv-head kvh): [G, d]."""
@@ -215,4 +221,4 @@ class DecodeRun:
         pages = self.bt[b, :n]
         kt = gpu_pages(self.run, "k", 0, pages, kvh)
         vt = gpu_pages(self.run, "v", 0, pages, kvh)
-        return O.decode_attention(q, kt, vt, w.softmax_scale)
+        return O.decode_attention(q, kt, vt, w.softmax_scale, block=w.block)

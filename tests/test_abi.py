@@ -62,9 +62,13 @@ def test_invalid_configs_rejected(kvq):
         c = kvq.make_config(num_pages=4, **kw)
         with pytest.raises(kvq.KvqError):
             kvq.kvq_cache_layout(c)
-    c = kvq.make_config(num_pages=4, hadamard_block=64)
     out = (ctypes.c_size_t * 7)()
-    assert kvq.lib.kvq_cache_layout(ctypes.byref(c), out) == kvq.KVQ_ERR_UNSUPPORTED
+    for blk, want in ((64, kvq.KVQ_OK), (8, kvq.KVQ_OK), (4, kvq.KVQ_ERR_UNSUPPORTED), (48, kvq.KVQ_ERR_INVALID_ARG),
+                      (256, kvq.KVQ_ERR_INVALID_ARG)):
+        c = kvq.make_config(num_pages=4, hadamard_block=blk)
+        assert kvq.lib.kvq_cache_layout(ctypes.byref(c), out) == want, blk
+    m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=4, hadamard_block=128)
+    assert kvq.lib.kvq_cache_layout(ctypes.byref(m), out) == kvq.KVQ_ERR_UNSUPPORTED  # the latent rotates in full
 
 
 def test_host_rejections_before_launch(kvq):

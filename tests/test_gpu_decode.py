@@ -35,6 +35,7 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("gqa", dict(batch=3, seq_len=512)),
     ("long", dict(batch=2, seq_len=2048)),
     ("g128", dict(batch=3, seq_len=1024)),
+    ("saw4", dict(batch=3, seq_len=512)),
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]
@@ -99,6 +100,18 @@ def test_decode_long_pages_ragged_and_empty():
 def test_decode_tile_lengths(tile, group, bits):
     # 3-bit keys come from the two planes of the page; one or two kv-heads per CTA
     w = dataclasses.replace(W.WORKLOADS["gqa"].scaled(batch=2, seq_len=1024), tile_tokens=tile,
+                            num_q_heads=8 * group, bits_k=bits[0], bits_v=bits[1])
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("block,group,bits", [(8, 4, (4, 4)), (16, 8, (3, 4)), (64, 1, (2, 2)), (32, 2, (8, 8))])
+def test_decode_block_diagonal_rotation(block, group, bits):
+    # query rotation and output un-rotation by blocks; one or two kv-heads per CTA
+    w = dataclasses.replace(W.WORKLOADS["saw4"].scaled(batch=2, seq_len=512), hadamard_block=block,
                             num_q_heads=8 * group, bits_k=bits[0], bits_v=bits[1])
     run = QuantRun(w)
     dec = DecodeRun(run)

@@ -14,7 +14,7 @@ from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_er
                      compare_quantized, oracle_fraction)
 
 
-@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128"])
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128", "saw4"])
 def test_fullsize_sampled_parity(name):
     w = W.WORKLOADS[name]
     run = QuantRun(w)
@@ -30,9 +30,9 @@ def test_fullsize_sampled_parity(name):
         for layer in layers:
             for head in heads:
                 x = run.input_tiles(which, layer, tiles, head)
-                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters)
+                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block)
                 gpu = run.gpu_tiles(which, layer, tiles, head)
-                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters),
+                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters, w.block),
                                            "%s %s L%d H%d" % (name, which, layer, head), check_rate=False)
                 total += gpu.q.size
     assert flips <= CODE_FLIP_RATE * total, "%d flips in %d sampled codes" % (flips, total)

@@ -17,6 +17,7 @@ SMALL = {
     "prefill": dict(seq_len=256, num_layers=3),
     "mla": dict(batch=2, seq_len=256),
     "g128": dict(batch=2, seq_len=512),
+    "saw4": dict(batch=2, seq_len=512),
 }
 
 
@@ -29,9 +30,9 @@ def _check_all(run: QuantRun, tiles=None, heads=None, layers=None):
         for layer in (range(w.num_layers) if layers is None else layers):
             for head in (range(w.num_kv_heads) if heads is None else heads):
                 x = run.input_tiles(which, layer, tiles, head)
-                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters)
+                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block)
                 gpu = run.gpu_tiles(which, layer, tiles, head)
-                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters),
+                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters, w.block),
                                            "%s L%d H%d" % (which, layer, head), check_rate=False)
                 total += gpu.q.size
     assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes" % (flips, total)
@@ -61,6 +62,18 @@ def test_quantize_parity_iteration_counts(name, iters):
     import dataclasses
     w = dataclasses.replace(W.WORKLOADS[name].scaled(batch=1, seq_len=256), sinkhorn_iters=iters)
     _check_all(QuantRun(w))
+
+
+@pytest.mark.parametrize("block,iters,bits,tile", [(8, 0, (4, 4), 16), (16, 4, (3, 2), 16), (32, 0, (4, 4), 16),
+                                                    (64, 6, (2, 8), 16), (32, 4, (4, 2), 128)])
+def test_quantize_parity_block_diagonal_rotation(block, iters, bits, tile):
+    # SAW-INT4-style ablation: blocks of 8..64 channels, with and without the normalisation
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["saw4"].scaled(batch=1, seq_len=512), hadamard_block=block,
+                            sinkhorn_iters=iters, bits_k=bits[0], bits_v=bits[1], tile_tokens=tile)
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
 
 
 @pytest.mark.parametrize("tile,bits", [(32, (3, 4)), (64, (4, 8)), (128, (3, 2)), (128, (8, 4))])
@@ -181,7 +194,7 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-@pytest.mark.parametrize("name", ["long", "mla", "g128"])
+@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4"])
 def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
     w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
@@ -197,7 +210,7 @@ def test_dequantize_matches_oracle_on_stored_codes(name):
             for h in range(w.num_kv_heads):
                 inv = np.argsort(run.pages)                      # page -> tile
                 g = run.gpu_tiles(which, 0, inv, h)              # tiles in page order
-                ref = O.dequantize_tiles(g.q, g.a, g.z, g.c, unrotate=bool(unrot))
+                ref = O.dequantize_tiles(g.q, g.a, g.z, g.c, unrotate=bool(unrot), block=w.block)
                 got = out[:, h].cpu().numpy().astype(np.float64)
                 scale = np.max(np.abs(ref), axis=(-1, -2), keepdims=True)
                 assert np.max(np.abs(got - ref) / scale) < 2e-6

@@ -37,6 +37,7 @@ def _check_tail(dec: DecodeRun, o: np.ndarray, layer=0, lens=None):
     ("g128", dict(batch=3, seq_len=1024), [1024, 0, 640]),
     ("rt1k", dict(batch=2, seq_len=256), [256, 16]),          # fp16 tail rows, one query head
     ("long", dict(batch=2, seq_len=512), [512, 128]),         # 8 query heads per kv-head, 3-bit keys
+    ("saw4", dict(batch=2, seq_len=256), [256, 64]),          # block-diagonal rotation
 ])
 def test_decode_with_tail_parity(name, kw, seq_lens):
     w = W.WORKLOADS[name].scaled(**kw)
@@ -115,13 +116,13 @@ def test_quantize_on_fill_skips_partial_tails(name):
         for layer in range(w.num_layers):
             for h in range(w.num_kv_heads):
                 x = W.half_bits_to_f64(src[layer, [1, 3], :, h], w.in_dtype)      # [2, T, d]
-                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters)
+                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block)
                 raw = codes[layer, [5, 2], h].cpu().numpy()
                 tok = run.cache.tok_scale(which)[layer, [5, 2], h].cpu().numpy()
                 ch = run.cache.chan_scale(which)[layer, [5, 2], h].cpu().numpy()
                 gpu = O.QuantizedTiles(O.unpack_codes(raw, bits, w.tile_tokens, w.head_dim), tok[..., 0],
                                        tok[..., 1], ch)
-                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters),
+                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters, w.block),
                                            "%s L%d H%d" % (which, layer, h), check_rate=False)
                 total += gpu.q.size
     assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes" % (flips, total)
