@@ -117,6 +117,30 @@ def test_tile_lengths_accepted_and_rejected(kvq):
     assert f(m, mview, fake, None, fake, 0, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
 
 
+def test_tail_entry_host_rejections(kvq):
+    # checked before any launch: missing or misaligned tail buffers, MLA caches
+    fake = 1 << 20
+    c = kvq.make_config(num_kv_heads=2, num_pages=8)
+    view = kvq.make_view([fake] * 6 + [None])
+    ws = kvq.kvq_decode_workspace_bytes(c, 4, 8, 1024)
+    f = kvq.kvq_decode_attention_tail
+    args = (0, fake, fake, 64, fake)
+    assert f(c, view, *args, None, fake, fake, 4, 8, 0.1, fake, fake, ws, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert f(c, view, *args, fake, fake, None, 4, 8, 0.1, fake, fake, ws, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert f(c, view, *args, fake + 8, fake, fake, 4, 8, 0.1, fake, fake, ws, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert f(c, view, *args, fake, fake, fake, 4, 8, 0.1, fake, fake, ws - 1, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    assert f(c, view, *args, None, None, None, 0, 8, 0.1, fake, fake, ws, fake, 0,
+             raise_on_error=False) == kvq.KVQ_OK                     # empty batch: nothing to do
+    m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=8)
+    mview = kvq.make_view([fake] * 3 + [None] * 3 + [fake])
+    assert f(m, mview, *args, fake, fake, fake, 4, 128, 0.1, fake, fake, 1 << 30, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
+
+
 def test_decode_workspace_counts_16_token_tiles(kvq):
     # decode works on 16-token tiles whatever the page length, so the split
     # plan (and the workspace) depends on the context length only
