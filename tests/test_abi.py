@@ -148,3 +148,18 @@ def test_decode_workspace_counts_16_token_tiles(kvq):
         sizes = {T: kvq.kvq_decode_workspace_bytes(kvq.make_config(num_kv_heads=8, num_pages=8, tile_tokens=T),
                                                    32, 32, seq) for T in (16, 32, 64, 128)}
         assert len(set(sizes.values())) == 1, (seq, sizes)
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    # the product path has no CPU fallback: without libkvq.so the binding refuses to import
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "kv_cache_quantization_03_b200"
+    pkg.mkdir()
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "kv_cache_quantization_03_b200")
+    for name in ("__init__.py", "kvq.py"):
+        shutil.copy(os.path.join(src, name), pkg / name)
+    r = subprocess.run([sys.executable, "-c", "import kv_cache_quantization_03_b200.kvq"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "libkvq.so is not built" in r.stderr
