@@ -163,3 +163,39 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import kv_cache_quantization_03_b200.kvq"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "ImportError" in r.stderr and "libkvq.so is not built" in r.stderr
+
+
+def test_header_is_plain_c_and_links(tmp_path, kvq):
+    # include/kvq.h compiles as C99 and a C program calls the library through it (host-only calls)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "kvq.h"
+int main(void) {
+  kvq_config c;
+  size_t sizes[7];
+  memset(&c, 0, sizeof c);
+  c.head_dim = 128; c.num_kv_heads = 8; c.sinkhorn_iters = 4; c.hadamard_block = 128;
+  c.num_layers = 2; c.num_pages = 10; c.in_dtype = KVQ_BF16;
+  if (kvq_config_from_string("kvarn_k4v2_g128", &c) != KVQ_OK) return 1;
+  if (c.bits_k != 4 || c.bits_v != 2 || c.tile_tokens != 128) return 2;
+  if (kvq_cache_layout(&c, sizes) != KVQ_OK) return 3;
+  printf("%s %zu %zu\n", kvq_version(), sizes[0], sizes[3]);
+  return strcmp(kvq_status_string(KVQ_ERR_PARTIAL_TILE), "KVQ_ERR_PARTIAL_TILE") != 0;
+}
+""")
+    lib = os.path.join(ROOT, "kv_cache_quantization_03_b200", "libkvq.so")
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), lib,
+                        "-Wl,-rpath," + os.path.dirname(lib), "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    n = 2 * 10 * 8
+    assert r.stdout.split()[1:] == [str(n * 128 * 128 * 4 // 8), str(n * 128 * 128 * 2 // 8)]
