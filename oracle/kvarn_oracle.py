@@ -45,6 +45,12 @@ Readings where the pages are silent (each is a declared choice):
 * the row and column factors are folded into what is stored: per token
   a = r * s and z = r * m, per channel c, all float32 (round to nearest);
   dequantisation in the rotated domain is (a * q + z) * c;
+* the pages fix no scale layout, and (a, z, c) is only defined up to moving
+  a factor between c and (a, z).  The stored tile is balanced by a power of
+  two: with k the integer for which max_j c_j (as float32) lies in
+  (2^(k-1), 2^k], c is stored times 2^-k and a, z times 2^k.  The scaling is
+  exact, so the dequantised tile is unchanged, and every stored c is <= 1
+  (a consumer can bound a dequantised row by max(|z|, |a (2^b - 1) + z|));
 * codes are packed little-endian inside each byte, lowest channel in the
   lowest bits, token rows one after the other; 3-bit codes are two planes
   per tile: all rows' low 2 bits (2-bit packing), then all rows' high bit
@@ -165,22 +171,35 @@ def rtn_rows(y: np.ndarray, bits: int):
 class QuantizedTiles:
     """What one or more quantised tiles store: logical codes and folded scales."""
     q: np.ndarray   # int64 [..., T, d]   codes in [0, 2^bits - 1]
-    a: np.ndarray   # float32 [..., T]    a = r * s
-    z: np.ndarray   # float32 [..., T]    z = r * m
-    c: np.ndarray   # float32 [..., d]    column factor
+    a: np.ndarray   # float32 [..., T]    a = r * s * 2^k
+    z: np.ndarray   # float32 [..., T]    z = r * m * 2^k
+    c: np.ndarray   # float32 [..., d]    column factor * 2^-k (max in (1/2, 1])
+
+
+def balance_exponent(c32: np.ndarray) -> np.ndarray:
+    """The integer k with max_j c_j in (2^(k-1), 2^k] of each tile's float32
+    column factors c32: [..., d] (positive).  Exact: from the binary exponent."""
+    cmax = np.max(np.asarray(c32, dtype=np.float64), axis=-1)
+    mant, e = np.frexp(cmax)                  # cmax = mant * 2^e, mant in [1/2, 1)
+    return np.where(mant == 0.5, e - 1, e).astype(np.int64)
 
 
 def quantize_tiles(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] = None) -> QuantizedTiles:
     """Rotate, normalise and quantise tiles x: [..., T, d] (any float dtype).
 
     The tiles are independent; leading axes only batch them.  block: the
-    rotation's block (None = full width).
+    rotation's block (None = full width).  The stored scales are balanced
+    by a power of two (max c in (1/2, 1]; see the module notes).
     """
     z = rotate(x, block)
     y, r, c = sinkhorn_normalize(z, n_iter)
     q, m, s = rtn_rows(y, bits)
-    return QuantizedTiles(q=q, a=(r * s).astype(np.float32), z=(r * m).astype(np.float32),
-                          c=c.astype(np.float32))
+    a32, z32, c32 = (r * s).astype(np.float32), (r * m).astype(np.float32), c.astype(np.float32)
+    k = balance_exponent(c32)
+    a32 = np.ldexp(a32, k[..., None]).astype(np.float32)
+    z32 = np.ldexp(z32, k[..., None]).astype(np.float32)
+    c32 = np.ldexp(c32, -k[..., None]).astype(np.float32)
+    return QuantizedTiles(q=q, a=a32, z=z32, c=c32)
 
 
 def dequantize_tiles(q, a, z, c, unrotate: bool = True, block: Optional[int] = None) -> np.ndarray:

@@ -124,7 +124,7 @@ def test_sinkhorn_golden_rank1():
     fx = _golden("tile_t2_d4_rank1.json")
     z = np.array(fx["z_rotated"])
     y, r, c = O.sinkhorn_normalize(z, fx["n_iter"])
-    assert np.allclose(c, fx["c"], rtol=1e-14, atol=0)
+    assert np.allclose(c, fx["c_normalisation"], rtol=1e-14, atol=0)   # before the stored balance
     s = np.array([[1, -1, 1, 1], [-1, 1, 1, -1]], dtype=float)
     assert np.allclose(y, s, rtol=0, atol=1e-14)
 
@@ -239,6 +239,47 @@ def test_quantize_homogeneity_and_token_permutation():
     assert np.array_equal(pm.q, base.q[perm])
     assert np.allclose(pm.a, base.a[perm], rtol=1e-6) and np.allclose(pm.z, base.z[perm], rtol=1e-6)
     assert np.allclose(pm.c, base.c, rtol=1e-6)
+
+
+def test_stored_scales_balanced_by_a_power_of_two():
+    # The stored (a, z, c) are the textbook (r s, r m, c) with an exact power
+    # of two 2^k moved from c into a and z, k chosen so that max c lies in
+    # (1/2, 1]; the dequantised tile is bit-for-bit the unbalanced one.
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((40, 16, 128)) * np.exp(rng.uniform(-3, 3, (40, 1, 128)))
+    x[:4] *= np.exp2(rng.integers(-40, 40, (4, 1, 1)))
+    for n_iter in (0, 1, 4):
+        qt = O.quantize_tiles(x, 4, n_iter)
+        cmax = qt.c.max(-1).astype(np.float64)
+        assert np.all(cmax > 0.5) and np.all(cmax <= 1.0)
+        # unbalanced, from the pipeline's steps taken one by one
+        y, r, c = O.sinkhorn_normalize(O.rotate(x), n_iter)
+        q, m, st = O.rtn_rows(y, 4)
+        a0, z0, c0 = (r * st).astype(np.float32), (r * m).astype(np.float32), c.astype(np.float32)
+        assert np.array_equal(q, qt.q)
+        k = np.log2(c0.max(-1).astype(np.float64) / cmax)
+        assert np.array_equal(k, np.round(k))                      # a power of two per tile
+        assert np.array_equal(O.dequantize_tiles(qt.q, qt.a, qt.z, qt.c, unrotate=False),
+                              O.dequantize_tiles(q, a0, z0, c0, unrotate=False))
+    # no normalisation: c = 1, already balanced (k = 0)
+    qt = O.quantize_tiles(x, 4, 0)
+    assert np.all(qt.c == 1.0)
+
+
+def test_quantize_row_scale_invariance():
+    # Scaling one token row by a power of two scales that row's a and z by it
+    # and changes no code and no column factor: the row step divides it out
+    # before any column step sees it.  Holds across the float range the input
+    # formats reach.
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-1, 1, 128))
+    base = O.quantize_tiles(x, 4, 4)
+    f = np.ones(16)
+    f[3], f[7], f[11] = 2.0 ** -64, 2.0 ** 60, 2.0 ** -100
+    sc = O.quantize_tiles(x * f[:, None], 4, 4)
+    assert np.array_equal(sc.q, base.q) and np.array_equal(sc.c, base.c)
+    assert np.array_equal(sc.a, (base.a * f).astype(np.float32))
+    assert np.array_equal(sc.z, (base.z * f).astype(np.float32))
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
