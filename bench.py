@@ -1,13 +1,18 @@
 """Throughput of the KVarN-style hot path on B200: quantize-append + decode attention.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa] [--impl kvq|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl kvq|reference]
+                    [--no-extra] [--no-cpu-baseline]
 
 One step = the whole hot path over one batch of the workload: every new K/V
 row of the batch is rotated, normalised, quantised and packed into the paged
 cache (kvq_quantize_append), then one decode step of attention runs over the
 quantised cache (kvq_decode_attention, split-KV + combine).  The default
-workload is the Llama-3-8B-shaped GQA case: 32 sequences x 8192 tokens, 8 kv /
-32 query heads, head_dim 128, bf16 inputs, 4-bit K and V, 16-token pages.
+workload is the largest single-GPU one, long-context decode: 4 sequences x
+131072 tokens, 8 kv / 64 query heads, head_dim 128, bf16 inputs (Student-t
+keys), 3-bit K, 4-bit V, 6 normalisation rounds, 16-token pages.  The other
+workloads (gqa, prefill, mla, the kvarn_k4v2_g128 preset, the saw4 ablation
+and the rt1k round trip) are timed after it with fewer steps and reported
+under "workloads" in the same line (--no-extra skips them).
 
 value  = KV tokens quantized per second (all ranks; one token = all kv-heads'
          K and V rows of one position), inputs resident in HBM;
@@ -178,12 +183,31 @@ def oracle_sample_inputs(w, tokens):
 
 
 def blas_threads():
+    """Threads the oracle's dense products run on (numpy's BLAS pool)."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return max(n) if n else 1
     except Exception:
         return 1
+
+
+def host_cpu():
+    """(logical CPUs this process may use, CPU model name)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return n, model
 
 
 def cpu_baseline(w, budget_s=12.0, tokens=4096):
@@ -197,7 +221,9 @@ def cpu_baseline(w, budget_s=12.0, tokens=4096):
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": done / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    nproc, model = host_cpu()
+    return {"value": done / dt, "unit": UNIT, "cores": blas_threads(), "nproc": nproc, "cpu_model": model,
+            "kind": "oracle",
             "sample": "%d x {quantize K and V of one kv-head over %d tokens of sequence 0 (float64, dense "
                       "Hadamard) + decode of its %d query heads over them}; %.1f s" % (n, tokens, w.group, dt)}
 
@@ -219,7 +245,8 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_dict(w, args),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "nproc": host_cpu()[0],
+                             "cpu_model": host_cpu()[1], "kind": "oracle",
                              "sample": "each step: one kv-head of sequence 0, %d tokens: quantize K and V + "
                                        "decode of its %d query heads (float64 oracle)" % (tokens, w.group)},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -233,8 +260,10 @@ def config_dict(w, args):
             "sinkhorn_iters": w.sinkhorn_iters, "hadamard_block": w.hadamard_block or w.head_dim,
             "layers": w.num_layers,
             "parallelism": "dp%d (independent shards)" % args.gpus,
-            "l2": "inputs larger than L2 (K+V bf16 %.2f GB per rank)" % (
-                2 * w.num_layers * w.n_tok * w.num_kv_heads * w.head_dim * 2 / 1e9)}
+            "l2": ("inputs larger than L2 (latent + rope bf16 %.2f GB per rank)" % (
+                w.num_layers * w.n_tok * (w.head_dim + w.rope_dim) * 2 / 1e9)) if w.mla else
+                  ("inputs larger than L2 (K+V bf16 %.2f GB per rank)" % (
+                      2 * w.num_layers * w.n_tok * w.num_kv_heads * w.head_dim * 2 / 1e9))}
 
 
 # --------------------------------------------------------------------------- ranks
@@ -263,44 +292,50 @@ def max_over_ranks(values, world: int, device=None):
 
 
 # --------------------------------------------------------------------------- GPU leg
-def run_gpu(args, w):
+QUANTIZE_ONLY = ("prefill",)       # workloads whose step is quantise-append alone
+EXTRA_WORKLOADS = ("gqa", "prefill", "mla", "g128", "saw4", "rt1k")
+
+
+def kernel_names(w):
+    """(quantize kernel, decode kernels) as launched for the workload."""
+    if w.mla:
+        return "quantize_kernel<D=512>", "mla_prep_q + decode_mla (tcgen05) + combine_mla"
+    return "quantize_kernel<D=128, T=%d>" % w.tile_tokens, "decode_d128 + combine_d128"
+
+
+def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
+    """Times `steps` steps of workload w on this rank's GPU (CUDA events on the
+    launching stream).  Returns a dict of seconds and byte counts."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     from kv_cache_quantization_03_b200 import kvq, workloads as W
     from kv_cache_quantization_03_b200.cache import QuantizedCache
 
-    world, rank, local = rank_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
     ws = shard(w, rank)
-
+    q_only = any(w.name == n or w.name.startswith(n + "-") for n in QUANTIZE_ONLY)
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                           bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                           rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype,
                           hadamard_block=w.hadamard_block or None)
     cache = QuantizedCache(cfg)
-    qb, pages = W.queries(ws), W.page_assignment(ws)
-    bt, sl = W.block_table(ws), W.seq_lens(ws)
-    host = {"k": torch.from_numpy(W.kv_inputs(ws, "k").view(np.int16)).pin_memory()}
+    host = {"k": torch.from_numpy(W.kv_inputs(ws, "k").view(np.int16))}
     if w.mla:
-        host["rope"] = torch.from_numpy(W.rope_inputs(ws).view(np.int16)).pin_memory()
+        host["rope"] = torch.from_numpy(W.rope_inputs(ws).view(np.int16))
     else:
-        host["v"] = torch.from_numpy(W.kv_inputs(ws, "v").view(np.int16)).pin_memory()
-    host.update({"q": torch.from_numpy(qb.view(np.int16)).pin_memory(),
-                 "dst": torch.from_numpy(pages).pin_memory(),
-                 "bt": torch.from_numpy(np.ascontiguousarray(bt)).pin_memory(),
-                 "sl": torch.from_numpy(sl).pin_memory()})
+        host["v"] = torch.from_numpy(W.kv_inputs(ws, "v").view(np.int16))
+    host["dst"] = torch.from_numpy(W.page_assignment(ws))
+    if not q_only:
+        host.update({"q": torch.from_numpy(W.queries(ws).view(np.int16)),
+                     "bt": torch.from_numpy(np.ascontiguousarray(W.block_table(ws))),
+                     "sl": torch.from_numpy(W.seq_lens(ws))})
+    if e2e:
+        host = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.cuda() for k, v in host.items()}
     out = torch.empty(w.batch, w.num_q_heads, w.head_dim, device="cuda")
-    out_host = torch.empty_like(out, device="cpu").pin_memory()
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     ws_bytes = kvq.kvq_decode_workspace_bytes(cfg, w.batch, w.num_q_heads, w.seq_len)
-    work = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    work = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     s_ptr = stream.cuda_stream
 
@@ -309,10 +344,11 @@ def run_gpu(args, w):
                                 s_ptr)
 
     def decode():
-        kvq.kvq_decode_attention(cfg, cache.view, 0, dev["q"], dev["bt"], w.tiles_per_seq, dev["sl"], w.batch,
-                                 w.num_q_heads, w.softmax_scale, out, work, ws_bytes, err, s_ptr)
+        if not q_only:
+            kvq.kvq_decode_attention(cfg, cache.view, 0, dev["q"], dev["bt"], w.tiles_per_seq, dev["sl"], w.batch,
+                                     w.num_q_heads, w.softmax_scale, out, work, ws_bytes, err, s_ptr)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         quantize()
         decode()
     torch.cuda.synchronize()
@@ -320,51 +356,97 @@ def run_gpu(args, w):
     if st != kvq.KVQ_OK or bits:
         raise RuntimeError("device error word %#x after warm-up" % bits)
 
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        for i in range(K):
-            ev[i][0].record(stream)
-            quantize()
-            ev[i][1].record(stream)
-            decode()
-            ev[i][2].record(stream)
-        end.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    elapsed = start.elapsed_time(end) / 1e3
-    t_q = sum(e[0].elapsed_time(e[1]) for e in ev) / K / 1e3
-    t_d = sum(e[1].elapsed_time(e[2]) for e in ev) / K / 1e3
-
-    # end to end: inputs from pinned host memory, output back to the host, each step
-    Ke = max(1, min(K, 10))
-    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
-    d2h = out.numel() * out.element_size()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(Ke):
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
+    clk = ClockSampler(local) if clocks else None
+    if clk:
+        clk.__enter__()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
         quantize()
+        ev[i][1].record(stream)
         decode()
-        out_host.copy_(out, non_blocking=True)
-    e1.record(stream)
+        ev[i][2].record(stream)
+    end.record(stream)
     torch.cuda.synchronize()
-    e2e_s = e0.elapsed_time(e1) / 1e3 / Ke
+    if clk:
+        clk.__exit__()
+    if world > 1:
+        dist.barrier()
+    r = {"elapsed": start.elapsed_time(end) / 1e3,
+         "t_q": sum(e[0].elapsed_time(e[1]) for e in ev) / steps / 1e3,
+         "t_d": sum(e[1].elapsed_time(e[2]) for e in ev) / steps / 1e3,
+         "q_only": q_only, "clocks": clk.summary() if clk else None}
+
+    if e2e:  # inputs from pinned host memory, output back to the host, each step
+        out_host = torch.empty_like(out, device="cpu").pin_memory()
+        Ke = max(1, min(steps, 10))
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            for k in host:
+                dev[k].copy_(host[k], non_blocking=True)
+            quantize()
+            decode()
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        r["e2e_s"] = e0.elapsed_time(e1) / 1e3 / Ke
+        r["h2d"] = sum(host[k].numel() * host[k].element_size() for k in host)
+        r["d2h"] = out.numel() * out.element_size()
     st, bits = kvq.kvq_read_error(err, s_ptr)
     if st != kvq.KVQ_OK or bits:
         raise RuntimeError("device error word %#x" % bits)
+    del cache, dev, host, work, out
+    torch.cuda.empty_cache()
+    return r
 
-    elapsed, e2e_s, t_q, t_d = max_over_ranks([elapsed, e2e_s, t_q, t_d], world, device="cuda")
+
+def summarize(w, r, peak, world=1):
+    """Per-kernel throughput of one measured workload."""
+    qb_bytes, db_bytes = algorithmic_bytes(w)
+    t_q, t_d = r["t_q"], r["t_d"]
+    qk, dk = kernel_names(w)
+    q_gbs = qb_bytes / t_q / 1e9
+    res = {"ms_per_step": 1e3 * r["elapsed"] / max(r.get("steps", 1), 1),
+           "quantize": {"kernel": qk, "us": 1e6 * t_q, "gbs": q_gbs, "frac_of_measured": q_gbs / peak,
+                        "frac_of_8tbs": q_gbs / 8000.0, "algorithmic_bytes": qb_bytes,
+                        "rows_per_s": w.num_layers * w.n_tok * w.num_kv_heads * (1 if w.mla else 2) / t_q}}
+    if not r["q_only"]:
+        d_gbs = db_bytes / t_d / 1e9
+        res["decode_attn"] = {"kernel": dk, "us": 1e6 * t_d, "gbs": d_gbs, "frac_of_measured": d_gbs / peak,
+                              "frac_of_8tbs": d_gbs / 8000.0, "algorithmic_bytes": db_bytes}
+        if w.mla:   # 128 heads share every latent: a dense contraction, tensor-bound
+            flops = 2.0 * w.batch * w.seq_len * w.num_q_heads * (w.head_dim + w.rope_dim + w.head_dim)
+            tf = flops / t_d / 1e12
+            tpeak, tsrc = load_tensor_peak()
+            res["decode_attn"].update({"tflops": tf, "frac_of_tensor_peak": tf / tpeak, "tensor_peak": tpeak,
+                                       "tensor_peak_source": tsrc, "flops": flops})
+    return res
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    K = args.steps
+    r = measure(w, K, args.warmup, rank, world, local, e2e=True, clocks=True)
+    elapsed, e2e_s, t_q, t_d = max_over_ranks([r["elapsed"], r["e2e_s"], r["t_q"], r["t_d"]], world, device="cuda")
+    r.update({"elapsed": elapsed, "e2e_s": e2e_s, "t_q": t_q, "t_d": t_d, "steps": K})
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -372,40 +454,56 @@ def run_gpu(args, w):
 
     tokens = w.batch * w.seq_len * world
     peak, peak_kind = load_peaks()
-    qb_bytes, db_bytes = algorithmic_bytes(w)
-    q_gbs = qb_bytes / t_q / 1e9
-    d_gbs = db_bytes / t_d / 1e9
-    traffic = traffic_from_profile("quantize.cu", "quantize_d128_gqa.md") if not w.mla else None
+    summ = summarize(w, r, peak, world)
+    qb_bytes, _ = algorithmic_bytes(w)
+    qk, dk = kernel_names(w)
+    profile = "quantize_d512_mla.md" if w.mla else "quantize_d128_%s.md" % w.name
+    traffic = traffic_from_profile("quantize.cu", profile)
     line = {
         "metric": METRIC, "value": tokens * K / elapsed, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; see workloads.py)",
         "config": config_dict(w, args),
-        "roofline": {"kernel": "quantize_d128", "bound": "hbm", "achieved": q_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": q_gbs / peak, "peak_source": peak_kind,
+        "roofline": {"kernel": qk, "bound": "hbm", "achieved": summ["quantize"]["gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": summ["quantize"]["gbs"] / peak, "peak_source": peak_kind,
                      "traffic": traffic, "algorithmic_bytes": qb_bytes},
-        "decode_attn": {"kernel": "decode_d128 + combine", "gbs": d_gbs, "frac_of_measured": d_gbs / peak,
-                        "frac_of_8tbs": d_gbs / 8000.0, "us": 1e6 * t_d, "algorithmic_bytes": db_bytes},
-        "quantize": {"rows_per_s": w.num_layers * w.n_tok * w.num_kv_heads * 2 / t_q, "gbs": q_gbs,
-                     "frac_of_8tbs": q_gbs / 8000.0, "us": 1e6 * t_q},
-        "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (3 if w.mla else 4) * K,  # quantize (K[, V]), decode, combine
-        "clocks": clk.summary(),
+        "quantize": summ["quantize"],
+        "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        # quantize: one launch per quantised stream (latent, or K and V); decode:
+        # decode + combine (MLA: query prep + decode + combine)
+        "gpu_launches": (1 if w.mla else 2) * K + (0 if r["q_only"] else (3 if w.mla else 2) * K),
+        "clocks": r["clocks"],
     }
-    if w.mla:   # decode attention is a dense contraction over 128 heads: tensor-bound
-        flops = 2.0 * w.batch * w.seq_len * w.num_q_heads * (w.head_dim + w.rope_dim + w.head_dim)
-        tf = flops / t_d / 1e12
-        tpeak = load_tensor_peak()
-        line["decode_attn"].update({"tflops": tf, "frac_of_tensor_peak": tf / tpeak[0], "tensor_peak": tpeak[0],
-                                    "tensor_peak_source": tpeak[1], "flops": flops})
-        if t_d >= t_q:
-            line["roofline"] = {"kernel": "decode_mla (tcgen05)", "bound": "tensor", "achieved": tf,
-                                "peak": tpeak[0], "unit": "TFLOP/s", "frac": tf / tpeak[0],
-                                "peak_source": tpeak[1] + " bf16 dense (f16 same rate)", "traffic": None,
-                                "algorithmic_flops": flops}
+    if "decode_attn" in summ:
+        line["decode_attn"] = summ["decode_attn"]
+        if w.mla and t_d >= t_q:
+            d = summ["decode_attn"]
+            line["roofline"] = {"kernel": dk, "bound": "tensor", "achieved": d["tflops"], "peak": d["tensor_peak"],
+                                "unit": "TFLOP/s", "frac": d["frac_of_tensor_peak"],
+                                "peak_source": d["tensor_peak_source"] + " bf16 dense (f16 same rate)",
+                                "traffic": None, "algorithmic_flops": d["flops"]}
+    if world == 1 and not args.no_extra:
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            wx = W_WORKLOADS()[name]
+            rx = measure(wx, min(K, 10), 3, e2e=False)
+            rx["steps"] = min(K, 10)
+            sx = summarize(wx, rx, peak)
+            sx["tokens_per_s"] = wx.batch * wx.seq_len / (rx["elapsed"] / rx["steps"])
+            if name == "rt1k":
+                sx["note"] = "L2-resident: latency, not a roofline figure"
+            extra[name] = sx
+        line["workloads"] = extra
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))
+
+
+def W_WORKLOADS():
+    from kv_cache_quantization_03_b200 import workloads as W
+    return W.WORKLOADS
 
 
 def main():
@@ -413,9 +511,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--workload", default="long")
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time the chosen workload only")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling small cases)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the context length")
     args = ap.parse_args()

@@ -234,8 +234,13 @@ kvq_status kvq_decode_attention_tail(const kvq_config* cfg, const kvq_cache_view
  * exits); nothing is allocated.  Shapes that need more than 8 MiB (see
  * kvq_decode_workspace_bytes with max_seq_len = max_pages_per_seq *
  * tile_tokens) return KVQ_ERR_WORKSPACE_TOO_SMALL before any launch.
- * The first call on a device looks up the array's address on that device,
- * so make that first call before any stream capture.  All calls share the
+ * The first call on a device looks up the array's address on that device
+ * and keeps it, so make that first call before any stream capture.  A
+ * device reset (cudaDeviceReset) invalidates the kept address: do not call
+ * this entry point again after one.  A call that fails with KVQ_ERR_CUDA
+ * drops the kept address, and the next call looks it up again.  Sizes are
+ * checked after every other argument: KVQ_ERR_WORKSPACE_TOO_SMALL means the
+ * call was otherwise valid.  All calls share the
  * array and it keeps the last call's contents (nothing in it needs to start
  * at zero): calls that overlap on the GPU, on any streams of the process,
  * race and give wrong results; serialise them. */
@@ -244,6 +249,17 @@ kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache_v
                                         int32_t max_pages_per_seq, const int32_t* seq_lens,
                                         int32_t batch, int32_t num_q_heads, float softmax_scale,
                                         float* out, uint32_t* dev_error, void* stream);
+
+/* Testing hook for the failure path of the bounded device waits (the pages
+ * have no counterpart).  With ns > 0, every CTA of each later GQA decode
+ * call (kvq_decode_attention and its variants) first waits, for at most ns
+ * nanoseconds of GPU time, on a device flag that nothing ever sets.  The
+ * wait runs out before the CTA issues any copy: the CTA sets
+ * KVQ_DEVERR_TIMEOUT, skips its tiles and returns, so the call ends with
+ * zeros in place of the attention output and kvq_read_error reports
+ * KVQ_ERR_TIMEOUT.  ns = 0 (the default) turns the hook off.  Process-wide;
+ * affects only calls made after it. */
+void kvq_set_test_wait(uint32_t ns);
 
 /* Synchronise `stream`, copy the device error word to *host_bits and reset
  * it to 0.  KVQ_ERR_TIMEOUT if the TIMEOUT bit was set, else KVQ_OK (other

@@ -4,6 +4,7 @@
 // include/kvq.h.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdio>
@@ -15,12 +16,29 @@ using namespace kvq;
 
 namespace {
 
-constexpr int kNumSMs = 148;           // B200
+// Testing hook (kvq_set_test_wait): 0 in normal use.
+std::atomic<uint32_t> g_test_wait_ns{0};
+
+constexpr int kDefaultSMs = 148;       // B200, when no device can be queried (host-only sizing)
 constexpr int kDecodeCtasPerSm = 4;      // resident decode CTAs per SM (registers and shared memory)
 constexpr int kDecodeWarps = 4;        // warps per decode CTA (tiles are dealt round robin)
 constexpr int kMaxGroup = 8;
 
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// SMs of the current device (the split plans size their grids by it); the
+// B200's 148 when there is no device.  kvq_decode_workspace_bytes and the
+// decode calls use the same count, so a workspace sized on a device fits
+// the calls made on it.
+int num_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();  // clear the error the failed query left behind
+    return kDefaultSMs;
+  }
+  return sms;
+}
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 
@@ -101,7 +119,7 @@ struct DecodePlan {
 DecodePlan decode_plan(int64_t pairs, int64_t max_tiles) {
   DecodePlan d{1, 0};
   if (pairs <= 0 || max_tiles <= 0) return d;
-  const int64_t slots = (int64_t)kDecodeCtasPerSm * kNumSMs;
+  const int64_t slots = (int64_t)kDecodeCtasPerSm * num_sms();
   const int64_t cap = (max_tiles + 4 * kDecodeWarps - 1) / (4 * kDecodeWarps);
   int64_t best = 1, best_cost = INT64_MAX;
   for (int64_t s = 1; s <= cap && s <= 256; ++s) {
@@ -121,7 +139,7 @@ size_t decode_ws_bytes(int64_t pairs, const DecodePlan& d, int head_dim) {
   return (size_t)pairs * d.splits * kMaxGroup * ((size_t)head_dim + 2) * sizeof(float);
 }
 
-// MLA: one CTA pair per (sequence, split), one CTA per SM, so kNumSMs / 2
+// MLA: one CTA pair per (sequence, split), one CTA per SM, so (SMs / 2)
 // pairs run at once.  The split count minimises (waves) x (32-token chunks
 // per split + a fixed cost of about four chunks for the query fetch, the
 // output write and the combine); a split has an even number of tiles.
@@ -129,7 +147,7 @@ constexpr int kMlaHeads = 128;
 DecodePlan decode_plan_mla(int64_t batch, int64_t max_tiles) {
   DecodePlan d{1, 2};
   if (batch <= 0 || max_tiles <= 0) return d;
-  const int64_t slots = kNumSMs / 2, chunks = (max_tiles + 1) / 2;
+  const int64_t slots = num_sms() / 2, chunks = (max_tiles + 1) / 2;
   int64_t best = 1, best_cost = INT64_MAX;
   for (int64_t s = 1; s <= chunks && s <= 64; ++s) {
     const int64_t per = (chunks + s - 1) / s, waves = (batch * s + slots - 1) / slots;
@@ -365,6 +383,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   p.tail_f16 = c->in_dtype == KVQ_F16;
   p.tail_tokens = c->tile_tokens;
   p.hblock = c->hadamard_block;
+  p.test_wait_ns = g_test_wait_ns.load(std::memory_order_relaxed);
   return cuda_status(launch_decode_d128(p, stream));
 }
 
@@ -395,6 +414,8 @@ kvq_status kvq_decode_attention_tail(const kvq_config* c, const kvq_cache_view* 
                 v_tail, tail_lens, batch, num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error,
                 stream);
 }
+
+void kvq_set_test_wait(uint32_t ns) { g_test_wait_ns.store(ns, std::memory_order_relaxed); }
 
 kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream) {
   if (!dev_error || !host_bits) return KVQ_ERR_INVALID_ARG;

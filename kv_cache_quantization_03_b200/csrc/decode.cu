@@ -206,6 +206,22 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+// A device word that nothing ever sets: the testing hook's wait polls it
+// until its time limit runs out.
+__device__ uint32_t g_never_set = 0;
+
+// Testing hook: lane 0 polls g_never_set for at most `ns` nanoseconds; true
+// if the flag was seen set (never, by construction).
+__device__ __forceinline__ bool wait_never_set(uint32_t ns) {
+  uint64_t t0, t1;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (;;) {
+    if (*reinterpret_cast<volatile uint32_t*>(&g_never_set)) return true;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+    if (t1 - t0 >= ns) return false;
+  }
+}
+
 // NH = 1: one kv-head per CTA, its (up to 8) query heads on the MMA's 8
 // columns.  NH = 2 (groups of at most 4 query heads): two adjacent kv-heads
 // per CTA; head slot n (column n of the MMAs) is query head n % 4 of kv-head
@@ -319,6 +335,18 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     tmem_st32(tq, qr);
   }
 
+  // Testing hook (kvq_set_test_wait): a bounded wait on a flag that nothing
+  // sets runs out before any copy is issued; the warp reports a timeout and
+  // skips its tiles, so nothing is in flight when it leaves.
+  int n_run = my_n;
+  if (p.test_wait_ns) {
+    const bool got = __shfl_sync(0xffffffffu, lane == 0 ? (int)wait_never_set(p.test_wait_ns) : 0, 0) != 0;
+    if (!got) {
+      n_run = 0;
+      if (lane == 0) set_error(p.err, KVQ_DEVERR_TIMEOUT);
+    }
+  }
+
   // ---- producer: lane 0 fills stage (i % kStages) with local tile i
   auto issue = [&](int i) {
     if (lane != 0) return;
@@ -362,7 +390,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       bulk_g2s(st + SL.off_vc + h * (kD * 4), p.v.chan + sh * kD, kD * 4, bar);
     }
   };
-  const int pre = my_n < kStages ? my_n : kStages;
+  const int pre = n_run < kStages ? n_run : kStages;
   for (int i = 0; i < pre; ++i) issue(i);
   int issued = pre;
 
@@ -374,7 +402,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
   int stop = -1;  // local tile whose wait ran out
-  for (int i = 0; i < my_n; ++i) {
+  for (int i = 0; i < n_run; ++i) {
     const bool ok = mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
     if (!__all_sync(0xffffffffu, ok)) {
       stop = i;
@@ -513,7 +541,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       }
     }
     __syncwarp();
-    if (issued < my_n) {
+    if (issued < n_run) {
       // the stage's shared-memory reads by all lanes precede the async refill
       if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       issue(issued++);

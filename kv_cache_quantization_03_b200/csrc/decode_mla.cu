@@ -63,6 +63,8 @@ constexpr int kSboK = kKf / 8 * 128;         // 9216: next 8 rows of a dequantis
 constexpr int kQsBytes = kH * kKS * 2;       // 73728
 constexpr int kQtBytes = kH * kKT * 2;       // 73728
 constexpr int kKbBytes = kChunk * kKf * 2;   // 36864 per buffer
+// prepared queries of one sequence: shared-memory part | tensor-memory part | per-head exponent (int)
+constexpr int kQprepBytes = kQsBytes + kQtBytes + kH * 4;
 constexpr int kOffQs = 0;
 constexpr int kOffKb = kOffQs + kQsBytes;
 __host__ __device__ constexpr int num_kb(int bits) { return bits == 8 ? 2 : 3; }  // dequantised chunk buffers
@@ -74,9 +76,11 @@ __host__ __device__ constexpr int stage_bytes(int bits) {
 }
 constexpr int kNS = 2;  // raw-tile stages
 __host__ __device__ constexpr int bar_offset(int bits) { return st_offset(bits) + kNS * stage_bytes(bits); }
-// full[2] dq[3] sfull[2] pfull[2] pv[4] qf qt, the TMEM address, then the tile-validity bits
-constexpr int kNumBars = kNS + 3 + 2 + 2 + 4 + 2;
-__host__ __device__ constexpr int vmask_offset(int bits) { return bar_offset(bits) + kNumBars * 8 + 8; }
+// full[2] dq[3] sfull[2] pfull[2] pv[4] qf qt fin, the TMEM address, the operand
+// exponents of the dequantised chunk buffers (int[4]), then the tile-validity bits
+constexpr int kNumBars = kNS + 3 + 2 + 2 + 4 + 3;
+__host__ __device__ constexpr int echunk_offset(int bits) { return bar_offset(bits) + kNumBars * 8 + 8; }
+__host__ __device__ constexpr int vmask_offset(int bits) { return echunk_offset(bits) + 16; }
 __host__ __device__ constexpr int smem_bytes(int bits, int tiles_per_split) {
   return vmask_offset(bits) + ((tiles_per_split + 31) / 32) * 4;
 }
@@ -170,8 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   uint64_t* pv = pfull + 2;
   uint64_t* qf = pv + 4;
   uint64_t* qt = qf + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qt + 1);
+  uint64_t* fin = qt + 1;  // every MMA of the CTA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + vmask_offset(BITS));
+  int* echunk = reinterpret_cast<int*>(smem + echunk_offset(BITS));  // [NB]: operand exponent of each buffer
   const uint32_t s_base = smem_u32(smem);
 
   const int seq_raw = p.seq_lens[b];
@@ -186,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   const int ntl = t1 > t0 ? t1 - t0 : 0;
   const int nchunks = (ntl + 1) / 2;
   const int32_t* btab = p.block_table + (size_t)b * p.max_pages + t0;
-  const uint8_t* qprep = p.qprep + (size_t)b * (kQsBytes + kQtBytes);
+  const uint8_t* qprep = p.qprep + (size_t)b * kQprepBytes;
 
   // which tiles of the split have a valid page (bit lt of vmask)
   for (int i = tid; i < (ntl + 31) / 32; i += kThreads) vmask[i] = 0u;
@@ -212,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
     for (int i = 0; i < 4; ++i) mbar_init(&pv[i], 1);
     mbar_init(qf, 1);
     mbar_init(qt, kH);
+    mbar_init(fin, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -267,10 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
         issue(c + NS, pg_next);
         pages_of(c + NS + 1, pg_next);  // in flight until the next chunk
       }
-      ok &= mbar_wait_bounded(qf, 0u, ok ? kWaitLimit : 0u);
-      // no bulk copy may still be writing when the CTA exits
+      // No bulk copy may still be writing when the CTA exits: every chunk is
+      // issued (also after a timeout), and only the last NS can be in flight.
+      // These waits take the full limit even after an earlier wait gave up.
+      ok &= mbar_wait_bounded(qf, 0u, kWaitLimit);
       for (int c = nchunks > NS ? nchunks - NS : 0; c < nchunks; ++c)
-        ok &= mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, ok ? kWaitLimit : 0u);
+        ok &= mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, kWaitLimit);
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA (one thread)
@@ -308,6 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
           umma_commit(&pv[x & 3]);
         }
       }
+      // every MMA issued above has completed before tensor memory is freed
+      // (full limit, also after a timeout)
+      umma_commit(fin);
+      ok &= mbar_wait_bounded(fin, 0u, kWaitLimit);
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- dequantisation
@@ -327,6 +340,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       const uint8_t* st = smem + kOffSt + (c % NS) * SB;
       uint8_t* kb = smem + kOffKb + (c % NB) * kKbBytes;
       const bool valid = tile_ok(2 * c + j);
+      // Operand scale of the chunk: the stored c is at most 1, so a row's
+      // dequantised latent is bounded by max(|z|, |a (2^b - 1) + z|).  The
+      // exact power of two 2^-e (e >= 0) that keeps the chunk's bound below
+      // 2^14 multiplies the latent and the rope keys, so the f16 operands
+      // cannot overflow; the softmax multiplies the chunk's scores by 2^e
+      // and weighs its values by it.  Every warp computes e from lane l's
+      // token (tile l / 16, row l % 16).
+      int e_chunk;
+      {
+        const float2 az = *reinterpret_cast<const float2*>(st + kStAz + (lane >> 4) * kT * 8 + (lane & 15) * 8);
+        constexpr float kQm = (float)((1 << BITS) - 1);
+        float bnd = tile_ok(2 * c + (lane >> 4)) ? fmaxf(fabsf(az.y), fabsf(fmaf(az.x, kQm, az.y))) : 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) bnd = fmaxf(bnd, __shfl_xor_sync(0xffffffffu, bnd, off));
+        e_chunk = max(0, (int)(__float_as_uint(bnd) >> 23) - 140);  // bnd < 2^(E - 126): 2^-e bnd < 2^14
+        if (dw == 0 && lane == 0) echunk[c % NB] = e_chunk;             // published by the dq arrive below
+      }
+      const float sE = __uint_as_float((uint32_t)(127 - e_chunk) << 23);
       f2 cc[4];
       {
         const float4* cp = reinterpret_cast<const float4*>(st + kStC + j * kLat * 4 + ch0 * 4);
@@ -337,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
 #pragma unroll
       for (int it = 0; it < 4; ++it) {
         const int tr = 8 * rh + ((lane + it + 4 * hf) & 7);
-        const float2 az = *reinterpret_cast<const float2*>(st + kStAz + j * kT * 8 + tr * 8);
+        float2 az = *reinterpret_cast<const float2*>(st + kStAz + j * kT * 8 + tr * 8);
+        az.x *= sE, az.y *= sE;
         float q[8];
         codes8<BITS>(st + j * CB, tr, ch0, q);
         uint32_t pk[4];
@@ -356,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
         const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pk[e] = v2 ? pack_f16x2(bf16f(w[e] & 0xFFFFu), bf16f(w[e] >> 16)) : 0u;
+        for (int e = 0; e < 4; ++e) pk[e] = v2 ? pack_f16x2(bf16f(w[e] & 0xFFFFu) * sE, bf16f(w[e] >> 16) * sE) : 0u;
         *reinterpret_cast<uint4*>(kb + cm_off(rrow, kLat + 8 * rgrp, kSboK)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       proxy_fence();
@@ -382,24 +414,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       tc_fence_before();
       mbar_arrive_local(qt);
     }
+    // the head's query was prepared times 2^-eq (see mla_prep_q_kernel)
+    const float s_q = __uint_as_float((uint32_t)(127 + reinterpret_cast<const int*>(qprep + kQsBytes + kQtBytes)[h])
+                                      << 23);
     float m_run = kNegBig, l_run = 0.f;
+    int e_ref = 0;  // the output accumulator holds sum p v 2^-e_ref (e_ref: largest chunk exponent so far)
     for (int x = 0; x < nchunks; ++x) {
       ok &= mbar_wait_bounded(&sfull[x & 1], (uint32_t)(x >> 1) & 1u, ok ? kWaitLimit : 0u);
+      // the chunk's operand exponent (its dequantisation is complete: the scores are)
+      ok &= mbar_wait_bounded(&dq[x % NB], (uint32_t)(x / NB) & 1u, ok ? kWaitLimit : 0u);
+      const int ex = echunk[x % NB];
       tc_fence_after();
       float sc[32];
       tmem_ld32(tmem + lane_base + kTmemS + 32 * (x & 1), sc);
       const bool tv[2] = {tile_ok(2 * x), tile_ok(2 * x + 1)};
+      // 2^ex 2^eq: the chunk's and the query's operand scales, undone
+      const float s_up = __uint_as_float((uint32_t)(127 + ex) << 23) * s_q;
       float mx = kNegBig;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        sc[i] = tv[i >> 4] ? sc[i] : kNegBig;
+        sc[i] = tv[i >> 4] ? sc[i] * s_up : kNegBig;
         mx = fmaxf(mx, sc[i]);
       }
       // lazy rescale; the TMEM accesses are warp-wide, so the whole warp
-      // joins (factor 1 where a head's max did not grow)
+      // joins (factor 1 where a head's max did not grow).  A chunk with a
+      // larger operand exponent rescales the accumulator too (chunk-uniform).
       const bool grow = mx > m_run + 8.f;
       const float alpha = grow ? ex2f(m_run - mx) : 1.f;
-      if (__any_sync(0xffffffffu, grow && x > 0)) {
+      const bool egrow = ex > e_ref;
+      const float alpha_o = egrow ? alpha * __uint_as_float((uint32_t)(127 + e_ref - ex) << 23) : alpha;
+      if (egrow) e_ref = ex;
+      if (__any_sync(0xffffffffu, (grow || egrow) && x > 0)) {
         ok &= mbar_wait_bounded(&pv[(x - 1) & 3], (uint32_t)((x - 1) >> 2) & 1u, ok ? kWaitLimit : 0u);
         tc_fence_after();
 #pragma unroll 1
@@ -407,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
           float o[32];
           tmem_ld32(tmem + lane_base + c0, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          for (int i = 0; i < 32; ++i) o[i] *= alpha_o;
           tmem_st32(tmem + lane_base + c0, o);
         }
       }
@@ -419,12 +464,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
         ok &= mbar_wait_bounded(&pv[(x - 2) & 3], (uint32_t)((x - 2) >> 2) & 1u, ok ? kWaitLimit : 0u);
       uint32_t pk[16];
       float ls = 0.f;
+      // weights of this chunk's (scaled) values: p 2^(ex - e_ref), ex <= e_ref
+      const float wsc = ex - e_ref >= -126 ? __uint_as_float((uint32_t)(127 + ex - e_ref) << 23) : 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float p0 = tv[i >> 3] ? ex2f(sc[2 * i] - m_run) : 0.f;
         const float p1 = tv[i >> 3] ? ex2f(sc[2 * i + 1] - m_run) : 0.f;
         ls += p0 + p1;
-        pk[i] = pack_f16x2(p0, p1);
+        pk[i] = pack_f16x2(p0 * wsc, p1 * wsc);
       }
       l_run += ls;
       tmem_st16(tmem + lane_base + kTmemP + 16 * (x & 1), pk);
@@ -439,9 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       ok &= mbar_wait_bounded(&pv[x & 3], (uint32_t)(x >> 2) & 1u, ok ? kWaitLimit : 0u);
       tc_fence_after();
 #pragma unroll 1
+      const float s_out = __uint_as_float((uint32_t)(127 + e_ref) << 23);  // 2^e_ref
       for (int c0 = 0; c0 < kHalf; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + c0, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= s_out;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           *reinterpret_cast<float4*>(po + c0 + 4 * i) = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
@@ -463,15 +513,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
 
 // Rotated, pre-scaled f16 queries of one sequence: element k of head h is
 // (H_512 q_lat)[k] * scale * log2(e) / sqrt(512) for k < 512 and
-// q_rope[k - 512] * scale * log2(e) after; k in [0, 288) row-major, k in
-// [288, 576) in the shared-memory operand layout.  One warp per head: lane l
-// keeps latent elements 16l..16l+15; index bits 0..3 are butterflies in
-// registers, bits 4..8 shuffles.
+// q_rope[k - 512] * scale * log2(e) after, both times 2^-eq_h; k in
+// [0, 288) row-major, k in [288, 576) in the shared-memory operand layout,
+// then eq_h (int) per head.  eq_h is the power of two that brings the
+// head's largest element into [2^7, 2^8): queries of any magnitude keep
+// f16's relative precision, and the softmax multiplies the head's scores by
+// 2^eq_h.  One warp per head: lane l keeps latent elements 16l..16l+15;
+// index bits 0..3 are butterflies in registers, bits 4..8 shuffles.
 __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
   const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* out_s = p.qprep + (size_t)b * (kQsBytes + kQtBytes);
+  uint8_t* out_s = p.qprep + (size_t)b * kQprepBytes;
   uint8_t* out_t = out_s + kQsBytes;
-  const float f = p.scale_log2 * 0.044194173824159216f;  // 1 / sqrt(512)
+  int* out_e = reinterpret_cast<int*>(out_t + kQtBytes);
+  const float f0 = p.scale_log2 * 0.044194173824159216f;  // 1 / sqrt(512)
   for (int h = warp; h < kH; h += 8) {
     float v[16];
     const bool live = h < p.num_q_heads;
@@ -504,6 +558,29 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
         v[i] = upper ? (o - v[i]) : (v[i] + o);
       }
     }
+    // the head's rope elements (lanes 0..7, eight each) and its exponent
+    float rp[8];
+    {
+      const uint4 x = lane < kRope / 8 ? *reinterpret_cast<const uint4*>(qh + kLat + 8 * lane) : make_uint4(0, 0, 0, 0);
+      const uint32_t a[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        rp[2 * e] = live ? bf16f(a[e] & 0xFFFFu) * p.scale_log2 : 0.f;
+        rp[2 * e + 1] = live ? bf16f(a[e] >> 16) * p.scale_log2 : 0.f;
+      }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i] * f0));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(rp[i]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    // mx in [2^(E-127), 2^(E-126)): eq = E - 134 puts it in [2^7, 2^8)
+    const int eq = mx > 0.f ? min(max((int)(__float_as_uint(mx) >> 23) - 134, -126), 126) : 0;
+    const float down = __uint_as_float((uint32_t)(127 - eq) << 23);  // 2^-eq, eq in [-126, 126]
+    const float f = f0 * down;
+    if (lane == 0) out_e[h] = eq;
     uint4 w[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k)
@@ -518,12 +595,9 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
       *reinterpret_cast<uint4*>(out_s + cm_off(h, k0 + 8 - kKT, kSboQ)) = w[1];
     }
     if (lane < kRope / 8) {
-      const uint4 x = *reinterpret_cast<const uint4*>(qh + kLat + 8 * lane);
-      const uint32_t a[4] = {x.x, x.y, x.z, x.w};
       uint32_t pk[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        pk[e] = live ? pack_f16x2(bf16f(a[e] & 0xFFFFu) * p.scale_log2, bf16f(a[e] >> 16) * p.scale_log2) : 0u;
+      for (int e = 0; e < 4; ++e) pk[e] = pack_f16x2(rp[2 * e] * down, rp[2 * e + 1] * down);
       *reinterpret_cast<uint4*>(out_s + cm_off(h, kLat - kKT + 8 * lane, kSboQ)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
@@ -568,7 +642,7 @@ int launch_mla_bits(const MlaDecodeParams& p, cudaStream_t s) {
 
 }  // namespace
 
-size_t mla_qprep_bytes(int64_t batch) { return (size_t)batch * (kQsBytes + kQtBytes); }
+size_t mla_qprep_bytes(int64_t batch) { return (size_t)batch * kQprepBytes; }
 
 int launch_decode_mla(const MlaDecodeParams& p, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -26,8 +26,10 @@ std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  The first
-// call on a device looks it up (cudaGetSymbolAddress) and caches it.
-kvq_status scratch_address(void** out) {
+// call on a device looks it up (cudaGetSymbolAddress) and caches it; a
+// device reset invalidates the cache, and a failed lookup or launch clears
+// the entry so that the next call looks it up again.
+kvq_status scratch_address(int* dev_out, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
@@ -36,8 +38,14 @@ kvq_status scratch_address(void** out) {
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
     g_scratch_addr[dev] = p;
   }
+  *dev_out = dev;
   *out = g_scratch_addr[dev];
   return KVQ_OK;
+}
+
+void forget_scratch_address(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_scratch_addr[dev] = nullptr;
 }
 
 }  // namespace
@@ -53,9 +61,18 @@ extern "C" kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const 
   kvq_status st = kvq_decode_workspace_bytes(cfg, batch, num_q_heads,
                                              max_pages_per_seq * cfg->tile_tokens, &need);
   if (st != KVQ_OK) return st;
-  if (need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE_TOO_SMALL;
+  if (need > kNoAllocScratchBytes) {
+    // Too big for the scratch array.  The workspace call validates every
+    // other argument first and launches nothing without a workspace, so a
+    // bad argument is reported as such rather than as the size.
+    return kvq_decode_attention(cfg, cache, layer, q, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                                softmax_scale, out, nullptr, 0, dev_error, stream);
+  }
   void* scratch = nullptr;
-  if ((st = scratch_address(&scratch)) != KVQ_OK) return st;
-  return kvq_decode_attention(cfg, cache, layer, q, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
-                              softmax_scale, out, scratch, kNoAllocScratchBytes, dev_error, stream);
+  int dev = 0;
+  if ((st = scratch_address(&dev, &scratch)) != KVQ_OK) return st;
+  st = kvq_decode_attention(cfg, cache, layer, q, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                            softmax_scale, out, scratch, kNoAllocScratchBytes, dev_error, stream);
+  if (st == KVQ_ERR_CUDA) forget_scratch_address(dev);
+  return st;
 }

@@ -91,6 +91,7 @@ struct DecodeParams {
   int tail_f16;                 // 1: fp16 rows, 0: bf16
   int tail_tokens;              // T
   int hblock;                   // Hadamard block: 8 .. 128 channels
+  uint32_t test_wait_ns;        // testing only: > 0 makes every CTA first wait this long on a flag nothing sets
 };
 
 struct MlaDecodeParams {

@@ -98,6 +98,30 @@ __device__ __forceinline__ float rsqrt_nr(float x) {
   return y * fmaf(-0.5f * x * y, y, 1.5f);
 }
 
+// Four per-lane values x[h][tp] of tokens 8h + 2t + tp (this lane's channels)
+// reduced with `op` over the eight lanes g that share t; returns the value of
+// the token this lane owns, 8 b2 + 2t + b1 (b1 = lane bit 3, b2 = lane bit 4).
+template <typename Op>
+__device__ __forceinline__ float reduce_tokens(const float (&x)[2][2], int b1, int b2, Op op) {
+  const float k0 = op(b2 ? x[1][0] : x[0][0], __shfl_xor_sync(0xffffffffu, b2 ? x[0][0] : x[1][0], 16));
+  const float k1 = op(b2 ? x[1][1] : x[0][1], __shfl_xor_sync(0xffffffffu, b2 ? x[0][1] : x[1][1], 16));
+  const float r = op(b1 ? k1 : k0, __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 8));
+  return op(r, __shfl_xor_sync(0xffffffffu, r, 4));
+}
+
+// Squares paired along channels: A[h][tp][q] = channels 2q, 2q+1 (of 16g + ..)
+// of token 8h + 2t + tp.
+__device__ __forceinline__ void square_pairs(const f2 (&P)[2][2][8], f2 (&A)[2][2][8]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const f2 x = P[h][q >> 2][2 * (q & 3)], y = P[h][q >> 2][2 * (q & 3) + 1];
+      A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
+      A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
+    }
+}
+
 // Byte 0 of four words, in order: the code held by a magic-number float.
 __device__ __forceinline__ uint32_t gather4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x4000u), 0x7610u);
@@ -152,6 +176,7 @@ struct TileShare {
   float2 x[4][32][32];   // per block, per register pair, per lane: values for the H_4 combination
   float row[2][4][kT];   // row partial sums, double-buffered by round parity
   float2 mm[4][kT];      // per block and token: (min, max)
+  float cmax[4];         // per block: largest column factor
 };
 
 template <int D>
@@ -259,7 +284,6 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
   // shared memory by cp.async (the next one while the current one is
   // processed), which keeps that kernel at 128 registers (four CTAs per SM).
   constexpr bool kStage = (W == 1);
-  constexpr bool kPark = true;
   constexpr int kLogDT = log2_dt<D, TW>();
   constexpr int kTmemCols = 64 * (kCW / 4);  // 64 columns per warp, four lane quarters
   __shared__ WarpScratch scratch[kCW];
@@ -284,7 +308,7 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
   const uint32_t stride = gridDim.x * TPC;
   uint32_t tile = blockIdx.x * TPC + slot_id;
   uint32_t tpark = 0;             // this warp's 64 TMEM columns
-  if constexpr (kPark) {
+  {
     if (warp == 0) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
                    "n"(kTmemCols));
@@ -346,17 +370,10 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
         P[i >> 4][(i >> 3) & 1][i & 7] = acc;
       }
     }
-    // squares paired along channels: A[h][tp][q] = channels 2q, 2q+1 of token 8h + 2t + tp
     f2 A[2][2][8];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const f2 x = P[h][q >> 2][2 * (q & 3)], y = P[h][q >> 2][2 * (q & 3) + 1];
-        A[h][0][q] = make_float2(x.x * x.x, y.x * y.x);
-        A[h][1][q] = make_float2(x.y * x.y, y.y * y.y);
-      }
-    if constexpr (kPark) {  // park the rotated tile in tensor memory until the factors are known
+    square_pairs(P, A);
+    // park the rotated tile in tensor memory until the factors are known
+    auto park = [&]() {
       float v[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -367,14 +384,24 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
         }
         tmem_st32(tpark + 32 * half, v);
       }
-    }
+    };
+    auto unpark = [&]() {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(tpark + 32 * half, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) P[half][i >> 3][i & 7] = make_float2(v[2 * i], v[2 * i + 1]);
+      }
+    };
+    park();
     float w[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 1.f;
-    float v_own = 1.f;
-    float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
-    f2 c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
-    for (int it = 0; it < p.iters; ++it) {
+    // Row sums of A / c^2 (the row step), for the token this lane owns
+    // (8 b2 + 2t + b1); at 512 channels the four blocks' sums are added through
+    // shared memory (buffer `par`, alternating between rounds).
+    auto row_sums = [&](int par) -> float {
       float R[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -389,21 +416,81 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
           const f2 s2 = add2(acc0, acc1);
           R[h][tp] = s2.x + s2.y;
         }
-      float k0 = b2 ? R[1][0] : R[0][0], k1 = b2 ? R[1][1] : R[0][1];
-      k0 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][0] : R[1][0], 16);
-      k1 += __shfl_xor_sync(0xffffffffu, b2 ? R[0][1] : R[1][1], 16);
-      float rk = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 8);
-      rk += __shfl_xor_sync(0xffffffffu, rk, 4);  // token 8*b2 + 2t + b1, this block's channels
+      float rk = reduce_tokens(R, b1, b2, [](float a, float b) { return a + b; });
       if constexpr (W > 1) {
         const int tok = 8 * b2 + 2 * t + b1;
-        if ((lane & 4) == 0) sh.row[it & 1][blk][tok] = rk;
+        if ((lane & 4) == 0) sh.row[par][blk][tok] = rk;
         __syncthreads();
-        rk = sh.row[it & 1][0][tok];
+        rk = sh.row[par][0][tok];
 #pragma unroll
-        for (int k = 1; k < W; ++k) rk += sh.row[it & 1][k][tok];
+        for (int k = 1; k < W; ++k) rk += sh.row[par][k][tok];
       }
-      // a zero row (rk = 0) only ever multiplies zeros, so its factor may be anything finite
-      v_own = rcp_fast(fmaxf(rk, 1e-30f));
+      return rk;
+    };
+    // Dynamic range.  The rounds run on fp32 squares of the rotated tile.  A
+    // row whose sum of squares is zero or outside [2^-60, 2^60] (an input row
+    // far from unit scale, or an all-zero row) is divided by a power of two
+    // 2^e taken from its largest |value| before squaring.  That is exact, and
+    // the method is invariant to it: the column factors only see A_ij / r_i^2,
+    // and the codes only the row's affine map; a and z are multiplied back by
+    // 2^e at the end.  An all-zero row keeps scale 1 and contributes nothing.
+    float rsc_own = 1.f;  // 2^e of the owned token's row
+    float rk = 0.f;
+    if (p.iters > 0) {
+      rk = row_sums(0);
+      const bool odd = !(rk >= 0x1p-60f && rk <= 0x1p60f);
+      if (__any_sync(0xffffffffu, odd)) {  // warp-uniform; at 512 channels tile-uniform too
+        unpark();
+        float mx[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int tp = 0; tp < 2; ++tp) {
+            float m = 0.f;
+#pragma unroll
+            for (int b = 0; b < 16; ++b) {
+              const f2 x = P[h][b >> 3][b & 7];
+              m = fmaxf(m, fabsf(tp ? x.y : x.x));
+            }
+            mx[h][tp] = m;
+          }
+        float omx = reduce_tokens(mx, b1, b2, [](float a, float b) { return fmaxf(a, b); });
+        if constexpr (W > 1) {
+          const int tok = 8 * b2 + 2 * t + b1;
+          if ((lane & 4) == 0) sh.mm[blk][tok] = make_float2(0.f, omx);
+          __syncthreads();
+#pragma unroll
+          for (int k = 0; k < W; ++k) omx = fmaxf(omx, sh.mm[k][tok].y);
+        }
+        // exponent field E of the row max, kept in [1, 253]: scale 2^(127-E)
+        // brings the max into [1, 2) (a subnormal max into (0, 1), a max of
+        // 2^127 or more into [2, 4)); a zero row keeps scale 1
+        const int e = min(max((int)(__float_as_uint(omx) >> 23), 1), 253);
+        const float s_own = omx > 0.f ? __uint_as_float((uint32_t)(254 - e) << 23) : 1.f;
+        rsc_own = omx > 0.f ? __uint_as_float((uint32_t)e << 23) : 1.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const f2 s2 = make_float2(__shfl_sync(0xffffffffu, s_own, (h << 4) | t),
+                                    __shfl_sync(0xffffffffu, s_own, (h << 4) | 8 | t));
+#pragma unroll
+          for (int b = 0; b < 16; ++b) P[h][b >> 3][b & 7] = mul2(P[h][b >> 3][b & 7], s2);
+        }
+        square_pairs(P, A);
+        park();
+        rk = row_sums(0);
+      }
+    }
+    // Per-round factors: v = (d/T) / R (row) and w = 1 / C (column) keep
+    // w = 1 / c^2 of the textbook recursion exactly, so the final column sums
+    // are c^2 itself.  A row or column whose sum is exactly 0 holds only
+    // zeros; its factor multiplies nothing and is set to 0 (its stored c is 1).
+    constexpr float kDT = kLogDT >= 0 ? (float)(1 << kLogDT) : 1.f / (float)(1 << -kLogDT);
+    float v_own = 1.f;
+    float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
+    f2 c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
+    for (int it = 0; it < p.iters; ++it) {
+      if (it > 0) rk = row_sums(it & 1);
+      v_own = rk > 0.f ? rcp_fast(rk) * kDT : 0.f;
       float v[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -439,11 +526,10 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
         }
         ++rounds;
       }
-      // likewise a zero column; its stored factor is set to 1 after the rounds
-      w_own.x = rcp_fast(fmaxf(c01.x, 1e-30f));
-      w_own.y = rcp_fast(fmaxf(c01.y, 1e-30f));
-      w_own.z = rcp_fast(fmaxf(c23.x, 1e-30f));
-      w_own.w = rcp_fast(fmaxf(c23.y, 1e-30f));
+      w_own.x = c01.x > 0.f ? rcp_fast(c01.x) : 0.f;
+      w_own.y = c01.y > 0.f ? rcp_fast(c01.y) : 0.f;
+      w_own.z = c23.x > 0.f ? rcp_fast(c23.x) : 0.f;
+      w_own.w = c23.y > 0.f ? rcp_fast(c23.y) : 0.f;
       sc.own[lane] = w_own;
       __syncwarp();
 #pragma unroll
@@ -453,36 +539,29 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       }
       __syncwarp();
     }
+    float cmax = 1.f;  // largest column factor of the tile
+    float4 cv4;        // this lane's four column factors
     {
       const bool norm = p.iters > 0;
-      // The rounds use v = 1 / R and w = 1 / C instead of d / R and T / C:
-      // every factor then differs from the textbook one by a power of two,
-      // and after n rounds c^2 = C / T = C' (d / T)^n, an exact scaling.
-      const float c2_scale = ldexpf(1.f, kLogDT * p.iters);
-      const float ct[4] = {c01.x, c01.y, c23.x, c23.y};
+      const float ct[4] = {c01.x, c01.y, c23.x, c23.y};  // c^2 of the owned channels
       float cv[4], ic[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float x = ct[i] * c2_scale;
+        const float x = ct[i];
         const float y = rsqrt_nr(x);
         const bool ok = norm && ct[i] > 0.f;
         ic[i] = ok ? y : 1.f;
         cv[i] = ok ? x * y : 1.f;
       }
-      if (wt == 0)
-        *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
-            make_float4(cv[0], cv[1], cv[2], cv[3]);
+      cmax = fmaxf(fmaxf(cv[0], cv[1]), fmaxf(cv[2], cv[3]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, off));
+      if constexpr (W > 1)
+        if (lane == 0) sh.cmax[blk] = cmax;  // read after the tile's min/max exchange below
+      cv4 = make_float4(cv[0], cv[1], cv[2], cv[3]);
       sc.dup[0][lane] = make_float4(ic[0], ic[0], ic[1], ic[1]);
       sc.dup[1][lane] = make_float4(ic[2], ic[2], ic[3], ic[3]);
-      if constexpr (kPark) {  // the rotated tile back from tensor memory
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float v[32];
-          tmem_ld32(tpark + 32 * half, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) P[half][i >> 3][i & 7] = make_float2(v[2 * i], v[2 * i + 1]);
-        }
-      }
+      unpark();  // the rotated tile back from tensor memory
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -525,14 +604,26 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       for (int k = 0; k < W; ++k) {
         const float2 x = sh.mm[k][tok];
         omn = fminf(omn, x.x), omx = fmaxf(omx, x.y);
+        cmax = fmaxf(cmax, sh.cmax[k]);
       }
+    }
+    // Stored balance: the power of two 2^kb with max c in (2^(kb-1), 2^kb]
+    // moves from c into a and z (exact; the dequantised tile is unchanged).
+    const uint32_t cbits = __float_as_uint(cmax);
+    const int kb = (int)(cbits >> 23) - 127 + ((cbits & 0x7FFFFFu) != 0u);
+    if (wt == 0) {
+      const float cs = __uint_as_float((uint32_t)(127 - kb) << 23);
+      *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
+          make_float4(cv4.x * cs, cv4.y * cs, cv4.z * cs, cv4.w * cs);
     }
     constexpr float kQmax = (float)((1 << BITS) - 1);
     const float s_own = (omx - omn) / kQmax;
     const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
+    // 1/sqrt(block) times the row's power of two times the balance 2^kb
+    const float fold = inv_sqrt_d * rsc_own * __uint_as_float((uint32_t)(127 + kb) << 23);
     if ((lane & 4) == 0 && blk == 0)
       *reinterpret_cast<float2*>(p.dst.tok + slot * (kTile * 2) + 2 * (kT * wt + 8 * b2 + 2 * t + b1)) =
-          make_float2(s_own * inv_sqrt_d, omn * inv_sqrt_d);
+          make_float2(s_own * fold, omn * fold);
     uint8_t* codes = p.dst.codes + slot * (kTile * D * BITS / 8);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -575,7 +666,7 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
     }
     tile_sync<W>();  // shared tile buffers are reused by the next tile
   }
-  if constexpr (kPark) {
+  {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 0)

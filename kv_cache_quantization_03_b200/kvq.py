@@ -40,7 +40,7 @@ KVQ_F16, KVQ_BF16, KVQ_F32 = 0, 1, 2
 EXPORTED = (
     "kvq_config_from_string", "kvq_cache_layout", "kvq_quantize_append", "kvq_dequantize",
     "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_tail",
-    "kvq_decode_attention_noalloc", "kvq_read_error",
+    "kvq_decode_attention_noalloc", "kvq_read_error", "kvq_set_test_wait",
     "kvq_status_string", "kvq_version",
 )
 
@@ -79,6 +79,7 @@ _sig = {
     "kvq_decode_attention_noalloc": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "kvq_read_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "kvq_set_test_wait": (None, [ctypes.c_uint32]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_version": (ctypes.c_char_p, []),
 }
@@ -204,6 +205,12 @@ def kvq_decode_attention_noalloc(cfg, view, layer, q, block_table, max_pages_per
                                           max_pages_per_seq, _ptr(seq_lens), batch, num_q_heads,
                                           float(softmax_scale), _ptr(out), _ptr(dev_error), _stream(stream))
     return _check("kvq_decode_attention_noalloc", st, raise_on_error)
+
+
+def kvq_set_test_wait(ns: int) -> None:
+    """Testing hook: later GQA decode calls first wait up to ns nanoseconds on a
+    device flag that nothing sets, report a timeout and skip their tiles (0: off)."""
+    lib.kvq_set_test_wait(int(ns))
 
 
 def kvq_read_error(dev_error, stream=None):

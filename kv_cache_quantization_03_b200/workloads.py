@@ -36,6 +36,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, Optional
 
 import numpy as np
@@ -192,19 +194,28 @@ def kv_inputs(w: Workload, which: str, tokens: Optional[slice] = None) -> np.nda
             for h in range(H):
                 ch = outlier_channels(dataclasses.replace(w, name=base), layer, h, which)
                 outl[layer, 0, h, ch] = factor
-    for layer in range(L):
-        for c0 in range(t0, t1, CHUNK_TOKENS):
-            c1 = min(c0 + CHUNK_TOKENS, t1)
-            r = _rng(w.seed, (kind << 40) | (layer << 24) | (c0 // CHUNK_TOKENS))
-            if base == "long" and which == "k":
-                x = r.standard_t(4.0, size=(c1 - c0, H, d)).astype(np.float32)
-            else:
-                x = r.standard_normal(size=(c1 - c0, H, d), dtype=np.float32)
-            if outl is not None:
-                x *= outl[layer]
-            if scale is not None:
-                x *= scale[layer]
-            out[layer, c0 - t0:c1 - t0] = _round_to(x, w.in_dtype)
+    def chunk(layer: int, c0: int) -> None:
+        c1 = min(c0 + CHUNK_TOKENS, t1)
+        r = _rng(w.seed, (kind << 40) | (layer << 24) | (c0 // CHUNK_TOKENS))
+        if base == "long" and which == "k":
+            x = r.standard_t(4.0, size=(c1 - c0, H, d)).astype(np.float32)
+        else:
+            x = r.standard_normal(size=(c1 - c0, H, d), dtype=np.float32)
+        if outl is not None:
+            x *= outl[layer]
+        if scale is not None:
+            x *= scale[layer]
+        out[layer, c0 - t0:c1 - t0] = _round_to(x, w.in_dtype)
+
+    # every chunk has its own stream, so the chunks may be drawn in any order
+    # (numpy's generators release the GIL: threads draw them in parallel)
+    jobs = [(layer, c0) for layer in range(L) for c0 in range(t0, t1, CHUNK_TOKENS)]
+    if len(jobs) <= 2:
+        for j in jobs:
+            chunk(*j)
+    else:
+        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda j: chunk(*j), jobs))
     return out
 
 

@@ -36,12 +36,55 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("long", dict(batch=2, seq_len=2048)),
     ("g128", dict(batch=3, seq_len=1024)),
     ("saw4", dict(batch=3, seq_len=512)),
+    ("prefill", dict(seq_len=1024, num_layers=2)),   # per-channel scales over two decades
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]
     w = w.scaled(**kw) if kw else w
     run = QuantRun(w)
     dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    _check(dec, o)
+
+
+def _pow2(bits: np.ndarray, dtype: str, e: int) -> np.ndarray:
+    """bf16/fp16 bit patterns times the exact power of two 2^e."""
+    return W._round_to((W.half_bits_to_f64(bits, dtype) * 2.0 ** e).astype(np.float32), dtype)
+
+
+@pytest.mark.parametrize("kv_exp,q_exp", [(20, 0), (-20, 0), (0, 8), (0, -8), (20, -8), (-20, 8)])
+@pytest.mark.parametrize("name", ["gqa", "long", "g128"])
+def test_decode_parity_input_magnitudes(name, kv_exp, q_exp):
+    # u = q~ c_K and w = p a_V / max(a_V) travel as f16 hi + lo pairs: the
+    # result must hold when keys, values and queries are far from unit scale
+    w = W.WORKLOADS[name].scaled(batch=2, seq_len=1024)
+    kb = _pow2(W.kv_inputs(w, "k"), w.in_dtype, kv_exp)
+    vb = _pow2(W.kv_inputs(w, "v"), w.in_dtype, -kv_exp)
+    run = QuantRun(w, inputs=(kb, vb))
+    dec = DecodeRun(run, q_bits=_pow2(W.queries(w), "bf16", q_exp))
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("lat_exp", [12, 14, 20, -12, -8])
+def test_mla_decode_parity_latent_magnitudes(lat_exp):
+    # The latent tiles meet the tensor cores as f16 operands: a chunk whose
+    # dequantised latent would pass the f16 range is scaled down by a power of
+    # two first (and the rope keys with it), and small latents keep f16's
+    # relative precision down to 2^-14.  The query's latent part is scaled the
+    # other way, so the logits stay at the workload's scale: with single f16
+    # operands the score carries ~2^-12 relative error, which the 2e-3
+    # tolerance absorbs only while |logits| stay of order ten (log2 units).
+    w = W.WORKLOADS["mla"].scaled(batch=2, seq_len=512)
+    kb = _pow2(W.kv_inputs(w, "k"), w.in_dtype, lat_exp)
+    run = QuantRun(w, inputs=(kb, None))
+    qb = W.queries(w).copy()
+    qb[..., : w.head_dim] = _pow2(qb[..., : w.head_dim], "bf16", -lat_exp)
+    dec = DecodeRun(run, q_bits=qb)
     o = dec()
     assert run.error_bits() == 0
     assert np.all(np.isfinite(o))
@@ -170,3 +213,23 @@ def test_decode_deterministic():
     a = dec()
     b = dec()
     assert np.array_equal(a, b)
+
+
+def test_decode_wait_timeout_reports_and_recovers():
+    # A bounded device wait that runs out (the testing hook makes every CTA
+    # wait 2 ms on a flag nothing sets) raises KVQ_DEVERR_TIMEOUT, the call
+    # still returns with nothing in flight, and the next call is correct.
+    w = W.WORKLOADS["gqa"].scaled(batch=2, seq_len=512)
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    kvq.kvq_set_test_wait(2_000_000)
+    try:
+        o = dec()
+    finally:
+        kvq.kvq_set_test_wait(0)
+    st, bits = kvq.kvq_read_error(run.err)
+    assert st == kvq.KVQ_ERR_TIMEOUT and bits & kvq.KVQ_DEVERR_TIMEOUT
+    assert np.all(o == 0)
+    o2 = dec()
+    assert run.error_bits() == 0
+    _check(dec, o2)

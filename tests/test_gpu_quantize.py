@@ -8,7 +8,7 @@ from oracle import kvarn_oracle as O
 
 pytestmark = pytest.mark.gpu
 
-from _parity import (CODE_FLIP_RATE, QuantRun, compare_quantized, oracle_fraction)  # noqa: E402
+from _parity import CODE_FLIP_RATE, QuantRun, check_tiles  # noqa: E402
 
 SMALL = {
     "rt1k": {},
@@ -24,19 +24,15 @@ SMALL = {
 def _check_all(run: QuantRun, tiles=None, heads=None, layers=None):
     w = run.w
     tiles = np.arange(w.n_tok // w.tile_tokens) if tiles is None else np.asarray(tiles)
-    flips = total = 0
+    flips = ties = total = 0
     for which in (("k",) if w.mla else ("k", "v")):
-        bits = w.bits_k if which == "k" else w.bits_v
         for layer in (range(w.num_layers) if layers is None else layers):
             for head in (range(w.num_kv_heads) if heads is None else heads):
-                x = run.input_tiles(which, layer, tiles, head)
-                ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block)
-                gpu = run.gpu_tiles(which, layer, tiles, head)
-                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters, w.block),
-                                           "%s L%d H%d" % (which, layer, head), check_rate=False)
-                total += gpu.q.size
-    assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes" % (flips, total)
-    return flips, total
+                f = check_tiles(run, which, layer, tiles, head, "%s L%d H%d" % (which, layer, head))
+                flips, ties = flips + f.counted, ties + f.exact_ties
+                total += len(tiles) * w.tile_tokens * w.head_dim
+    assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes (%d more at exact ties)" % (flips, total, ties)
+    return flips, ties, total
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -56,7 +52,7 @@ def test_quantize_parity_other_bit_widths(bits):
     _check_all(run)
 
 
-@pytest.mark.parametrize("iters", [0, 1, 9])
+@pytest.mark.parametrize("iters", [0, 1, 9, 64])
 @pytest.mark.parametrize("name", ["gqa", "g128"])
 def test_quantize_parity_iteration_counts(name, iters):
     import dataclasses
@@ -122,6 +118,46 @@ def test_quantize_parity_degenerate_tiles(tile):
     if tile == 16:
         zero = run.gpu_tiles("k", 0, [0], 0)
         assert np.all(zero.q == 0) and np.all(zero.a == 0) and np.all(zero.z == 0) and np.all(zero.c == 1)
+
+
+def _scaled(w, which, row_exp):
+    """The workload's inputs with token row i of every tile scaled by the exact
+    power of two 2^row_exp[i % T], rounded back to the input format (exact for
+    normal values)."""
+    x = W.half_bits_to_f64(W.kv_inputs(w, which), w.in_dtype)
+    e = np.asarray(row_exp, dtype=np.float64)
+    f = np.exp2(np.tile(e, x.shape[1] // e.size))[None, :, None, None]
+    return W._round_to((x * f).astype(np.float32), w.in_dtype)
+
+
+# exponent of every token row of a tile: unit rows, single rows far from the
+# others, and whole tiles near the ends of the bf16 range (kept in its normal
+# range: elements below 2^-126 would be subnormal inputs)
+ROW_SCALES = {
+    "one_row_2^-64": [0] * 5 + [-64] + [0] * 10,
+    "rows_2^-100_to_2^100": [0, -100, 60, 0, -30, 30, 0, -64, 0, 64, 0, 0, -96, 0, 100, 0],
+    "tile_2^-100": [-100] * 16,
+    "tile_2^+100": [100] * 16,
+}
+
+
+@pytest.mark.parametrize("scales", list(ROW_SCALES))
+@pytest.mark.parametrize("name,iters", [("gqa", 4), ("gqa", 0), ("long", 6), ("g128", 4), ("mla", 4)])
+def test_quantize_parity_dynamic_range(name, iters, scales):
+    # The method is invariant to a power-of-two scale of a token row (codes
+    # and column factors unchanged, a and z scaled): the kernel must follow
+    # the float64 oracle across the bf16 exponent range, including tiles whose
+    # rows differ by 2^200.
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS[name].scaled(batch=1, seq_len=256), sinkhorn_iters=iters)
+    e = ROW_SCALES[scales]
+    e = (e * (w.tile_tokens // 16))[: w.tile_tokens] if w.tile_tokens > 16 else e
+    kb = _scaled(w, "k", e)
+    vb = None if w.mla else _scaled(w, "v", e[::-1])
+    run = QuantRun(w, inputs=(kb, vb))
+    assert run.error_bits() == 0
+    flips, ties, total = _check_all(run)
+    assert flips + ties <= 1e-3 * total
 
 
 def test_quantize_bad_page_sets_error_and_skips_tile():

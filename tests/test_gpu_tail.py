@@ -14,7 +14,7 @@ from oracle import kvarn_oracle as O
 pytestmark = pytest.mark.gpu
 
 from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_error,  # noqa: E402
-                     compare_quantized, oracle_fraction)
+                     compare_quantized)
 
 
 def _check_tail(dec: DecodeRun, o: np.ndarray, layer=0, lens=None):
@@ -122,8 +122,8 @@ def test_quantize_on_fill_skips_partial_tails(name):
                 ch = run.cache.chan_scale(which)[layer, [5, 2], h].cpu().numpy()
                 gpu = O.QuantizedTiles(O.unpack_codes(raw, bits, w.tile_tokens, w.head_dim), tok[..., 0],
                                        tok[..., 1], ch)
-                flips += compare_quantized(gpu, ora, oracle_fraction(x, bits, w.sinkhorn_iters, w.block),
-                                           "%s L%d H%d" % (which, layer, h), check_rate=False)
+                flips += compare_quantized(gpu, ora, x, bits, w.sinkhorn_iters, w.block,
+                                           "%s L%d H%d" % (which, layer, h), check_rate=False).counted
                 total += gpu.q.size
     assert flips <= CODE_FLIP_RATE * total, "%d tie flips in %d codes" % (flips, total)
 
