@@ -51,12 +51,16 @@ Readings where the pages are silent (each is a declared choice):
   (2^(k-1), 2^k], c is stored times 2^-k and a, z times 2^k.  The scaling is
   exact, so the dequantised tile is unchanged, and every stored c is <= 1
   (a consumer can bound a dequantised row by max(|z|, |a (2^b - 1) + z|));
+* metadata format: float32 by default; the compact layout stores a, z, c
+  as IEEE half precision (round to nearest even from the balanced float64
+  values).  Codes do not depend on it;
 * codes are packed little-endian inside each byte, lowest channel in the
   lowest bits, token rows one after the other; 3-bit codes are two planes
   per tile: all rows' low 2 bits (2-bit packing), then all rows' high bit
   (1-bit packing).
 
-All arithmetic is float64 except the float32 rounding of the stored a, z, c.
+All arithmetic is float64 except the rounding of the stored a, z, c to the
+metadata format.
 Parity of every function here is pinned in tests/test_oracle_pins.py against
 closed forms, library routines, brute force and hand-worked fixtures.
 """
@@ -184,22 +188,36 @@ def balance_exponent(c32: np.ndarray) -> np.ndarray:
     return np.where(mant == 0.5, e - 1, e).astype(np.int64)
 
 
-def quantize_tiles(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] = None) -> QuantizedTiles:
+def quantize_stages(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] = None):
+    """The pipeline up to storage: rotate, normalise, RTN, balance.
+
+    Returns (q, a, z, c) with a, z, c in float64, already balanced by the
+    power of two 2^k (k decided on the float32 column factors, the precision
+    in which the stored c lives).  quantize_tiles rounds them for storage."""
+    z = rotate(x, block)
+    y, r, c = sinkhorn_normalize(z, n_iter)
+    q, m, s = rtn_rows(y, bits)
+    k = balance_exponent(c.astype(np.float32))
+    return q, np.ldexp(r * s, k[..., None]), np.ldexp(r * m, k[..., None]), np.ldexp(c, -k[..., None])
+
+
+def quantize_tiles(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] = None,
+                   meta: str = "f32") -> QuantizedTiles:
     """Rotate, normalise and quantise tiles x: [..., T, d] (any float dtype).
 
     The tiles are independent; leading axes only batch them.  block: the
     rotation's block (None = full width).  The stored scales are balanced
-    by a power of two (max c in (1/2, 1]; see the module notes).
+    by a power of two (max c in (1/2, 1]; see the module notes) and rounded
+    to nearest in the metadata format: meta "f32" (float32) or "f16" (IEEE
+    half: the compact layout, same codes, scales to 11 significant bits).
     """
-    z = rotate(x, block)
-    y, r, c = sinkhorn_normalize(z, n_iter)
-    q, m, s = rtn_rows(y, bits)
-    a32, z32, c32 = (r * s).astype(np.float32), (r * m).astype(np.float32), c.astype(np.float32)
-    k = balance_exponent(c32)
-    a32 = np.ldexp(a32, k[..., None]).astype(np.float32)
-    z32 = np.ldexp(z32, k[..., None]).astype(np.float32)
-    c32 = np.ldexp(c32, -k[..., None]).astype(np.float32)
-    return QuantizedTiles(q=q, a=a32, z=z32, c=c32)
+    q, a, z, c = quantize_stages(x, bits, n_iter, block)
+    if meta == "f32":
+        # the unbalanced float32 values times an exact power of two
+        return QuantizedTiles(q=q, a=a.astype(np.float32), z=z.astype(np.float32), c=c.astype(np.float32))
+    if meta == "f16":
+        return QuantizedTiles(q=q, a=a.astype(np.float16), z=z.astype(np.float16), c=c.astype(np.float16))
+    raise ValueError("meta must be 'f32' or 'f16'")
 
 
 def dequantize_tiles(q, a, z, c, unrotate: bool = True, block: Optional[int] = None) -> np.ndarray:

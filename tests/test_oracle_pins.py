@@ -266,6 +266,38 @@ def test_stored_scales_balanced_by_a_power_of_two():
     assert np.all(qt.c == 1.0)
 
 
+def _f16_neighbours(v16):
+    """The fp16 values just below and just above each fp16 value (brute force on the bit patterns)."""
+    b = v16.astype(np.float16).view(np.uint16).astype(np.int64)
+    up = np.where(b & 0x8000, b - 1, b + 1)           # toward +inf
+    dn = np.where(b & 0x8000, b + 1, b - 1)           # toward -inf
+    dn = np.where(b == 0, 0x8001, dn)                 # below +0: the smallest negative subnormal
+    return up.astype(np.uint16).view(np.float16).astype(np.float64), dn.astype(np.uint16).view(np.float16).astype(np.float64)
+
+
+def test_fp16_metadata_is_the_nearest_half_and_leaves_codes_alone():
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((24, 16, 128)) * np.exp(rng.uniform(-2, 2, (24, 1, 128)))
+    for n_iter, bits in ((4, 4), (0, 3), (6, 2)):
+        f32 = O.quantize_tiles(x, bits, n_iter)
+        f16 = O.quantize_tiles(x, bits, n_iter, meta="f16")
+        assert f16.a.dtype == np.float16 and f16.c.dtype == np.float16
+        assert np.array_equal(f16.q, f32.q)                       # codes do not see the format
+        _, a64, z64, c64 = O.quantize_stages(x, bits, n_iter)
+        for got, exact in ((f16.a, a64), (f16.z, z64), (f16.c, c64)):
+            g = got.astype(np.float64)
+            up, dn = _f16_neighbours(got)
+            err = np.abs(g - exact)
+            assert np.all(err <= np.abs(up - exact)) and np.all(err <= np.abs(dn - exact))   # nearest half
+        assert np.all(f16.c.astype(np.float64) <= 1.0) and np.all(f16.c.max(-1).astype(np.float64) >= 0.5)
+        # dequantised with half scales: within 2^-10 (relative, per element bound) of the float32 ones
+        d32 = O.dequantize_tiles(f32.q, f32.a, f32.z, f32.c, unrotate=False)
+        d16 = O.dequantize_tiles(f16.q, f16.a, f16.z, f16.c, unrotate=False)
+        bound = 2.0 ** -10 * (np.abs(f32.a)[..., None] * f32.q + np.abs(f32.z)[..., None] + 1e-30) * \
+            f32.c.astype(np.float64)[..., None, :] * 1.5
+        assert np.all(np.abs(d16 - d32) <= bound)
+
+
 def test_quantize_row_scale_invariance():
     # Scaling one token row by a power of two scales that row's a and z by it
     # and changes no code and no column factor: the row step divides it out
