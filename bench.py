@@ -69,8 +69,9 @@ def load_tensor_peak():
 def algorithmic_bytes(w):
     """(quantize bytes, decode bytes) one step must move, from the cache format."""
     T, d, H = w.tile_tokens, w.head_dim, w.num_kv_heads
+    mb = 2 if w.meta_f16 else 4                           # bytes of one a, z or c
     if w.mla:
-        lat_row = d * w.bits_k / 8 + 8 + d * 4 / T          # codes + (a, z) + channel-scale share
+        lat_row = d * w.bits_k / 8 + 2 * mb + d * mb / T    # codes + (a, z) + channel-scale share
         rope_row = w.rope_dim * 2
         tokens = w.num_layers * w.n_tok
         q_bytes = tokens * (d * 2 + rope_row) + tokens * (lat_row + rope_row)
@@ -79,7 +80,7 @@ def algorithmic_bytes(w):
     rows = w.num_layers * w.n_tok * H
     per_row_in = d * 2
     def cache_row(bits):                       # codes + (a, z) + c share of one row
-        return d * bits / 8 + 8 + d * 4 / T
+        return d * bits / 8 + 2 * mb + d * mb / T
     q_bytes = rows * 2 * per_row_in + rows * (cache_row(w.bits_k) + cache_row(w.bits_v))
     dec_bytes = w.batch * w.seq_len * H * (cache_row(w.bits_k) + cache_row(w.bits_v)) \
         + w.batch * w.num_q_heads * d * (2 + 4)
@@ -258,7 +259,7 @@ def config_dict(w, args):
             "num_kv_heads": w.num_kv_heads, "num_q_heads": w.num_q_heads, "head_dim": w.head_dim,
             "bits_k": w.bits_k, "bits_v": w.bits_v, "tile_tokens": w.tile_tokens,
             "sinkhorn_iters": w.sinkhorn_iters, "hadamard_block": w.hadamard_block or w.head_dim,
-            "layers": w.num_layers,
+            "metadata": "f16" if w.meta_f16 else "f32", "layers": w.num_layers,
             "parallelism": "dp%d (independent shards)" % args.gpus,
             "l2": ("inputs larger than L2 (latent + rope bf16 %.2f GB per rank)" % (
                 w.num_layers * w.n_tok * (w.head_dim + w.rope_dim) * 2 / 1e9)) if w.mla else
@@ -293,7 +294,7 @@ def max_over_ranks(values, world: int, device=None):
 
 # --------------------------------------------------------------------------- GPU leg
 QUANTIZE_ONLY = ("prefill",)       # workloads whose step is quantise-append alone
-EXTRA_WORKLOADS = ("gqa", "prefill", "mla", "g128", "saw4", "rt1k")
+EXTRA_WORKLOADS = ("gqa", "gqa16", "prefill", "mla", "g128", "saw4", "rt1k")
 
 
 def kernel_names(w):
@@ -317,7 +318,7 @@ def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                           bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                           rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype,
-                          hadamard_block=w.hadamard_block or None)
+                          hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16)
     cache = QuantizedCache(cfg)
     host = {"k": torch.from_numpy(W.kv_inputs(ws, "k").view(np.int16))}
     if w.mla:

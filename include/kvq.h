@@ -55,8 +55,11 @@
  *               lowest channel in the lowest bits (2, 4 or 8 bits); 3-bit
  *               codes are a plane of all rows' low 2 bits (2-bit packing)
  *               followed by a plane of all rows' high bits (1-bit packing);
- *   tok_scale:  float32 [T][2] = (a, z) per token;
- *   chan_scale: float32 [d] = c per channel;
+ *   tok_scale:  [T][2] = (a, z) per token;
+ *   chan_scale: [d] = c per channel;
+ *               both float32, or IEEE half when meta_f16 = 1; each tile's
+ *               scales are balanced by a power of two so that max c lies in
+ *               (1/2, 1] (the dequantised tile does not change);
  *   rope (MLA): bf16 [layer][page][T][rope_dim], unquantised.
  *
  * Supported on the GPU: head_dim 128 (GQA) with tile_tokens 16, 32, 64 or
@@ -112,6 +115,11 @@ typedef struct kvq_config {
   int32_t num_layers;     /* layers in the pool */
   int64_t num_pages;      /* pages per layer in the pool */
   kvq_dtype in_dtype;     /* dtype of the new K/V rows: KVQ_F16 or KVQ_BF16 */
+  int32_t meta_f16;       /* metadata format of a, z and c: 0 = float32 (a
+                           * zero-filled config gets it), 1 = IEEE half
+                           * (the compact layout: same codes, scales rounded
+                           * to 11 significant bits; rows must stay within the
+                           * half range, |a|, |z| < 65504) */
 } kvq_config;
 
 /* Caller-owned device arrays of one cache; byte sizes from kvq_cache_layout

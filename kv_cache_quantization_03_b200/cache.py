@@ -24,6 +24,8 @@ class QuantizedCache:
                 self.arrays[name] = torch.zeros(nbytes, dtype=torch.uint8, device=device)
             elif name == "rope":
                 self.arrays[name] = torch.zeros(nbytes // 2, dtype=torch.bfloat16, device=device)
+            elif cfg.meta_f16:     # a, z, c as IEEE half
+                self.arrays[name] = torch.zeros(nbytes // 2, dtype=torch.float16, device=device)
             else:
                 self.arrays[name] = torch.zeros(nbytes // 4, dtype=torch.float32, device=device)
         self.view = kvq.make_view([self.arrays[n] for n in NAMES])

@@ -51,6 +51,7 @@ kvq_status check_config(const kvq_config* c) {
   if (!valid_bits(c->bits_k)) return KVQ_ERR_INVALID_ARG;
   if (!c->mla && !valid_bits(c->bits_v)) return KVQ_ERR_INVALID_ARG;
   if (c->in_dtype != KVQ_F16 && c->in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (c->meta_f16 != 0 && c->meta_f16 != 1) return KVQ_ERR_INVALID_ARG;
   if (c->mla) {
     if (c->num_kv_heads != 1 || c->rope_dim < 0 || (c->rope_dim % 8)) return KVQ_ERR_INVALID_ARG;
   }
@@ -86,9 +87,10 @@ int64_t slots(const kvq_config* c) { return (int64_t)c->num_layers * c->num_page
 CacheArrays arrays(const kvq_cache_view* v, int which, int bits) {
   CacheArrays a;
   a.codes = static_cast<uint8_t*>(which == 0 ? v->k_codes : v->v_codes);
-  a.tok = static_cast<float*>(which == 0 ? v->k_tok_scale : v->v_tok_scale);
-  a.chan = static_cast<float*>(which == 0 ? v->k_chan_scale : v->v_chan_scale);
+  a.tok = which == 0 ? v->k_tok_scale : v->v_tok_scale;
+  a.chan = which == 0 ? v->k_chan_scale : v->v_chan_scale;
   a.bits = bits;
+  a.meta16 = 0;
   return a;
 }
 
@@ -203,13 +205,14 @@ kvq_status kvq_cache_layout(const kvq_config* c, size_t bytes_out[7]) {
   const kvq_status st = check_config(c);
   if (st != KVQ_OK) return st;
   const size_t n = (size_t)slots(c), T = c->tile_tokens, d = c->head_dim;
+  const size_t msz = c->meta_f16 ? 2 : 4;  // bytes of one a, z or c
   bytes_out[0] = n * T * d * c->bits_k / 8;
-  bytes_out[1] = n * T * 2 * sizeof(float);
-  bytes_out[2] = n * d * sizeof(float);
+  bytes_out[1] = n * T * 2 * msz;
+  bytes_out[2] = n * d * msz;
   const bool has_v = !c->mla;
   bytes_out[3] = has_v ? n * T * d * c->bits_v / 8 : 0;
-  bytes_out[4] = has_v ? n * T * 2 * sizeof(float) : 0;
-  bytes_out[5] = has_v ? n * d * sizeof(float) : 0;
+  bytes_out[4] = has_v ? n * T * 2 * msz : 0;
+  bytes_out[5] = has_v ? n * d * msz : 0;
   bytes_out[6] = c->mla ? (size_t)c->num_layers * c->num_pages * T * c->rope_dim * 2 : 0;
   return KVQ_OK;
 }
@@ -232,6 +235,7 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.src[1] = v_new;
   p.dst[0] = arrays(cache, 0, c->bits_k);
   p.dst[1] = arrays(cache, 1, c->bits_v);
+  p.dst[0].meta16 = p.dst[1].meta16 = c->meta_f16;
   p.kinds = c->mla ? 1 : 2;
   p.n_tok = n_tok;
   p.num_layers = c->num_layers;
@@ -263,6 +267,7 @@ kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int3
   DequantParams p{};
   p.src[0] = arrays(cache, 0, c->bits_k);
   p.src[1] = arrays(cache, 1, c->bits_v);
+  p.src[0].meta16 = p.src[1].meta16 = c->meta_f16;
   p.kinds = c->mla ? 1 : 2;
   p.layer = layer;
   p.num_heads = c->num_kv_heads;
@@ -323,8 +328,9 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
       return workspace_bytes < need ? KVQ_ERR_WORKSPACE_TOO_SMALL : KVQ_ERR_INVALID_ARG;
     MlaDecodeParams m{};
     m.codes = static_cast<const uint8_t*>(cache->k_codes);
-    m.tok = static_cast<const float*>(cache->k_tok_scale);
-    m.chan = static_cast<const float*>(cache->k_chan_scale);
+    m.tok = cache->k_tok_scale;
+    m.chan = cache->k_chan_scale;
+    m.meta16 = c->meta_f16;
     m.rope = static_cast<const uint16_t*>(cache->rope);
     m.bits = c->bits_k;
     m.layer = layer;
@@ -359,6 +365,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   DecodeParams p{};
   p.k = arrays(cache, 0, c->bits_k);
   p.v = arrays(cache, 1, c->bits_v);
+  p.k.meta16 = p.v.meta16 = c->meta_f16;
   p.layer = layer;
   p.num_kv_heads = c->num_kv_heads;
   p.num_pages = c->num_pages;

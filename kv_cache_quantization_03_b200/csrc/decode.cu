@@ -45,16 +45,36 @@ struct StageLayout {
 };
 
 // One stage: the tile of nh adjacent kv-heads (their pages are contiguous in
-// every cache array): K codes | K (a, z) | K c | V codes | V (a, z) | V c.
-__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv, int nh) {
+// every cache array): K codes | K (a, z) | K c | V codes | V (a, z) | V c,
+// with m bytes per a, z or c (4: float32, 2: half).
+__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv, int nh, int m) {
   return StageLayout{nh * kT * kD * bk / 8,
                      nh * kT * kD * bv / 8,
                      nh * (kT * kD * bk / 8),
-                     nh * (kT * kD * bk / 8 + kT * 8),
-                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4),
-                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4) + nh * kT * kD * bv / 8,
-                     nh * (kT * kD * bk / 8 + kT * 8 + kD * 4) + nh * (kT * kD * bv / 8 + kT * 8),
-                     nh * (kT * kD * (bk + bv) / 8 + 2 * (kT * 8 + kD * 4))};
+                     nh * (kT * kD * bk / 8 + kT * 2 * m),
+                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m),
+                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m) + nh * kT * kD * bv / 8,
+                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m) + nh * (kT * kD * bv / 8 + kT * 2 * m),
+                     nh * (kT * kD * (bk + bv) / 8 + 2 * (kT * 2 * m + kD * m))};
+}
+
+// (a, z) of token i, and c of channels i .. i + 3, from a stage's metadata
+// (M = 4: float32, 2: half).
+template <int M>
+__device__ __forceinline__ float2 ld_az(const uint8_t* base, int i) {
+  if constexpr (M == 4) return reinterpret_cast<const float2*>(base)[i];
+  else return __half22float2(reinterpret_cast<const __half2*>(base)[i]);
+}
+template <int M>
+__device__ __forceinline__ float4 ld_c4(const uint8_t* base, int i) {
+  if constexpr (M == 4) {
+    return *reinterpret_cast<const float4*>(base + 4 * i);
+  } else {
+    const uint2 h = *reinterpret_cast<const uint2*>(base + 2 * i);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
 }
 // Ring depth per warp: 3 stages of one kv-head, 2 of a pair (four CTAs per SM).
 __host__ __device__ constexpr int num_stages(int nh) { return nh == 2 ? 2 : kStages; }
@@ -229,10 +249,10 @@ __device__ __forceinline__ bool wait_never_set(uint32_t ns) {
 // 2t, 2t+1, i.e. kv-head hs = t / 2.  The score MMAs run once per kv-head
 // (each lane keeps the result of its own kv-head); for P V each kv-head's
 // weights are masked to its own columns, so both MMAs add into one result.
-template <int BK, int BV, int NH>
+template <int BK, int BV, int NH, int M>
 __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr StageLayout SL = stage_layout(BK, BV, NH);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH, M);
   constexpr int kStages = num_stages(NH);
   constexpr int KCB = SL.kcb / NH, VCB = SL.vcb / NH;  // code bytes of one kv-head's tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -361,13 +381,17 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     }
     const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_kv_heads + kvh;
     mbar_arrive_expect_tx(bar, (uint32_t)SL.bytes);
+    const uint8_t* ktok = static_cast<const uint8_t*>(p.k.tok);
+    const uint8_t* kch = static_cast<const uint8_t*>(p.k.chan);
+    const uint8_t* vtok = static_cast<const uint8_t*>(p.v.tok);
+    const uint8_t* vch = static_cast<const uint8_t*>(p.v.chan);
     if (p.sub_log2 == 0) {  // 16-token pages: the nh kv-heads' pages are contiguous in every array
       bulk_g2s(st, p.k.codes + slot * KCB, SL.kcb, bar);
-      bulk_g2s(st + SL.off_kaz, p.k.tok + slot * (kT * 2), NH * kT * 8, bar);
-      bulk_g2s(st + SL.off_kc, p.k.chan + slot * kD, NH * kD * 4, bar);
+      bulk_g2s(st + SL.off_kaz, ktok + slot * (kT * 2 * M), NH * kT * 2 * M, bar);
+      bulk_g2s(st + SL.off_kc, kch + slot * (kD * M), NH * kD * M, bar);
       bulk_g2s(st + SL.off_v, p.v.codes + slot * VCB, SL.vcb, bar);
-      bulk_g2s(st + SL.off_vaz, p.v.tok + slot * (kT * 2), NH * kT * 8, bar);
-      bulk_g2s(st + SL.off_vc, p.v.chan + slot * kD, NH * kD * 4, bar);
+      bulk_g2s(st + SL.off_vaz, vtok + slot * (kT * 2 * M), NH * kT * 2 * M, bar);
+      bulk_g2s(st + SL.off_vc, vch + slot * (kD * M), NH * kD * M, bar);
       return;
     }
     // longer pages: slice `sub` of each kv-head's page, in the same stage layout
@@ -382,12 +406,12 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       } else {
         bulk_g2s(st + h * KCB, kc + sub * KCB, KCB, bar);
       }
-      bulk_g2s(st + SL.off_kaz + h * (kT * 8), p.k.tok + (sh * spt + sub) * (kT * 2), kT * 8, bar);
-      bulk_g2s(st + SL.off_kc + h * (kD * 4), p.k.chan + sh * kD, kD * 4, bar);
+      bulk_g2s(st + SL.off_kaz + h * (kT * 2 * M), ktok + (sh * spt + sub) * (kT * 2 * M), kT * 2 * M, bar);
+      bulk_g2s(st + SL.off_kc + h * (kD * M), kch + sh * (kD * M), kD * M, bar);
       static_assert(BV != 3, "3-bit values have two planes");
       bulk_g2s(st + SL.off_v + h * VCB, p.v.codes + (sh * spt + sub) * VCB, VCB, bar);
-      bulk_g2s(st + SL.off_vaz + h * (kT * 8), p.v.tok + (sh * spt + sub) * (kT * 2), kT * 8, bar);
-      bulk_g2s(st + SL.off_vc + h * (kD * 4), p.v.chan + sh * kD, kD * 4, bar);
+      bulk_g2s(st + SL.off_vaz + h * (kT * 2 * M), vtok + (sh * spt + sub) * (kT * 2 * M), kT * 2 * M, bar);
+      bulk_g2s(st + SL.off_vc + h * (kD * M), vch + sh * (kD * M), kD * M, bar);
     }
   };
   const int pre = n_run < kStages ? n_run : kStages;
@@ -413,10 +437,10 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     if (page >= 0 && page < p.num_pages) {
       const uint8_t* st = wsm + (i % kStages) * SL.bytes;
       const int hu = NH == 2 ? (g >> 2) : 0, hs = NH == 2 ? (t >> 1) : 0;  // kv-head of this lane's u / columns
-      const float* kaz = reinterpret_cast<const float*>(st + SL.off_kaz) + hs * 2 * kT;
-      const float* kc = reinterpret_cast<const float*>(st + SL.off_kc) + hu * kD;
-      const float* vaz = reinterpret_cast<const float*>(st + SL.off_vaz) + hs * 2 * kT;
-      const float* vc = reinterpret_cast<const float*>(st + SL.off_vc) + hs * kD;
+      const uint8_t* kaz = st + SL.off_kaz + hs * (2 * kT * M);
+      const uint8_t* kc = st + SL.off_kc + hu * (kD * M);
+      const uint8_t* vaz = st + SL.off_vaz + hs * (2 * kT * M);
+      const uint8_t* vc = st + SL.off_vc + hs * (kD * M);
 
       // u = q~ * c_K on this lane's 32 channels (slot order), and its sum
       float u[32];
@@ -428,7 +452,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int kk = 4 * ((k + rq) & 7);
-          const float4 c4 = *reinterpret_cast<const float4*>(kc + 32 * t + kk);
+          const float4 c4 = ld_c4<M>(kc, 32 * t + kk);
           const f2 a = mul2(make_float2(qv[4 * k], qv[4 * k + 1]), make_float2(c4.x, c4.y));
           const f2 d = mul2(make_float2(qv[4 * k + 2], qv[4 * k + 3]), make_float2(c4.z, c4.w));
           su2 = add2(su2, add2(a, d));
@@ -466,8 +490,8 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
         for (int e = 0; e < 4; ++e)
           if (h == 0 || hs == h) S[e] = Sh[e] + Sl[e];
       }
-      const float2 az0 = *reinterpret_cast<const float2*>(kaz + 2 * g);
-      const float2 az1 = *reinterpret_cast<const float2*>(kaz + 2 * (g + 8));
+      const float2 az0 = ld_az<M>(kaz, g);
+      const float2 az1 = ld_az<M>(kaz, g + 8);
       float sc[4];
       sc[0] = fmaf(az0.x, S[0], az0.y * su0);
       sc[1] = fmaf(az0.x, S[1], az0.y * su1);
@@ -490,8 +514,8 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       lrun[1] = fmaf(lrun[1], al1, p1 + p3);
 
       // value weights w = p * a_V / max(a_V) (f16, transposed into B fragments)
-      const float2 vz0 = *reinterpret_cast<const float2*>(vaz + 2 * g);
-      const float2 vz1 = *reinterpret_cast<const float2*>(vaz + 2 * (g + 8));
+      const float2 vz0 = ld_az<M>(vaz, g);
+      const float2 vz1 = ld_az<M>(vaz, g + 8);
       float amax = fmaxf(vz0.x, vz1.x);
       float bz0 = fmaf(p0, vz0.y, p2 * vz1.y), bz1 = fmaf(p1, vz0.y, p3 * vz1.y);
 #pragma unroll
@@ -512,7 +536,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       float cv[16];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float4 c4 = *reinterpret_cast<const float4*>(vc + 16 * g + 4 * k);
+        const float4 c4 = ld_c4<M>(vc, 16 * g + 4 * k);
         cv[4 * k] = c4.x, cv[4 * k + 1] = c4.y, cv[4 * k + 2] = c4.z, cv[4 * k + 3] = c4.w;
       }
       const f2 alpha = make_float2(al0, al1), bz = make_float2(bz0, bz1), am = splat2(amax);
@@ -703,15 +727,15 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
   }
 }
 
-template <int BK, int BV, int NH>
+template <int BK, int BV, int NH, int M>
 int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
-  constexpr StageLayout SL = stage_layout(BK, BV, NH);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH, M);
   constexpr int kStages = num_stages(NH);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
   const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
-  auto kern = decode_d128_kernel<BK, BV, NH>;
+  auto kern = decode_d128_kernel<BK, BV, NH, M>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.splits, p.batch * p.num_kv_heads / NH);
   kern<<<grid, kDW * 32, smem, s>>>(p);
@@ -727,8 +751,11 @@ int launch_decode_d128(const DecodeParams& p, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bk = p.k.bits, bv = p.v.bits;
   const bool pairs = decode_kv_heads_per_cta(p.group, p.num_kv_heads) == 2;
-#define KVQ_CASE(K, V) \
-  if (bk == K && bv == V) return pairs ? launch_bk_bv<K, V, 2>(p, s) : launch_bk_bv<K, V, 1>(p, s);
+#define KVQ_CASE(K, V)                                                                        \
+  if (bk == K && bv == V) {                                                                   \
+    if (p.k.meta16) return pairs ? launch_bk_bv<K, V, 2, 2>(p, s) : launch_bk_bv<K, V, 1, 2>(p, s); \
+    return pairs ? launch_bk_bv<K, V, 2, 4>(p, s) : launch_bk_bv<K, V, 1, 4>(p, s);           \
+  }
   KVQ_CASE(4, 4) KVQ_CASE(3, 4) KVQ_CASE(2, 4) KVQ_CASE(8, 4)
   KVQ_CASE(4, 2) KVQ_CASE(3, 2) KVQ_CASE(2, 2) KVQ_CASE(8, 2)
   KVQ_CASE(4, 8) KVQ_CASE(3, 8) KVQ_CASE(2, 8) KVQ_CASE(8, 8)

@@ -69,22 +69,43 @@ constexpr int kOffQs = 0;
 constexpr int kOffKb = kOffQs + kQsBytes;
 __host__ __device__ constexpr int num_kb(int bits) { return bits == 8 ? 2 : 3; }  // dequantised chunk buffers
 __host__ __device__ constexpr int st_offset(int bits) { return kOffKb + num_kb(bits) * kKbBytes; }
-// a stage holds two tiles: codes | (a, z) | channel scales | rope
+// a stage holds two tiles: codes | (a, z) | channel scales | rope; m bytes per
+// a, z or c (4: float32, 2: half)
 __host__ __device__ constexpr int tile_code_bytes(int bits) { return kT * kLat * bits / 8; }
-__host__ __device__ constexpr int stage_bytes(int bits) {
-  return 2 * (tile_code_bytes(bits) + kT * 8 + kLat * 4 + kT * kRope * 2);
+__host__ __device__ constexpr int stage_bytes(int bits, int m) {
+  return 2 * (tile_code_bytes(bits) + kT * 2 * m + kLat * m + kT * kRope * 2);
 }
 constexpr int kNS = 2;  // raw-tile stages
-__host__ __device__ constexpr int bar_offset(int bits) { return st_offset(bits) + kNS * stage_bytes(bits); }
+__host__ __device__ constexpr int bar_offset(int bits, int m) { return st_offset(bits) + kNS * stage_bytes(bits, m); }
 // full[2] dq[3] sfull[2] pfull[2] pv[4] qf qt fin, the TMEM address, the operand
 // exponents of the dequantised chunk buffers (int[4]), then the tile-validity bits
 constexpr int kNumBars = kNS + 3 + 2 + 2 + 4 + 3;
-__host__ __device__ constexpr int echunk_offset(int bits) { return bar_offset(bits) + kNumBars * 8 + 8; }
-__host__ __device__ constexpr int vmask_offset(int bits) { return echunk_offset(bits) + 16; }
-__host__ __device__ constexpr int smem_bytes(int bits, int tiles_per_split) {
-  return vmask_offset(bits) + ((tiles_per_split + 31) / 32) * 4;
+__host__ __device__ constexpr int echunk_offset(int bits, int m) { return bar_offset(bits, m) + kNumBars * 8 + 8; }
+__host__ __device__ constexpr int vmask_offset(int bits, int m) { return echunk_offset(bits, m) + 16; }
+__host__ __device__ constexpr int smem_bytes(int bits, int m, int tiles_per_split) {
+  return vmask_offset(bits, m) + ((tiles_per_split + 31) / 32) * 4;
 }
-static_assert(smem_bytes(4, 8192) <= 232448 && smem_bytes(8, 8192) <= 232448, "shared memory");
+static_assert(smem_bytes(4, 4, 8192) <= 232448 && smem_bytes(8, 4, 8192) <= 232448, "shared memory");
+
+// (a, z) of a stage's token and c of eight channels (M = 4: float32, 2: half)
+template <int M>
+__device__ __forceinline__ float2 mla_az(const uint8_t* base) {
+  if constexpr (M == 4) return *reinterpret_cast<const float2*>(base);
+  else return __half22float2(*reinterpret_cast<const __half2*>(base));
+}
+template <int M>
+__device__ __forceinline__ void mla_c8(const uint8_t* base, f2 (&cc)[4]) {
+  if constexpr (M == 4) {
+    const float4 c0 = reinterpret_cast<const float4*>(base)[0], c1 = reinterpret_cast<const float4*>(base)[1];
+    cc[0] = make_float2(c0.x, c0.y), cc[1] = make_float2(c0.z, c0.w);
+    cc[2] = make_float2(c1.x, c1.y), cc[3] = make_float2(c1.z, c1.w);
+  } else {
+    const uint4 h = *reinterpret_cast<const uint4*>(base);
+    const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cc[e] = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+  }
+}
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
@@ -159,15 +180,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
 }
 
-template <int BITS>
+template <int BITS, int M>
 __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams p) {
-  constexpr int NS = kNS, NB = num_kb(BITS), SB = stage_bytes(BITS), CB = tile_code_bytes(BITS);
+  constexpr int NS = kNS, NB = num_kb(BITS), SB = stage_bytes(BITS, M), CB = tile_code_bytes(BITS);
   constexpr int kOffSt = st_offset(BITS);
-  constexpr int kStAz = 2 * CB, kStC = kStAz + 2 * kT * 8, kStRope = kStC + 2 * kLat * 4;
+  constexpr int kStAz = 2 * CB, kStC = kStAz + 2 * kT * 2 * M, kStRope = kStC + 2 * kLat * M;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x & 1, split = blockIdx.x >> 1, b = blockIdx.y;  // r: output half
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + bar_offset(BITS));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + bar_offset(BITS, M));
   uint64_t* dq = full + kNS;
   uint64_t* sfull = dq + 3;
   uint64_t* pfull = sfull + 2;
@@ -176,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   uint64_t* qt = qf + 1;
   uint64_t* fin = qt + 1;  // every MMA of the CTA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
-  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + vmask_offset(BITS));
-  int* echunk = reinterpret_cast<int*>(smem + echunk_offset(BITS));  // [NB]: operand exponent of each buffer
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + vmask_offset(BITS, M));
+  int* echunk = reinterpret_cast<int*>(smem + echunk_offset(BITS, M));  // [NB]: operand exponent of each buffer
   const uint32_t s_base = smem_u32(smem);
 
   const int seq_raw = p.seq_lens[b];
@@ -247,15 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
         uint32_t bytes = 0;
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          if (tile_ok(2 * c + j)) bytes += CB + kT * 8 + kLat * 4 + kT * kRope * 2;
+          if (tile_ok(2 * c + j)) bytes += CB + kT * 2 * M + kLat * M + kT * kRope * 2;
         mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (!tile_ok(2 * c + j)) continue;
           const size_t slot = (size_t)p.layer * p.num_pages + pg[j];
           bulk_g2s(st + j * CB, p.codes + slot * CB, CB, bar);
-          bulk_g2s(st + kStAz + j * kT * 8, p.tok + slot * kT * 2, kT * 8, bar);
-          bulk_g2s(st + kStC + j * kLat * 4, p.chan + slot * kLat, kLat * 4, bar);
+          bulk_g2s(st + kStAz + j * kT * 2 * M, static_cast<const uint8_t*>(p.tok) + slot * (kT * 2 * M), kT * 2 * M,
+                   bar);
+          bulk_g2s(st + kStC + j * kLat * M, static_cast<const uint8_t*>(p.chan) + slot * (kLat * M), kLat * M, bar);
           bulk_g2s(st + kStRope + j * kT * kRope * 2, p.rope + slot * kT * kRope, kT * kRope * 2, bar);
         }
       };
@@ -349,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       // token (tile l / 16, row l % 16).
       int e_chunk;
       {
-        const float2 az = *reinterpret_cast<const float2*>(st + kStAz + (lane >> 4) * kT * 8 + (lane & 15) * 8);
+        const float2 az = mla_az<M>(st + kStAz + (lane >> 4) * kT * 2 * M + (lane & 15) * 2 * M);
         constexpr float kQm = (float)((1 << BITS) - 1);
         float bnd = tile_ok(2 * c + (lane >> 4)) ? fmaxf(fabsf(az.y), fabsf(fmaf(az.x, kQm, az.y))) : 0.f;
 #pragma unroll
@@ -359,16 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       }
       const float sE = __uint_as_float((uint32_t)(127 - e_chunk) << 23);
       f2 cc[4];
-      {
-        const float4* cp = reinterpret_cast<const float4*>(st + kStC + j * kLat * 4 + ch0 * 4);
-        const float4 c0 = cp[0], c1 = cp[1];
-        cc[0] = make_float2(c0.x, c0.y), cc[1] = make_float2(c0.z, c0.w);
-        cc[2] = make_float2(c1.x, c1.y), cc[3] = make_float2(c1.z, c1.w);
-      }
+      mla_c8<M>(st + kStC + j * kLat * M + ch0 * M, cc);
 #pragma unroll
       for (int it = 0; it < 4; ++it) {
         const int tr = 8 * rh + ((lane + it + 4 * hf) & 7);
-        float2 az = *reinterpret_cast<const float2*>(st + kStAz + j * kT * 8 + tr * 8);
+        float2 az = mla_az<M>(st + kStAz + j * kT * 2 * M + tr * 2 * M);
         az.x *= sE, az.y *= sE;
         float q[8];
         codes8<BITS>(st + j * CB, tr, ch0, q);
@@ -627,17 +644,17 @@ __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
   p.out[((size_t)b * p.num_q_heads + h) * kLat + j] = buf[j] * 0.044194173824159216f;
 }
 
-template <int BITS>
+template <int BITS, int M>
 int launch_mla_bits(const MlaDecodeParams& p, cudaStream_t s) {
-  const int smem = smem_bytes(BITS, p.tiles_per_split);
-  cudaError_t e = cudaFuncSetAttribute(decode_mla_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = smem_bytes(BITS, M, p.tiles_per_split);
+  cudaError_t e = cudaFuncSetAttribute(decode_mla_kernel<BITS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.splits, p.batch, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  return (int)cudaLaunchKernelEx(&cfg, decode_mla_kernel<BITS>, p);
+  return (int)cudaLaunchKernelEx(&cfg, decode_mla_kernel<BITS, M>, p);
 }
 
 }  // namespace
@@ -649,11 +666,12 @@ int launch_decode_mla(const MlaDecodeParams& p, void* stream) {
   mla_prep_q_kernel<<<p.batch, 256, 0, s>>>(p);
   int e = (int)cudaGetLastError();
   if (e != cudaSuccess) return e;
+  const bool h = p.meta16 != 0;
   switch (p.bits) {
-    case 2: e = launch_mla_bits<2>(p, s); break;
-    case 3: e = launch_mla_bits<3>(p, s); break;
-    case 4: e = launch_mla_bits<4>(p, s); break;
-    default: e = launch_mla_bits<8>(p, s); break;
+    case 2: e = h ? launch_mla_bits<2, 2>(p, s) : launch_mla_bits<2, 4>(p, s); break;
+    case 3: e = h ? launch_mla_bits<3, 2>(p, s) : launch_mla_bits<3, 4>(p, s); break;
+    case 4: e = h ? launch_mla_bits<4, 2>(p, s) : launch_mla_bits<4, 4>(p, s); break;
+    default: e = h ? launch_mla_bits<8, 2>(p, s) : launch_mla_bits<8, 4>(p, s); break;
   }
   if (e != cudaSuccess) return e;
   combine_mla_kernel<<<p.batch * p.num_q_heads, kLat, 0, s>>>(p);

@@ -41,13 +41,17 @@ __global__ void __launch_bounds__(kD) dequantize_kernel(DequantParams p) {
   const int T = p.tile_tokens;
   const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_heads + head;
   const uint8_t* codes = src.codes + slot * ((size_t)T * kD * src.bits / 8);
-  const float* tok = src.tok + slot * T * 2;
-  const float c = src.chan[slot * kD + ch];
+  // a, z, c: float32 or IEEE half
+  auto meta = [&](const void* base, size_t i) {
+    return src.meta16 ? __half2float(static_cast<const __half*>(base)[i]) : static_cast<const float*>(base)[i];
+  };
+  const size_t tok0 = slot * T * 2;
+  const float c = meta(src.chan, slot * kD + ch);
   float* out = p.out[kind] + (((size_t)pi * p.num_heads + head) * T) * kD;
   for (int r0 = 0; r0 < T; r0 += kT) {  // kT rows at a time
     for (int r = 0; r < kT; ++r)
-      tile[r][ch] =
-          fmaf(tok[2 * (r0 + r)], (float)read_code<kD>(codes, src.bits, T, r0 + r, ch), tok[2 * (r0 + r) + 1]) * c;
+      tile[r][ch] = fmaf(meta(src.tok, tok0 + 2 * (r0 + r)), (float)read_code<kD>(codes, src.bits, T, r0 + r, ch),
+                         meta(src.tok, tok0 + 2 * (r0 + r) + 1)) * c;
     __syncthreads();
     if (p.unrotate) {  // H / sqrt(b) on each block of b = hblock channels
       for (int r = 0; r < kT; ++r) {

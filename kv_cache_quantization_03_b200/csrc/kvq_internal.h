@@ -25,9 +25,10 @@ constexpr uint32_t kWaitLimit = 1000000000u;
 // One quantised stream (K, V or the MLA latent) of the cache.
 struct CacheArrays {
   uint8_t* codes;    // [layer][page][head][T*d*bits/8]
-  float* tok;        // [layer][page][head][T][2]
-  float* chan;       // [layer][page][head][d]
+  void* tok;         // [layer][page][head][T][2]  float32, or half when meta16
+  void* chan;        // [layer][page][head][d]     float32, or half when meta16
   int bits;
+  int meta16;        // 1: a, z, c stored as IEEE half
 };
 
 struct QuantizeParams {
@@ -96,8 +97,9 @@ struct DecodeParams {
 
 struct MlaDecodeParams {
   const uint8_t* codes;         // latent codes [layer][page][T*512*bits/8]
-  const float* tok;             // [layer][page][T][2]
-  const float* chan;            // [layer][page][512]
+  const void* tok;              // [layer][page][T][2]  float32, or half when meta16
+  const void* chan;             // [layer][page][512]   float32, or half when meta16
+  int meta16;
   const uint16_t* rope;         // bf16 [layer][page][T][64]
   int bits;
   int layer;

@@ -613,17 +613,28 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
     const int kb = (int)(cbits >> 23) - 127 + ((cbits & 0x7FFFFFu) != 0u);
     if (wt == 0) {
       const float cs = __uint_as_float((uint32_t)(127 - kb) << 23);
-      *reinterpret_cast<float4*>(p.dst.chan + slot * D + kBlk * blk + 16 * g + 4 * t) =
-          make_float4(cv4.x * cs, cv4.y * cs, cv4.z * cs, cv4.w * cs);
+      const size_t ci = slot * D + kBlk * blk + 16 * g + 4 * t;
+      if (p.dst.meta16) {  // half metadata: rounded to nearest from the float32 value
+        const __half2 lo = __floats2half2_rn(cv4.x * cs, cv4.y * cs), hi = __floats2half2_rn(cv4.z * cs, cv4.w * cs);
+        *reinterpret_cast<uint2*>(static_cast<__half*>(p.dst.chan) + ci) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+      } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.dst.chan) + ci) =
+            make_float4(cv4.x * cs, cv4.y * cs, cv4.z * cs, cv4.w * cs);
+      }
     }
     constexpr float kQmax = (float)((1 << BITS) - 1);
     const float s_own = (omx - omn) / kQmax;
     const float is_own = s_own > 0.f ? rcp_nr(s_own) : 0.f;
     // 1/sqrt(block) times the row's power of two times the balance 2^kb
     const float fold = inv_sqrt_d * rsc_own * __uint_as_float((uint32_t)(127 + kb) << 23);
-    if ((lane & 4) == 0 && blk == 0)
-      *reinterpret_cast<float2*>(p.dst.tok + slot * (kTile * 2) + 2 * (kT * wt + 8 * b2 + 2 * t + b1)) =
-          make_float2(s_own * fold, omn * fold);
+    if ((lane & 4) == 0 && blk == 0) {
+      const size_t ti = slot * (kTile * 2) + 2 * (kT * wt + 8 * b2 + 2 * t + b1);
+      if (p.dst.meta16)
+        *reinterpret_cast<__half2*>(static_cast<__half*>(p.dst.tok) + ti) = __floats2half2_rn(s_own * fold, omn * fold);
+      else
+        *reinterpret_cast<float2*>(static_cast<float*>(p.dst.tok) + ti) = make_float2(s_own * fold, omn * fold);
+    }
     uint8_t* codes = p.dst.codes + slot * (kTile * D * BITS / 8);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {

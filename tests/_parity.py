@@ -11,7 +11,10 @@ Tolerances (readings as stated in the oracle's header):
   only happen without normalisation rounds (with them y involves square
   roots).  Counted flips and exact ties are reported separately;
 * a, z, c: |gpu - oracle| <= 1e-6 |oracle| (purely relative, so it holds at
-  any magnitude; a zero must be an exact zero);
+  any magnitude; a zero must be an exact zero); with half-precision metadata
+  the stored half must equal the oracle's, or be its neighbour where the
+  oracle's float64 value lies within 1e-6 (relative) of the midpoint between
+  the two (the kernel rounds its float32 value, the oracle the exact one);
 * attention: per (sequence, head) max_j |o_j - o'_j| / max_j |o'_j| <= 2e-3,
   with the oracle run on the GPU's stored codes and scales.
 """
@@ -39,7 +42,7 @@ def config_for(w: W.Workload, num_pages=None) -> kvq.kvq_config:
                            bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                            rope_dim=w.rope_dim, num_layers=w.num_layers,
                            num_pages=w.num_pages if num_pages is None else num_pages, in_dtype=w.in_dtype,
-                           hadamard_block=w.hadamard_block or None)
+                           hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16)
 
 
 class QuantRun:
@@ -156,6 +159,17 @@ def compare_quantized(gpu: O.QuantizedTiles, ora: O.QuantizedTiles, x: np.ndarra
         counted = int(diff.sum()) - ties
     if check_rate:
         assert counted <= CODE_FLIP_RATE * gpu.q.size, "%s: %d flips in %d codes" % (label, counted, gpu.q.size)
+    if np.asarray(gpu.a).dtype == np.float16:
+        _, a64, z64, c64 = O.quantize_stages(x, bits, n_iter, block)
+        for name, exact in (("a", a64), ("z", z64), ("c", c64)):
+            g16, o16 = np.asarray(getattr(gpu, name), np.float16), np.asarray(getattr(ora, name), np.float16)
+            g, o = g16.astype(np.float64), o16.astype(np.float64)
+            gb, ob = g16.view(np.uint16).astype(np.int64), o16.view(np.uint16).astype(np.int64)
+            neighbour = (np.abs(gb - ob) == 1) & ((gb ^ ob) & 0x8000 == 0)
+            at_mid = np.abs(exact - (g + o) / 2) <= SCALE_RTOL * np.abs(exact)
+            ok = (gb == ob) | (neighbour & at_mid)
+            assert np.all(ok), "%s: half %s differs from the oracle's (%d values)" % (label, name, int((~ok).sum()))
+        return Flips(counted, ties)
     for name in ("a", "z", "c"):
         g = getattr(gpu, name).astype(np.float64)
         o = getattr(ora, name).astype(np.float64)
@@ -170,7 +184,7 @@ def check_tiles(run, which: str, layer: int, tiles, head: int, label="", check_r
     w = run.w
     bits = w.bits_k if which == "k" else w.bits_v
     x = run.input_tiles(which, layer, tiles, head)
-    ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block)
+    ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block, meta="f16" if w.meta_f16 else "f32")
     gpu = run.gpu_tiles(which, layer, tiles, head)
     return compare_quantized(gpu, ora, x, bits, w.sinkhorn_iters, w.block, label, check_rate)
 

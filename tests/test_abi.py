@@ -54,6 +54,14 @@ def test_cache_layout_sizes(kvq):
     m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=4)
     s = kvq.kvq_cache_layout(m)
     assert s[3:6] == [0, 0, 0] and s[6] == 4 * 16 * 64 * 2 and s[0] == 4 * 16 * 512 // 2
+    # half-precision metadata: a, z, c take two bytes each, codes unchanged
+    h = kvq.make_config(num_kv_heads=8, num_layers=2, num_pages=10, bits_k=3, bits_v=4, meta_f16=True)
+    assert kvq.kvq_cache_layout(h) == [n * 16 * 128 * 3 // 8, n * 16 * 2 * 2, n * 128 * 2, n * 16 * 128 * 4 // 8,
+                                       n * 16 * 2 * 2, n * 128 * 2, 0]
+    bad = kvq.make_config(num_pages=4)
+    bad.meta_f16 = 2
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_layout(bad)
 
 
 def test_invalid_configs_rejected(kvq):
@@ -186,7 +194,7 @@ int main(void) {
   if (kvq_config_from_string("kvarn_k4v2_g128", &c) != KVQ_OK) return 1;
   if (c.bits_k != 4 || c.bits_v != 2 || c.tile_tokens != 128) return 2;
   if (kvq_cache_layout(&c, sizes) != KVQ_OK) return 3;
-  printf("%s %zu %zu\n", kvq_version(), sizes[0], sizes[3]);
+  printf("%s %zu %zu %zu\n", kvq_version(), sizes[0], sizes[3], sizeof(kvq_config));
   return strcmp(kvq_status_string(KVQ_ERR_PARTIAL_TILE), "KVQ_ERR_PARTIAL_TILE") != 0;
 }
 """)
@@ -198,4 +206,5 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     n = 2 * 10 * 8
-    assert r.stdout.split()[1:] == [str(n * 128 * 128 * 4 // 8), str(n * 128 * 128 * 2 // 8)]
+    assert r.stdout.split()[1:] == [str(n * 128 * 128 * 4 // 8), str(n * 128 * 128 * 2 // 8),
+                                     str(ctypes.sizeof(kvq.kvq_config))]     # the binding's struct is the header's

@@ -37,6 +37,7 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("g128", dict(batch=3, seq_len=1024)),
     ("saw4", dict(batch=3, seq_len=512)),
     ("prefill", dict(seq_len=1024, num_layers=2)),   # per-channel scales over two decades
+    ("gqa16", dict(batch=3, seq_len=512)),            # a, z, c as IEEE half
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]
@@ -108,6 +109,20 @@ def test_mla_decode_fewer_heads_ragged():
     dec = DecodeRun(run, seq_lens=[256, 48, 0])
     o = dec()
     assert run.error_bits() == 0
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("name,kw", [("long", dict(batch=2, seq_len=1024)), ("g128", dict(batch=3, seq_len=1024)),
+                                     ("mla", dict(batch=2, seq_len=512))])
+def test_decode_parity_half_metadata(name, kw):
+    # the half-precision layout through both decode kernels (one and two
+    # kv-heads per CTA, 128-token pages, the MLA latent)
+    w = dataclasses.replace(W.WORKLOADS[name].scaled(**kw), meta_f16=True)
+    run = QuantRun(w)
+    dec = DecodeRun(run)
+    o = dec()
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
     _check(dec, o)
 
 

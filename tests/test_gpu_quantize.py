@@ -160,6 +160,23 @@ def test_quantize_parity_dynamic_range(name, iters, scales):
     assert flips + ties <= 1e-3 * total
 
 
+@pytest.mark.parametrize("name", ["gqa16", "long", "g128", "mla", "prefill"])
+def test_quantize_parity_half_metadata(name):
+    # a, z, c stored as IEEE half: the codes are the float32 layout's, bit for
+    # bit (the format does not enter the code decision), and each half is the
+    # oracle's rounding of the exact value (or its neighbour at a midpoint)
+    import dataclasses
+    w = W.WORKLOADS[name]
+    w = dataclasses.replace(w.scaled(batch=1, seq_len=256, num_layers=2 if w.num_layers > 1 else None),
+                            meta_f16=True)
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
+    ref = QuantRun(dataclasses.replace(w, meta_f16=False))
+    for which in (("k",) if w.mla else ("k", "v")):
+        assert torch.equal(run.cache.codes(which), ref.cache.codes(which)), which
+
+
 def test_quantize_bad_page_sets_error_and_skips_tile():
     w = W.WORKLOADS["gqa"].scaled(batch=1, seq_len=64)
     pages = np.array([0, 7, 2, 3], dtype=np.int32)        # pool of 4 pages: 7 is out of range
@@ -230,7 +247,7 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4"])
+@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4", "gqa16"])
 def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
     w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
