@@ -220,6 +220,42 @@ def quantize_tiles(x: np.ndarray, bits: int, n_iter: int, block: Optional[int] =
     raise ValueError("meta must be 'f32' or 'f16'")
 
 
+@dataclasses.dataclass
+class ChannelQuantizedTiles:
+    """Keys quantised along the other axis: one (step, minimum) per channel."""
+    q: np.ndarray   # int64 [..., T, d]   codes in [0, 2^bits - 1]
+    s: np.ndarray   # float32 [..., d]    step of each channel
+    m: np.ndarray   # float32 [..., d]    minimum of each channel
+
+
+def quantize_tiles_per_channel(x: np.ndarray, bits: int, block: Optional[int] = None) -> ChannelQuantizedTiles:
+    """KIVI-style key quantisation (the KIVI entry of the Hugging Face paper
+    listing: keys quantised per channel, values per token, asymmetric,
+    tuning-free), as the ablation of the dual-axis normalisation: the tile
+    is rotated (block 1 = no rotation, as in KIVI), not normalised, and every
+    channel (a column of the tile: its T tokens) is one asymmetric RTN group
+    with its own minimum m_j and step s_j = (max_j - m_j) / (2^b - 1).
+    Dequantised (rotated domain): s_j q_tj + m_j."""
+    z = rotate(x, block)
+    qt, m, st = rtn_rows(np.swapaxes(z, -1, -2), bits)     # the channels as the groups
+    return ChannelQuantizedTiles(q=np.swapaxes(qt, -1, -2), s=st.astype(np.float32), m=m.astype(np.float32))
+
+
+def dequantize_channel_tiles(t: ChannelQuantizedTiles, unrotate: bool = True,
+                             block: Optional[int] = None) -> np.ndarray:
+    """s_j q_tj + m_j (float64), then optionally un-rotated."""
+    zh = np.asarray(t.s, np.float64)[..., None, :] * np.asarray(t.q, np.float64) + \
+        np.asarray(t.m, np.float64)[..., None, :]
+    return rotate(zh, block) if unrotate else zh
+
+
+def _rotated_rows(t) -> np.ndarray:
+    """Dequantised rows, rotated domain, of either kind of quantised tiles."""
+    if isinstance(t, ChannelQuantizedTiles):
+        return dequantize_channel_tiles(t, unrotate=False)
+    return dequantize_tiles(t.q, t.a, t.z, t.c, unrotate=False)
+
+
 def dequantize_tiles(q, a, z, c, unrotate: bool = True, block: Optional[int] = None) -> np.ndarray:
     """(a q + z) c in the rotated domain (float64), then optionally un-rotated."""
     a = np.asarray(a, dtype=np.float64)
@@ -300,8 +336,8 @@ def decode_attention(q: np.ndarray, k: QuantizedTiles, v: QuantizedTiles,
     output is rotated back.
     """
     d = q.shape[-1]
-    kh = dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=False).reshape(-1, d)
-    vh = dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=False).reshape(-1, d)
+    kh = _rotated_rows(k).reshape(-1, d)      # keys: per-token tiles, or per-channel (KIVI-style axes)
+    vh = _rotated_rows(v).reshape(-1, d)
     qr = rotate(q, block)
     p = _softmax(softmax_scale * (qr @ kh.T))
     return rotate(p @ vh, block)
@@ -328,7 +364,7 @@ def decode_attention_with_tail(q: np.ndarray, k: Optional[QuantizedTiles], v: Op
     keys = [np.asarray(k_tail, dtype=np.float64).reshape(-1, d)]
     vals = [np.asarray(v_tail, dtype=np.float64).reshape(-1, d)]
     if k is not None and k.q.shape[0] > 0:
-        keys.insert(0, dequantize_tiles(k.q, k.a, k.z, k.c, unrotate=True, block=block).reshape(-1, d))
+        keys.insert(0, rotate(_rotated_rows(k), block).reshape(-1, d))
         vals.insert(0, dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=True, block=block).reshape(-1, d))
     kk = np.concatenate(keys, 0)
     vv = np.concatenate(vals, 0)

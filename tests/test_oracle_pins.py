@@ -298,6 +298,56 @@ def test_fp16_metadata_is_the_nearest_half_and_leaves_codes_alone():
         assert np.all(np.abs(d16 - d32) <= bound)
 
 
+# ---------------------------------------------------------------- KIVI-style axes (ablation)
+def test_block_one_rotation_is_the_identity():
+    x = np.random.default_rng(41).standard_normal((3, 16, 128))
+    assert np.array_equal(O.rotate(x, 1), x)
+    assert np.array_equal(O.block_hadamard_matrix(128, 1), np.eye(128, dtype=np.int64))
+
+
+def test_per_channel_golden():
+    fx = _golden("tile_per_channel.json")
+    t = O.quantize_tiles_per_channel(np.array(fx["x"]), fx["bits"], block=1)
+    assert np.array_equal(t.q, fx["q"])
+    assert np.allclose(t.s, np.array(fx["s"], np.float32), rtol=0, atol=0)
+    assert np.array_equal(t.m, np.array(fx["m"], np.float32))
+    assert np.allclose(O.dequantize_channel_tiles(t, unrotate=False, block=1), fx["x"], rtol=0, atol=1e-7)
+
+
+@pytest.mark.parametrize("bits,block", [(2, 1), (4, 1), (3, 32), (8, 128)])
+def test_per_channel_rtn_is_nearest_level_brute_force(bits, block):
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((6, 16, 128)) * np.exp(rng.uniform(-2, 2, (6, 1, 128)))
+    t = O.quantize_tiles_per_channel(x, bits, block)
+    z = O.rotate(x, block)
+    s, m = t.s.astype(np.float64), t.m.astype(np.float64)
+    levels = np.arange(1 << bits)
+    # every code is the nearest level of its own channel's grid (the stored
+    # float32 step and minimum reproduce it to float32 rounding)
+    recon = m[..., None, :, None] + s[..., None, :, None] * levels
+    best = np.argmin(np.abs(z[..., None] - recon), axis=-1)
+    assert np.mean(best == t.q) > 0.9999
+    assert np.all(np.abs(z - (m[..., None, :] + s[..., None, :] * t.q)) <= s[..., None, :] / 2 * (1 + 1e-5) + 1e-12)
+    lo, hi = np.argmin(z, axis=-2), np.argmax(z, axis=-2)          # per channel
+    assert np.all(np.take_along_axis(t.q, lo[..., None, :], -2) == 0)
+    assert np.all(np.take_along_axis(t.q, hi[..., None, :], -2) == (1 << bits) - 1)
+
+
+def test_attention_with_per_channel_keys_matches_torch_sdpa():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((2, 5, 16, 128))
+    k = O.quantize_tiles_per_channel(x[0], 2, block=1)
+    v = O.quantize_tiles(x[1], 2, 0, block=1)
+    q = rng.standard_normal((4, 128))
+    got = O.decode_attention(q, k, v, 0.1, block=1)
+    kk = torch.from_numpy(O.dequantize_channel_tiles(k, unrotate=True, block=1).reshape(-1, 128))
+    vv = torch.from_numpy(O.dequantize_tiles(v.q, v.a, v.z, v.c, unrotate=True, block=1).reshape(-1, 128))
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q)[None], kk[None], vv[None],
+                                                           scale=0.1)[0].numpy()
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
 def test_quantize_row_scale_invariance():
     # Scaling one token row by a power of two scales that row's a and z by it
     # and changes no code and no column factor: the row step divides it out
