@@ -390,3 +390,32 @@ def mla_decode_attention(q: np.ndarray, lat: QuantizedTiles, rope: np.ndarray,
     s = qr @ ch.T + q[:, d:] @ np.asarray(rope, dtype=np.float64).T
     p = _softmax(softmax_scale * s)
     return rotate(p @ ch)
+
+
+def mla_decode_attention_with_tail(q: np.ndarray, lat: Optional[QuantizedTiles], rope: Optional[np.ndarray],
+                                   lat_tail: np.ndarray, rope_tail: np.ndarray, softmax_scale: float) -> np.ndarray:
+    """MLA decode step over a sequence whose newest tokens do not fill a tile.
+
+    Same reading as decode_attention_with_tail: the last L < T tokens stay
+    unquantised (latent row and rope key as given) and attention runs over
+    all of the sequence's tokens.  Written in the input basis: the cached
+    latent tiles are dequantised and rotated back, the tail rows join them
+    as they are; score = scale * (q_lat . latent + q_rope . rope), output =
+    sum p latent.  q: [H, d + rope_dim]; lat: [n_tiles, T, d] quantised (or
+    None); rope: [n_tiles * T, rope_dim]; lat_tail: [L, d]; rope_tail:
+    [L, rope_dim].  Returns [H, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = np.asarray(lat_tail).shape[-1]
+    rd = q.shape[-1] - d
+    keys = [np.asarray(lat_tail, dtype=np.float64).reshape(-1, d)]
+    ropes = [np.asarray(rope_tail, dtype=np.float64).reshape(-1, rd)]
+    if lat is not None and lat.q.shape[0] > 0:
+        keys.insert(0, dequantize_tiles(lat.q, lat.a, lat.z, lat.c, unrotate=True).reshape(-1, d))
+        ropes.insert(0, np.asarray(rope, dtype=np.float64).reshape(-1, rd))
+    kk, rr = np.concatenate(keys, 0), np.concatenate(ropes, 0)
+    if kk.shape[0] == 0:
+        return np.zeros((q.shape[0], d))
+    p = _softmax(softmax_scale * (q[:, :d] @ kk.T + q[:, d:] @ rr.T))
+    return p @ kk
+

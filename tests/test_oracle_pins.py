@@ -514,3 +514,31 @@ def test_mla_attention_matches_torch_sdpa_float64():
         torch.from_numpy(q)[None, :, None, :], torch.from_numpy(key)[None, None].expand(1, H, -1, -1),
         torch.from_numpy(ch)[None, None].expand(1, H, -1, -1), scale=scale)[0, :, 0, :].numpy()
     assert np.max(np.abs(o - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_mla_tail_attention_pins():
+    # an empty tail gives the cache-only formula (rotated domain, 1e-12); no
+    # cached tiles gives SDPA over the tail rows; moving the last tile's
+    # dequantised rows into the tail changes nothing
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(44)
+    d, rd, H = 512, 64, 8
+    lat = O.quantize_tiles(rng.standard_normal((3, 16, d)), 4, 4)
+    rope = rng.standard_normal((48, rd))
+    q = rng.standard_normal((H, d + rd))
+    base = O.mla_decode_attention(q, lat, rope, 0.04)
+    got = O.mla_decode_attention_with_tail(q, lat, rope, np.zeros((0, d)), np.zeros((0, rd)), 0.04)
+    assert np.max(np.abs(got - base)) < 1e-12
+    lt, rt = rng.standard_normal((7, d)), rng.standard_normal((7, rd))
+    only = O.mla_decode_attention_with_tail(q, None, None, lt, rt, 0.04)
+    kk = torch.from_numpy(np.concatenate([lt, rt], 1))[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q)[None], kk,
+                                                           torch.from_numpy(lt)[None], scale=0.04)[0].numpy()
+    assert np.max(np.abs(only - ref)) < 1e-12
+    rows = O.dequantize_tiles(lat.q[2], lat.a[2], lat.z[2], lat.c[2], unrotate=True)
+    two = O.QuantizedTiles(lat.q[:2], lat.a[:2], lat.z[:2], lat.c[:2])
+    moved = O.mla_decode_attention_with_tail(q, two, rope[:32], np.concatenate([rows, lt]),
+                                             np.concatenate([rope[32:], rt]), 0.04)
+    whole = O.mla_decode_attention_with_tail(q, lat, rope, lt, rt, 0.04)
+    assert np.max(np.abs(moved - whole)) < 1e-12
+
