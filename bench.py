@@ -81,8 +81,9 @@ def algorithmic_bytes(w):
     per_row_in = d * 2
     def cache_row(bits):                       # codes + (a, z) + c share of one row
         return d * bits / 8 + 2 * mb + d * mb / T
-    q_bytes = rows * 2 * per_row_in + rows * (cache_row(w.bits_k) + cache_row(w.bits_v))
-    dec_bytes = w.batch * w.seq_len * H * (cache_row(w.bits_k) + cache_row(w.bits_v)) \
+    k_row = (d * w.bits_k / 8 + d * 2 * mb / T) if w.k_per_channel else cache_row(w.bits_k)  # (s, m) per channel
+    q_bytes = rows * 2 * per_row_in + rows * (k_row + cache_row(w.bits_v))
+    dec_bytes = w.batch * w.seq_len * H * (k_row + cache_row(w.bits_v)) \
         + w.batch * w.num_q_heads * d * (2 + 4)
     return q_bytes, dec_bytes
 
@@ -157,11 +158,13 @@ def oracle_sample_step(w, sample):
     from oracle import kvarn_oracle as O
     from kv_cache_quantization_03_b200 import workloads as W
     xk, xv, q = sample
-    kt = O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters, w.block)
+    meta = "f16" if w.meta_f16 else "f32"
+    kt = O.quantize_tiles_per_channel(xk, w.bits_k, w.block) if w.k_per_channel else \
+        O.quantize_tiles(xk, w.bits_k, w.sinkhorn_iters, w.block, meta=meta)
     if w.mla:   # xv holds the rope keys
         O.mla_decode_attention(q, kt, xv, w.softmax_scale)
         return xk.shape[0] * xk.shape[1]
-    vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters, w.block)
+    vt = O.quantize_tiles(xv, w.bits_v, w.sinkhorn_iters, w.block, meta=meta)
     O.decode_attention(q, kt, vt, w.softmax_scale, block=w.block)
     return xk.shape[0] * xk.shape[1] / w.num_kv_heads
 
@@ -259,7 +262,8 @@ def config_dict(w, args):
             "num_kv_heads": w.num_kv_heads, "num_q_heads": w.num_q_heads, "head_dim": w.head_dim,
             "bits_k": w.bits_k, "bits_v": w.bits_v, "tile_tokens": w.tile_tokens,
             "sinkhorn_iters": w.sinkhorn_iters, "hadamard_block": w.hadamard_block or w.head_dim,
-            "metadata": "f16" if w.meta_f16 else "f32", "layers": w.num_layers,
+            "metadata": "f16" if w.meta_f16 else "f32", "key_groups": "channel" if w.k_per_channel else "token",
+            "layers": w.num_layers,
             "parallelism": "dp%d (independent shards)" % args.gpus,
             "l2": ("inputs larger than L2 (latent + rope bf16 %.2f GB per rank)" % (
                 w.num_layers * w.n_tok * (w.head_dim + w.rope_dim) * 2 / 1e9)) if w.mla else
@@ -294,7 +298,7 @@ def max_over_ranks(values, world: int, device=None):
 
 # --------------------------------------------------------------------------- GPU leg
 QUANTIZE_ONLY = ("prefill",)       # workloads whose step is quantise-append alone
-EXTRA_WORKLOADS = ("gqa", "gqa16", "prefill", "mla", "g128", "saw4", "rt1k")
+EXTRA_WORKLOADS = ("gqa", "gqa16", "prefill", "mla", "g128", "saw4", "kivi", "rt1k")
 
 
 def kernel_names(w):
@@ -318,7 +322,8 @@ def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
     cfg = kvq.make_config(head_dim=w.head_dim, num_kv_heads=w.num_kv_heads, tile_tokens=w.tile_tokens,
                           bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                           rope_dim=w.rope_dim, num_layers=w.num_layers, num_pages=w.num_pages, in_dtype=w.in_dtype,
-                          hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16)
+                          hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16,
+                          k_per_channel=w.k_per_channel)
     cache = QuantizedCache(cfg)
     host = {"k": torch.from_numpy(W.kv_inputs(ws, "k").view(np.int16))}
     if w.mla:

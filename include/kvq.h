@@ -60,12 +60,18 @@
  *               both float32, or IEEE half when meta_f16 = 1; each tile's
  *               scales are balanced by a power of two so that max c lies in
  *               (1/2, 1] (the dequantised tile does not change);
+ *   keys with k_per_channel = 1: k_tok_scale holds [d][2] = (s, m) per
+ *               channel, the step and minimum of the channel's T rotated
+ *               values, and k_chan_scale is unused (size 0, may be NULL);
+ *               dequantised rotated value s q + m;
  *   rope (MLA): bf16 [layer][page][T][rope_dim], unquantised.
  *
  * Supported on the GPU: head_dim 128 (GQA) with tile_tokens 16, 32, 64 or
  * 128 (the shipped "4-bit Keys, 2-bit Values Preset" uses 128), or 512 (MLA
  * latent) with tile_tokens 16; bits_k in {2,3,4,8}, bits_v in {2,4,8}, query
- * group size 1..8 for GQA and 1..128 heads for MLA; inputs fp16 or bf16.
+ * group size 1..8 for GQA and 1..128 heads for MLA; inputs fp16 or bf16;
+ * rotation blocks 1 (no rotation) .. head_dim for K/V caches; per-channel
+ * keys with 2-, 4- or 8-bit codes at tile_tokens 16.
  * Other shapes return KVQ_ERR_UNSUPPORTED.
  */
 #ifndef KVQ_H_
@@ -107,9 +113,10 @@ typedef struct kvq_config {
   int32_t bits_v;         /* value code width: 2, 4 or 8; ignored when mla */
   int32_t sinkhorn_iters; /* n >= 0 normalisation rounds (0 = rotation + RTN only) */
   int32_t hadamard_block; /* channels per block of the rotation: head_dim = the full
-                           * Sylvester rotation; 8..head_dim/2 (K/V caches only) = a
+                           * Sylvester rotation; 1..head_dim/2 (K/V caches only) = a
                            * block-diagonal rotation of consecutive channels (the
-                           * SAW-INT4 entry on the Hugging Face paper listing) */
+                           * SAW-INT4 entry on the Hugging Face paper listing);
+                           * 1 = no rotation */
   int32_t mla;            /* 1: one latent per token is key and value; no V arrays */
   int32_t rope_dim;       /* MLA: width of the unquantised bf16 rope key (64) */
   int32_t num_layers;     /* layers in the pool */
@@ -120,6 +127,11 @@ typedef struct kvq_config {
                            * (the compact layout: same codes, scales rounded
                            * to 11 significant bits; rows must stay within the
                            * half range, |a|, |z| < 65504) */
+  int32_t k_per_channel;  /* key quantisation axis: 0 = per token (KVarN; a
+                           * zero-filled config gets it), 1 = per channel
+                           * (the KIVI-style axes ablation: each channel's T
+                           * tokens are one RTN group; needs sinkhorn_iters = 0;
+                           * head_dim 128, tile_tokens 16).  Values stay per token */
 } kvq_config;
 
 /* Caller-owned device arrays of one cache; byte sizes from kvq_cache_layout

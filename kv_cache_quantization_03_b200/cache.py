@@ -44,8 +44,10 @@ class QuantizedCache:
         return self.arrays[which + "_codes"].view(*self.slot_shape(), c.tile_tokens * c.head_dim * bits // 8)
 
     def tok_scale(self, which="k"):
+        """Group scales: (a, z) per token [..][T][2], or, for per-channel keys, (s, m) per channel [..][d][2]."""
         c = self.cfg
-        return self.arrays[which + "_tok_scale"].view(*self.slot_shape(), c.tile_tokens, 2)
+        groups = c.head_dim if (which == "k" and c.k_per_channel) else c.tile_tokens
+        return self.arrays[which + "_tok_scale"].view(*self.slot_shape(), groups, 2)
 
     def chan_scale(self, which="k"):
         c = self.cfg

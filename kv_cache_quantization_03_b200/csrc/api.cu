@@ -52,12 +52,16 @@ kvq_status check_config(const kvq_config* c) {
   if (!c->mla && !valid_bits(c->bits_v)) return KVQ_ERR_INVALID_ARG;
   if (c->in_dtype != KVQ_F16 && c->in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (c->meta_f16 != 0 && c->meta_f16 != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->k_per_channel != 0 && c->k_per_channel != 1) return KVQ_ERR_INVALID_ARG;
+  // per-channel key groups are the ablation without normalisation (a row factor
+  // could not be folded into per-channel scales)
+  if (c->k_per_channel && (c->mla || c->sinkhorn_iters != 0)) return KVQ_ERR_INVALID_ARG;
   if (c->mla) {
     if (c->num_kv_heads != 1 || c->rope_dim < 0 || (c->rope_dim % 8)) return KVQ_ERR_INVALID_ARG;
   }
   if (!is_pow2(c->hadamard_block) || c->hadamard_block > c->head_dim) return KVQ_ERR_INVALID_ARG;
-  // block-diagonal rotations (blocks of 8 .. head_dim channels) for K/V caches; the MLA latent full width
-  if (c->hadamard_block < 8 || (c->mla && c->hadamard_block != c->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  // block-diagonal rotations (blocks of 1 .. head_dim channels) for K/V caches; the MLA latent full width
+  if (c->mla && c->hadamard_block != c->head_dim) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 
@@ -65,6 +69,9 @@ kvq_status check_config(const kvq_config* c) {
 // 16, 32, 64 or 128 tokens; a 512-wide MLA latent with 16-token tiles.
 kvq_status check_gpu_shape(const kvq_config* c) {
   if (c->head_dim != (c->mla ? 512 : 128)) return KVQ_ERR_UNSUPPORTED;
+  // per-channel keys and rotation blocks below 8 channels: 16-token tiles
+  if ((c->k_per_channel || c->hadamard_block < 8) && c->tile_tokens != 16) return KVQ_ERR_UNSUPPORTED;
+  if (c->k_per_channel && c->bits_k == 3) return KVQ_ERR_UNSUPPORTED;
   if (c->mla ? c->tile_tokens != 16 : (c->tile_tokens < 16 || c->tile_tokens > 128)) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
@@ -91,6 +98,7 @@ CacheArrays arrays(const kvq_cache_view* v, int which, int bits) {
   a.chan = which == 0 ? v->k_chan_scale : v->v_chan_scale;
   a.bits = bits;
   a.meta16 = 0;
+  a.per_channel = 0;
   return a;
 }
 
@@ -98,7 +106,7 @@ kvq_status check_view(const kvq_config* c, const kvq_cache_view* v) {
   if (!v) return KVQ_ERR_INVALID_ARG;
   const void* need[4] = {v->k_codes, v->k_tok_scale, v->k_chan_scale, nullptr};
   for (int i = 0; i < 3; ++i)
-    if (!need[i] || !aligned16(need[i])) return KVQ_ERR_INVALID_ARG;
+    if ((!need[i] && !(i == 2 && c->k_per_channel)) || !aligned16(need[i])) return KVQ_ERR_INVALID_ARG;
   if (!c->mla) {
     const void* vv[3] = {v->v_codes, v->v_tok_scale, v->v_chan_scale};
     for (int i = 0; i < 3; ++i)
@@ -207,8 +215,8 @@ kvq_status kvq_cache_layout(const kvq_config* c, size_t bytes_out[7]) {
   const size_t n = (size_t)slots(c), T = c->tile_tokens, d = c->head_dim;
   const size_t msz = c->meta_f16 ? 2 : 4;  // bytes of one a, z or c
   bytes_out[0] = n * T * d * c->bits_k / 8;
-  bytes_out[1] = n * T * 2 * msz;
-  bytes_out[2] = n * d * msz;
+  bytes_out[1] = c->k_per_channel ? n * d * 2 * msz : n * T * 2 * msz;  // (s, m) per channel, or (a, z) per token
+  bytes_out[2] = c->k_per_channel ? 0 : n * d * msz;
   const bool has_v = !c->mla;
   bytes_out[3] = has_v ? n * T * d * c->bits_v / 8 : 0;
   bytes_out[4] = has_v ? n * T * 2 * msz : 0;
@@ -236,6 +244,7 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   p.dst[0] = arrays(cache, 0, c->bits_k);
   p.dst[1] = arrays(cache, 1, c->bits_v);
   p.dst[0].meta16 = p.dst[1].meta16 = c->meta_f16;
+  p.dst[0].per_channel = c->k_per_channel;
   p.kinds = c->mla ? 1 : 2;
   p.n_tok = n_tok;
   p.num_layers = c->num_layers;
@@ -268,6 +277,7 @@ kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int3
   p.src[0] = arrays(cache, 0, c->bits_k);
   p.src[1] = arrays(cache, 1, c->bits_v);
   p.src[0].meta16 = p.src[1].meta16 = c->meta_f16;
+  p.src[0].per_channel = c->k_per_channel;
   p.kinds = c->mla ? 1 : 2;
   p.layer = layer;
   p.num_heads = c->num_kv_heads;
@@ -366,6 +376,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   p.k = arrays(cache, 0, c->bits_k);
   p.v = arrays(cache, 1, c->bits_v);
   p.k.meta16 = p.v.meta16 = c->meta_f16;
+  p.k.per_channel = c->k_per_channel;
   p.layer = layer;
   p.num_kv_heads = c->num_kv_heads;
   p.num_pages = c->num_pages;

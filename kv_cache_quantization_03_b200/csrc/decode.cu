@@ -45,17 +45,21 @@ struct StageLayout {
 };
 
 // One stage: the tile of nh adjacent kv-heads (their pages are contiguous in
-// every cache array): K codes | K (a, z) | K c | V codes | V (a, z) | V c,
-// with m bytes per a, z or c (4: float32, 2: half).
-__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv, int nh, int m) {
+// every cache array): K codes | K group scales | K c | V codes | V (a, z) |
+// V c, with m bytes per scale (4: float32, 2: half).  Key group scales are
+// (a, z) per token, or (s, m) per channel with per-channel keys (kpc), which
+// have no c.
+__host__ __device__ constexpr int kgroup_bytes(int m, int kpc) { return kpc ? kD * 2 * m : kT * 2 * m; }
+__host__ __device__ constexpr StageLayout stage_layout(int bk, int bv, int nh, int m, int kpc) {
   return StageLayout{nh * kT * kD * bk / 8,
                      nh * kT * kD * bv / 8,
                      nh * (kT * kD * bk / 8),
-                     nh * (kT * kD * bk / 8 + kT * 2 * m),
-                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m),
-                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m) + nh * kT * kD * bv / 8,
-                     nh * (kT * kD * bk / 8 + kT * 2 * m + kD * m) + nh * (kT * kD * bv / 8 + kT * 2 * m),
-                     nh * (kT * kD * (bk + bv) / 8 + 2 * (kT * 2 * m + kD * m))};
+                     nh * (kT * kD * bk / 8 + kgroup_bytes(m, kpc)),
+                     nh * (kT * kD * bk / 8 + kgroup_bytes(m, kpc) + (kpc ? 0 : kD * m)),
+                     nh * (kT * kD * bk / 8 + kgroup_bytes(m, kpc) + (kpc ? 0 : kD * m)) + nh * kT * kD * bv / 8,
+                     nh * (kT * kD * bk / 8 + kgroup_bytes(m, kpc) + (kpc ? 0 : kD * m)) +
+                         nh * (kT * kD * bv / 8 + kT * 2 * m),
+                     nh * (kT * kD * (bk + bv) / 8 + kgroup_bytes(m, kpc) + (kpc ? 0 : kD * m) + kT * 2 * m + kD * m)};
 }
 
 // (a, z) of token i, and c of channels i .. i + 3, from a stage's metadata
@@ -249,10 +253,11 @@ __device__ __forceinline__ bool wait_never_set(uint32_t ns) {
 // 2t, 2t+1, i.e. kv-head hs = t / 2.  The score MMAs run once per kv-head
 // (each lane keeps the result of its own kv-head); for P V each kv-head's
 // weights are masked to its own columns, so both MMAs add into one result.
-template <int BK, int BV, int NH, int M>
+template <int BK, int BV, int NH, int M, int KPC>
 __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr StageLayout SL = stage_layout(BK, BV, NH, M);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH, M, KPC);
+  constexpr int KG = kgroup_bytes(M, KPC);  // key group-scale bytes of one kv-head's tile
   constexpr int kStages = num_stages(NH);
   constexpr int KCB = SL.kcb / NH, VCB = SL.vcb / NH;  // code bytes of one kv-head's tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -387,14 +392,15 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     const uint8_t* vch = static_cast<const uint8_t*>(p.v.chan);
     if (p.sub_log2 == 0) {  // 16-token pages: the nh kv-heads' pages are contiguous in every array
       bulk_g2s(st, p.k.codes + slot * KCB, SL.kcb, bar);
-      bulk_g2s(st + SL.off_kaz, ktok + slot * (kT * 2 * M), NH * kT * 2 * M, bar);
-      bulk_g2s(st + SL.off_kc, kch + slot * (kD * M), NH * kD * M, bar);
+      bulk_g2s(st + SL.off_kaz, ktok + slot * KG, NH * KG, bar);
+      if constexpr (!KPC) bulk_g2s(st + SL.off_kc, kch + slot * (kD * M), NH * kD * M, bar);
       bulk_g2s(st + SL.off_v, p.v.codes + slot * VCB, SL.vcb, bar);
       bulk_g2s(st + SL.off_vaz, vtok + slot * (kT * 2 * M), NH * kT * 2 * M, bar);
       bulk_g2s(st + SL.off_vc, vch + slot * (kD * M), NH * kD * M, bar);
       return;
     }
     // longer pages: slice `sub` of each kv-head's page, in the same stage layout
+    // (per-channel keys come with 16-token pages only)
     const int spt = 1 << p.sub_log2, sub = (t0 + li) & (spt - 1);
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
@@ -406,8 +412,10 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       } else {
         bulk_g2s(st + h * KCB, kc + sub * KCB, KCB, bar);
       }
-      bulk_g2s(st + SL.off_kaz + h * (kT * 2 * M), ktok + (sh * spt + sub) * (kT * 2 * M), kT * 2 * M, bar);
-      bulk_g2s(st + SL.off_kc + h * (kD * M), kch + sh * (kD * M), kD * M, bar);
+      if constexpr (!KPC) {
+        bulk_g2s(st + SL.off_kaz + h * (kT * 2 * M), ktok + (sh * spt + sub) * (kT * 2 * M), kT * 2 * M, bar);
+        bulk_g2s(st + SL.off_kc + h * (kD * M), kch + sh * (kD * M), kD * M, bar);
+      }
       static_assert(BV != 3, "3-bit values have two planes");
       bulk_g2s(st + SL.off_v + h * VCB, p.v.codes + (sh * spt + sub) * VCB, VCB, bar);
       bulk_g2s(st + SL.off_vaz + h * (kT * 2 * M), vtok + (sh * spt + sub) * (kT * 2 * M), kT * 2 * M, bar);
@@ -437,8 +445,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     if (page >= 0 && page < p.num_pages) {
       const uint8_t* st = wsm + (i % kStages) * SL.bytes;
       const int hu = NH == 2 ? (g >> 2) : 0, hs = NH == 2 ? (t >> 1) : 0;  // kv-head of this lane's u / columns
-      const uint8_t* kaz = st + SL.off_kaz + hs * (2 * kT * M);
-      const uint8_t* kc = st + SL.off_kc + hu * (kD * M);
+      const uint8_t* kaz = st + SL.off_kaz + hs * KG;
+      // per-token keys: c of kv-head hu; per-channel keys: its (s, m) pairs
+      const uint8_t* kc = KPC ? st + SL.off_kaz + hu * KG : st + SL.off_kc + hu * (kD * M);
       const uint8_t* vaz = st + SL.off_vaz + hs * (2 * kT * M);
       const uint8_t* vc = st + SL.off_vc + hs * (kD * M);
 
@@ -452,10 +461,20 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int kk = 4 * ((k + rq) & 7);
-          const float4 c4 = ld_c4<M>(kc, 32 * t + kk);
-          const f2 a = mul2(make_float2(qv[4 * k], qv[4 * k + 1]), make_float2(c4.x, c4.y));
-          const f2 d = mul2(make_float2(qv[4 * k + 2], qv[4 * k + 3]), make_float2(c4.z, c4.w));
-          su2 = add2(su2, add2(a, d));
+          const f2 q01 = make_float2(qv[4 * k], qv[4 * k + 1]), q23 = make_float2(qv[4 * k + 2], qv[4 * k + 3]);
+          f2 a, d;
+          if constexpr (KPC) {  // u = q~ s; su2 gathers beta = sum q~ m, which takes z's place
+            const float2 p0 = ld_az<M>(kc, 32 * t + kk), p1 = ld_az<M>(kc, 32 * t + kk + 1);
+            const float2 p2 = ld_az<M>(kc, 32 * t + kk + 2), p3 = ld_az<M>(kc, 32 * t + kk + 3);
+            a = mul2(q01, make_float2(p0.x, p1.x));
+            d = mul2(q23, make_float2(p2.x, p3.x));
+            su2 = fma2(q01, make_float2(p0.y, p1.y), fma2(q23, make_float2(p2.y, p3.y), su2));
+          } else {
+            const float4 c4 = ld_c4<M>(kc, 32 * t + kk);
+            a = mul2(q01, make_float2(c4.x, c4.y));
+            d = mul2(q23, make_float2(c4.z, c4.w));
+            su2 = add2(su2, add2(a, d));
+          }
           u[4 * k] = a.x, u[4 * k + 1] = a.y, u[4 * k + 2] = d.x, u[4 * k + 3] = d.y;
         }
       }
@@ -490,8 +509,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
         for (int e = 0; e < 4; ++e)
           if (h == 0 || hs == h) S[e] = Sh[e] + Sl[e];
       }
-      const float2 az0 = ld_az<M>(kaz, g);
-      const float2 az1 = ld_az<M>(kaz, g + 8);
+      // per-channel keys: score = S + beta (a = 1, and su0, su1 hold beta)
+      const float2 az0 = KPC ? make_float2(1.f, 1.f) : ld_az<M>(kaz, g);
+      const float2 az1 = KPC ? make_float2(1.f, 1.f) : ld_az<M>(kaz, g + 8);
       float sc[4];
       sc[0] = fmaf(az0.x, S[0], az0.y * su0);
       sc[1] = fmaf(az0.x, S[1], az0.y * su1);
@@ -727,15 +747,15 @@ __global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
   }
 }
 
-template <int BK, int BV, int NH, int M>
+template <int BK, int BV, int NH, int M, int KPC>
 int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
-  constexpr StageLayout SL = stage_layout(BK, BV, NH, M);
+  constexpr StageLayout SL = stage_layout(BK, BV, NH, M, KPC);
   constexpr int kStages = num_stages(NH);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
   const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
-  auto kern = decode_d128_kernel<BK, BV, NH, M>;
+  auto kern = decode_d128_kernel<BK, BV, NH, M, KPC>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.splits, p.batch * p.num_kv_heads / NH);
   kern<<<grid, kDW * 32, smem, s>>>(p);
@@ -751,10 +771,20 @@ int launch_decode_d128(const DecodeParams& p, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bk = p.k.bits, bv = p.v.bits;
   const bool pairs = decode_kv_heads_per_cta(p.group, p.num_kv_heads) == 2;
-#define KVQ_CASE(K, V)                                                                        \
-  if (bk == K && bv == V) {                                                                   \
-    if (p.k.meta16) return pairs ? launch_bk_bv<K, V, 2, 2>(p, s) : launch_bk_bv<K, V, 1, 2>(p, s); \
-    return pairs ? launch_bk_bv<K, V, 2, 4>(p, s) : launch_bk_bv<K, V, 1, 4>(p, s);           \
+  if (p.k.per_channel) {  // the KIVI-style axes ablation: 2-, 4- and 8-bit codes (same widths for K and V)
+#define KVQ_KPC(K)                                                                                            \
+  if (bk == K && bv == K) {                                                                                   \
+    if (p.k.meta16) return pairs ? launch_bk_bv<K, K, 2, 2, 1>(p, s) : launch_bk_bv<K, K, 1, 2, 1>(p, s); \
+    return pairs ? launch_bk_bv<K, K, 2, 4, 1>(p, s) : launch_bk_bv<K, K, 1, 4, 1>(p, s);                 \
+  }
+    KVQ_KPC(2) KVQ_KPC(4) KVQ_KPC(8)
+#undef KVQ_KPC
+    return (int)cudaErrorInvalidValue;
+  }
+#define KVQ_CASE(K, V)                                                                              \
+  if (bk == K && bv == V) {                                                                         \
+    if (p.k.meta16) return pairs ? launch_bk_bv<K, V, 2, 2, 0>(p, s) : launch_bk_bv<K, V, 1, 2, 0>(p, s); \
+    return pairs ? launch_bk_bv<K, V, 2, 4, 0>(p, s) : launch_bk_bv<K, V, 1, 4, 0>(p, s);                 \
   }
   KVQ_CASE(4, 4) KVQ_CASE(3, 4) KVQ_CASE(2, 4) KVQ_CASE(8, 4)
   KVQ_CASE(4, 2) KVQ_CASE(3, 2) KVQ_CASE(2, 2) KVQ_CASE(8, 2)

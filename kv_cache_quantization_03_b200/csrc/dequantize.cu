@@ -45,13 +45,19 @@ __global__ void __launch_bounds__(kD) dequantize_kernel(DequantParams p) {
   auto meta = [&](const void* base, size_t i) {
     return src.meta16 ? __half2float(static_cast<const __half*>(base)[i]) : static_cast<const float*>(base)[i];
   };
+  // per-token groups: (a, z) per row and c per channel; per-channel key
+  // groups: (s, m) of this thread's channel, no row scales
   const size_t tok0 = slot * T * 2;
-  const float c = meta(src.chan, slot * kD + ch);
+  const float c = src.per_channel ? 1.f : meta(src.chan, slot * kD + ch);
+  const float cs = src.per_channel ? meta(src.tok, slot * kD * 2 + 2 * ch) : 0.f;
+  const float cm = src.per_channel ? meta(src.tok, slot * kD * 2 + 2 * ch + 1) : 0.f;
   float* out = p.out[kind] + (((size_t)pi * p.num_heads + head) * T) * kD;
   for (int r0 = 0; r0 < T; r0 += kT) {  // kT rows at a time
     for (int r = 0; r < kT; ++r)
-      tile[r][ch] = fmaf(meta(src.tok, tok0 + 2 * (r0 + r)), (float)read_code<kD>(codes, src.bits, T, r0 + r, ch),
-                         meta(src.tok, tok0 + 2 * (r0 + r) + 1)) * c;
+      tile[r][ch] = src.per_channel
+                        ? fmaf(cs, (float)read_code<kD>(codes, src.bits, T, r0 + r, ch), cm)
+                        : fmaf(meta(src.tok, tok0 + 2 * (r0 + r)), (float)read_code<kD>(codes, src.bits, T, r0 + r, ch),
+                               meta(src.tok, tok0 + 2 * (r0 + r) + 1)) * c;
     __syncthreads();
     if (p.unrotate) {  // H / sqrt(b) on each block of b = hblock channels
       for (int r = 0; r < kT; ++r) {

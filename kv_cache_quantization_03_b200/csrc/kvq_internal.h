@@ -29,6 +29,7 @@ struct CacheArrays {
   void* chan;        // [layer][page][head][d]     float32, or half when meta16
   int bits;
   int meta16;        // 1: a, z, c stored as IEEE half
+  int per_channel;   // 1: one (s, m) pair per channel in `tok` ([d][2]); no `chan`
 };
 
 struct QuantizeParams {

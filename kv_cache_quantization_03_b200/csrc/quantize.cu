@@ -198,9 +198,11 @@ __device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLau
 }
 
 // Channel bits 0..6 of the 128-channel block: bits 3..6 on the tensor cores
-// (16 MMAs), bits 0..2 as three butterfly stages on fp32 pairs.
-template <bool F16>
-__device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const uint32_t (&afrag)[4], f2 (&P)[2][2][8]) {
+// (16 MMAs), bits 0..2 as three butterfly stages on fp32 pairs (only the
+// stages inside the rotation's block: none for block 1, no rotation).
+template <bool F16, bool SMALL_BLOCKS>
+__device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const uint32_t (&afrag)[4], f2 (&P)[2][2][8],
+                                            int hblock) {
   const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int h = 0; h < 2; ++h)
@@ -221,7 +223,7 @@ __device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const 
       for (int s = 1; s < 8; s <<= 1)
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
-          if (b & s) continue;
+          if ((b & s) || (SMALL_BLOCKS && s >= hblock)) continue;
           const f2 x = P[h][m3][b], y = P[h][m3][b + s];
           P[h][m3][b] = add2(x, y);
           P[h][m3][b + s] = sub2(x, y);
@@ -271,10 +273,15 @@ __device__ __forceinline__ void slice_sync(int slot) {
 template <int TW>
 constexpr size_t stage_bytes() { return (size_t)cta_warps<TW>() * 2 * 8 * 32 * sizeof(uint4); }
 
-template <bool F16, int BITS, int D, int TW>
+// AXES = 1: the ablation instantiation (16-token tiles at head_dim 128):
+// rotation blocks below 8 channels, and per-channel key groups when the
+// stream asks for them; the standard instantiation (AXES = 0) carries
+// neither.
+template <bool F16, int BITS, int D, int TW, int AXES>
 __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_warps<TW>() : 3))
     quantize_kernel(QuantLaunch p) {
   static_assert(TW == 1 || D == kBlk, "tiles longer than 16 tokens need head_dim 128");
+  static_assert(AXES == 0 || (D == kBlk && TW == 1), "the ablation instantiation is for 16 x 128 tiles");
   constexpr int kCW = cta_warps<TW>();
   constexpr int W = D / kBlk;     // warps per tile along channels
   constexpr int kTile = kT * TW;  // tokens per tile
@@ -320,6 +327,45 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
     // a warp reaches the TMEM lanes 32 (warp % 4) .. +31 only
     tpark = tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) + 64 * (warp >> 2);
   }
+  // Packs and stores the codes of this lane's rows of the tile in `slot`:
+  // tq_of(h, j) gives the magic-number-rounded codes of P[h][j >> 3][j & 7]
+  // (tokens 8h + 2t, 8h + 2t + 1 at channel 16g + j of the warp's block).
+  auto emit_codes = [&](size_t slot, auto&& tq_of) {
+    uint8_t* codes = p.dst.codes + slot * (kTile * D * BITS / 8);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t q[2][16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const f2 tq = tq_of(h, j);
+        q[0][j] = __float_as_uint(tq.x);
+        q[1][j] = __float_as_uint(tq.y);
+      }
+#pragma unroll
+      for (int tp = 0; tp < 2; ++tp) {
+        const int tok = kT * wt + 8 * h + 2 * t + tp;  // row of the tile
+        const uint32_t* f = q[tp];
+        constexpr int row_bytes = D * BITS / 8, seg = kBlk * BITS / 8;
+        if constexpr (BITS == 4) {
+          *reinterpret_cast<uint2*>(codes + tok * row_bytes + seg * blk + 8 * g) =
+              make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
+        } else if constexpr (BITS == 8) {
+          *reinterpret_cast<uint4*>(codes + tok * row_bytes + seg * blk + 16 * g) =
+              make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
+                         gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
+        } else if constexpr (BITS == 2) {
+          *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = pack_crumbs(f);
+        } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
+          *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
+          *reinterpret_cast<uint16_t*>(codes + kTile * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) =
+              (uint16_t)hi;
+        }
+      }
+    }
+  };
   uint32_t L[2][4][4];
   int32_t page = 0;
   uint32_t rounds = 0;  // rounds done by this warp (parity of the column-partial buffer)
@@ -336,7 +382,7 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       read_staged(staged[warp][buf], lane, L);
       if (tile + stride < p.total) stage_tile<TW>(staged[warp][buf ^ 1], p, tile + stride, wt, g, t, lane, page);
     }
-    hadamard128<F16>(L, afrag, P);
+    hadamard128<F16, AXES == 1>(L, afrag, P, D == kBlk ? p.hblock : kBlk);
     const uint32_t cur = tile;
     const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
     const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
@@ -368,6 +414,58 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
           acc = (__popc(blk & k) & 1) ? sub2(acc, y) : add2(acc, y);
         }
         P[i >> 4][(i >> 3) & 1][i & 7] = acc;
+      }
+    }
+    if constexpr (AXES == 1 && BITS != 3) {
+      if (p.dst.per_channel) {
+        // Per-channel groups (the KIVI-style axes, no normalisation): channel
+        // 16g + j is tokens {2t, 2t+1, 2t+8, 2t+9} of this lane and of the
+        // lanes t' = t ^ 1, t ^ 2; its minimum and step go to the group
+        // scales as (s, m) pairs, lane t writing channels 16g + 4t .. + 3.
+        float cmn[16], cmx[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const f2 a = P[0][j >> 3][j & 7], b = P[1][j >> 3][j & 7];
+          cmn[j] = fminf(fminf(a.x, a.y), fminf(b.x, b.y));
+          cmx[j] = fmaxf(fmaxf(a.x, a.y), fmaxf(b.x, b.y));
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            cmn[j] = fminf(cmn[j], __shfl_xor_sync(0xffffffffu, cmn[j], off));
+            cmx[j] = fmaxf(cmx[j], __shfl_xor_sync(0xffffffffu, cmx[j], off));
+          }
+        constexpr float kQm = (float)((1 << BITS) - 1);
+        float st[4], mt[4];  // the lane's four channels 16g + 4t + i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = t == 0 ? cmn[i] : t == 1 ? cmn[4 + i] : t == 2 ? cmn[8 + i] : cmn[12 + i];
+          const float hi = t == 0 ? cmx[i] : t == 1 ? cmx[4 + i] : t == 2 ? cmx[8 + i] : cmx[12 + i];
+          st[i] = (hi - lo) / kQm * inv_sqrt_d;
+          mt[i] = lo * inv_sqrt_d;
+        }
+        const size_t gi = slot * (D * 2) + 2 * (16 * g + 4 * t);
+        if (p.dst.meta16) {
+          const __half2 h0 = __floats2half2_rn(st[0], mt[0]), h1 = __floats2half2_rn(st[1], mt[1]);
+          const __half2 h2 = __floats2half2_rn(st[2], mt[2]), h3 = __floats2half2_rn(st[3], mt[3]);
+          *reinterpret_cast<uint4*>(static_cast<__half*>(p.dst.tok) + gi) =
+              make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                         *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+        } else {
+          float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(p.dst.tok) + gi);
+          d4[0] = make_float4(st[0], mt[0], st[1], mt[1]);
+          d4[1] = make_float4(st[2], mt[2], st[3], mt[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {  // cmx becomes 1 / step
+          const float sj = (cmx[j] - cmn[j]) / kQm;
+          cmx[j] = sj > 0.f ? rcp_nr(sj) : 0.f;
+        }
+        emit_codes(slot, [&](int h, int j) {
+          return fma2(sub2(P[h][j >> 3][j & 7], splat2(cmn[j])), splat2(cmx[j]), splat2(kMagic));
+        });
+        continue;  // (one warp per tile here: no tile barrier to meet)
       }
     }
     f2 A[2][2][8];
@@ -635,46 +733,16 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       else
         *reinterpret_cast<float2*>(static_cast<float*>(p.dst.tok) + ti) = make_float2(s_own * fold, omn * fold);
     }
-    uint8_t* codes = p.dst.codes + slot * (kTile * D * BITS / 8);
+    f2 m2h[2], is2h[2];  // row minimum and 1/step of the lane's tokens 8h + 2t, 8h + 2t + 1
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const f2 m2 = make_float2(__shfl_sync(0xffffffffu, omn, (h << 4) | t),
-                                __shfl_sync(0xffffffffu, omn, (h << 4) | 8 | t));
-      const f2 is2 = make_float2(__shfl_sync(0xffffffffu, is_own, (h << 4) | t),
-                                 __shfl_sync(0xffffffffu, is_own, (h << 4) | 8 | t));
-      uint32_t q[2][16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        // (y - m) / s rounded to the nearest integer (ties to even) by the
-        // single rounding of the fused multiply-add into the magic number
-        const f2 tq = fma2(sub2(P[h][j >> 3][j & 7], m2), is2, splat2(kMagic));
-        q[0][j] = __float_as_uint(tq.x);
-        q[1][j] = __float_as_uint(tq.y);
-      }
-#pragma unroll
-      for (int tp = 0; tp < 2; ++tp) {
-        const int tok = kT * wt + 8 * h + 2 * t + tp;  // row of the tile
-        const uint32_t* f = q[tp];
-        constexpr int row_bytes = D * BITS / 8, seg = kBlk * BITS / 8;
-        if constexpr (BITS == 4) {
-          *reinterpret_cast<uint2*>(codes + tok * row_bytes + seg * blk + 8 * g) =
-              make_uint2(pack_nibbles(f), pack_nibbles(f + 8));
-        } else if constexpr (BITS == 8) {
-          *reinterpret_cast<uint4*>(codes + tok * row_bytes + seg * blk + 16 * g) =
-              make_uint4(gather4(f[0], f[1], f[2], f[3]), gather4(f[4], f[5], f[6], f[7]),
-                         gather4(f[8], f[9], f[10], f[11]), gather4(f[12], f[13], f[14], f[15]));
-        } else if constexpr (BITS == 2) {
-          *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = pack_crumbs(f);
-        } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
-          uint32_t lo = 0, hi = 0;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
-          *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
-          *reinterpret_cast<uint16_t*>(codes + kTile * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) =
-              (uint16_t)hi;
-        }
-      }
+      m2h[h] = make_float2(__shfl_sync(0xffffffffu, omn, (h << 4) | t), __shfl_sync(0xffffffffu, omn, (h << 4) | 8 | t));
+      is2h[h] = make_float2(__shfl_sync(0xffffffffu, is_own, (h << 4) | t),
+                            __shfl_sync(0xffffffffu, is_own, (h << 4) | 8 | t));
     }
+    // (y - m) / s rounded to the nearest integer (ties to even) by the single
+    // rounding of the fused multiply-add into the magic number
+    emit_codes(slot, [&](int h, int j) { return fma2(sub2(P[h][j >> 3][j & 7], m2h[h]), is2h[h], splat2(kMagic)); });
     tile_sync<W>();  // shared tile buffers are reused by the next tile
   }
   {
@@ -684,7 +752,6 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "n"(kTmemCols));
   }
 }
-
 FastDiv make_div(uint32_t d) {
   FastDiv f{d, 0, 0};
   uint32_t s = 0;
@@ -694,26 +761,26 @@ FastDiv make_div(uint32_t d) {
   return f;
 }
 
-template <bool F16, int BITS, int D, int TW>
+template <bool F16, int BITS, int D, int TW, int AXES>
 void launch_one(const QuantLaunch& q, int sms, cudaStream_t s) {
   constexpr int kCW = cta_warps<TW>(), tpc = kCW / ((D / kBlk) * TW);
   constexpr size_t dyn = D == kBlk ? stage_bytes<TW>() : 0;  // raw-tile staging at head_dim 128
   const int64_t need = (q.total + tpc - 1) / tpc;
   const int64_t cap = (int64_t)sms * (D == kBlk ? 16 / kCW : 3);  // resident CTAs per SM
   const int grid = (int)(need < cap ? need : cap);
-  auto kern = quantize_kernel<F16, BITS, D, TW>;
+  auto kern = quantize_kernel<F16, BITS, D, TW, AXES>;
   // static + dynamic shared memory may pass 48 KB, which needs the opt-in
   if (dyn > 0) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
   kern<<<grid, kCW * 32, dyn, s>>>(q);
 }
 
-template <bool F16, int D, int TW>
+template <bool F16, int D, int TW, int AXES = 0>
 int launch_bits(const QuantLaunch& q, int bits, int sms, cudaStream_t s) {
   switch (bits) {
-    case 2: launch_one<F16, 2, D, TW>(q, sms, s); break;
-    case 3: launch_one<F16, 3, D, TW>(q, sms, s); break;
-    case 4: launch_one<F16, 4, D, TW>(q, sms, s); break;
-    case 8: launch_one<F16, 8, D, TW>(q, sms, s); break;
+    case 2: launch_one<F16, 2, D, TW, AXES>(q, sms, s); break;
+    case 3: launch_one<F16, 3, D, TW, AXES>(q, sms, s); break;
+    case 4: launch_one<F16, 4, D, TW, AXES>(q, sms, s); break;
+    case 8: launch_one<F16, 8, D, TW, AXES>(q, sms, s); break;
     default: return (int)cudaErrorInvalidValue;
   }
   return (int)cudaGetLastError();
@@ -725,7 +792,9 @@ int launch_shape(const QuantLaunch& q, int head_dim, int tile_tokens, int sms, c
   if (head_dim == 512 && tile_tokens == 16) return launch_bits<F16, 512, 1>(q, bits, sms, s);
   if (head_dim != 128) return (int)cudaErrorInvalidValue;
   switch (tile_tokens) {
-    case 16: return launch_bits<F16, 128, 1>(q, bits, sms, s);
+    case 16:  // blocks below 8 channels or per-channel key groups: the ablation instantiation
+      return (q.hblock < 8 || q.dst.per_channel) ? launch_bits<F16, 128, 1, 1>(q, bits, sms, s)
+                                                 : launch_bits<F16, 128, 1>(q, bits, sms, s);
     case 32: return launch_bits<F16, 128, 2>(q, bits, sms, s);
     case 64: return launch_bits<F16, 128, 4>(q, bits, sms, s);
     case 128: return launch_bits<F16, 128, 8>(q, bits, sms, s);

@@ -51,7 +51,7 @@ class kvq_config(ctypes.Structure):
         ("bits_k", ctypes.c_int32), ("bits_v", ctypes.c_int32), ("sinkhorn_iters", ctypes.c_int32),
         ("hadamard_block", ctypes.c_int32), ("mla", ctypes.c_int32), ("rope_dim", ctypes.c_int32),
         ("num_layers", ctypes.c_int32), ("num_pages", ctypes.c_int64), ("in_dtype", ctypes.c_int),
-        ("meta_f16", ctypes.c_int32),
+        ("meta_f16", ctypes.c_int32), ("k_per_channel", ctypes.c_int32),
     ]
 
 
@@ -134,11 +134,11 @@ def kvq_version() -> str:
 
 def make_config(head_dim=128, num_kv_heads=1, tile_tokens=16, bits_k=4, bits_v=4, sinkhorn_iters=4,
                 mla=False, rope_dim=0, num_layers=1, num_pages=0, in_dtype="bf16",
-                hadamard_block=None, meta_f16=False) -> kvq_config:
+                hadamard_block=None, meta_f16=False, k_per_channel=False) -> kvq_config:
     return kvq_config(head_dim, num_kv_heads, tile_tokens, bits_k, bits_v, sinkhorn_iters,
                       head_dim if hadamard_block is None else hadamard_block, int(bool(mla)), rope_dim,
                       num_layers, num_pages, {"fp16": KVQ_F16, "bf16": KVQ_BF16}.get(in_dtype, in_dtype),
-                      int(bool(meta_f16)))
+                      int(bool(meta_f16)), int(bool(k_per_channel)))
 
 
 def make_view(ptrs: Sequence) -> kvq_cache_view:

@@ -26,6 +26,8 @@ mla    64 seq x 32768 tok, latent 512 (4-bit) + rope 64 (bf16), 128
 g128   the shipped preset kvarn_k4v2_g128 on the gqa shapes and
        distribution: 4-bit K, 2-bit V, 128-token tiles (= pages)
 gqa16  gqa (same seed and inputs) with a, z, c stored as IEEE half
+kivi   ablation on gqa's inputs: KIVI-style axes (keys per channel, values
+       per token), 2-bit codes, no rotation, no normalisation
 saw4   ablation on the gqa shapes and distribution: block-diagonal
        Hadamard (32-channel blocks) and per-token INT4, no normalisation
 =====  ==================================================================
@@ -63,6 +65,7 @@ class Workload:
     rope_dim: int = 0
     hadamard_block: int = 0         # channels per block of a block-diagonal rotation; 0 = full head_dim
     meta_f16: bool = False          # a, z, c stored as IEEE half (the compact layout)
+    k_per_channel: bool = False     # keys quantised per channel (the KIVI-style axes ablation)
     description: str = ""
 
     @property
@@ -118,6 +121,9 @@ WORKLOADS: Dict[str, Workload] = {
                                  "no normalisation rounds, gqa shapes"),
     "gqa16": Workload("gqa16", 32, 8192, 8, 32, 128, 4, 4, 4, 2, meta_f16=True,
                       description="gqa with the compact layout: a, z, c as IEEE half (same inputs as gqa)"),
+    "kivi": Workload("kivi", 32, 8192, 8, 32, 128, 2, 2, 0, 2, hadamard_block=1, k_per_channel=True,
+                     description="ablation: KIVI-style axes, 2-bit keys per channel and values per token, "
+                                 "no rotation, no normalisation (same inputs as gqa)"),
 }
 
 
@@ -153,7 +159,7 @@ def outlier_channels(w: Workload, layer: int, head: int, which: str) -> np.ndarr
         return np.array([3, 17, 64, 101])
     if w.mla:
         n = round(0.01 * w.head_dim)
-    elif _base_name(w) in ("gqa", "g128", "saw4", "gqa16"):
+    elif _base_name(w) in ("gqa", "g128", "saw4", "gqa16", "kivi"):
         n = round(0.02 * w.head_dim)
     else:
         return np.zeros(0, dtype=np.int64)
@@ -191,8 +197,8 @@ def kv_inputs(w: Workload, which: str, tokens: Optional[slice] = None) -> np.nda
         r = _rng(w.seed, 10 * kind)
         scale = np.exp(r.uniform(math.log(0.1), math.log(10.0), size=(L, 1, H, d))).astype(np.float32)
     outl = None
-    if base in ("rt1k", "gqa", "mla", "g128", "saw4", "gqa16"):
-        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0, "g128": 15.0, "saw4": 15.0, "gqa16": 15.0}[base]
+    if base in ("rt1k", "gqa", "mla", "g128", "saw4", "gqa16", "kivi"):
+        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0, "g128": 15.0, "saw4": 15.0, "gqa16": 15.0, "kivi": 15.0}[base]
         outl = np.ones((L, 1, H, d), dtype=np.float32)
         for layer in range(L):
             for h in range(H):

@@ -42,7 +42,8 @@ def config_for(w: W.Workload, num_pages=None) -> kvq.kvq_config:
                            bits_k=w.bits_k, bits_v=w.bits_v, sinkhorn_iters=w.sinkhorn_iters, mla=w.mla,
                            rope_dim=w.rope_dim, num_layers=w.num_layers,
                            num_pages=w.num_pages if num_pages is None else num_pages, in_dtype=w.in_dtype,
-                           hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16)
+                           hadamard_block=w.hadamard_block or None, meta_f16=w.meta_f16,
+                           k_per_channel=w.k_per_channel)
 
 
 class QuantRun:
@@ -76,16 +77,9 @@ class QuantRun:
         st, bits = kvq.kvq_read_error(self.err)
         return bits
 
-    def gpu_tiles(self, which: str, layer: int, tiles, head: int) -> O.QuantizedTiles:
+    def gpu_tiles(self, which: str, layer: int, tiles, head: int):
         """Stored codes (unpacked with the oracle's unpack) and scales of tiles (append order)."""
-        w = self.w
-        bits = w.bits_k if which == "k" else w.bits_v
-        pg = torch.from_numpy(self.pages[np.asarray(tiles)].astype(np.int64)).cuda()
-        raw = self.cache.codes(which)[layer, pg, head].cpu().numpy()
-        tok = self.cache.tok_scale(which)[layer, pg, head].cpu().numpy()
-        ch = self.cache.chan_scale(which)[layer, pg, head].cpu().numpy()
-        q = O.unpack_codes(raw, bits, w.tile_tokens, w.head_dim)
-        return O.QuantizedTiles(q=q, a=tok[..., 0], z=tok[..., 1], c=ch)
+        return gpu_pages(self, which, layer, self.pages[np.asarray(tiles)], head)
 
     def input_tiles(self, which: str, layer: int, tiles, head: int) -> np.ndarray:
         w = self.w
@@ -94,15 +88,17 @@ class QuantRun:
         return W.half_bits_to_f64(src[layer, idx, head, :], w.in_dtype)   # [n, T, d]
 
 
-def oracle_fraction(x: np.ndarray, bits: int, n_iter: int, block=None) -> np.ndarray:
-    """The oracle's (y - m) / s of every element (to locate rounding ties)."""
+def oracle_fraction(x: np.ndarray, bits: int, n_iter: int, block=None, per_channel=False) -> np.ndarray:
+    """The oracle's (y - m) / s of every element (to locate rounding ties);
+    the groups are token rows, or channels with per_channel."""
     y, _, _ = O.sinkhorn_normalize(O.rotate(x, block), n_iter)
-    m = y.min(-1, keepdims=True)
-    s = (y.max(-1, keepdims=True) - m) / ((1 << bits) - 1)
+    ax = -2 if per_channel else -1
+    m = y.min(ax, keepdims=True)
+    s = (y.max(ax, keepdims=True) - m) / ((1 << bits) - 1)
     return (y - m) / np.where(s > 0, s, 1.0)
 
 
-def exact_half_ties(x: np.ndarray, bits: int, n_iter: int, block, idx) -> np.ndarray:
+def exact_half_ties(x: np.ndarray, bits: int, n_iter: int, block, idx, per_channel=False) -> np.ndarray:
     """Whether the codes at idx (index arrays into tiles x: [n, T, d]) sit at
     an exact rounding tie: (y - m) / s a half-integer in real arithmetic.
 
@@ -117,19 +113,20 @@ def exact_half_ties(x: np.ndarray, bits: int, n_iter: int, block, idx) -> np.nda
     d = x.shape[-1]
     h = O.block_hadamard_matrix(d, block or d).astype(object)
     qmax = (1 << bits) - 1
-    rows = {}
+    tiles = {}
     out = np.zeros(n, dtype=bool)
     for e, (i, t, j) in enumerate(zip(*idx)):
-        if (i, t) not in rows:
-            fr = [Fraction(float(v)) for v in x[i, t]]
-            den = max(f.denominator for f in fr)           # a power of two
-            ints = np.array([f.numerator * (den // f.denominator) for f in fr], dtype=object)
-            y = ints.dot(h)                                # den * sqrt(b) * y, exact
-            rows[(i, t)] = (y, min(y), max(y))
-        y, lo, hi = rows[(i, t)]
+        if i not in tiles:   # the whole tile, exactly: den * sqrt(b) * y as integers
+            fr = [[Fraction(float(v)) for v in row] for row in x[i]]
+            den = max(f.denominator for row in fr for f in row)   # a power of two
+            ints = np.array([[f.numerator * (den // f.denominator) for f in row] for row in fr], dtype=object)
+            tiles[i] = ints.dot(h)
+        y = tiles[i]
+        grp = y[:, j] if per_channel else y[t, :]        # the RTN group of the element
+        lo, hi = min(grp), max(grp)
         if hi == lo:
             continue
-        num = 2 * qmax * (y[j] - lo)                       # 2 (y - m) / s = num / (hi - lo)
+        num = 2 * qmax * (y[t, j] - lo)                    # 2 (y - m) / s = num / (hi - lo)
         out[e] = num % (hi - lo) == 0 and (num // (hi - lo)) % 2 == 1
     return out
 
@@ -139,26 +136,35 @@ class Flips(NamedTuple):
     exact_ties: int   # flips at exact ties (both codes correct)
 
 
-def compare_quantized(gpu: O.QuantizedTiles, ora: O.QuantizedTiles, x: np.ndarray, bits: int, n_iter: int,
-                      block=None, label="", check_rate=True) -> Flips:
+def compare_quantized(gpu, ora, x: np.ndarray, bits: int, n_iter: int, block=None, label="",
+                      check_rate=True) -> Flips:
     """Asserts the code and scale tolerances of quantised tiles against the
     oracle's on the same inputs x: [n, T, d]; returns the flip counts.
 
     With check_rate=False the caller aggregates the counted flips over
     several comparisons and checks the 1e-5 rate itself."""
+    per_channel = isinstance(ora, O.ChannelQuantizedTiles)
     diff = gpu.q != ora.q
     counted = ties = 0
     if diff.any():
         assert np.all(np.abs(gpu.q[diff] - ora.q[diff]) == 1), label + ": code off by more than 1"
-        frac = oracle_fraction(x, bits, n_iter, block)
+        frac = oracle_fraction(x, bits, n_iter, block, per_channel)
         f = frac[diff]
         dist = np.abs(f - np.floor(f) - 0.5)
         assert np.all(dist <= CODE_TIE_BAND), "%s: flip away from a tie (distance %g)" % (label, dist.max())
-        exact = exact_half_ties(x, bits, n_iter, block, np.nonzero(diff))
+        exact = exact_half_ties(x, bits, n_iter, block, np.nonzero(diff), per_channel)
         ties = int(exact.sum())
         counted = int(diff.sum()) - ties
     if check_rate:
         assert counted <= CODE_FLIP_RATE * gpu.q.size, "%s: %d flips in %d codes" % (label, counted, gpu.q.size)
+    if per_channel:   # the per-channel step and minimum
+        for name in ("s", "m"):
+            g = getattr(gpu, name).astype(np.float64)
+            o = getattr(ora, name).astype(np.float64)
+            tol = (2.0 ** -10 if np.asarray(getattr(gpu, name)).dtype == np.float16 else SCALE_RTOL) * np.abs(o)
+            assert np.all(np.abs(g - o) <= tol), "%s: %s off by %g relative" % (
+                label, name, float(np.max(np.abs(g - o) / np.maximum(np.abs(o), 1e-300))))
+        return Flips(counted, ties)
     if np.asarray(gpu.a).dtype == np.float16:
         _, a64, z64, c64 = O.quantize_stages(x, bits, n_iter, block)
         for name, exact in (("a", a64), ("z", z64), ("c", c64)):
@@ -184,7 +190,10 @@ def check_tiles(run, which: str, layer: int, tiles, head: int, label="", check_r
     w = run.w
     bits = w.bits_k if which == "k" else w.bits_v
     x = run.input_tiles(which, layer, tiles, head)
-    ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block, meta="f16" if w.meta_f16 else "f32")
+    if which == "k" and w.k_per_channel:
+        ora = O.quantize_tiles_per_channel(x, bits, w.block)
+    else:
+        ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block, meta="f16" if w.meta_f16 else "f32")
     gpu = run.gpu_tiles(which, layer, tiles, head)
     return compare_quantized(gpu, ora, x, bits, w.sinkhorn_iters, w.block, label, check_rate)
 
@@ -200,16 +209,18 @@ def seq_tiles(w: W.Workload, b: int) -> np.ndarray:
     return b * w.tiles_per_seq + np.arange(w.tiles_per_seq)
 
 
-def gpu_pages(run: QuantRun, which: str, layer: int, pages, head: int) -> O.QuantizedTiles:
+def gpu_pages(run: QuantRun, which: str, layer: int, pages, head: int):
     """Stored tiles of the given physical pages (unpacked with the oracle)."""
     w = run.w
     bits = w.bits_k if which == "k" else w.bits_v
     pg = torch.as_tensor(np.asarray(pages, dtype=np.int64)).cuda()
     raw = run.cache.codes(which)[layer, pg, head].cpu().numpy()
     tok = run.cache.tok_scale(which)[layer, pg, head].cpu().numpy()
+    q = O.unpack_codes(raw, bits, w.tile_tokens, w.head_dim)
+    if which == "k" and w.k_per_channel:       # (s, m) per channel
+        return O.ChannelQuantizedTiles(q=q, s=tok[..., 0], m=tok[..., 1])
     ch = run.cache.chan_scale(which)[layer, pg, head].cpu().numpy()
-    return O.QuantizedTiles(q=O.unpack_codes(raw, bits, w.tile_tokens, w.head_dim), a=tok[..., 0],
-                            z=tok[..., 1], c=ch)
+    return O.QuantizedTiles(q=q, a=tok[..., 0], z=tok[..., 1], c=ch)
 
 
 class DecodeRun:

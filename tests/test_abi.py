@@ -62,6 +62,15 @@ def test_cache_layout_sizes(kvq):
     bad.meta_f16 = 2
     with pytest.raises(kvq.KvqError):
         kvq.kvq_cache_layout(bad)
+    # per-channel keys (KIVI-style axes): (s, m) per channel, no key c
+    kc = kvq.make_config(num_kv_heads=8, num_layers=2, num_pages=10, bits_k=2, bits_v=2, sinkhorn_iters=0,
+                         hadamard_block=1, k_per_channel=True)
+    assert kvq.kvq_cache_layout(kc) == [n * 16 * 128 * 2 // 8, n * 128 * 2 * 4, 0, n * 16 * 128 * 2 // 8,
+                                        n * 16 * 2 * 4, n * 128 * 4, 0]
+    for kw in (dict(sinkhorn_iters=4), dict(mla=True, head_dim=512, num_kv_heads=1, rope_dim=64)):
+        bad = kvq.make_config(num_pages=4, k_per_channel=True, **kw)
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_cache_layout(bad)
 
 
 def test_invalid_configs_rejected(kvq):
@@ -71,8 +80,8 @@ def test_invalid_configs_rejected(kvq):
         with pytest.raises(kvq.KvqError):
             kvq.kvq_cache_layout(c)
     out = (ctypes.c_size_t * 7)()
-    for blk, want in ((64, kvq.KVQ_OK), (8, kvq.KVQ_OK), (4, kvq.KVQ_ERR_UNSUPPORTED), (48, kvq.KVQ_ERR_INVALID_ARG),
-                      (256, kvq.KVQ_ERR_INVALID_ARG)):
+    for blk, want in ((64, kvq.KVQ_OK), (8, kvq.KVQ_OK), (4, kvq.KVQ_OK), (1, kvq.KVQ_OK),
+                      (48, kvq.KVQ_ERR_INVALID_ARG), (256, kvq.KVQ_ERR_INVALID_ARG), (0, kvq.KVQ_ERR_INVALID_ARG)):
         c = kvq.make_config(num_pages=4, hadamard_block=blk)
         assert kvq.lib.kvq_cache_layout(ctypes.byref(c), out) == want, blk
     m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=4, hadamard_block=128)
@@ -108,6 +117,15 @@ def test_host_rejections_before_launch(kvq):
                raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # layer out of range
     assert dec(c, view, 0, fake, fake, 64, fake, 0, 8, 0.1, fake, fake, ws, fake, 0,
                raise_on_error=False) == kvq.KVQ_OK                    # empty batch: nothing to do
+    # per-channel keys: no key c array needed; 16-token tiles and 2/4/8-bit keys only
+    kc = kvq.make_config(num_kv_heads=2, num_pages=8, bits_k=2, bits_v=2, sinkhorn_iters=0, hadamard_block=1,
+                         k_per_channel=True)
+    no_kc = kvq.make_view([fake, fake, None, fake, fake, fake, None])
+    assert f(kc, no_kc, fake, fake, None, 0, fake, fake, 0, raise_on_error=False) == kvq.KVQ_OK
+    for kw in (dict(tile_tokens=32), dict(bits_k=3)):
+        k2 = kvq.make_config(num_kv_heads=2, num_pages=8, bits_v=2, sinkhorn_iters=0, k_per_channel=True,
+                             **dict(dict(bits_k=2), **kw))
+        assert f(k2, no_kc, fake, fake, None, 32, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def test_tile_lengths_accepted_and_rejected(kvq):

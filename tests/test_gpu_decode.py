@@ -38,6 +38,7 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("saw4", dict(batch=3, seq_len=512)),
     ("prefill", dict(seq_len=1024, num_layers=2)),   # per-channel scales over two decades
     ("gqa16", dict(batch=3, seq_len=512)),            # a, z, c as IEEE half
+    ("kivi", dict(batch=3, seq_len=512)),             # keys per channel, no rotation
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]
@@ -123,6 +124,19 @@ def test_decode_parity_half_metadata(name, kw):
     o = dec()
     assert run.error_bits() == 0
     assert np.all(np.isfinite(o))
+    _check(dec, o)
+
+
+@pytest.mark.parametrize("group,bits,block,meta16", [(8, 4, 1, False), (4, 8, 128, True), (1, 2, 32, False),
+                                                 (2, 4, 1, True)])
+def test_decode_parity_per_channel_keys(group, bits, block, meta16):
+    # KIVI-style axes through one and two kv-heads per CTA, with and without a rotation
+    w = dataclasses.replace(W.WORKLOADS["kivi"].scaled(batch=2, seq_len=768), num_q_heads=8 * group, bits_k=bits,
+                            bits_v=bits, hadamard_block=block, meta_f16=meta16)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=[768, 400 // 16 * 16])
+    o = dec()
+    assert run.error_bits() == 0
     _check(dec, o)
 
 

@@ -18,6 +18,7 @@ SMALL = {
     "mla": dict(batch=2, seq_len=256),
     "g128": dict(batch=2, seq_len=512),
     "saw4": dict(batch=2, seq_len=512),
+    "kivi": dict(batch=2, seq_len=512),
 }
 
 
@@ -177,6 +178,19 @@ def test_quantize_parity_half_metadata(name):
         assert torch.equal(run.cache.codes(which), ref.cache.codes(which)), which
 
 
+@pytest.mark.parametrize("bits,block,meta16", [(4, 1, False), (8, 1, False), (2, 32, False), (4, 128, True),
+                                           (2, 1, True)])
+def test_quantize_parity_per_channel_keys(bits, block, meta16):
+    # KIVI-style axes: keys per channel (with and without a rotation, either
+    # metadata format), values per token
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["kivi"].scaled(batch=2, seq_len=256), bits_k=bits, bits_v=bits,
+                            hadamard_block=block, meta_f16=meta16)
+    run = QuantRun(w)
+    assert run.error_bits() == 0
+    _check_all(run)
+
+
 def test_quantize_bad_page_sets_error_and_skips_tile():
     w = W.WORKLOADS["gqa"].scaled(batch=1, seq_len=64)
     pages = np.array([0, 7, 2, 3], dtype=np.int32)        # pool of 4 pages: 7 is out of range
@@ -247,7 +261,7 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4", "gqa16"])
+@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4", "gqa16", "kivi"])
 def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
     w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
@@ -263,7 +277,10 @@ def test_dequantize_matches_oracle_on_stored_codes(name):
             for h in range(w.num_kv_heads):
                 inv = np.argsort(run.pages)                      # page -> tile
                 g = run.gpu_tiles(which, 0, inv, h)              # tiles in page order
-                ref = O.dequantize_tiles(g.q, g.a, g.z, g.c, unrotate=bool(unrot), block=w.block)
+                if isinstance(g, O.ChannelQuantizedTiles):
+                    ref = O.dequantize_channel_tiles(g, unrotate=bool(unrot), block=w.block)
+                else:
+                    ref = O.dequantize_tiles(g.q, g.a, g.z, g.c, unrotate=bool(unrot), block=w.block)
                 got = out[:, h].cpu().numpy().astype(np.float64)
                 scale = np.max(np.abs(ref), axis=(-1, -2), keepdims=True)
                 assert np.max(np.abs(got - ref) / scale) < 2e-6
