@@ -220,21 +220,24 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache_view* cac
                                 uint32_t* dev_error, void* stream);
 
 /* kvq_decode_attention for sequences whose newest tokens do not fill a page
- * yet (GQA caches).  The KVarN pages are silent on partial tiles; here the
- * last tail_lens[b] < T tokens of sequence b stay unquantised in a tail
- * buffer and attention runs over its cached tokens and its tail together
- * (a tail token is scored with q . k and weighted by its value row as is;
- * the result is the softmax over all of the sequence's keys).
- *   k_tail, v_tail: device, in_dtype [num_layers][batch][tile_tokens]
- *                [num_kv_heads][head_dim], 16-byte aligned: rows 0 ..
+ * yet.  The KVarN pages are silent on partial tiles; here the last
+ * tail_lens[b] < T tokens of sequence b stay unquantised in a tail buffer
+ * and attention runs over its cached tokens and its tail together (a tail
+ * token is scored with q . k and weighted by its value row as is; the
+ * result is the softmax over all of the sequence's keys).
+ *   k_tail, v_tail: device, 16-byte aligned, [num_layers][batch]
+ *                [tile_tokens][num_kv_heads][head_dim] in in_dtype: rows 0 ..
  *                tail_lens[b] - 1 of sequence b are its tail in this layer;
  *                the same layout as kvq_quantize_append's input with
  *                n_tok = batch * tile_tokens, so full tails are quantised in
- *                one append call (dst_page[b] = -1 skips the others);
+ *                one append call (dst_page[b] = -1 skips the others).
+ *                MLA caches: k_tail holds the latent rows [num_layers]
+ *                [batch][tile_tokens][head_dim] in in_dtype and v_tail the
+ *                rope keys [num_layers][batch][tile_tokens][rope_dim] bf16;
  *   tail_lens:   device int32 [batch], 0 .. tile_tokens (a value outside
  *                sets KVQ_DEVERR_BAD_SEQ and the tail is ignored);
  * the other arguments and the workspace are those of kvq_decode_attention.
- * MLA caches and tiles longer than 128 tokens return KVQ_ERR_UNSUPPORTED. */
+ * Tiles longer than 128 tokens return KVQ_ERR_UNSUPPORTED. */
 kvq_status kvq_decode_attention_tail(const kvq_config* cfg, const kvq_cache_view* cache, int32_t layer,
                                      const void* q, const int32_t* block_table,
                                      int32_t max_pages_per_seq, const int32_t* seq_lens,
@@ -242,6 +245,29 @@ kvq_status kvq_decode_attention_tail(const kvq_config* cfg, const kvq_cache_view
                                      int32_t batch, int32_t num_q_heads, float softmax_scale,
                                      float* out, void* workspace, size_t workspace_bytes,
                                      uint32_t* dev_error, void* stream);
+
+/* One decode step with quantise-on-fill: for every sequence b with
+ * fill_page[b] >= 0, the full tail of this layer (all tile_tokens rows of
+ * k_tail / v_tail for b) is first quantised into page fill_page[b] of this
+ * layer, exactly as kvq_quantize_append would; then attention runs over the
+ * cached pages and the remaining tails as in kvq_decode_attention_tail.
+ * Both steps are enqueued on `stream` in that order by this one call.
+ * (The pages are silent on tokens short of a tile; this is the serving
+ * reading of the unquantised tail: a tail is quantised when it fills.)
+ *   fill_page:   device int32 [batch]: the page that receives b's full tail,
+ *                or -1 (no fill); pages must be distinct and outside what
+ *                other calls are reading;
+ * the caller describes the state after the fill: block_table row b already
+ * ends with fill_page[b], seq_lens[b] counts it, and tail_lens[b] = 0 for a
+ * filled sequence (its tail buffer rows are read by the fill only).  The
+ * other arguments are those of kvq_decode_attention_tail. */
+kvq_status kvq_decode_attention_fill(const kvq_config* cfg, const kvq_cache_view* cache, int32_t layer,
+                                     const void* q, const int32_t* block_table,
+                                     int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                     const void* k_tail, const void* v_tail, const int32_t* tail_lens,
+                                     const int32_t* fill_page, int32_t batch, int32_t num_q_heads,
+                                     float softmax_scale, float* out, void* workspace,
+                                     size_t workspace_bytes, uint32_t* dev_error, void* stream);
 
 /* kvq_decode_attention for callers that cannot allocate device memory when
  * they decode (a plug-in whose host process owns all device allocations and

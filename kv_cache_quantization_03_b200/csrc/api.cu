@@ -176,6 +176,45 @@ size_t decode_ws_bytes_mla(int64_t batch, const DecodePlan& d) {
 
 kvq_status cuda_status(int e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
+// Quantise n_tok rows of `layers` consecutive layers, the first being
+// `layer0`, into the cache (arguments already validated).  The rows are
+// [layers][n_tok][H][d] (MLA rope [layers][n_tok][rope_dim]); the kernel
+// sees a cache whose first layer is layer0.
+kvq_status quantize_rows(const kvq_config* c, const kvq_cache_view* cache, const void* k_rows, const void* v_rows,
+                         const void* rope_rows, int64_t n_tok, const int32_t* dst_page, uint32_t* dev_error,
+                         int layers, int layer0, void* stream) {
+  const size_t slot0 = (size_t)layer0 * c->num_pages * c->num_kv_heads;  // slots before layer0
+  const size_t msz = c->meta_f16 ? 2 : 4, T = c->tile_tokens, d = c->head_dim;
+  QuantizeParams p{};
+  p.src[0] = k_rows;
+  p.src[1] = v_rows;
+  for (int kind = 0; kind < 2; ++kind) {
+    p.dst[kind] = arrays(cache, kind, kind == 0 ? c->bits_k : c->bits_v);
+    p.dst[kind].meta16 = c->meta_f16;
+    const bool pc = kind == 0 && c->k_per_channel;
+    p.dst[kind].per_channel = pc;
+    if (p.dst[kind].codes) p.dst[kind].codes += slot0 * (T * d * p.dst[kind].bits / 8);
+    if (p.dst[kind].tok) p.dst[kind].tok = static_cast<uint8_t*>(p.dst[kind].tok) + slot0 * (pc ? d * 2 : T * 2) * msz;
+    if (p.dst[kind].chan && !pc) p.dst[kind].chan = static_cast<uint8_t*>(p.dst[kind].chan) + slot0 * d * msz;
+  }
+  p.kinds = c->mla ? 1 : 2;
+  p.n_tok = n_tok;
+  p.num_layers = layers;
+  p.num_heads = c->num_kv_heads;
+  p.num_pages = c->num_pages;
+  p.iters = c->sinkhorn_iters;
+  p.dst_page = dst_page;
+  p.err = dev_error;
+  p.total_tiles = (int64_t)p.kinds * layers * (n_tok / c->tile_tokens) * c->num_kv_heads;
+  if (p.total_tiles >= (int64_t)1 << 31) return KVQ_ERR_UNSUPPORTED;  // tile ids are 32-bit in the kernel
+  p.rope_src = (c->mla && c->rope_dim > 0) ? rope_rows : nullptr;
+  p.rope_dst = cache->rope ? static_cast<uint8_t*>(cache->rope) + (size_t)layer0 * c->num_pages * T * c->rope_dim * 2
+                           : nullptr;
+  p.rope_dim = c->rope_dim;
+  p.hblock = c->hadamard_block;
+  return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, c->tile_tokens, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -238,29 +277,8 @@ kvq_status kvq_quantize_append(const kvq_config* c, const kvq_cache_view* cache,
   if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new))) return KVQ_ERR_INVALID_ARG;
   if ((st = check_gpu_shape(c)) != KVQ_OK) return st;
   if (n_tok == 0) return KVQ_OK;
-  QuantizeParams p{};
-  p.src[0] = k_new;
-  p.src[1] = v_new;
-  p.dst[0] = arrays(cache, 0, c->bits_k);
-  p.dst[1] = arrays(cache, 1, c->bits_v);
-  p.dst[0].meta16 = p.dst[1].meta16 = c->meta_f16;
-  p.dst[0].per_channel = c->k_per_channel;
-  p.kinds = c->mla ? 1 : 2;
-  p.n_tok = n_tok;
-  p.num_layers = c->num_layers;
-  p.num_heads = c->num_kv_heads;
-  p.num_pages = c->num_pages;
-  p.iters = c->sinkhorn_iters;
-  p.dst_page = dst_page;
-  p.err = dev_error;
-  p.total_tiles = (int64_t)p.kinds * c->num_layers * (n_tok / c->tile_tokens) * c->num_kv_heads;
-  if (p.total_tiles >= (int64_t)1 << 31) return KVQ_ERR_UNSUPPORTED;  // tile ids are 32-bit in the kernel
-  p.rope_src = (c->mla && c->rope_dim > 0) ? rope_new : nullptr;
-  p.rope_dst = cache->rope;
-  p.rope_dim = c->rope_dim;
-  p.hblock = c->hadamard_block;
-  if (p.rope_src && !aligned16(p.rope_src)) return KVQ_ERR_INVALID_ARG;
-  return cuda_status(launch_quantize(p, c->in_dtype == KVQ_F16, c->head_dim, c->tile_tokens, stream));
+  if (c->mla && c->rope_dim > 0 && !aligned16(rope_new)) return KVQ_ERR_INVALID_ARG;
+  return quantize_rows(c, cache, k_new, v_new, rope_new, n_tok, dst_page, dev_error, c->num_layers, 0, stream);
 }
 
 kvq_status kvq_dequantize(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
@@ -359,6 +377,11 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
     m.tiles_per_split = plan.tiles_per_split;
     m.qprep = reinterpret_cast<uint8_t*>(m.part_ml + (size_t)batch * plan.splits * kMlaHeads * 2);
     m.err = dev_error;
+    m.lat_tail = static_cast<const uint16_t*>(k_tail);  // latent rows; v_tail holds the rope keys
+    m.rope_tail = static_cast<const uint16_t*>(v_tail);
+    m.tail_lens = tail_lens;
+    m.tail_f16 = c->in_dtype == KVQ_F16;
+    m.tail_tokens = c->tile_tokens;
     return cuda_status(launch_decode_mla(m, stream));
   }
   const int group = num_q_heads / c->num_kv_heads;
@@ -424,7 +447,6 @@ kvq_status kvq_decode_attention_tail(const kvq_config* c, const kvq_cache_view* 
                                      const int32_t* tail_lens, int32_t batch, int32_t num_q_heads,
                                      float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                                      uint32_t* dev_error, void* stream) {
-  if (c && c->mla) return check_config(c) == KVQ_OK ? KVQ_ERR_UNSUPPORTED : check_config(c);
   if (batch > 0 && (!k_tail || !v_tail || !tail_lens)) return KVQ_ERR_INVALID_ARG;
   if ((k_tail && !aligned16(k_tail)) || (v_tail && !aligned16(v_tail))) return KVQ_ERR_INVALID_ARG;
   if (c && c->tile_tokens > 128) return KVQ_ERR_UNSUPPORTED;
@@ -434,6 +456,40 @@ kvq_status kvq_decode_attention_tail(const kvq_config* c, const kvq_cache_view* 
 }
 
 void kvq_set_test_wait(uint32_t ns) { g_test_wait_ns.store(ns, std::memory_order_relaxed); }
+
+kvq_status kvq_decode_attention_fill(const kvq_config* c, const kvq_cache_view* cache, int32_t layer,
+                                     const void* q, const int32_t* block_table, int32_t max_pages_per_seq,
+                                     const int32_t* seq_lens, const void* k_tail, const void* v_tail,
+                                     const int32_t* tail_lens, const int32_t* fill_page, int32_t batch,
+                                     int32_t num_q_heads, float softmax_scale, float* out, void* workspace,
+                                     size_t workspace_bytes, uint32_t* dev_error, void* stream) {
+  kvq_status st = check_config(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_view(c, cache)) != KVQ_OK) return st;
+  if (layer < 0 || layer >= c->num_layers || batch < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch > 0 && (!k_tail || !v_tail || !tail_lens || !fill_page)) return KVQ_ERR_INVALID_ARG;
+  if ((k_tail && !aligned16(k_tail)) || (v_tail && !aligned16(v_tail))) return KVQ_ERR_INVALID_ARG;
+  if (c->tile_tokens > 128) return KVQ_ERR_UNSUPPORTED;
+  if ((st = check_decode_shape(c)) != KVQ_OK) return st;
+  if (batch == 0) return KVQ_OK;
+  // the decode's own checks (shapes, workspace) before anything is launched
+  size_t need = 0;
+  if ((st = kvq_decode_workspace_bytes(c, batch, num_q_heads, max_pages_per_seq * c->tile_tokens, &need)) != KVQ_OK)
+    return st;
+  if (workspace_bytes < need) return KVQ_ERR_WORKSPACE_TOO_SMALL;
+  // 1) this layer's full tails into their pages: the rows of every sequence
+  //    (fill_page[b] = -1 skips b), as one append of batch * T tokens
+  const size_t row_elems = (size_t)c->tile_tokens * c->num_kv_heads * c->head_dim;  // one sequence's tail
+  const uint8_t* kl = static_cast<const uint8_t*>(k_tail) + (size_t)layer * batch * row_elems * 2;
+  const uint8_t* vl = static_cast<const uint8_t*>(v_tail) +
+                      (size_t)layer * batch * (c->mla ? (size_t)c->tile_tokens * c->rope_dim : row_elems) * 2;
+  st = quantize_rows(c, cache, kl, c->mla ? nullptr : vl, c->mla ? vl : nullptr, (int64_t)batch * c->tile_tokens,
+                     fill_page, dev_error, 1, layer, stream);
+  if (st != KVQ_OK) return st;
+  // 2) attention over the cache (now holding the filled pages) and the remaining tails
+  return decode(c, cache, layer, q, block_table, max_pages_per_seq, seq_lens, k_tail, v_tail, tail_lens, batch,
+                num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error, stream);
+}
 
 kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream) {
   if (!dev_error || !host_bits) return KVQ_ERR_INVALID_ARG;

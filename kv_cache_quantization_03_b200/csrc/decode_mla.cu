@@ -620,11 +620,58 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
   }
 }
 
-// Merge the splits of one (sequence, head), normalise, rotate back with H_512.
+// Merge the splits of one (sequence, head), rotate back with H_512,
+// normalise.  With a tail, its tokens join as one more partial: their scores
+// q_lat . latent + q_rope . rope and their latent sum are taken in the input
+// basis (the rotation is orthogonal), and the sum is added after the splits'
+// sum has been rotated back.
+constexpr int kMlaMaxTail = 16;
 __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
   __shared__ float buf[kLat];
+  __shared__ float red[kLat / 32][kMlaMaxTail];  // per warp, per tail token: partial scores
+  __shared__ float ts[kMlaMaxTail];              // tail scores (log2 units)
   const int b = blockIdx.x / p.num_q_heads, h = blockIdx.x % p.num_q_heads, j = threadIdx.x;
-  float mx = kNegBig;
+  const int warp = j >> 5, lane = j & 31;
+  int L = 0;
+  if (p.lat_tail) {
+    L = p.tail_lens[b];
+    if (L < 0 || L > p.tail_tokens || L > kMlaMaxTail) {
+      if (j == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+      L = 0;
+    }
+  }
+  float tm = kNegBig, tl = 0.f, tv = 0.f;  // tail: max, sum, value sum of channel j
+  if (L > 0) {
+    const size_t row0 = ((size_t)p.layer * p.batch + b) * p.tail_tokens;
+    const uint16_t* qh = p.q + ((size_t)b * p.num_q_heads + h) * kKf;
+    auto lat = [&](int t) {
+      const uint16_t x = p.lat_tail[(row0 + t) * kLat + j];
+      return p.tail_f16 ? __half2float(__ushort_as_half(x)) : bf16f(x);
+    };
+    const float qj = bf16f(qh[j]), qr = j < kRope ? bf16f(qh[kLat + j]) : 0.f;
+    for (int t = 0; t < L; ++t) {
+      float s = qj * lat(t);
+      if (j < kRope) s = fmaf(qr, bf16f(p.rope_tail[(row0 + t) * kRope + j]), s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (lane == 0) red[warp][t] = s;
+    }
+    __syncthreads();
+    if (j < L) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kLat / 32; ++w) s += red[w][j];
+      ts[j] = s * p.scale_log2;
+    }
+    __syncthreads();
+    for (int t = 0; t < L; ++t) tm = fmaxf(tm, ts[t]);
+    for (int t = 0; t < L; ++t) {
+      const float e = ex2f(ts[t] - tm);
+      tl += e;
+      tv = fmaf(e, lat(t), tv);
+    }
+  }
+  float mx = tm;
   for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)b * p.splits + s) * kH + h) * 2]);
   float acc = 0.f, l = 0.f;
   for (int s = 0; s < p.splits; ++s) {
@@ -633,7 +680,7 @@ __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
     acc = fmaf(f, p.part_o[i * kLat + j], acc);
     l = fmaf(f, p.part_ml[i * 2 + 1], l);
   }
-  buf[j] = l > 0.f ? acc / l : 0.f;
+  buf[j] = acc;
   __syncthreads();
   for (int s = 1; s < kLat; s <<= 1) {
     const float x = buf[j & ~s], y = buf[j | s];
@@ -641,7 +688,13 @@ __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
     buf[j] = (j & s) ? (x - y) : (x + y);
     __syncthreads();
   }
-  p.out[((size_t)b * p.num_q_heads + h) * kLat + j] = buf[j] * 0.044194173824159216f;
+  float o = buf[j] * 0.044194173824159216f;
+  if (L > 0) {
+    const float f = ex2f(tm - mx);
+    o = fmaf(f, tv, o);
+    l = fmaf(f, tl, l);
+  }
+  p.out[((size_t)b * p.num_q_heads + h) * kLat + j] = l > 0.f ? o / l : 0.f;
 }
 
 template <int BITS, int M>

@@ -119,6 +119,13 @@ struct MlaDecodeParams {
   int tiles_per_split;          // even
   uint8_t* qprep;               // [B][2][128 x 288 f16]: rotated queries in the score-operand layout
   uint32_t* err;
+  // unquantised tail of each sequence, merged by the combine kernel;
+  // lat_tail == nullptr: no tail
+  const uint16_t* lat_tail;     // [layers][B][T][512], fp16 or bf16
+  const uint16_t* rope_tail;    // [layers][B][T][64] bf16
+  const int32_t* tail_lens;     // [B], 0..T
+  int tail_f16;                 // 1: fp16 latent rows, 0: bf16
+  int tail_tokens;              // T
 };
 
 // Launchers (defined in the .cu files); return a cudaError_t value.

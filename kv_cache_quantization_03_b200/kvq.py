@@ -39,7 +39,7 @@ KVQ_F16, KVQ_BF16, KVQ_F32 = 0, 1, 2
 
 EXPORTED = (
     "kvq_config_from_string", "kvq_cache_layout", "kvq_quantize_append", "kvq_dequantize",
-    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_tail",
+    "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_tail", "kvq_decode_attention_fill",
     "kvq_decode_attention_noalloc", "kvq_read_error", "kvq_set_test_wait",
     "kvq_status_string", "kvq_version",
 )
@@ -76,6 +76,9 @@ _sig = {
                                             ctypes.c_size_t, _P, _P]),
     "kvq_decode_attention_tail": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                                  _P, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P,
+                                                 _P, ctypes.c_size_t, _P, _P]),
+    "kvq_decode_attention_fill": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
+                                                 _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P,
                                                  _P, ctypes.c_size_t, _P, _P]),
     "kvq_decode_attention_noalloc": (ctypes.c_int, [_cfgp, _viewp, ctypes.c_int32, _P, _P, ctypes.c_int32, _P,
                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
@@ -195,6 +198,17 @@ def kvq_decode_attention_tail(cfg, view, layer, q, block_table, max_pages_per_se
                                        _ptr(tail_lens), batch, num_q_heads, float(softmax_scale), _ptr(out),
                                        _ptr(workspace), workspace_bytes, _ptr(dev_error), _stream(stream))
     return _check("kvq_decode_attention_tail", st, raise_on_error)
+
+
+def kvq_decode_attention_fill(cfg, view, layer, q, block_table, max_pages_per_seq, seq_lens, k_tail, v_tail,
+                              tail_lens, fill_page, batch, num_q_heads, softmax_scale, out, workspace,
+                              workspace_bytes, dev_error, stream=None, raise_on_error=True) -> int:
+    """Quantise this layer's full tails into fill_page (-1: none), then decode with the remaining tails."""
+    st = lib.kvq_decode_attention_fill(ctypes.byref(cfg), ctypes.byref(view), layer, _ptr(q), _ptr(block_table),
+                                       max_pages_per_seq, _ptr(seq_lens), _ptr(k_tail), _ptr(v_tail),
+                                       _ptr(tail_lens), _ptr(fill_page), batch, num_q_heads, float(softmax_scale),
+                                       _ptr(out), _ptr(workspace), workspace_bytes, _ptr(dev_error), _stream(stream))
+    return _check("kvq_decode_attention_fill", st, raise_on_error)
 
 
 def kvq_decode_attention_noalloc(cfg, view, layer, q, block_table, max_pages_per_seq, seq_lens, batch,

@@ -253,6 +253,14 @@ def tail_inputs(w: Workload, which: str) -> np.ndarray:
     return _round_to(x, w.in_dtype)
 
 
+def tail_rope_inputs(w: Workload) -> np.ndarray:
+    """Unquantised rope keys of an MLA tail buffer: uint16 bf16 bits
+    [layers][B][T][rope_dim], N(0,1)."""
+    r = _rng(w.seed, 9)
+    x = r.standard_normal(size=(w.num_layers, w.batch, w.tile_tokens, w.rope_dim), dtype=np.float32)
+    return _round_to(x, "bf16")
+
+
 def tail_lens(w: Workload) -> np.ndarray:
     """Tail length of every sequence: int32 [B], uniform in [0, T)."""
     r = _rng(w.seed, 8)

@@ -35,6 +35,15 @@ CODE_TIE_BAND = 1e-4
 CODE_FLIP_RATE = 1e-5
 SCALE_RTOL = 1e-6
 ATTN_TOL = 2e-3
+# MLA decode on short contexts (tens of tokens, outside the MLA workload):
+# its 128-head contraction runs on single-f16 operands, and the query's f16
+# rounding shifts every token's score the same way, so it does not average
+# out over a few tokens.  A CPU emulation of that rounding (f16 query, f16
+# latent chunk, f16 P, fp32 accumulation) on 32..256-token contexts of the
+# mla distribution gives up to 2.7e-3 max relative error over 128 heads
+# (1.65e-3 at 4096 tokens; 5.9e-4 with an exact query).  The MLA workload
+# itself is checked at ATTN_TOL.
+MLA_SHORT_ATTN_TOL = 3.5e-3
 
 
 def config_for(w: W.Workload, num_pages=None) -> kvq.kvq_config:

@@ -161,10 +161,21 @@ def test_tail_entry_host_rejections(kvq):
              raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
     assert f(c, view, *args, None, None, None, 0, 8, 0.1, fake, fake, ws, fake, 0,
              raise_on_error=False) == kvq.KVQ_OK                     # empty batch: nothing to do
+    # MLA caches take a tail too (latent rows + rope keys); their checks run before any launch
     m = kvq.make_config(head_dim=512, num_kv_heads=1, mla=True, rope_dim=64, num_pages=8)
     mview = kvq.make_view([fake] * 3 + [None] * 3 + [fake])
-    assert f(m, mview, *args, fake, fake, fake, 4, 128, 0.1, fake, fake, 1 << 30, fake, 0,
-             raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
+    assert f(m, mview, *args, fake, fake + 8, fake, 4, 128, 0.1, fake, fake, 1 << 30, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG          # misaligned rope tail
+    assert f(m, mview, *args, fake, fake, fake, 4, 128, 0.1, fake, fake, 16, fake, 0,
+             raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    g = kvq.kvq_decode_attention_fill    # the fill call: every check before the fill's launch
+    for mm, vv, heads in ((c, view, 8), (m, mview, 128)):
+        assert g(mm, vv, *args, fake, fake, fake, None, 4, heads, 0.1, fake, fake, 1 << 30, fake, 0,
+                 raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG      # no fill pages
+        assert g(mm, vv, *args, fake, fake, fake, fake, 4, heads, 0.1, fake, fake, 16, fake, 0,
+                 raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    assert g(c, view, 0, fake, fake, 64, fake, fake, fake, fake, fake, 0, 8, 0.1, fake, fake, 0, fake, 0,
+             raise_on_error=False) == kvq.KVQ_OK                       # empty batch
 
 
 def test_decode_workspace_counts_16_token_tiles(kvq):

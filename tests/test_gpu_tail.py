@@ -13,8 +13,8 @@ from oracle import kvarn_oracle as O
 
 pytestmark = pytest.mark.gpu
 
-from _parity import (ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_error,  # noqa: E402
-                     compare_quantized)
+from _parity import (ATTN_TOL, CODE_FLIP_RATE, MLA_SHORT_ATTN_TOL, DecodeRun, QuantRun,  # noqa: E402
+                     attention_error, compare_quantized)
 
 
 def _check_tail(dec: DecodeRun, o: np.ndarray, layer=0, lens=None):
@@ -139,7 +139,107 @@ def test_tail_entry_rejections():
              w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
     assert f(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, kt.data_ptr() + 2, kt, tl, 2, dec.hq,
              w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
-    m = dataclasses.replace(W.WORKLOADS["mla"].scaled(batch=1, seq_len=32))
-    mrun = QuantRun(m)
-    assert f(mrun.cfg, mrun.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, kt, kt, tl, 1, 128,
-             m.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
+    g = kvq.kvq_decode_attention_fill
+    assert g(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, kt, kt, tl, None, 2, dec.hq,
+             w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert g(run.cfg, run.cache.view, 3, dec.q, dec.bt_d, dec.maxp, dec.sl_d, kt, kt, tl, tl, 2, dec.hq,
+             w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err, raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
+    assert g(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d, kt, kt, tl, tl, 2, dec.hq,
+             w.softmax_scale, dec.out, dec.ws, 16, run.err, raise_on_error=False) == kvq.KVQ_ERR_WORKSPACE_TOO_SMALL
+    torch.cuda.synchronize()
+    assert run.error_bits() == 0                               # nothing was launched
+
+
+def _mla_oracle_tail(dec: DecodeRun, b: int, layer=0):
+    w = dec.run.w
+    n = int(dec.sl[b]) // w.tile_tokens
+    L = int(dec.tl[b])
+    q = W.half_bits_to_f64(dec.q_bits[b], "bf16")
+    lt = W.half_bits_to_f64(dec.k_tail_bits[layer, b, :L].reshape(L, w.head_dim), w.in_dtype)
+    rt = W.half_bits_to_f64(dec.v_tail_bits[layer, b, :L], "bf16")
+    lat = rope = None
+    if n:
+        from _parity import gpu_pages
+        pages = dec.bt[b, :n]
+        lat = gpu_pages(dec.run, "k", layer, pages, 0)
+        rope_all = dec.run.cache["rope"].view(w.num_layers, -1, w.tile_tokens, w.rope_dim)
+        pg = torch.as_tensor(np.asarray(pages, dtype=np.int64)).cuda()
+        rope = rope_all[layer, pg].float().cpu().numpy().astype(np.float64).reshape(-1, w.rope_dim)
+    return O.mla_decode_attention_with_tail(q, lat, rope, lt, rt, w.softmax_scale)
+
+
+@pytest.mark.parametrize("kw,seq_lens,lens", [(dict(batch=3, seq_len=256), [256, 0, 112], [15, 9, 0]),
+                                              (dict(batch=2, seq_len=64, num_q_heads=16), [64, 32], [16, 3])])
+def test_mla_decode_with_tail_parity(kw, seq_lens, lens):
+    # latent and rope tail rows merged in the MLA combine; a sequence with no
+    # cached page, a full tail and an empty one
+    nq = kw.pop("num_q_heads", None)
+    w = W.WORKLOADS["mla"].scaled(**kw)
+    if nq:
+        w = dataclasses.replace(w, num_q_heads=nq)
+    run = QuantRun(w)
+    dec = DecodeRun(run, seq_lens=seq_lens)
+    o = dec.with_tail(W.tail_inputs(w, "k"), W.tail_rope_inputs(w), lens)
+    assert run.error_bits() == 0
+    assert np.all(np.isfinite(o))
+    for b in range(dec.batch):
+        err = attention_error(o[b], _mla_oracle_tail(dec, b))
+        assert err <= MLA_SHORT_ATTN_TOL, "seq %d: %g" % (b, err)
+
+
+@pytest.mark.parametrize("name,layer", [("gqa", 0), ("gqa", 1), ("g128", 1), ("mla", 1), ("kivi", 0), ("gqa16", 1)])
+def test_decode_with_fill_parity(name, layer):
+    # kvq_decode_attention_fill: sequences 0 and 2 have full tails in `layer`,
+    # quantised into spare pages by the call, then attention runs over the
+    # cache (with those pages) and the other sequences' partial tails
+    w = W.WORKLOADS[name].scaled(batch=3, seq_len=2 * W.WORKLOADS[name].tile_tokens, num_layers=2)
+    T = w.tile_tokens
+    run = QuantRun(w, num_pages=w.num_pages + 3)             # three spare pages past the appended ones
+    bt = np.zeros((w.batch, w.tiles_per_seq + 1), dtype=np.int32)
+    bt[:, :w.tiles_per_seq] = W.block_table(w)
+    fill = np.array([w.num_pages + 1, -1, w.num_pages + 2], dtype=np.int32)
+    seq = np.full(w.batch, w.seq_len, dtype=np.int32)
+    tl = np.array([0, 5, 0], dtype=np.int32)
+    for b in (0, 2):
+        bt[b, w.tiles_per_seq] = fill[b]
+        seq[b] += T
+    dec = DecodeRun(run, seq_lens=seq, block_table=bt)
+    kt = W.tail_inputs(w, "k")
+    vt = W.tail_rope_inputs(w) if w.mla else W.tail_inputs(w, "v")
+    dec.k_tail_bits, dec.v_tail_bits, dec.tl = kt, vt, tl
+    kvq.kvq_decode_attention_fill(run.cfg, run.cache.view, layer, dec.q, dec.bt_d, dec.maxp, dec.sl_d,
+                                  torch.from_numpy(kt.view(np.int16)).cuda(), torch.from_numpy(vt.view(np.int16)).cuda(),
+                                  torch.from_numpy(tl).cuda(), torch.from_numpy(fill).cuda(), dec.batch, dec.hq,
+                                  w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err)
+    torch.cuda.synchronize()
+    o = dec.out.cpu().numpy().astype(np.float64)
+    assert run.error_bits() == 0
+    from _parity import gpu_pages
+    # the filled pages hold the quantised tails (oracle on the same rows)
+    for b in (0, 2):
+        for which in (("k",) if w.mla else ("k", "v")):
+            bits = w.bits_k if which == "k" else w.bits_v
+            for h in range(w.num_kv_heads):
+                src = kt if which == "k" else vt
+                x = W.half_bits_to_f64(src[layer, b, :, h], w.in_dtype)[None]      # [1, T, d]
+                if which == "k" and w.k_per_channel:
+                    ora = O.quantize_tiles_per_channel(x, bits, w.block)
+                else:
+                    ora = O.quantize_tiles(x, bits, w.sinkhorn_iters, w.block, meta="f16" if w.meta_f16 else "f32")
+                compare_quantized(gpu_pages(run, which, layer, [fill[b]], h), ora, x, bits, w.sinkhorn_iters,
+                                  w.block, "seq %d %s H%d" % (b, which, h), check_rate=False)
+        if w.mla:   # the rope rows of the filled page
+            rope_all = run.cache["rope"].view(w.num_layers, -1, T, w.rope_dim)
+            got = rope_all[layer, int(fill[b])].cpu().view(torch.int16).numpy()
+            assert np.array_equal(got, vt[layer, b].view(np.int16))
+    # attention over the cache with the filled pages and the remaining tails
+    for b in range(w.batch):
+        if w.mla:   # 32..48-token contexts
+            err = attention_error(o[b], _mla_oracle_tail(dec, b, layer))
+            assert err <= MLA_SHORT_ATTN_TOL, "seq %d: %g" % (b, err)
+            continue
+        G = dec.hq // w.num_kv_heads
+        for h in range(w.num_kv_heads):
+            err = attention_error(o[b, h * G:(h + 1) * G], dec.oracle_tail(b, h, layer))
+            assert err <= ATTN_TOL, "seq %d kv-head %d: %g" % (b, h, err)
+
