@@ -356,9 +356,17 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
         } else if constexpr (BITS == 2) {
           *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = pack_crumbs(f);
         } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
+          // Codes 4k..4k+3 gathered into the bytes of one word; a multiply
+          // then compacts their low crumbs (to bits 18..25) and their high
+          // bits (to bits 21..24): the partial products are disjoint fields,
+          // so nothing carries into the result bits.
           uint32_t lo = 0, hi = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) lo |= (f[j] & 3u) << (2 * j), hi |= ((f[j] >> 2) & 1u) << j;
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t x = gather4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
+            lo |= ((((x & 0x03030303u) * 0x41041u) >> 18) & 0xFFu) << (8 * k);
+            hi |= (((((x >> 2) & 0x01010101u) * 0x204081u) >> 21) & 0xFu) << (4 * k);
+          }
           *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
           *reinterpret_cast<uint16_t*>(codes + kTile * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) =
               (uint16_t)hi;
