@@ -644,107 +644,101 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   }
 }
 
-// Merge the splits of one (sequence, kv-head), rotate back, normalise.  With
-// a tail, its tokens join as one more partial: their scores q . k and their
-// value sum are taken in the input basis (the rotation is orthogonal, so
-// q~ . k~ = q . k), and that sum is added after the splits' sum is rotated
+// Merge the splits of one (sequence, kv-head) for up to four of its query
+// heads, one warp each (blockIdx.y picks the group of four), rotate back and
+// normalise.  Lane l holds channels 4l .. 4l+3: the rotation's channel bits
+// 0 and 1 are in-register butterflies, bits 2..6 shuffles across the lanes.
+// With a tail, its tokens join as one more partial: their scores q . k and
+// their value sum are taken in the input basis (the rotation is orthogonal,
+// so q~ . k~ = q . k), and the sum is added after the splits' sum is rotated
 // back.
 constexpr int kMaxTail = 128;
-__global__ void __launch_bounds__(kD) combine_d128_kernel(DecodeParams p) {
-  __shared__ float buf[kD];
-  __shared__ float tq[8][kD];        // tail: the group's query heads
-  __shared__ float ts[8][kMaxTail];  // tail: scores (log2 units), then softmax numerators
-  __shared__ float tov[8][kD];       // tail: sum_t p_t v_t per head
-  __shared__ float tml[8][2];        // tail: (max, sum) per head
+__global__ void __launch_bounds__(128) combine_d128_kernel(DecodeParams p) {
   const int pair = blockIdx.x;
   const int b = pair / p.num_kv_heads, kvh = pair % p.num_kv_heads;
-  const int ch = threadIdx.x, warp = ch >> 5, lane = ch & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 4 + warp;  // query head of the kv-head's group
+  if (h >= p.group) return;             // (the kernel has no block-wide barrier)
   int L = 0;
   if (p.k_tail) {
     L = p.tail_lens[b];
     if (L < 0 || L > p.tail_tokens || L > kMaxTail) {
-      if (ch == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+      if (h == 0 && lane == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
       L = 0;
     }
   }
+  float tm = kNegBig, tl = 0.f, tv[4] = {0.f, 0.f, 0.f, 0.f};  // tail: running max, sum, value sums
   if (L > 0) {
-    const size_t row_stride = (size_t)p.num_kv_heads * kD;  // elements between tail tokens
-    const size_t base = (((size_t)p.layer * p.batch + b) * p.tail_tokens * p.num_kv_heads + kvh) * kD;
-    const uint16_t* kt = p.k_tail + base;
-    const uint16_t* vt = p.v_tail + base;
     auto elem = [&](uint16_t x) { return p.tail_f16 ? __half2float(__ushort_as_half(x)) : bf16_to_f(x); };
-    for (int h = 0; h < p.group; ++h)
-      tq[h][ch] = bf16_to_f(p.q[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch]);
-    __syncthreads();
-    for (int t = warp; t < L; t += kD / 32) {  // warp w: tokens w, w + 4, ...; lane: channels 4 lane .. +3
-      const uint2 raw = *reinterpret_cast<const uint2*>(kt + t * row_stride + 4 * lane);
-      const float k4[4] = {elem((uint16_t)(raw.x & 0xFFFF)), elem((uint16_t)(raw.x >> 16)),
-                           elem((uint16_t)(raw.y & 0xFFFF)), elem((uint16_t)(raw.y >> 16))};
-      for (int h = 0; h < p.group; ++h) {
-        float s = tq[h][4 * lane] * k4[0];
-        s = fmaf(tq[h][4 * lane + 1], k4[1], s);
-        s = fmaf(tq[h][4 * lane + 2], k4[2], s);
-        s = fmaf(tq[h][4 * lane + 3], k4[3], s);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) ts[h][t] = s * p.scale_log2;
-      }
-    }
-    __syncthreads();
-    for (int h = warp; h < p.group; h += kD / 32) {
-      float m = kNegBig;
-      for (int t = lane; t < L; t += 32) m = fmaxf(m, ts[h][t]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      float l = 0.f;
-      for (int t = lane; t < L; t += 32) {
-        const float e = ex2(ts[h][t] - m);
-        ts[h][t] = e;
-        l += e;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      if (lane == 0) tml[h][0] = m, tml[h][1] = l;
-    }
-    __syncthreads();
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint2 qw = *reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD +
+                                                     4 * lane);
+    const float q4[4] = {bf16_to_f((uint16_t)(qw.x & 0xFFFF)), bf16_to_f((uint16_t)(qw.x >> 16)),
+                         bf16_to_f((uint16_t)(qw.y & 0xFFFF)), bf16_to_f((uint16_t)(qw.y >> 16))};
+    const size_t row0 = ((size_t)p.layer * p.batch + b) * p.tail_tokens;
     for (int t = 0; t < L; ++t) {
-      const float v = elem(vt[t * row_stride + ch]);
+      const size_t off = ((row0 + t) * p.num_kv_heads + kvh) * kD + 4 * lane;
+      const uint2 kr = *reinterpret_cast<const uint2*>(p.k_tail + off);
+      const uint2 vr = *reinterpret_cast<const uint2*>(p.v_tail + off);
+      float s = q4[0] * elem((uint16_t)(kr.x & 0xFFFF));
+      s = fmaf(q4[1], elem((uint16_t)(kr.x >> 16)), s);
+      s = fmaf(q4[2], elem((uint16_t)(kr.y & 0xFFFF)), s);
+      s = fmaf(q4[3], elem((uint16_t)(kr.y >> 16)), s);
 #pragma unroll
-      for (int h = 0; h < 8; ++h)
-        if (h < p.group) acc[h] = fmaf(ts[h][t], v, acc[h]);
-    }
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      s *= p.scale_log2;
+      const float mn = fmaxf(tm, s), al = ex2(tm - mn), e = ex2(s - mn);
+      tm = mn;
+      tl = fmaf(tl, al, e);
+      const float v4[4] = {elem((uint16_t)(vr.x & 0xFFFF)), elem((uint16_t)(vr.x >> 16)),
+                           elem((uint16_t)(vr.y & 0xFFFF)), elem((uint16_t)(vr.y >> 16))};
 #pragma unroll
-    for (int h = 0; h < 8; ++h)
-      if (h < p.group) tov[h][ch] = acc[h];
+      for (int i = 0; i < 4; ++i) tv[i] = fmaf(tv[i], al, e * v4[i]);
+    }
   }
-  for (int h = 0; h < p.group; ++h) {
-    float mx = L > 0 ? tml[h][0] : kNegBig;
-    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)pair * p.splits + s) * 8 + h) * 2]);
-    float acc = 0.f, l = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const size_t i = ((size_t)pair * p.splits + s) * 8 + h;
-      const float f = ex2(p.part_ml[i * 2] - mx);
-      acc = fmaf(f, p.part_o[i * kD + ch], acc);
-      l = fmaf(f, p.part_ml[i * 2 + 1], l);
-    }
-    __syncthreads();
-    buf[ch] = acc;
-    __syncthreads();
-    for (int s = 1; s < p.hblock; s <<= 1) {  // H / sqrt(b) on each block of b = hblock channels
-      const float x = buf[ch & ~s], y = buf[ch | s];
-      __syncthreads();
-      buf[ch] = (ch & s) ? (x - y) : (x + y);
-      __syncthreads();
-    }
-    float o = buf[ch] * inv_sqrt_pow2(p.hblock);
-    if (L > 0) {
-      const float f = ex2(tml[h][0] - mx);
-      o = fmaf(f, tov[h][ch], o);
-      l = fmaf(f, tml[h][1], l);
-    }
-    p.out[((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + ch] = l > 0.f ? o / l : 0.f;
+  const float* pml = p.part_ml + ((size_t)pair * p.splits * 8 + h) * 2;       // split s at pml + 16 s
+  const float* po = p.part_o + ((size_t)pair * p.splits * 8 + h) * kD + 4 * lane;  // split s at po + 8 kD s
+  float mx = tm;
+  for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, pml[16 * s]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+  for (int s = 0; s < p.splits; ++s) {
+    const float f = ex2(pml[16 * s] - mx);
+    const float4 x = *reinterpret_cast<const float4*>(po + (size_t)8 * kD * s);
+    acc[0] = fmaf(f, x.x, acc[0]), acc[1] = fmaf(f, x.y, acc[1]);
+    acc[2] = fmaf(f, x.z, acc[2]), acc[3] = fmaf(f, x.w, acc[3]);
+    l = fmaf(f, pml[16 * s + 1], l);
   }
+  // H / sqrt(b) on each block of b = hblock channels
+  if (p.hblock > 1) {
+    const float a0 = acc[0] + acc[1], a1 = acc[0] - acc[1], a2 = acc[2] + acc[3], a3 = acc[2] - acc[3];
+    acc[0] = a0, acc[1] = a1, acc[2] = a2, acc[3] = a3;
+  }
+  if (p.hblock > 2) {
+    const float a0 = acc[0] + acc[2], a1 = acc[1] + acc[3], a2 = acc[0] - acc[2], a3 = acc[1] - acc[3];
+    acc[0] = a0, acc[1] = a1, acc[2] = a2, acc[3] = a3;
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    if (4 * off >= p.hblock) break;
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, acc[i], off);
+      acc[i] = upper ? (o - acc[i]) : (acc[i] + o);
+    }
+  }
+  const float sc = inv_sqrt_pow2(p.hblock);
+  float o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = acc[i] * sc;
+  if (L > 0) {
+    const float f = ex2(tm - mx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = fmaf(f, tv[i], o[i]);
+    l = fmaf(f, tl, l);
+  }
+  const float il = l > 0.f ? 1.f / l : 0.f;
+  *reinterpret_cast<float4*>(p.out + ((size_t)b * p.num_q_heads + (size_t)kvh * p.group + h) * kD + 4 * lane) =
+      make_float4(o[0] * il, o[1] * il, o[2] * il, o[3] * il);
 }
 
 template <int BK, int BV, int NH, int M, int KPC>
@@ -759,7 +753,7 @@ int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.splits, p.batch * p.num_kv_heads / NH);
   kern<<<grid, kDW * 32, smem, s>>>(p);
-  combine_d128_kernel<<<p.batch * p.num_kv_heads, kD, 0, s>>>(p);
+  combine_d128_kernel<<<dim3(p.batch * p.num_kv_heads, (p.group + 3) / 4), 128, 0, s>>>(p);
   return (int)cudaGetLastError();
 }
 
