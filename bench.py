@@ -89,13 +89,14 @@ def algorithmic_bytes(w):
 
 
 def traffic_from_profile(kernel_file: str, profile_name: str):
-    """Bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+    """DRAM bytes of one quantize-append call (the K and the V launch, or the latent launch) from a
+    committed ncu summary, if the kernel source is unchanged since the counters were taken."""
     path = os.path.join(ROOT, "profiles", profile_name)
     src = os.path.join(ROOT, "kv_cache_quantization_03_b200", "csrc", kernel_file)
     try:
         txt = open(path).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha256_16:\s*([0-9a-f]+)", txt)
+        m = re.search(r"traffic_bytes_per_call:\s*([0-9.eE+]+)\s+source_sha256_16:\s*([0-9a-f]+)", txt)
         if m and m.group(2) == sha:
             return float(m.group(1))
     except OSError:
@@ -472,7 +473,8 @@ def run_gpu(args, w):
         "config": config_dict(w, args),
         "roofline": {"kernel": qk, "bound": "hbm", "achieved": summ["quantize"]["gbs"], "peak": peak,
                      "unit": "GB/s", "frac": summ["quantize"]["gbs"] / peak, "peak_source": peak_kind,
-                     "traffic": traffic, "algorithmic_bytes": qb_bytes},
+                     "traffic": traffic, "algorithmic_bytes": qb_bytes,
+                     "per": "one quantize-append call (the K and the V launch; MLA: the latent launch)"},
         "quantize": summ["quantize"],
         "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         # quantize: one launch per quantised stream (latent, or K and V); decode:
