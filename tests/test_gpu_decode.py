@@ -180,7 +180,8 @@ def test_decode_tile_lengths(tile, group, bits):
     _check(dec, o)
 
 
-@pytest.mark.parametrize("block,group,bits", [(8, 4, (4, 4)), (16, 8, (3, 4)), (64, 1, (2, 2)), (32, 2, (8, 8))])
+@pytest.mark.parametrize("block,group,bits", [(1, 4, (4, 4)), (2, 8, (3, 4)), (4, 2, (4, 2)), (8, 4, (4, 4)),
+                                             (16, 8, (3, 4)), (64, 1, (2, 2)), (32, 2, (8, 8))])
 def test_decode_block_diagonal_rotation(block, group, bits):
     # query rotation and output un-rotation by blocks; one or two kv-heads per CTA
     w = dataclasses.replace(W.WORKLOADS["saw4"].scaled(batch=2, seq_len=512), hadamard_block=block,

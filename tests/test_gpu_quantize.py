@@ -61,10 +61,11 @@ def test_quantize_parity_iteration_counts(name, iters):
     _check_all(QuantRun(w))
 
 
-@pytest.mark.parametrize("block,iters,bits,tile", [(8, 0, (4, 4), 16), (16, 4, (3, 2), 16), (32, 0, (4, 4), 16),
+@pytest.mark.parametrize("block,iters,bits,tile", [(1, 4, (4, 4), 16), (2, 0, (4, 4), 16), (4, 4, (3, 2), 16),
+                                                    (8, 0, (4, 4), 16), (16, 4, (3, 2), 16), (32, 0, (4, 4), 16),
                                                     (64, 6, (2, 8), 16), (32, 4, (4, 2), 128)])
 def test_quantize_parity_block_diagonal_rotation(block, iters, bits, tile):
-    # SAW-INT4-style ablation: blocks of 8..64 channels, with and without the normalisation
+    # SAW-INT4-style ablation: blocks of 1..64 channels (1: no rotation), with and without the normalisation
     import dataclasses
     w = dataclasses.replace(W.WORKLOADS["saw4"].scaled(batch=1, seq_len=512), hadamard_block=block,
                             sinkhorn_iters=iters, bits_k=bits[0], bits_v=bits[1], tile_tokens=tile)
