@@ -101,6 +101,19 @@ __device__ __forceinline__ uint32_t h2_field(uint32_t word, uint32_t mask) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ uint32_t h2_codes(uint32_t masked) { return h2_field<0>(masked, 0xFFFFFFFFu); }
+// The same conversion for a word whose two fields (at bit `shift` of each
+// half) are already masked and OR-ed into 0x6400 (shift constant after
+// unrolling).
+__device__ __forceinline__ uint32_t h2_scaled(uint32_t v, int shift) {
+  __half2 h = *reinterpret_cast<__half2*>(&v);
+  if (shift == 0) {
+    h = __hsub2(h, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  } else {
+    const float sc = 1.0f / (float)(1 << shift);
+    h = __hfma2(h, __float2half2_rn(sc), __float2half2_rn(-1024.0f * sc));
+  }
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
 // Four code pairs of one word of 4-bit codes: (nibble e, nibble e+4), e = 0..3.
 __device__ __forceinline__ void nib_pairs(uint32_t w, uint32_t* out) {
@@ -173,16 +186,21 @@ __device__ __forceinline__ void key_pairs(const uint8_t* codes, int row, int t, 
     const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r + 4 * ((t + 1) & 1));
     uint32_t hw = *reinterpret_cast<const uint32_t*>(codes + kT * 32 + row * 16 + 4 * t);
     hw = (t & 1) ? __funnelshift_r(hw, hw, 16) : hw;
-    uint32_t lo[16];
-    crumb_pairs(w0, lo);
-    crumb_pairs(w1, lo + 8);
     const uint32_t hs[2] = {__byte_perm(hw, 0u, 0x4140u), __byte_perm(hw, 0u, 0x4342u)};
-    const __half2 four = __halves2half2(__ushort_as_half(0x4400), __ushort_as_half(0x4400));
+    // Pair pi = channels (pi, pi + 8) of word pi >> 3: its low crumbs sit at
+    // bit s = 2 (pi & 3) of each half (of the word, or of the word >> 8 for
+    // pi & 4), its high bits at bit pi & 7 of each half of hs[pi >> 3].  The
+    // high bits are moved next to the crumbs (bit s + 2), so one field of
+    // 3-bit codes times 2^s goes through a single f16 conversion.
+    const uint32_t w8[2] = {w0 >> 8, w1 >> 8};
 #pragma unroll
     for (int pi = 0; pi < 16; ++pi) {
-      uint32_t hi = h2_codes((hs[pi >> 3] >> (pi & 7)) & 0x00010001u);
-      __half2 r = __hfma2(*reinterpret_cast<__half2*>(&hi), four, *reinterpret_cast<__half2*>(&lo[pi]));
-      pr[pi] = *reinterpret_cast<uint32_t*>(&r);
+      const int s = 2 * (pi & 3), sh = s + 2 - (pi & 7);
+      const uint32_t v = (pi & 4) ? w8[pi >> 3] : ((pi >> 3) ? w1 : w0);
+      const uint32_t h = hs[pi >> 3];
+      const uint32_t hb = sh >= 0 ? (h << sh) : (h >> -sh);
+      const uint32_t f = (v & (0x00030003u << s)) | (hb & (0x00040004u << s)) | 0x64006400u;
+      pr[pi] = h2_scaled(f, s);
     }
   }
 }
