@@ -88,6 +88,22 @@ def algorithmic_bytes(w):
     return q_bytes, dec_bytes
 
 
+def fill_bytes(w, fill_tiles, tail_tokens):
+    """Bytes a decode step with quantise-on-fill moves beyond the plain
+    decode: the filled tails (input rows in, cache rows out) and the
+    remaining tails' rows read by the attention."""
+    mb = 2 if w.meta_f16 else 4
+    d, T, H = w.head_dim, w.tile_tokens, w.num_kv_heads
+    if w.mla:
+        lat_row = d * w.bits_k / 8 + 2 * mb + d * mb / T
+        rope = w.rope_dim * 2
+        return fill_tiles * T * (d * 2 + rope + lat_row + rope) + tail_tokens * (d * 2 + rope)
+    def cache_row(bits):
+        return d * bits / 8 + 2 * mb + d * mb / T
+    k_row = (d * w.bits_k / 8 + d * 2 * mb / T) if w.k_per_channel else cache_row(w.bits_k)
+    return fill_tiles * T * H * (2 * d * 2 + k_row + cache_row(w.bits_v)) + tail_tokens * H * 2 * d * 2
+
+
 def traffic_from_profile(kernel_file: str, profile_name: str):
     """DRAM bytes of one quantize-append call (the K and the V launch, or the latent launch) from a
     committed ncu summary, if the kernel source is unchanged since the counters were taken."""
@@ -409,12 +425,66 @@ def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
         r["e2e_s"] = e0.elapsed_time(e1) / 1e3 / Ke
         r["h2d"] = sum(host[k].numel() * host[k].element_size() for k in host)
         r["d2h"] = out.numel() * out.element_size()
+    if not q_only:
+        r.update(measure_fill(w, ws, cfg, cache, dev, out, work, ws_bytes, err, stream, steps))
     st, bits = kvq.kvq_read_error(err, s_ptr)
     if st != kvq.KVQ_OK or bits:
         raise RuntimeError("device error word %#x" % bits)
     del cache, dev, host, work, out
     torch.cuda.empty_cache()
     return r
+
+
+def fill_state(ws):
+    """A decode step of the serving reading with unquantised tails: every
+    sequence b with b % 16 == 0 has just filled its tail (quantised into the
+    last page of its block table row, which the step's decode then reads);
+    the others keep a tail of tail_lens[b] < T tokens.  Returns (tail_lens,
+    fill_page) as int32 arrays."""
+    import numpy as np
+
+    from kv_cache_quantization_03_b200 import workloads as W
+
+    tl = W.tail_lens(ws).copy()
+    bt = W.block_table(ws)
+    fill = np.full(ws.batch, -1, dtype=np.int32)
+    for b in range(0, ws.batch, 16):
+        tl[b] = 0
+        fill[b] = bt[b, ws.tiles_per_seq - 1]
+    return tl, fill
+
+
+def measure_fill(w, ws, cfg, cache, dev, out, work, ws_bytes, err, stream, steps):
+    """Times kvq_decode_attention_fill (decode-time append): the filled tails
+    are quantised into their pages and attention runs over the cached pages
+    plus the remaining tails, in one call."""
+    import numpy as np
+    import torch
+
+    from kv_cache_quantization_03_b200 import kvq, workloads as W
+
+    tl, fill = fill_state(ws)
+    kt = torch.from_numpy(W.tail_inputs(ws, "k").view(np.int16)).cuda()
+    vt = torch.from_numpy((W.tail_rope_inputs(ws) if w.mla else W.tail_inputs(ws, "v")).view(np.int16)).cuda()
+    tl_d, fill_d = torch.from_numpy(tl).cuda(), torch.from_numpy(fill).cuda()
+    s_ptr = stream.cuda_stream
+
+    def step():
+        kvq.kvq_decode_attention_fill(cfg, cache.view, 0, dev["q"], dev["bt"], w.tiles_per_seq, dev["sl"], kt, vt,
+                                      tl_d, fill_d, w.batch, w.num_q_heads, w.softmax_scale, out, work, ws_bytes,
+                                      err, s_ptr)
+
+    for _ in range(3):
+        step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"t_f": e0.elapsed_time(e1) / 1e3 / steps, "fill_tiles": int((fill >= 0).sum()),
+            "tail_tokens": int(tl.sum())}
 
 
 def summarize(w, r, peak, world=1):
@@ -431,6 +501,12 @@ def summarize(w, r, peak, world=1):
         d_gbs = db_bytes / t_d / 1e9
         res["decode_attn"] = {"kernel": dk, "us": 1e6 * t_d, "gbs": d_gbs, "frac_of_measured": d_gbs / peak,
                               "frac_of_8tbs": d_gbs / 8000.0, "algorithmic_bytes": db_bytes}
+        if "t_f" in r:  # decode-time append: filled tails quantised, then decode over cache + tails
+            fb = fill_bytes(w, r["fill_tiles"], r["tail_tokens"])
+            res["decode_fill"] = {"us": 1e6 * r["t_f"], "filled_pages": r["fill_tiles"],
+                                  "tail_tokens": r["tail_tokens"], "algorithmic_bytes": db_bytes + fb,
+                                  "gbs": (db_bytes + fb) / r["t_f"] / 1e9,
+                                  "frac_of_measured": (db_bytes + fb) / r["t_f"] / 1e9 / peak}
         if w.mla:   # 128 heads share every latent: a dense contraction, tensor-bound
             flops = 2.0 * w.batch * w.seq_len * w.num_q_heads * (w.head_dim + w.rope_dim + w.head_dim)
             tf = flops / t_d / 1e12
@@ -452,8 +528,11 @@ def run_gpu(args, w):
                                 device_id=torch.device("cuda", local))
     K = args.steps
     r = measure(w, K, args.warmup, rank, world, local, e2e=True, clocks=True)
-    elapsed, e2e_s, t_q, t_d = max_over_ranks([r["elapsed"], r["e2e_s"], r["t_q"], r["t_d"]], world, device="cuda")
+    elapsed, e2e_s, t_q, t_d, t_f = max_over_ranks([r["elapsed"], r["e2e_s"], r["t_q"], r["t_d"], r.get("t_f", 0.0)],
+                                                   world, device="cuda")
     r.update({"elapsed": elapsed, "e2e_s": e2e_s, "t_q": t_q, "t_d": t_d, "steps": K})
+    if "t_f" in r:
+        r["t_f"] = t_f
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -484,6 +563,7 @@ def run_gpu(args, w):
     }
     if "decode_attn" in summ:
         line["decode_attn"] = summ["decode_attn"]
+        line["decode_fill"] = summ["decode_fill"]
         if w.mla and t_d >= t_q:
             d = summ["decode_attn"]
             line["roofline"] = {"kernel": dk, "bound": "tensor", "achieved": d["tflops"], "peak": d["tensor_peak"],

@@ -693,24 +693,52 @@ __global__ void __launch_bounds__(128) combine_d128_kernel(DecodeParams p) {
     const float q4[4] = {bf16_to_f((uint16_t)(qw.x & 0xFFFF)), bf16_to_f((uint16_t)(qw.x >> 16)),
                          bf16_to_f((uint16_t)(qw.y & 0xFFFF)), bf16_to_f((uint16_t)(qw.y >> 16))};
     const size_t row0 = ((size_t)p.layer * p.batch + b) * p.tail_tokens;
-    for (int t = 0; t < L; ++t) {
-      const size_t off = ((row0 + t) * p.num_kv_heads + kvh) * kD + 4 * lane;
-      const uint2 kr = *reinterpret_cast<const uint2*>(p.k_tail + off);
-      const uint2 vr = *reinterpret_cast<const uint2*>(p.v_tail + off);
-      float s = q4[0] * elem((uint16_t)(kr.x & 0xFFFF));
-      s = fmaf(q4[1], elem((uint16_t)(kr.x >> 16)), s);
-      s = fmaf(q4[2], elem((uint16_t)(kr.y & 0xFFFF)), s);
-      s = fmaf(q4[3], elem((uint16_t)(kr.y >> 16)), s);
+    // Eight tail tokens at a time: their rows are loaded together and their
+    // eight dot products reduced side by side, so the load and shuffle
+    // latencies are paid once per group.  Rows past L are not read (the
+    // last valid row stands in) and take no weight.
+    constexpr int kG = 8;
+    for (int t0 = 0; t0 < L; t0 += kG) {
+      uint2 kr[kG], vr[kG];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      s *= p.scale_log2;
-      const float mn = fmaxf(tm, s), al = ex2(tm - mn), e = ex2(s - mn);
+      for (int j = 0; j < kG; ++j) {
+        const int t = min(t0 + j, L - 1);
+        const size_t off = ((row0 + t) * p.num_kv_heads + kvh) * kD + 4 * lane;
+        kr[j] = *reinterpret_cast<const uint2*>(p.k_tail + off);
+        vr[j] = *reinterpret_cast<const uint2*>(p.v_tail + off);
+      }
+      float s[kG];
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        float x = q4[0] * elem((uint16_t)(kr[j].x & 0xFFFF));
+        x = fmaf(q4[1], elem((uint16_t)(kr[j].x >> 16)), x);
+        x = fmaf(q4[2], elem((uint16_t)(kr[j].y & 0xFFFF)), x);
+        s[j] = fmaf(q4[3], elem((uint16_t)(kr[j].y >> 16)), x);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int j = 0; j < kG; ++j) s[j] += __shfl_xor_sync(0xffffffffu, s[j], o);
+      float cm = kNegBig;
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        s[j] = t0 + j < L ? s[j] * p.scale_log2 : kNegBig;
+        cm = fmaxf(cm, s[j]);
+      }
+      const float mn = fmaxf(tm, cm), al = ex2(tm - mn);
       tm = mn;
-      tl = fmaf(tl, al, e);
-      const float v4[4] = {elem((uint16_t)(vr.x & 0xFFFF)), elem((uint16_t)(vr.x >> 16)),
-                           elem((uint16_t)(vr.y & 0xFFFF)), elem((uint16_t)(vr.y >> 16))};
+      tl *= al;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tv[i] = fmaf(tv[i], al, e * v4[i]);
+      for (int i = 0; i < 4; ++i) tv[i] *= al;
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        const float e = t0 + j < L ? ex2(s[j] - mn) : 0.f;
+        tl += e;
+        tv[0] = fmaf(e, elem((uint16_t)(vr[j].x & 0xFFFF)), tv[0]);
+        tv[1] = fmaf(e, elem((uint16_t)(vr[j].x >> 16)), tv[1]);
+        tv[2] = fmaf(e, elem((uint16_t)(vr[j].y & 0xFFFF)), tv[2]);
+        tv[3] = fmaf(e, elem((uint16_t)(vr[j].y >> 16)), tv[3]);
+      }
     }
   }
   const float* pml = p.part_ml + ((size_t)pair * p.splits * 8 + h) * 2;       // split s at pml + 16 s
