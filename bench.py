@@ -315,7 +315,7 @@ def max_over_ranks(values, world: int, device=None):
 
 # --------------------------------------------------------------------------- GPU leg
 QUANTIZE_ONLY = ("prefill",)       # workloads whose step is quantise-append alone
-EXTRA_WORKLOADS = ("gqa", "gqa16", "prefill", "mla", "g128", "saw4", "kivi", "rt1k")
+EXTRA_WORKLOADS = ("gqa", "gqa16", "prefill", "mla", "g128", "saw4", "hadonly", "kivi", "rt1k")
 
 
 def kernel_names(w):

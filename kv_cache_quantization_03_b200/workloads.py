@@ -121,6 +121,9 @@ WORKLOADS: Dict[str, Workload] = {
                                  "no normalisation rounds, gqa shapes"),
     "gqa16": Workload("gqa16", 32, 8192, 8, 32, 128, 4, 4, 4, 2, meta_f16=True,
                       description="gqa with the compact layout: a, z, c as IEEE half (same inputs as gqa)"),
+    "hadonly": Workload("hadonly", 32, 8192, 8, 32, 128, 4, 4, 0, 2,
+                        description="ablation: full Hadamard rotation + per-token 4-bit RTN, no normalisation "
+                                    "(same inputs as gqa)"),
     "kivi": Workload("kivi", 32, 8192, 8, 32, 128, 2, 2, 0, 2, hadamard_block=1, k_per_channel=True,
                      description="ablation: KIVI-style axes, 2-bit keys per channel and values per token, "
                                  "no rotation, no normalisation (same inputs as gqa)"),
@@ -159,7 +162,7 @@ def outlier_channels(w: Workload, layer: int, head: int, which: str) -> np.ndarr
         return np.array([3, 17, 64, 101])
     if w.mla:
         n = round(0.01 * w.head_dim)
-    elif _base_name(w) in ("gqa", "g128", "saw4", "gqa16", "kivi"):
+    elif _base_name(w) in ("gqa", "g128", "saw4", "gqa16", "kivi", "hadonly"):
         n = round(0.02 * w.head_dim)
     else:
         return np.zeros(0, dtype=np.int64)
@@ -197,8 +200,9 @@ def kv_inputs(w: Workload, which: str, tokens: Optional[slice] = None) -> np.nda
         r = _rng(w.seed, 10 * kind)
         scale = np.exp(r.uniform(math.log(0.1), math.log(10.0), size=(L, 1, H, d))).astype(np.float32)
     outl = None
-    if base in ("rt1k", "gqa", "mla", "g128", "saw4", "gqa16", "kivi"):
-        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0, "g128": 15.0, "saw4": 15.0, "gqa16": 15.0, "kivi": 15.0}[base]
+    if base in ("rt1k", "gqa", "mla", "g128", "saw4", "gqa16", "kivi", "hadonly"):
+        factor = {"rt1k": 20.0, "gqa": 15.0, "mla": 25.0, "g128": 15.0, "saw4": 15.0, "gqa16": 15.0, "kivi": 15.0,
+                  "hadonly": 15.0}[base]
         outl = np.ones((L, 1, H, d), dtype=np.float32)
         for layer in range(L):
             for h in range(H):

@@ -39,6 +39,7 @@ def _check(dec: DecodeRun, o: np.ndarray, pairs=None):
     ("prefill", dict(seq_len=1024, num_layers=2)),   # per-channel scales over two decades
     ("gqa16", dict(batch=3, seq_len=512)),            # a, z, c as IEEE half
     ("kivi", dict(batch=3, seq_len=512)),             # keys per channel, no rotation
+    ("hadonly", dict(batch=3, seq_len=512)),          # full rotation, no normalisation
 ])
 def test_decode_parity_small(name, kw):
     w = W.WORKLOADS[name]

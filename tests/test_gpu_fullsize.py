@@ -12,7 +12,8 @@ pytestmark = pytest.mark.gpu
 from _parity import ATTN_TOL, CODE_FLIP_RATE, DecodeRun, QuantRun, attention_error, check_tiles  # noqa: E402
 
 
-@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128", "saw4", "gqa16", "kivi"])
+@pytest.mark.parametrize("name", ["rt1k", "gqa", "long", "prefill", "mla", "g128", "saw4", "hadonly", "gqa16",
+                                  "kivi"])
 def test_fullsize_sampled_parity(name):
     w = W.WORKLOADS[name]
     run = QuantRun(w)

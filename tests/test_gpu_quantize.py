@@ -18,6 +18,7 @@ SMALL = {
     "mla": dict(batch=2, seq_len=256),
     "g128": dict(batch=2, seq_len=512),
     "saw4": dict(batch=2, seq_len=512),
+    "hadonly": dict(batch=2, seq_len=512),
     "kivi": dict(batch=2, seq_len=512),
 }
 
@@ -262,7 +263,7 @@ def test_quantize_deterministic():
         assert torch.equal(run.cache.arrays[n], t), n
 
 
-@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4", "gqa16", "kivi"])
+@pytest.mark.parametrize("name", ["long", "mla", "g128", "saw4", "hadonly", "gqa16", "kivi"])
 def test_dequantize_matches_oracle_on_stored_codes(name):
     from kv_cache_quantization_03_b200 import kvq
     w = W.WORKLOADS[name].scaled(batch=1, seq_len=256)
