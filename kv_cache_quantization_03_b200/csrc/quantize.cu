@@ -173,29 +173,10 @@ struct QuantLaunch {
 
 // Shared memory of one tile whose 512 channels are split over four warps.
 struct TileShare {
-  float2 x[4][32][32];   // per block, per register pair, per lane: values for the H_4 combination
   float row[2][4][kT];   // row partial sums, double-buffered by round parity
   float2 mm[4][kT];      // per block and token: (min, max)
   float cmax[4];         // per block: largest column factor
 };
-
-template <int D>
-__device__ __forceinline__ void load_tile(uint32_t (&L)[2][4][4], const QuantLaunch& p, uint32_t tile, int blk, int g,
-                                          int t, int32_t& page) {
-  const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
-  const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
-  page = __ldg(p.dst_page + tt);
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {  // (16-token tiles only)
-    const uint16_t* row = p.src + (((size_t)layer * p.n_tok + (size_t)tt * kT + 8 * h + g) * p.num_heads + head) * D +
-                          kBlk * blk + 8 * t;
-#pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      const uint4 v = ldg_nc_v4(row + 32 * l);
-      L[h][l][0] = v.x, L[h][l][1] = v.y, L[h][l][2] = v.z, L[h][l][3] = v.w;
-    }
-  }
-}
 
 // Channel bits 0..6 of the 128-channel block: bits 3..6 on the tensor cores
 // (16 MMAs), bits 0..2 as three butterfly stages on fp32 pairs (only the
@@ -230,20 +211,21 @@ __device__ __forceinline__ void hadamard128(const uint32_t (&L)[2][4][4], const 
         }
 }
 
-// Raw 16 tokens x 128 channels (token slice wt of a tile of TW slices)
-// staged per lane in shared memory by cp.async: slot [h * 4 + l][lane] holds
-// what load_tile keeps in L[h][l].
-template <int TW>
-__device__ __forceinline__ void stage_tile(uint4 (*dst)[32], const QuantLaunch& p, uint32_t tile, int wt, int g, int t,
-                                           int lane, int32_t& page) {
+// Raw 16 tokens x 128 channels (token slice wt of a tile of TW slices; at
+// D = 512 channel block blk of the latent) staged per lane in shared memory
+// by cp.async: slot [h * 4 + l][lane] holds tokens 8h + g, channels
+// 128 blk + 8t + 32 l .. + 7, which read_staged puts in L[h][l].
+template <int TW, int D>
+__device__ __forceinline__ void stage_tile(uint4 (*dst)[32], const QuantLaunch& p, uint32_t tile, int wt, int blk, int g,
+                                           int t, int lane, int32_t& page) {
   const uint32_t r1 = fdiv(tile, p.div_h), head = tile - r1 * p.div_h.d;
   const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
   page = __ldg(p.dst_page + tt);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint16_t* row =
-        p.src + (((size_t)layer * p.n_tok + (size_t)tt * (kT * TW) + kT * wt + 8 * h + g) * p.num_heads + head) * kBlk +
-        8 * t;
+        p.src + (((size_t)layer * p.n_tok + (size_t)tt * (kT * TW) + kT * wt + 8 * h + g) * p.num_heads + head) * D +
+        kBlk * blk + 8 * t;
 #pragma unroll
     for (int l = 0; l < 4; ++l)
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&dst[h * 4 + l][lane])), "l"(row + 32 * l)
@@ -278,7 +260,7 @@ constexpr size_t stage_bytes() { return (size_t)cta_warps<TW>() * 2 * 8 * 32 * s
 // stream asks for them; the standard instantiation (AXES = 0) carries
 // neither.
 template <bool F16, int BITS, int D, int TW, int AXES>
-__global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_warps<TW>() : 3))
+__global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     quantize_kernel(QuantLaunch p) {
   static_assert(TW == 1 || D == kBlk, "tiles longer than 16 tokens need head_dim 128");
   static_assert(AXES == 0 || (D == kBlk && TW == 1), "the ablation instantiation is for 16 x 128 tiles");
@@ -287,17 +269,16 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
   constexpr int kTile = kT * TW;  // tokens per tile
   constexpr int TPC = kCW / (W * TW);  // tiles per CTA
   // The rotated tile waits out the rounds in tensor memory (64 columns of the
-  // warp's lane quarter).  At head_dim 128 the raw tiles are also staged in
-  // shared memory by cp.async (the next one while the current one is
-  // processed), which keeps that kernel at 128 registers (four CTAs per SM).
-  constexpr bool kStage = (W == 1);
+  // warp's lane quarter).  The raw tiles are staged in shared memory by
+  // cp.async (the next one while the current one is processed), which keeps
+  // the kernel at 128 registers or fewer (four CTAs per SM).
   constexpr int kLogDT = log2_dt<D, TW>();
   constexpr int kTmemCols = 64 * (kCW / 4);  // 64 columns per warp, four lane quarters
   __shared__ WarpScratch scratch[kCW];
   __shared__ TileShare share[W > 1 ? 1 : 0 + 1];
   __shared__ float4 colw[TW > 1 ? TPC : 1][2][TW][32];  // column partials of the token slices, by round parity
   extern __shared__ uint4 dyn_smem[];
-  uint4(*staged)[2][8][32] = reinterpret_cast<uint4(*)[2][8][32]>(dyn_smem);  // [kCW] when kStage
+  uint4(*staged)[2][8][32] = reinterpret_cast<uint4(*)[2][8][32]>(dyn_smem);  // [kCW]
   __shared__ uint32_t tmem_slot;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int warp = threadIdx.x >> 5, blk = warp % W, wt = (warp / W) % TW, slot_id = warp / (W * TW);
@@ -377,25 +358,17 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
   uint32_t L[2][4][4];
   int32_t page = 0;
   uint32_t rounds = 0;  // rounds done by this warp (parity of the column-partial buffer)
-  if constexpr (kStage) {
-    if (tile < p.total) stage_tile<TW>(staged[warp][0], p, tile, wt, g, t, lane, page);
-  } else {
-    if (tile < p.total) load_tile<D>(L, p, tile, blk, g, t, page);
-  }
+  if (tile < p.total) stage_tile<TW, D>(staged[warp][0], p, tile, wt, blk, g, t, lane, page);
   for (int buf = 0; tile < p.total; tile += stride, buf ^= 1) {
     f2 P[2][2][8];  // [h][m3][b]: tokens (8h+2t, 8h+2t+1) at channel 16g + 8m3 + b of the block
     const int32_t cur_page = page;
-    if constexpr (kStage) {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");  // this lane's copies of the current tile
-      read_staged(staged[warp][buf], lane, L);
-      if (tile + stride < p.total) stage_tile<TW>(staged[warp][buf ^ 1], p, tile + stride, wt, g, t, lane, page);
-    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");  // this lane's copies of the current tile
+    read_staged(staged[warp][buf], lane, L);
+    if (tile + stride < p.total) stage_tile<TW, D>(staged[warp][buf ^ 1], p, tile + stride, wt, blk, g, t, lane, page);
     hadamard128<F16, AXES == 1>(L, afrag, P, D == kBlk ? p.hblock : kBlk);
     const uint32_t cur = tile;
     const uint32_t r1 = fdiv(cur, p.div_h), head = cur - r1 * p.div_h.d;
     const uint32_t layer = fdiv(r1, p.div_ntt), tt = r1 - layer * p.div_ntt.d;
-    if constexpr (!kStage)
-      if (tile + stride < p.total) load_tile<D>(L, p, tile + stride, blk, g, t, page);
     if (cur_page < 0 || cur_page >= p.num_pages) {  // same decision in every warp of the tile
       // page -1: the caller skips this tile (a sequence whose tail is not full)
       if (cur_page != -1 && lane == 0 && blk == 0 && wt == 0) set_error(p.err, KVQ_DEVERR_BAD_PAGE);
@@ -409,19 +382,29 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, (D == 128 ? 16 / cta_war
       for (int i = lane * 8; i < kT * rd; i += 32 * 8)
         *reinterpret_cast<uint4*>(rdst + i) = *reinterpret_cast<const uint4*>(rs + i);
     }
-    if constexpr (W > 1) {  // channel bits 7, 8: H_4 across the four blocks of the tile
+    if constexpr (W > 1) {
+      // Channel bits 7, 8: H_4 across the four blocks of the tile, one token
+      // half at a time, through the tile warps' staging buffers of the
+      // current tile (the raw tile is in registers by now, and the next
+      // tile's copies go to the other buffer).
+      const int w0 = warp - blk;  // the tile's first warp
 #pragma unroll
-      for (int i = 0; i < 32; ++i) sh.x[blk][i][lane] = P[i >> 4][(i >> 3) & 1][i & 7];
-      __syncthreads();
+      for (int h = 0; h < 2; ++h) {
+        f2(*own)[32] = reinterpret_cast<f2(*)[32]>(staged[warp][buf]);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        f2 acc = sh.x[0][i][lane];
+        for (int i = 0; i < 16; ++i) own[i][lane] = P[h][i >> 3][i & 7];
+        __syncthreads();
 #pragma unroll
-        for (int k = 1; k < W; ++k) {
-          const f2 y = sh.x[k][i][lane];
-          acc = (__popc(blk & k) & 1) ? sub2(acc, y) : add2(acc, y);
+        for (int i = 0; i < 16; ++i) {
+          f2 acc = reinterpret_cast<const f2(*)[32]>(staged[w0][buf])[i][lane];
+#pragma unroll
+          for (int k = 1; k < W; ++k) {
+            const f2 y = reinterpret_cast<const f2(*)[32]>(staged[w0 + k][buf])[i][lane];
+            acc = (__popc(blk & k) & 1) ? sub2(acc, y) : add2(acc, y);
+          }
+          P[h][i >> 3][i & 7] = acc;
         }
-        P[i >> 4][(i >> 3) & 1][i & 7] = acc;
+        __syncthreads();  // every warp has read this half before the next one is written
       }
     }
     if constexpr (AXES == 1 && BITS != 3) {
@@ -772,9 +755,9 @@ FastDiv make_div(uint32_t d) {
 template <bool F16, int BITS, int D, int TW, int AXES>
 void launch_one(const QuantLaunch& q, int sms, cudaStream_t s) {
   constexpr int kCW = cta_warps<TW>(), tpc = kCW / ((D / kBlk) * TW);
-  constexpr size_t dyn = D == kBlk ? stage_bytes<TW>() : 0;  // raw-tile staging at head_dim 128
+  constexpr size_t dyn = stage_bytes<TW>();  // raw-tile staging
   const int64_t need = (q.total + tpc - 1) / tpc;
-  const int64_t cap = (int64_t)sms * (D == kBlk ? 16 / kCW : 3);  // resident CTAs per SM
+  const int64_t cap = (int64_t)sms * (16 / kCW);  // resident CTAs per SM
   const int grid = (int)(need < cap ? need : cap);
   auto kern = quantize_kernel<F16, BITS, D, TW, AXES>;
   // static + dynamic shared memory may pass 48 KB, which needs the opt-in
