@@ -311,3 +311,23 @@ class DecodeRun:
         kt = gpu_pages(self.run, "k", 0, pages, kvh)
         vt = gpu_pages(self.run, "v", 0, pages, kvh)
         return O.decode_attention(q, kt, vt, w.softmax_scale, block=w.block)
+
+
+def mla_oracle_tail(dec: "DecodeRun", b: int, layer=0) -> np.ndarray:
+    """Oracle MLA attention of sequence b over its cached pages (the GPU's
+    stored latents and rope rows) and its unquantised tail (dec.tl[b] rows of
+    dec.k_tail_bits / dec.v_tail_bits)."""
+    w = dec.run.w
+    n = int(dec.sl[b]) // w.tile_tokens
+    L = int(dec.tl[b])
+    q = W.half_bits_to_f64(dec.q_bits[b], "bf16")
+    lt = W.half_bits_to_f64(dec.k_tail_bits[layer, b, :L].reshape(L, w.head_dim), w.in_dtype)
+    rt = W.half_bits_to_f64(dec.v_tail_bits[layer, b, :L], "bf16")
+    lat = rope = None
+    if n:
+        pages = dec.bt[b, :n]
+        lat = gpu_pages(dec.run, "k", layer, pages, 0)
+        rope_all = dec.run.cache["rope"].view(w.num_layers, -1, w.tile_tokens, w.rope_dim)
+        pg = torch.as_tensor(np.asarray(pages, dtype=np.int64)).cuda()
+        rope = rope_all[layer, pg].float().cpu().numpy().astype(np.float64).reshape(-1, w.rope_dim)
+    return O.mla_decode_attention_with_tail(q, lat, rope, lt, rt, w.softmax_scale)

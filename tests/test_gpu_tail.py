@@ -14,7 +14,7 @@ from oracle import kvarn_oracle as O
 pytestmark = pytest.mark.gpu
 
 from _parity import (ATTN_TOL, CODE_FLIP_RATE, MLA_SHORT_ATTN_TOL, DecodeRun, QuantRun,  # noqa: E402
-                     attention_error, compare_quantized)
+                     attention_error, compare_quantized, mla_oracle_tail)
 
 
 def _check_tail(dec: DecodeRun, o: np.ndarray, layer=0, lens=None):
@@ -150,24 +150,6 @@ def test_tail_entry_rejections():
     assert run.error_bits() == 0                               # nothing was launched
 
 
-def _mla_oracle_tail(dec: DecodeRun, b: int, layer=0):
-    w = dec.run.w
-    n = int(dec.sl[b]) // w.tile_tokens
-    L = int(dec.tl[b])
-    q = W.half_bits_to_f64(dec.q_bits[b], "bf16")
-    lt = W.half_bits_to_f64(dec.k_tail_bits[layer, b, :L].reshape(L, w.head_dim), w.in_dtype)
-    rt = W.half_bits_to_f64(dec.v_tail_bits[layer, b, :L], "bf16")
-    lat = rope = None
-    if n:
-        from _parity import gpu_pages
-        pages = dec.bt[b, :n]
-        lat = gpu_pages(dec.run, "k", layer, pages, 0)
-        rope_all = dec.run.cache["rope"].view(w.num_layers, -1, w.tile_tokens, w.rope_dim)
-        pg = torch.as_tensor(np.asarray(pages, dtype=np.int64)).cuda()
-        rope = rope_all[layer, pg].float().cpu().numpy().astype(np.float64).reshape(-1, w.rope_dim)
-    return O.mla_decode_attention_with_tail(q, lat, rope, lt, rt, w.softmax_scale)
-
-
 @pytest.mark.parametrize("kw,seq_lens,lens", [(dict(batch=3, seq_len=256), [256, 0, 112], [15, 9, 0]),
                                               (dict(batch=2, seq_len=64, num_q_heads=16), [64, 32], [16, 3])])
 def test_mla_decode_with_tail_parity(kw, seq_lens, lens):
@@ -183,7 +165,7 @@ def test_mla_decode_with_tail_parity(kw, seq_lens, lens):
     assert run.error_bits() == 0
     assert np.all(np.isfinite(o))
     for b in range(dec.batch):
-        err = attention_error(o[b], _mla_oracle_tail(dec, b))
+        err = attention_error(o[b], mla_oracle_tail(dec, b))
         assert err <= MLA_SHORT_ATTN_TOL, "seq %d: %g" % (b, err)
 
 
@@ -235,7 +217,7 @@ def test_decode_with_fill_parity(name, layer):
     # attention over the cache with the filled pages and the remaining tails
     for b in range(w.batch):
         if w.mla:   # 32..48-token contexts
-            err = attention_error(o[b], _mla_oracle_tail(dec, b, layer))
+            err = attention_error(o[b], mla_oracle_tail(dec, b, layer))
             assert err <= MLA_SHORT_ATTN_TOL, "seq %d: %g" % (b, err)
             continue
         G = dec.hq // w.num_kv_heads
