@@ -100,7 +100,6 @@ __device__ __forceinline__ uint32_t h2_field(uint32_t word, uint32_t mask) {
   }
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ uint32_t h2_codes(uint32_t masked) { return h2_field<0>(masked, 0xFFFFFFFFu); }
 // The same conversion for a word whose two fields (at bit `shift` of each
 // half) are already masked and OR-ed into 0x6400 (shift constant after
 // unrolling).
