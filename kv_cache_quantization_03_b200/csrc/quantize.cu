@@ -92,6 +92,17 @@ __device__ __forceinline__ float rcp_fast(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+// 1 / x for a row or column sum x >= 0 of the normalisation rounds, finite
+// for x = 0 (an all-zero row or column, whose factor multiplies only zeros).
+// Tiles of one 16-token slice floor x at 2^-100 (one min); longer tiles
+// select 0 for x = 0 (with the floor ptxas spills registers there).  The two
+// agree for x = 0 in effect (a finite factor times zeros) and for every
+// x >= 2^-100.
+template <int TW>
+__device__ __forceinline__ float rcp_sum(float x) {
+  if constexpr (TW == 1) return rcp_fast(fmaxf(x, 0x1p-100f));
+  else return x > 0.f ? rcp_fast(x) : 0.f;
+}
 __device__ __forceinline__ float rsqrt_nr(float x) {
   float y;
   asm("rsqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -572,14 +583,20 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     // Per-round factors: v = (d/T) / R (row) and w = 1 / C (column) keep
     // w = 1 / c^2 of the textbook recursion exactly, so the final column sums
     // are c^2 itself.  A row or column whose sum is exactly 0 holds only
-    // zeros; its factor multiplies nothing and is set to 0 (its stored c is 1).
+    // zeros; its factor multiplies nothing, so it only has to be finite
+    // (rcp_sum; times d/T <= 32 it stays finite; its stored c is 1).  Every
+    // nonzero row sum is at least 2^-60 (2^-46 after the prescale), so the
+    // 2^-100 floor changes no other row.  A nonzero column sum below 2^-100
+    // would need every entry of the column ~2^-50 below its row's largest,
+    // which the rotation of bf16/fp16 rows reaches only by exact cancellation
+    // (an exact zero).
     constexpr float kDT = kLogDT >= 0 ? (float)(1 << kLogDT) : 1.f / (float)(1 << -kLogDT);
     float v_own = 1.f;
     float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
     f2 c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
     for (int it = 0; it < p.iters; ++it) {
       if (it > 0) rk = row_sums(it & 1);
-      v_own = rk > 0.f ? rcp_fast(rk) * kDT : 0.f;
+      v_own = rcp_sum<TW>(rk) * kDT;
       float v[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -615,10 +632,10 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
         }
         ++rounds;
       }
-      w_own.x = c01.x > 0.f ? rcp_fast(c01.x) : 0.f;
-      w_own.y = c01.y > 0.f ? rcp_fast(c01.y) : 0.f;
-      w_own.z = c23.x > 0.f ? rcp_fast(c23.x) : 0.f;
-      w_own.w = c23.y > 0.f ? rcp_fast(c23.y) : 0.f;
+      w_own.x = rcp_sum<TW>(c01.x);
+      w_own.y = rcp_sum<TW>(c01.y);
+      w_own.z = rcp_sum<TW>(c23.x);
+      w_own.w = rcp_sum<TW>(c23.y);
       sc.own[lane] = w_own;
       __syncwarp();
 #pragma unroll
