@@ -611,9 +611,12 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
       for (int k = 0; k < 4; ++k)
         sc.col[k][(lane & ~3) | (t ^ k)] = make_float4(C[2 * k].x, C[2 * k].y, C[2 * k + 1].x, C[2 * k + 1].y);
       __syncwarp();
-      c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
+      {
+        const float4 x0 = sc.col[t][(lane & ~3) | t];
+        c01 = make_float2(x0.x, x0.y), c23 = make_float2(x0.z, x0.w);
+      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 1; i < 4; ++i) {
         const float4 x = sc.col[t][(lane & ~3) | (i ^ t)];
         c01 = add2(c01, make_float2(x.x, x.y));
         c23 = add2(c23, make_float2(x.z, x.w));
