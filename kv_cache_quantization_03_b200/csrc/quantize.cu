@@ -507,14 +507,23 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int tp = 0; tp < 2; ++tp) {
-          f2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+          // one chain of paired FMAs (the ablation instance keeps two, which
+          // spares it a register spill)
+          if constexpr (AXES == 0) {
+            f2 acc = mul2(A[h][tp][0], make_float2(w[0], w[1]));
 #pragma unroll
-          for (int q = 0; q < 8; q += 2) {
-            acc0 = fma2(A[h][tp][q], make_float2(w[2 * q], w[2 * q + 1]), acc0);
-            acc1 = fma2(A[h][tp][q + 1], make_float2(w[2 * q + 2], w[2 * q + 3]), acc1);
+            for (int q = 1; q < 8; ++q) acc = fma2(A[h][tp][q], make_float2(w[2 * q], w[2 * q + 1]), acc);
+            R[h][tp] = acc.x + acc.y;
+          } else {
+            f2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 8; q += 2) {
+              acc0 = fma2(A[h][tp][q], make_float2(w[2 * q], w[2 * q + 1]), acc0);
+              acc1 = fma2(A[h][tp][q + 1], make_float2(w[2 * q + 2], w[2 * q + 3]), acc1);
+            }
+            const f2 s2 = add2(acc0, acc1);
+            R[h][tp] = s2.x + s2.y;
           }
-          const f2 s2 = add2(acc0, acc1);
-          R[h][tp] = s2.x + s2.y;
         }
       float rk = reduce_tokens(R, b1, b2, [](float a, float b) { return a + b; });
       if constexpr (W > 1) {
