@@ -644,6 +644,7 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
         }
         ++rounds;
       }
+      if (it + 1 == p.iters) break;  // the last round's column sums are c^2 itself
       w_own.x = rcp_sum<TW>(c01.x);
       w_own.y = rcp_sum<TW>(c01.y);
       w_own.z = rcp_sum<TW>(c23.x);
