@@ -348,17 +348,25 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
         } else if constexpr (BITS == 2) {
           *reinterpret_cast<uint32_t*>(codes + tok * row_bytes + seg * blk + 4 * g) = pack_crumbs(f);
         } else {  // 3 bits: low-2-bit plane [T][D/4 B], then high-bit plane [T][D/8 B]
-          // Codes 4k..4k+3 gathered into the bytes of one word; a multiply
-          // then compacts their low crumbs (to bits 18..25) and their high
-          // bits (to bits 21..24): the partial products are disjoint fields,
-          // so nothing carries into the result bits.
-          uint32_t lo = 0, hi = 0;
+          // Codes 4k..4k+3 gathered into the bytes of word x[k].  One
+          // multiply moves the word's four low crumbs to its top byte (crumb
+          // of byte j to bits 24 + 2j); one multiply moves the high bits of
+          // two words (the second shifted up by 4) to the top byte (bit j of
+          // the first word to 24 + j, of the second to 28 + j).  Below bit 24
+          // the crumb products sum to less than 2^24 and the high-bit
+          // products are disjoint bits, so nothing carries into the top
+          // byte; byte permutes then collect the top bytes.
+          uint32_t x[4], yl[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint32_t x = gather4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
-            lo |= ((((x & 0x03030303u) * 0x41041u) >> 18) & 0xFFu) << (8 * k);
-            hi |= (((((x >> 2) & 0x01010101u) * 0x204081u) >> 21) & 0xFu) << (4 * k);
+            x[k] = gather4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
+            yl[k] = (x[k] & 0x03030303u) * 0x01041040u;
           }
+          const uint32_t lo =
+              __byte_perm(__byte_perm(yl[0], yl[1], 0x0073u), __byte_perm(yl[2], yl[3], 0x7300u), 0x7610u);
+          const uint32_t y01 = ((x[0] & 0x04040404u) + ((x[1] & 0x04040404u) << 4)) * 0x00408102u;
+          const uint32_t y23 = ((x[2] & 0x04040404u) + ((x[3] & 0x04040404u) << 4)) * 0x00408102u;
+          const uint32_t hi = __byte_perm(y01, y23, 0x0073u);
           *reinterpret_cast<uint32_t*>(codes + tok * (D / 4) + (kBlk / 4) * blk + 4 * g) = lo;
           *reinterpret_cast<uint16_t*>(codes + kTile * (D / 4) + tok * (D / 8) + (kBlk / 8) * blk + 2 * g) =
               (uint16_t)hi;
