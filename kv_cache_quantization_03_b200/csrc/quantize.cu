@@ -611,8 +611,9 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     float v_own = 1.f;
     float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
     f2 c01 = make_float2(0.f, 0.f), c23 = make_float2(0.f, 0.f);
-    for (int it = 0; it < p.iters; ++it) {
-      if (it > 0) rk = row_sums(it & 1);
+    // Column step of a round: the row factors from the row sums rk, then the
+    // column sums c01, c23 of this lane's four channels.
+    auto col_step = [&]() {
       v_own = rcp_sum<TW>(rk) * kDT;
       float v[2][2];
 #pragma unroll
@@ -652,7 +653,11 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
         }
         ++rounds;
       }
-      if (it + 1 == p.iters) break;  // the last round's column sums are c^2 itself
+    };
+    // The column factors of the round just done, to the lanes that hold the
+    // channels.  (The next round's column step passes a __syncwarp before
+    // this buffer is written again.)
+    auto w_step = [&]() {
       w_own.x = rcp_sum<TW>(c01.x);
       w_own.y = rcp_sum<TW>(c01.y);
       w_own.z = rcp_sum<TW>(c23.x);
@@ -664,7 +669,16 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
         const float4 x = sc.own[(lane & ~3) | k];
         w[4 * k] = x.x, w[4 * k + 1] = x.y, w[4 * k + 2] = x.z, w[4 * k + 3] = x.w;
       }
-      __syncwarp();
+    };
+    // Round 0 takes the row sums from above; the last round's column sums
+    // are c^2 itself, so its column factors are not formed.
+    if (p.iters > 0) {
+      col_step();
+      for (int it = 1; it < p.iters; ++it) {
+        w_step();
+        rk = row_sums(it & 1);
+        col_step();
+      }
     }
     float cmax = 1.f;  // largest column factor of the tile
     float4 cv4;        // this lane's four column factors
