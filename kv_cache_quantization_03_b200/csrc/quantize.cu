@@ -103,10 +103,13 @@ __device__ __forceinline__ float rcp_sum(float x) {
   if constexpr (TW == 1) return rcp_fast(fmaxf(x, 0x1p-100f));
   else return x > 0.f ? rcp_fast(x) : 0.f;
 }
-__device__ __forceinline__ float rsqrt_nr(float x) {
-  float y;
-  asm("rsqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y * fmaf(-0.5f * x * y, y, 1.5f);
+// 1 / sqrt(x) of a pair: the approximation and one Newton step,
+// y (1.5 - 0.5 x y y), in paired arithmetic.
+__device__ __forceinline__ f2 rsqrt_nr2(f2 x) {
+  f2 y;
+  asm("rsqrt.approx.f32 %0, %1;" : "=f"(y.x) : "f"(x.x));
+  asm("rsqrt.approx.f32 %0, %1;" : "=f"(y.y) : "f"(x.y));
+  return mul2(y, fma2(mul2(mul2(splat2(-0.5f), x), y), y, splat2(1.5f)));
 }
 
 // Four per-lane values x[h][tp] of tokens 8h + 2t + tp (this lane's channels)
@@ -685,14 +688,15 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     {
       const bool norm = p.iters > 0;
       const float ct[4] = {c01.x, c01.y, c23.x, c23.y};  // c^2 of the owned channels
+      const f2 y01 = rsqrt_nr2(c01), y23 = rsqrt_nr2(c23);
+      const f2 x01 = mul2(c01, y01), x23 = mul2(c23, y23);  // c = c^2 / c
+      const float ys[4] = {y01.x, y01.y, y23.x, y23.y}, cs[4] = {x01.x, x01.y, x23.x, x23.y};
       float cv[4], ic[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float x = ct[i];
-        const float y = rsqrt_nr(x);
         const bool ok = norm && ct[i] > 0.f;
-        ic[i] = ok ? y : 1.f;
-        cv[i] = ok ? x * y : 1.f;
+        ic[i] = ok ? ys[i] : 1.f;
+        cv[i] = ok ? cs[i] : 1.f;
       }
       cmax = fmaxf(fmaxf(cv[0], cv[1]), fmaxf(cv[2], cv[3]));
 #pragma unroll
