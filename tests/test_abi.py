@@ -101,6 +101,8 @@ def test_host_rejections_before_launch(kvq):
     d512 = kvq.make_config(head_dim=256, num_kv_heads=2, num_pages=8)
     assert f(d512, view, fake, fake, None, 16, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
     assert f(c, view, fake, fake, None, 0, fake, fake, 0, raise_on_error=False) == kvq.KVQ_OK
+    # tile ids are 32-bit in the kernel: 2 kinds x 2 kv-heads x 2^29 tiles = 2^31 tiles is refused
+    assert f(c, view, fake, fake, None, 1 << 33, fake, fake, 0, raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED
     dec = kvq.kvq_decode_attention
     ws = kvq.kvq_decode_workspace_bytes(c, 4, 8, 1024)
     assert ws > 0
