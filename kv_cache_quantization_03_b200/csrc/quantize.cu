@@ -607,9 +607,10 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     // (rcp_sum; times d/T <= 32 it stays finite; its stored c is 1).  Every
     // nonzero row sum is at least 2^-60 (2^-46 after the prescale), so the
     // 2^-100 floor changes no other row.  A nonzero column sum below 2^-100
-    // would need every entry of the column ~2^-50 below its row's largest,
-    // which the rotation of bf16/fp16 rows reaches only by exact cancellation
-    // (an exact zero).
+    // needs every entry of the column ~2^-50 below its row's largest in all
+    // rows of the tile (rows whose inputs span ~2^50 and cancel their large
+    // parts exactly in the same channels); such a column gets the factor of
+    // a sum of 2^-100.
     constexpr float kDT = kLogDT >= 0 ? (float)(1 << kLogDT) : 1.f / (float)(1 << -kLogDT);
     float v_own = 1.f;
     float4 w_own = make_float4(1.f, 1.f, 1.f, 1.f);
