@@ -325,9 +325,40 @@ def kernel_names(w):
     return "quantize_kernel<D=128, T=%d>" % w.tile_tokens, "decode_d128 + combine_d128"
 
 
-def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
+def graph_time(fns, steps):
+    """Mean device time (s) of one replay of the calls fns(sp=stream), captured
+    once into a CUDA graph.  A sleep kernel queued first lets the host enqueue
+    every replay before the first one runs, so the time is the graph's own:
+    its kernels and the gaps between them, without host launch costs."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+        for f in fns:
+            f(sp=cap.cuda_stream)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda._sleep(2_000_000)
+    for a, b in ev:
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    t = sum(a.elapsed_time(b) for a, b in ev) / steps / 1e3
+    del g
+    return t
+
+
+def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False, graph=False):
     """Times `steps` steps of workload w on this rank's GPU (CUDA events on the
-    launching stream).  Returns a dict of seconds and byte counts."""
+    launching stream).  Returns a dict of seconds and byte counts.  With
+    graph, the step (and the decode alone) is also timed as a replayed CUDA
+    graph."""
     import numpy as np
     import torch
 
@@ -362,13 +393,15 @@ def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
     stream = torch.cuda.current_stream()
     s_ptr = stream.cuda_stream
 
-    def quantize(d=dev):
-        kvq.kvq_quantize_append(cfg, cache.view, d["k"], d.get("v"), d.get("rope"), w.n_tok, d["dst"], err, s_ptr)
+    def quantize(d=dev, sp=None):
+        kvq.kvq_quantize_append(cfg, cache.view, d["k"], d.get("v"), d.get("rope"), w.n_tok, d["dst"], err,
+                                s_ptr if sp is None else sp)
 
-    def decode(d=dev):
+    def decode(d=dev, sp=None):
         if not q_only:
             kvq.kvq_decode_attention(cfg, cache.view, 0, d["q"], d["bt"], w.tiles_per_seq, d["sl"], w.batch,
-                                     w.num_q_heads, w.softmax_scale, out, work, ws_bytes, err, s_ptr)
+                                     w.num_q_heads, w.softmax_scale, out, work, ws_bytes, err,
+                                     s_ptr if sp is None else sp)
 
     for _ in range(max(warmup, 3)):
         quantize()
@@ -405,6 +438,10 @@ def measure(w, steps, warmup, rank=0, world=1, local=0, e2e=True, clocks=False):
          "t_q": sum(e[0].elapsed_time(e[1]) for e in ev) / steps / 1e3,
          "t_d": sum(e[1].elapsed_time(e[2]) for e in ev) / steps / 1e3,
          "q_only": q_only, "clocks": clk.summary() if clk else None}
+    if graph:
+        r["graph_step_s"] = graph_time([quantize, decode], steps)
+        if not q_only:
+            r["graph_decode_s"] = graph_time([decode], steps)
 
     if e2e:  # inputs from pinned host memory, output back to the host, each step
         # Two input buffers, as a serving loop would keep them: the copy of
@@ -595,12 +632,18 @@ def run_gpu(args, w):
             if name == w.name:
                 continue
             wx = W_WORKLOADS()[name]
-            rx = measure(wx, min(K, 10), 3, e2e=False)
+            rx = measure(wx, min(K, 10), 3, e2e=False, graph=(name == "rt1k"))
             rx["steps"] = min(K, 10)
             sx = summarize(wx, rx, peak)
             sx["tokens_per_s"] = wx.batch * wx.seq_len / (rx["elapsed"] / rx["steps"])
             if name == "rt1k":
                 sx["note"] = "L2-resident: latency, not a roofline figure"
+            if "graph_step_s" in rx:  # the same step replayed as one CUDA graph (no host cost per launch)
+                n_launch = (1 if wx.mla else 2) + (0 if rx["q_only"] else (3 if wx.mla else 2))
+                sx["graph"] = {"step_us": 1e6 * rx["graph_step_s"], "launches_per_step": n_launch,
+                               "note": "device time per replay of the step captured as one CUDA graph"}
+                if "graph_decode_s" in rx:
+                    sx["graph"]["decode_us"] = 1e6 * rx["graph_decode_s"]
             extra[name] = sx
         line["workloads"] = extra
     if world == 1 and not args.no_cpu_baseline:

@@ -123,19 +123,22 @@ struct DecodePlan {
 };
 
 // Split the tiles of each (sequence, kv-head) over CTAs.  kDecodeCtasPerSm
-// CTAs fit on an SM at once, so the split count minimises (waves) x (tiles
-// per warp + a fixed cost of about six tiles for the prologue, the merge of
-// the CTA's warps and the combine), with at least 4 tiles per warp.
+// CTAs fit on an SM at once, so the split count minimises, in sixteenths of
+// a tile's time, (waves) x (tiles per warp + a fixed cost of about six tiles
+// for the prologue and the merge of the CTA's warps) plus one sixteenth per
+// split for its share of the combine (the split partials it reads).  Measured
+// on one B200 for short contexts, a warp's tile costs ~1.5 us and a split
+// ~0.1 us of the combine; at full-GPU sizes the waves term decides.
 DecodePlan decode_plan(int64_t pairs, int64_t max_tiles) {
   DecodePlan d{1, 0};
   if (pairs <= 0 || max_tiles <= 0) return d;
   const int64_t slots = (int64_t)kDecodeCtasPerSm * num_sms();
-  const int64_t cap = (max_tiles + 4 * kDecodeWarps - 1) / (4 * kDecodeWarps);
+  const int64_t cap = (max_tiles + kDecodeWarps - 1) / kDecodeWarps;  // at least one tile per warp
   int64_t best = 1, best_cost = INT64_MAX;
   for (int64_t s = 1; s <= cap && s <= 256; ++s) {
     const int64_t per_warp = (max_tiles + s * kDecodeWarps - 1) / (s * kDecodeWarps);
     const int64_t waves = (pairs * s + slots - 1) / slots;
-    const int64_t cost = waves * (per_warp + 6);
+    const int64_t cost = waves * 16 * (per_warp + 6) + s;
     if (cost < best_cost) best_cost = cost, best = s;
   }
   int64_t tps = (max_tiles + best - 1) / best;

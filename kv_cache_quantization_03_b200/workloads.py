@@ -158,7 +158,7 @@ def half_bits_to_f64(bits: np.ndarray, dtype: str) -> np.ndarray:
 
 def outlier_channels(w: Workload, layer: int, head: int, which: str) -> np.ndarray:
     """Seeded outlier channel set of one (layer, kv-head, K/V); fixed across tokens."""
-    if w.name == "rt1k":
+    if _base_name(w) == "rt1k":
         return np.array([3, 17, 64, 101])
     if w.mla:
         n = round(0.01 * w.head_dim)
