@@ -251,12 +251,18 @@ kvq_status kvq_decode_attention_tail(const kvq_config* cfg, const kvq_cache_view
  * k_tail / v_tail for b) is first quantised into page fill_page[b] of this
  * layer, exactly as kvq_quantize_append would; then attention runs over the
  * cached pages and the remaining tails as in kvq_decode_attention_tail.
- * Both steps are enqueued on `stream` in that order by this one call.
+ * Both steps are enqueued on `stream` in that order by this one call.  For
+ * K/V caches the attention kernel is enqueued as the programmatic dependent
+ * of the fill's quantize launch, so the two overlap: a CTA waits for the
+ * fill only before it reads a page of fill_page (the call's result is the
+ * same as with the steps run one after the other, and the call completes
+ * after both).
  * (The pages are silent on tokens short of a tile; this is the serving
  * reading of the unquantised tail: a tail is quantised when it fills.)
  *   fill_page:   device int32 [batch]: the page that receives b's full tail,
  *                or -1 (no fill); pages must be distinct and outside what
- *                other calls are reading;
+ *                other calls are reading, and in this call fill_page[b]
+ *                appears in no block-table row but b's;
  * the caller describes the state after the fill: block_table row b already
  * ends with fill_page[b], seq_lens[b] counts it, and tail_lens[b] = 0 for a
  * filled sequence (its tail buffer rows are read by the fill only).  The

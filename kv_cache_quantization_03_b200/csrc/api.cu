@@ -337,7 +337,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
                   const int32_t* block_table, int32_t max_pages_per_seq, const int32_t* seq_lens,
                   const void* k_tail, const void* v_tail, const int32_t* tail_lens, int32_t batch,
                   int32_t num_q_heads, float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
-                  uint32_t* dev_error, void* stream) {
+                  uint32_t* dev_error, void* stream, const int32_t* fill_page = nullptr) {
   kvq_status st = check_config(c);
   if (st != KVQ_OK) return st;
   if ((st = check_view(c, cache)) != KVQ_OK) return st;
@@ -428,6 +428,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   p.tail_tokens = c->tile_tokens;
   p.hblock = c->hadamard_block;
   p.test_wait_ns = g_test_wait_ns.load(std::memory_order_relaxed);
+  p.fill_page = fill_page;
   return cuda_status(launch_decode_d128(p, stream));
 }
 
@@ -490,8 +491,10 @@ kvq_status kvq_decode_attention_fill(const kvq_config* c, const kvq_cache_view* 
                      fill_page, dev_error, 1, layer, stream);
   if (st != KVQ_OK) return st;
   // 2) attention over the cache (now holding the filled pages) and the remaining tails
+  // (GQA: the decode overlaps the fill's quantize launch and waits for it
+  // only where it reads a filled page)
   return decode(c, cache, layer, q, block_table, max_pages_per_seq, seq_lens, k_tail, v_tail, tail_lens, batch,
-                num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error, stream);
+                num_q_heads, softmax_scale, out, workspace, workspace_bytes, dev_error, stream, fill_page);
 }
 
 kvq_status kvq_read_error(uint32_t* dev_error, uint32_t* host_bits, void* stream) {

@@ -247,6 +247,11 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+// Waits until the grid this one was launched after as a programmatic
+// dependent has completed and its writes are visible (returns at once in an
+// ordinary launch).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // A device word that nothing ever sets: the testing hook's wait polls it
 // until its time limit runs out.
 __device__ uint32_t g_never_set = 0;
@@ -270,7 +275,10 @@ __device__ __forceinline__ bool wait_never_set(uint32_t ns) {
 // 2t, 2t+1, i.e. kv-head hs = t / 2.  The score MMAs run once per kv-head
 // (each lane keeps the result of its own kv-head); for P V each kv-head's
 // weights are masked to its own columns, so both MMAs add into one result.
-template <int BK, int BV, int NH, int M, int KPC>
+// FILL: the instance for quantise-on-fill calls (p.fill_page set), launched as
+// the programmatic dependent of the fill's quantize launch; the other
+// instance carries none of its waits.
+template <int BK, int BV, int NH, int M, int KPC, bool FILL>
 __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr StageLayout SL = stage_layout(BK, BV, NH, M, KPC);
@@ -309,10 +317,21 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   const int my_n = (t1 > t0 + warp) ? (t1 - t0 - warp + kDW - 1) / kDW : 0;
   // the page id of each of this split's tiles, staged once in shared memory
   int32_t* spg = reinterpret_cast<int32_t*>(bars + kDW * kStages);
+  // quantise-on-fill: the first of this split's tiles on the page the fill
+  // writes for sequence b (INT_MAX: none); copies from there on wait for the
+  // fill's grid
+  __shared__ int fill_lo;
+  int my_fill = INT_MAX;
   {
     const int32_t* btab = p.block_table + (size_t)b * p.max_pages;
-    for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) spg[i] = btab[(t0 + i) >> p.sub_log2];
+    const int32_t fp = FILL ? p.fill_page[b] : -1;
+    for (int i = threadIdx.x; i < t1 - t0; i += kDW * 32) {
+      const int32_t pg = btab[(t0 + i) >> p.sub_log2];
+      spg[i] = pg;
+      if (FILL && fp >= 0 && pg == fp) my_fill = min(my_fill, i);
+    }
   }
+  if (FILL && threadIdx.x == 0) fill_lo = INT_MAX;
   __shared__ uint32_t tmem_slot;
   if (warp == 0) {  // 32 TMEM columns: each warp keeps its lanes' rotated query in its lane quarter
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 32;" ::"r"(smem_u32(&tmem_slot)));
@@ -322,6 +341,10 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tq = tmem_slot + ((uint32_t)(warp * 32) << 16);
+  if constexpr (FILL) {
+    if (my_fill != INT_MAX) atomicMin(&fill_lo, my_fill);
+    __syncthreads();
+  }
 
   // ---- rotated, pre-scaled query of the CTA's 8 heads: lane (g, t) computes head
   // slot g, channels 32t..32t+31, puts them in its slot order (through this
@@ -402,6 +425,7 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
       return;
     }
     const size_t slot = ((size_t)p.layer * p.num_pages + page) * p.num_kv_heads + kvh;
+    if (FILL && li >= fill_lo) wait_prior_grid();  // the fill's quantize grid writes this page
     mbar_arrive_expect_tx(bar, (uint32_t)SL.bytes);
     const uint8_t* ktok = static_cast<const uint8_t*>(p.k.tok);
     const uint8_t* kch = static_cast<const uint8_t*>(p.k.chan);
@@ -613,6 +637,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
     for (int i = stop + 1; i < issued; ++i)
       mbar_wait_bounded(&wbar[i % kStages], (uint32_t)(i / kStages) & 1u, kWaitLimit);
   }
+  // after a fill, this grid ends only after the fill's quantize grid: work
+  // later on the stream sees both complete
+  if (FILL && threadIdx.x == 0) wait_prior_grid();
 
   // ---- merge the CTA's warps, write this split's partial
 #pragma unroll
@@ -786,20 +813,39 @@ __global__ void __launch_bounds__(128) combine_d128_kernel(DecodeParams p) {
       make_float4(o[0] * il, o[1] * il, o[2] * il, o[3] * il);
 }
 
-template <int BK, int BV, int NH, int M, int KPC>
-int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
+template <int BK, int BV, int NH, int M, int KPC, bool FILL>
+int launch_fill(const DecodeParams& p, cudaStream_t s) {
   constexpr StageLayout SL = stage_layout(BK, BV, NH, M, KPC);
   constexpr int kStages = num_stages(NH);
   // stages, then one mbarrier per stage; the warp-merge buffer reuses the stage space
   static_assert(kDW * kStages * SL.bytes >= kDW * 8 * kD * 4 + kDW * 8 * 2 * 4, "merge buffer");
   const size_t smem = (size_t)kDW * kStages * SL.bytes + kDW * kStages * sizeof(uint64_t) +
                       ((size_t)p.tiles_per_split * sizeof(int32_t) + 15) / 16 * 16;
-  auto kern = decode_d128_kernel<BK, BV, NH, M, KPC>;
+  auto kern = decode_d128_kernel<BK, BV, NH, M, KPC, FILL>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.splits, p.batch * p.num_kv_heads / NH);
-  kern<<<grid, kDW * 32, smem, s>>>(p);
+  if constexpr (FILL) {  // a programmatic dependent of the fill's quantize launch just before it
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kDW * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return (int)e;
+  } else {
+    kern<<<grid, kDW * 32, smem, s>>>(p);
+  }
   combine_d128_kernel<<<dim3(p.batch * p.num_kv_heads, (p.group + 3) / 4), 128, 0, s>>>(p);
   return (int)cudaGetLastError();
+}
+template <int BK, int BV, int NH, int M, int KPC>
+int launch_bk_bv(const DecodeParams& p, cudaStream_t s) {
+  return p.fill_page ? launch_fill<BK, BV, NH, M, KPC, true>(p, s) : launch_fill<BK, BV, NH, M, KPC, false>(p, s);
 }
 
 }  // namespace

@@ -94,6 +94,11 @@ struct DecodeParams {
   int tail_tokens;              // T
   int hblock;                   // Hadamard block: 8 .. 128 channels
   uint32_t test_wait_ns;        // testing only: > 0 makes every CTA first wait this long on a flag nothing sets
+  // quantise-on-fill: [B], the page the preceding quantize launch of the same
+  // call writes for sequence b (-1: none); the decode is then launched as its
+  // programmatic dependent and waits for that grid only before it copies a
+  // filled page (and once before it exits); nullptr: an ordinary launch
+  const int32_t* fill_page;
 };
 
 struct MlaDecodeParams {

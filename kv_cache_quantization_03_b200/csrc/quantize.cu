@@ -183,6 +183,7 @@ struct QuantLaunch {
   int rope_dim;
   int hblock;                // Hadamard block (8 .. 128 channels; 512 for the MLA latent)
   float inv_sqrt_b;          // 1/sqrt(hblock)
+  int after_k;               // 1: the V launch, enqueued as the programmatic dependent of the K launch
 };
 
 // Shared memory of one tile whose 512 channels are split over four warps.
@@ -278,6 +279,11 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     quantize_kernel(QuantLaunch p) {
   static_assert(TW == 1 || D == kBlk, "tiles longer than 16 tokens need head_dim 128");
   static_assert(AXES == 0 || (D == kBlk && TW == 1), "the ablation instantiation is for 16 x 128 tiles");
+  // A launch enqueued as this grid's programmatic dependent may start now:
+  // the call's V launch (independent of this K launch), or the decode of a
+  // quantise-on-fill call, which waits for this grid before it reads a page
+  // written here.
+  asm volatile("griddepcontrol.launch_dependents;");
   constexpr int kCW = cta_warps<TW>();
   constexpr int W = D / kBlk;     // warps per tile along channels
   constexpr int kTile = kT * TW;  // tokens per tile
@@ -799,6 +805,10 @@ __global__ void __launch_bounds__(cta_warps<TW>() * 32, 16 / cta_warps<TW>())
     if (warp == 0)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "n"(kTmemCols));
   }
+  // Launched as the programmatic dependent of the call's K launch (the V
+  // launch), the grid ends only after that one: later work on the stream
+  // sees both complete.  In an ordinary launch this returns at once.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 FastDiv make_div(uint32_t d) {
   FastDiv f{d, 0, 0};
@@ -819,7 +829,21 @@ void launch_one(const QuantLaunch& q, int sms, cudaStream_t s) {
   auto kern = quantize_kernel<F16, BITS, D, TW, AXES>;
   // static + dynamic shared memory may pass 48 KB, which needs the opt-in
   if (dyn > 0) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-  kern<<<grid, kCW * 32, dyn, s>>>(q);
+  if (q.after_k) {  // the V launch: independent of the K launch before it, so it may overlap that one's tail
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kCW * 32);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, q);
+  } else {
+    kern<<<grid, kCW * 32, dyn, s>>>(q);
+  }
 }
 
 template <bool F16, int D, int TW, int AXES = 0>
@@ -879,6 +903,7 @@ int launch_quantize(const QuantizeParams& p, bool f16, int head_dim, int tile_to
     q.rope_dim = p.rope_dim;
     q.hblock = p.hblock;
     q.inv_sqrt_b = inv_sqrt_pow2(p.hblock);
+    q.after_k = kind == 1;
     const int e = f16 ? launch_shape<true>(q, head_dim, tile_tokens, sms, s)
                       : launch_shape<false>(q, head_dim, tile_tokens, sms, s);
     if (e != cudaSuccess) return e;

@@ -225,3 +225,36 @@ def test_decode_with_fill_parity(name, layer):
             err = attention_error(o[b, h * G:(h + 1) * G], dec.oracle_tail(b, h, layer))
             assert err <= ATTN_TOL, "seq %d kv-head %d: %g" % (b, h, err)
 
+
+
+@pytest.mark.parametrize("name", ["gqa", "long", "g128"])
+def test_decode_with_fill_of_a_first_page(name):
+    # The fill's pages are read by the decode kernel as soon as its grid
+    # completes: sequence 0's only page is the one being filled (its tiles
+    # are the first copies of their warps), sequence 1 has no page and a
+    # tail, sequence 2 two cached pages and then its filled one.
+    w = W.WORKLOADS[name].scaled(batch=3, seq_len=2 * W.WORKLOADS[name].tile_tokens)
+    T = w.tile_tokens
+    run = QuantRun(w, num_pages=w.num_pages + 2)
+    bt = np.full((w.batch, w.tiles_per_seq + 1), -1, dtype=np.int32)
+    bt[:, :w.tiles_per_seq] = W.block_table(w)
+    fill = np.array([w.num_pages, -1, w.num_pages + 1], dtype=np.int32)
+    bt[0, 0], bt[0, 1:] = fill[0], -1
+    bt[2, w.tiles_per_seq] = fill[2]
+    seq = np.array([T, 0, w.seq_len + T], dtype=np.int32)
+    tl = np.array([0, 7, 0], dtype=np.int32)
+    dec = DecodeRun(run, seq_lens=seq, block_table=bt)
+    kt, vt = W.tail_inputs(w, "k"), W.tail_inputs(w, "v")
+    dec.k_tail_bits, dec.v_tail_bits, dec.tl = kt, vt, tl
+    kvq.kvq_decode_attention_fill(run.cfg, run.cache.view, 0, dec.q, dec.bt_d, dec.maxp, dec.sl_d,
+                                  torch.from_numpy(kt.view(np.int16)).cuda(), torch.from_numpy(vt.view(np.int16)).cuda(),
+                                  torch.from_numpy(tl).cuda(), torch.from_numpy(fill).cuda(), dec.batch, dec.hq,
+                                  w.softmax_scale, dec.out, dec.ws, dec.ws_bytes, run.err)
+    torch.cuda.synchronize()
+    o = dec.out.cpu().numpy().astype(np.float64)
+    assert run.error_bits() == 0
+    G = dec.hq // w.num_kv_heads
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            err = attention_error(o[b, h * G:(h + 1) * G], dec.oracle_tail(b, h, 0))
+            assert err <= ATTN_TOL, "seq %d kv-head %d: %g" % (b, h, err)
