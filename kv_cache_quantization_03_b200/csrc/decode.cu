@@ -281,6 +281,9 @@ __device__ __forceinline__ bool wait_never_set(uint32_t ns) {
 template <int BK, int BV, int NH, int M, int KPC, bool FILL>
 __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // the combine kernel (this grid's programmatic dependent) may start now: it
+  // scores the unquantised tails, then waits for this grid's partials
+  asm volatile("griddepcontrol.launch_dependents;");
   constexpr StageLayout SL = stage_layout(BK, BV, NH, M, KPC);
   constexpr int KG = kgroup_bytes(M, KPC);  // key group-scale bytes of one kv-head's tile
   constexpr int kStages = num_stages(NH);
@@ -695,7 +698,9 @@ __global__ void __launch_bounds__(kDW * 32, 4) decode_d128_kernel(DecodeParams p
 // With a tail, its tokens join as one more partial: their scores q . k and
 // their value sum are taken in the input basis (the rotation is orthogonal,
 // so q~ . k~ = q . k), and the sum is added after the splits' sum is rotated
-// back.
+// back.  The kernel is launched as the decode grid's programmatic dependent:
+// it scores the tail while that grid runs and waits for it before it reads
+// the partials.
 constexpr int kMaxTail = 128;
 __global__ void __launch_bounds__(128) combine_d128_kernel(DecodeParams p) {
   const int pair = blockIdx.x;
@@ -767,6 +772,8 @@ __global__ void __launch_bounds__(128) combine_d128_kernel(DecodeParams p) {
       }
     }
   }
+  // the partials: written by the decode grid this one depends on
+  wait_prior_grid();
   const float* pml = p.part_ml + ((size_t)pair * p.splits * 8 + h) * 2;       // split s at pml + 16 s
   const float* po = p.part_o + ((size_t)pair * p.splits * 8 + h) * kD + 4 * lane;  // split s at po + 8 kD s
   float mx = tm;
@@ -840,7 +847,20 @@ int launch_fill(const DecodeParams& p, cudaStream_t s) {
   } else {
     kern<<<grid, kDW * 32, smem, s>>>(p);
   }
-  combine_d128_kernel<<<dim3(p.batch * p.num_kv_heads, (p.group + 3) / 4), 128, 0, s>>>(p);
+  {  // the combine: a programmatic dependent of the decode grid (its tail scoring overlaps that grid)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(p.batch * p.num_kv_heads, (p.group + 3) / 4);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_d128_kernel, p);
+    if (e != cudaSuccess) return (int)e;
+  }
   return (int)cudaGetLastError();
 }
 template <int BK, int BV, int NH, int M, int KPC>

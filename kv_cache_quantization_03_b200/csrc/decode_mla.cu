@@ -186,6 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
   constexpr int kOffSt = st_offset(BITS);
   constexpr int kStAz = 2 * CB, kStC = kStAz + 2 * kT * 2 * M, kStRope = kStC + 2 * kLat * M;
   extern __shared__ __align__(1024) uint8_t smem[];
+  // the combine kernel (this grid's programmatic dependent) may start now: it
+  // scores the unquantised tails, then waits for this grid's partials
+  asm volatile("griddepcontrol.launch_dependents;");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x & 1, split = blockIdx.x >> 1, b = blockIdx.y;  // r: output half
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + bar_offset(BITS, M));
@@ -624,7 +627,9 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
 // normalise.  With a tail, its tokens join as one more partial: their scores
 // q_lat . latent + q_rope . rope and their latent sum are taken in the input
 // basis (the rotation is orthogonal), and the sum is added after the splits'
-// sum has been rotated back.
+// sum has been rotated back.  Launched as the decode grid's programmatic
+// dependent, it scores the tail while that grid runs and waits for it before
+// it reads the partials.
 constexpr int kMlaMaxTail = 16;
 __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
   __shared__ float buf[kLat];
@@ -671,6 +676,7 @@ __global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
       tv = fmaf(e, lat(t), tv);
     }
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the decode grid's partials
   float mx = tm;
   for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)b * p.splits + s) * kH + h) * 2]);
   float acc = 0.f, l = 0.f;
@@ -727,7 +733,20 @@ int launch_decode_mla(const MlaDecodeParams& p, void* stream) {
     default: e = h ? launch_mla_bits<8, 2>(p, s) : launch_mla_bits<8, 4>(p, s); break;
   }
   if (e != cudaSuccess) return e;
-  combine_mla_kernel<<<p.batch * p.num_q_heads, kLat, 0, s>>>(p);
+  {  // the combine: a programmatic dependent of the decode grid
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(p.batch * p.num_q_heads);
+    cfg.blockDim = dim3(kLat);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = (int)cudaLaunchKernelEx(&cfg, combine_mla_kernel, p);
+    if (e != cudaSuccess) return e;
+  }
   return (int)cudaGetLastError();
 }
 
