@@ -189,6 +189,29 @@ def test_decode_workspace_counts_16_token_tiles(kvq):
         assert len(set(sizes.values())) == 1, (seq, sizes)
 
 
+def test_decode_split_plan(kvq):
+    # The split count, read back from the workspace size (batch x kv-heads x
+    # splits x 8 head slots x (d + 2) floats), on a 148-SM sizing (no device
+    # here): a short sequence spreads its tiles down to one per warp, the
+    # combine's share per split stops it at two per warp for 4096 tokens,
+    # and once the grid is full the wave count decides.
+    import torch
+    if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("split plans are sized by the SM count")
+
+    def splits(batch, seq, kv, hq, T=16):
+        c = kvq.make_config(num_kv_heads=kv, num_pages=8, tile_tokens=T)
+        return kvq.kvq_decode_workspace_bytes(c, batch, hq, seq) / (batch * kv * 8 * 130 * 4)
+
+    assert splits(1, 64, 1, 1) == 1            # 4 tiles: one per warp of one CTA
+    assert splits(1, 1024, 1, 1) == 16         # 64 tiles: one per warp
+    assert splits(1, 4096, 1, 1) == 32         # 256 tiles: two per warp
+    assert splits(3, 512, 8, 32) == 8          # 12 kv-head pairs (two per CTA), 32 tiles each
+    assert splits(32, 8192, 8, 32) == 4        # 128 kv-head pairs x 4 = 512 CTAs of 592 slots
+    assert splits(32, 8192, 8, 32, T=128) == 4  # 128-token pages: the same 16-token tiles
+    assert splits(4, 131072, 8, 64) == 18      # 32 kv-heads (one per CTA) x 18 = 576 CTAs of 592
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     # the product path has no CPU fallback: without libkvq.so the binding refuses to import
     import shutil
