@@ -207,8 +207,8 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch,
  *   num_q_heads: a multiple of num_kv_heads; q head h reads kv-head
  *                h / (num_q_heads / num_kv_heads);
  *   softmax_scale: multiplies q.k (1/sqrt(128) for GQA, 1/sqrt(576) for MLA);
- *   out:         device float32 [batch][num_q_heads][head_dim], un-rotated;
- *                a sequence of length 0 gets zeros;
+ *   out:         device float32 [batch][num_q_heads][head_dim], un-rotated,
+ *                16-byte aligned; a sequence of length 0 gets zeros;
  *   workspace:   device scratch of at least kvq_decode_workspace_bytes(...,
  *                max_seq_len >= every seq_len) bytes, 256-byte aligned; its
  *                contents need no initialisation and are overwritten. */

@@ -347,7 +347,7 @@ kvq_status decode(const kvq_config* c, const kvq_cache_view* cache, int32_t laye
   if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (batch > 0 && (!q || !seq_lens || !out || (max_pages_per_seq > 0 && !block_table)))
     return KVQ_ERR_INVALID_ARG;
-  if (q && !aligned16(q)) return KVQ_ERR_INVALID_ARG;
+  if ((q && !aligned16(q)) || (out && !aligned16(out))) return KVQ_ERR_INVALID_ARG;  // both moved in 16-byte units
   if ((st = check_decode_shape(c)) != KVQ_OK) return st;
   if (c->mla) {
     if (num_q_heads > kMlaHeads) return KVQ_ERR_UNSUPPORTED;

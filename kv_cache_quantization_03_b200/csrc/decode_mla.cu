@@ -624,83 +624,141 @@ __global__ void __launch_bounds__(256) mla_prep_q_kernel(MlaDecodeParams p) {
 }
 
 // Merge the splits of one (sequence, head), rotate back with H_512,
-// normalise.  With a tail, its tokens join as one more partial: their scores
-// q_lat . latent + q_rope . rope and their latent sum are taken in the input
-// basis (the rotation is orthogonal), and the sum is added after the splits'
-// sum has been rotated back.  Launched as the decode grid's programmatic
-// dependent, it scores the tail while that grid runs and waits for it before
-// it reads the partials.
+// normalise: one warp per (sequence, head), four per CTA.  Lane l holds
+// channels 16l .. 16l+15: the rotation's channel bits 0..3 are in-register
+// butterflies, bits 4..8 shuffles across the lanes.  With a tail, its tokens
+// join as one more partial: their scores q_lat . latent + q_rope . rope and
+// their latent sum are taken in the input basis (the rotation is
+// orthogonal), and the sum is added after the splits' sum has been rotated
+// back.  Launched as the decode grid's programmatic dependent, it scores the
+// tail while that grid runs and waits for it before it reads the partials.
 constexpr int kMlaMaxTail = 16;
-__global__ void __launch_bounds__(kLat) combine_mla_kernel(MlaDecodeParams p) {
-  __shared__ float buf[kLat];
-  __shared__ float red[kLat / 32][kMlaMaxTail];  // per warp, per tail token: partial scores
-  __shared__ float ts[kMlaMaxTail];              // tail scores (log2 units)
-  const int b = blockIdx.x / p.num_q_heads, h = blockIdx.x % p.num_q_heads, j = threadIdx.x;
-  const int warp = j >> 5, lane = j & 31;
+__device__ __forceinline__ void unpack8(uint4 w, bool f16, float* x) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (f16) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+      x[2 * e] = v.x, x[2 * e + 1] = v.y;
+    } else {
+      x[2 * e] = bf16f(ws[e] & 0xFFFFu), x[2 * e + 1] = bf16f(ws[e] >> 16);
+    }
+  }
+}
+__global__ void __launch_bounds__(128) combine_mla_kernel(MlaDecodeParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 4 + warp;          // (sequence, head) of this warp
+  if (gw >= p.batch * p.num_q_heads) return;     // (the kernel has no block-wide barrier)
+  const int b = gw / p.num_q_heads, h = gw % p.num_q_heads;
   int L = 0;
   if (p.lat_tail) {
     L = p.tail_lens[b];
     if (L < 0 || L > p.tail_tokens || L > kMlaMaxTail) {
-      if (j == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
+      if (h == 0 && lane == 0) set_error(p.err, KVQ_DEVERR_BAD_SEQ);
       L = 0;
     }
   }
-  float tm = kNegBig, tl = 0.f, tv = 0.f;  // tail: max, sum, value sum of channel j
+  float tm = kNegBig, tl = 0.f, tv[16];  // tail: max, sum, value sums of this lane's channels
+#pragma unroll
+  for (int i = 0; i < 16; ++i) tv[i] = 0.f;
   if (L > 0) {
-    const size_t row0 = ((size_t)p.layer * p.batch + b) * p.tail_tokens;
     const uint16_t* qh = p.q + ((size_t)b * p.num_q_heads + h) * kKf;
-    auto lat = [&](int t) {
-      const uint16_t x = p.lat_tail[(row0 + t) * kLat + j];
-      return p.tail_f16 ? __half2float(__ushort_as_half(x)) : bf16f(x);
+    float ql[16], x[16];
+    unpack8(reinterpret_cast<const uint4*>(qh + 16 * lane)[0], false, ql);
+    unpack8(reinterpret_cast<const uint4*>(qh + 16 * lane)[1], false, ql + 8);
+    const uint32_t qrw = *reinterpret_cast<const uint32_t*>(qh + kLat + 2 * lane);
+    const float qr0 = bf16f(qrw & 0xFFFFu), qr1 = bf16f(qrw >> 16);
+    const size_t row0 = ((size_t)p.layer * p.batch + b) * p.tail_tokens;
+    const bool f16 = p.tail_f16 != 0;
+    auto lat_row = [&](int t, float* v) {
+      const uint4* r = reinterpret_cast<const uint4*>(p.lat_tail + (row0 + t) * kLat + 16 * lane);
+      unpack8(r[0], f16, v);
+      unpack8(r[1], f16, v + 8);
     };
-    const float qj = bf16f(qh[j]), qr = j < kRope ? bf16f(qh[kLat + j]) : 0.f;
-    for (int t = 0; t < L; ++t) {
-      float s = qj * lat(t);
-      if (j < kRope) s = fmaf(qr, bf16f(p.rope_tail[(row0 + t) * kRope + j]), s);
+    float sc[kMlaMaxTail];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      if (lane == 0) red[warp][t] = s;
-    }
-    __syncthreads();
-    if (j < L) {
-      float s = 0.f;
+    for (int t = 0; t < kMlaMaxTail; ++t) {
+      float a = 0.f;
+      if (t < L) {
+        lat_row(t, x);
 #pragma unroll
-      for (int w = 0; w < kLat / 32; ++w) s += red[w][j];
-      ts[j] = s * p.scale_log2;
+        for (int i = 0; i < 16; ++i) a = fmaf(ql[i], x[i], a);
+        const uint32_t rw = *reinterpret_cast<const uint32_t*>(p.rope_tail + (row0 + t) * kRope + 2 * lane);
+        a = fmaf(qr0, bf16f(rw & 0xFFFFu), a);
+        a = fmaf(qr1, bf16f(rw >> 16), a);
+      }
+      sc[t] = a;
     }
-    __syncthreads();
-    for (int t = 0; t < L; ++t) tm = fmaxf(tm, ts[t]);
-    for (int t = 0; t < L; ++t) {
-      const float e = ex2f(ts[t] - tm);
-      tl += e;
-      tv = fmaf(e, lat(t), tv);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int t = 0; t < kMlaMaxTail; ++t) sc[t] += __shfl_xor_sync(0xffffffffu, sc[t], off);
+#pragma unroll
+    for (int t = 0; t < kMlaMaxTail; ++t) {
+      sc[t] = t < L ? sc[t] * p.scale_log2 : kNegBig;
+      tm = fmaxf(tm, sc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kMlaMaxTail; ++t) {
+      if (t < L) {
+        const float e = ex2f(sc[t] - tm);
+        tl += e;
+        lat_row(t, x);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) tv[i] = fmaf(e, x[i], tv[i]);
+      }
     }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the decode grid's partials
   float mx = tm;
   for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_ml[(((size_t)b * p.splits + s) * kH + h) * 2]);
-  float acc = 0.f, l = 0.f;
+  float acc[16], l = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   for (int s = 0; s < p.splits; ++s) {
     const size_t i = ((size_t)b * p.splits + s) * kH + h;
     const float f = ex2f(p.part_ml[i * 2] - mx);
-    acc = fmaf(f, p.part_o[i * kLat + j], acc);
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + i * kLat + 16 * lane);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = po[k];
+      acc[4 * k] = fmaf(f, v.x, acc[4 * k]), acc[4 * k + 1] = fmaf(f, v.y, acc[4 * k + 1]);
+      acc[4 * k + 2] = fmaf(f, v.z, acc[4 * k + 2]), acc[4 * k + 3] = fmaf(f, v.w, acc[4 * k + 3]);
+    }
     l = fmaf(f, p.part_ml[i * 2 + 1], l);
   }
-  buf[j] = acc;
-  __syncthreads();
-  for (int s = 1; s < kLat; s <<= 1) {
-    const float x = buf[j & ~s], y = buf[j | s];
-    __syncthreads();
-    buf[j] = (j & s) ? (x - y) : (x + y);
-    __syncthreads();
+  // H_512: channel bits 0..3 within the lane, bits 4..8 across lanes 1, 2, 4, 8, 16
+#pragma unroll
+  for (int st = 1; st < 16; st <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (!(i & st)) {
+        const float u = acc[i], v = acc[i + st];
+        acc[i] = u + v;
+        acc[i + st] = u - v;
+      }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, acc[i], off);
+      acc[i] = upper ? (o - acc[i]) : (acc[i] + o);
+    }
   }
-  float o = buf[j] * 0.044194173824159216f;
+  float o[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i] = acc[i] * 0.044194173824159216f;  // 1/sqrt(512)
   if (L > 0) {
     const float f = ex2f(tm - mx);
-    o = fmaf(f, tv, o);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = fmaf(f, tv[i], o[i]);
     l = fmaf(f, tl, l);
   }
-  p.out[((size_t)b * p.num_q_heads + h) * kLat + j] = l > 0.f ? o / l : 0.f;
+  const float il = l > 0.f ? 1.f / l : 0.f;
+  float4* out = reinterpret_cast<float4*>(p.out + ((size_t)b * p.num_q_heads + h) * kLat + 16 * lane);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) out[k] = make_float4(o[4 * k] * il, o[4 * k + 1] * il, o[4 * k + 2] * il, o[4 * k + 3] * il);
 }
 
 template <int BITS, int M>
@@ -738,8 +796,8 @@ int launch_decode_mla(const MlaDecodeParams& p, void* stream) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(p.batch * p.num_q_heads);
-    cfg.blockDim = dim3(kLat);
+    cfg.gridDim = dim3((p.batch * p.num_q_heads + 3) / 4);  // one warp per (sequence, head)
+    cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cfg.attrs = attr;

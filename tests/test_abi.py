@@ -113,6 +113,8 @@ def test_host_rejections_before_launch(kvq):
                raise_on_error=False) == kvq.KVQ_ERR_UNSUPPORTED       # group 9 > 8
     assert dec(c, view, 0, fake, fake, 64, fake, 4, 5, 0.1, fake, fake, ws, fake, 0,
                raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # 5 q heads over 2 kv heads
+    assert dec(c, view, 0, fake, fake, 64, fake, 4, 8, 0.1, fake + 4, fake, ws, fake, 0,
+               raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG       # out not 16-byte aligned
     assert dec(c, view, 0, fake, fake, 64, fake, 4, 8, float("nan"), fake, fake, ws, fake, 0,
                raise_on_error=False) == kvq.KVQ_ERR_INVALID_ARG
     assert dec(c, view, 1, fake, fake, 64, fake, 4, 8, 0.1, fake, fake, ws, fake, 0,
