@@ -38,7 +38,15 @@
  * word).  The library never allocates, frees or synchronises, except
  * kvq_read_error, which synchronises the given stream.  Every call that
  * takes a stream only enqueues work on it (a cudaStream_t passed as void*;
- * NULL = the legacy default stream) and returns.  Calls are thread-safe.
+ * NULL = the legacy default stream) and returns.  Calls are thread-safe,
+ * and the work they enqueue can be captured into a CUDA graph.  Within a
+ * call, a kernel may be enqueued as the programmatic dependent of the one
+ * before it (CUDA's programmatic dependent launch); a call's last kernel
+ * completes only after all of the call's kernels.  The library's kernels
+ * also let a dependent start early: a kernel the caller enqueues right
+ * after a call with programmatic stream serialisation must wait for its
+ * prerequisite grid (cudaGridDependencySynchronize) before it reads the
+ * call's results.
  *
  * Errors: every function returns kvq_status; nothing is thrown across the
  * ABI.  Host-detectable problems (null pointers, unsupported shapes or bit
