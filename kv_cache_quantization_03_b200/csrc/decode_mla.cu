@@ -505,7 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mla_kernel(MlaDecodeParams
       const int x = nchunks - 1;
       ok &= mbar_wait_bounded(&pv[x & 3], (uint32_t)(x >> 2) & 1u, ok ? kWaitLimit : 0u);
       tc_fence_after();
-#pragma unroll 1
       const float s_out = __uint_as_float((uint32_t)(127 + e_ref) << 23);  // 2^e_ref
       for (int c0 = 0; c0 < kHalf; c0 += 32) {
         float o[32];
