@@ -72,3 +72,21 @@ def test_traffic_lookup_needs_the_matching_source_hash(tmp_path, monkeypatch):
     assert bench.traffic_from_profile("k.cu", "q.md") is None      # the kernel changed since the capture
     assert bench.traffic_from_profile("k.cu", "missing.md") is None
 
+
+
+def test_algorithmic_bytes_of_the_benched_configs():
+    # the totals behind the reported bandwidths, from the per-row byte counts of the cache format
+    lng = W.WORKLOADS["long"]          # 3-bit K: 48 B codes + 8 B (a, z) + 32 B of c; 4-bit V: 64 + 8 + 32
+    q, d = bench.algorithmic_bytes(lng)
+    rows = lng.n_tok * lng.num_kv_heads
+    assert q == rows * 2 * 256 + rows * (88 + 104) == 2952790016
+    assert d == lng.batch * lng.seq_len * 8 * 192 + lng.batch * 64 * 128 * 6 == 805502976
+    mla = W.WORKLOADS["mla"]           # latent 256 B codes + 8 B (a, z) + 128 B of c, rope 128 B in and out
+    q, d = bench.algorithmic_bytes(mla)
+    assert q == mla.n_tok * (1024 + 128) + mla.n_tok * (392 + 128) == 3506438144
+    assert d == mla.batch * mla.seq_len * 520 + mla.batch * 128 * (576 * 2 + 512 * 4) == 1116733440
+    g = W.WORKLOADS["g128"]            # 128-token pages: 4-bit K 64 + 8 + 4, 2-bit V 32 + 8 + 4 = 120 B
+    q, d = bench.algorithmic_bytes(g)
+    rows = g.n_tok * g.num_kv_heads
+    assert q == rows * 2 * 256 + rows * 120
+    assert d == g.batch * g.seq_len * 8 * 120 + g.batch * 32 * 128 * 6
